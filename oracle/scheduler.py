@@ -1,0 +1,187 @@
+"""Iteration-level (continuous) batching, plain Python model (oracle; test
+infrastructure only).
+
+Policy ([P1] "大模型推理引擎高频优化：连续批处理、PagedAttention 与 KV Cache 实战拆解",
+section 2.2, Scheduler.schedule; [P3] "大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置",
+section "连续批处理Continuous Batching配置"), one call of ``step()``:
+
+1. Finished sequences leave the batch and return their blocks.
+2. Admission, first-come first-served: with a block budget equal to the free
+   block count, take the head of the waiting queue while its required blocks
+   fit the budget, charge the budget, and stop at the first request that does
+   not fit (it stays at the head; the pages' pseudocode stops with ``break``).
+   ``required = ceil(unshared_tokens / block_size) + 1`` (room for the first
+   generated token; +1 more when the request forks a parallel-sampling child).
+   The number of running sequences is also capped (``max_running``, the
+   pages' max-num-seqs).  An admitted request's prompt is placed: a
+   prefix-sharing request forks the resident prefix holder (shares its blocks
+   by reference) and appends its own tokens; any other request allocates its
+   tokens.  A request with a fork child then forks it (the child shares every
+   block, including a partly filled last one).
+3. Every running sequence, in admission order, reserves the slot of its next
+   token.  When the pool is exhausted, the most recently admitted running
+   sequence is preempted: its blocks are freed and it goes back to the FRONT of
+   the waiting queue, keeping its progress; on re-admission its whole history
+   is written again (recompute).  ([P2] "vLLM推理加速框架：PagedAttention与连续批处理技术解析",
+   section 3.2 names preemptive scheduling without an algorithm; this is the
+   reading adopted.)  Copy-on-write pairs from the block manager are reported.
+4. Each running sequence has generated one more token; it finishes once it has
+   generated ``output_len`` tokens (removed at the start of the next step).
+
+``step()`` returns a record of everything the device must do and everything a
+checker compares: cache writes (seq, position, slot) in issue order, CoW
+pairs, admitted / preempted / finished ids, and the running batch with its
+context lengths.  ``ops`` holds the writes and CoW copies interleaved in
+issue order: a copy must see every earlier write to its source block and none
+of the later ones, so the device has to apply them in that order.
+"""
+
+from dataclasses import dataclass, field
+
+from .block_manager import NoBlocks, ceil_div
+
+
+@dataclass
+class Request:
+    seq_id: int
+    prompt_len: int            # tokens of the request's own (unshared) prompt
+    output_len: int            # tokens to generate before finishing
+    shares_prefix: bool = False
+    fork_child: int = -1       # id of a parallel-sampling child, -1 for none
+    fork_output_len: int = 0
+
+
+@dataclass
+class _Seq:
+    seq_id: int
+    output_len: int
+    shares_prefix: bool
+    history: int               # tokens held (prefix included) while running
+    generated: int = 0
+    fork_child: int = -1
+    fork_output_len: int = 0
+    forked: bool = False
+    is_child: bool = False
+
+
+@dataclass
+class StepRecord:
+    finished: list = field(default_factory=list)
+    admitted: list = field(default_factory=list)
+    preempted: list = field(default_factory=list)
+    writes: list = field(default_factory=list)      # (seq, position, slot)
+    cow: list = field(default_factory=list)         # (src, dst)
+    ops: list = field(default_factory=list)         # ("w", seq, pos, slot) | ("c", src, dst)
+    running: list = field(default_factory=list)     # seq ids, admission order
+    context_lens: list = field(default_factory=list)
+
+    def write(self, seq, pos, slot):
+        self.writes.append((seq, pos, slot))
+        self.ops.append(("w", seq, pos, slot))
+
+    def copy(self, src, dst):
+        self.cow.append((src, dst))
+        self.ops.append(("c", src, dst))
+
+
+class Scheduler:
+    def __init__(self, bm, max_running, prefix_seq=-1):
+        self.bm = bm
+        self.max_running = int(max_running)
+        self.prefix_seq = prefix_seq
+        self.prefix_len = bm.context_len(prefix_seq) if prefix_seq >= 0 else 0
+        self.waiting = []          # list of _Seq, FCFS order
+        self.running = []          # list of _Seq, admission order
+
+    def add_request(self, req):
+        if req.shares_prefix and self.prefix_seq < 0:
+            raise ValueError("prefix-sharing request without a prefix holder")
+        base = self.prefix_len if req.shares_prefix else 0
+        self.waiting.append(_Seq(req.seq_id, req.output_len, req.shares_prefix,
+                                 base + req.prompt_len, 0, req.fork_child,
+                                 req.fork_output_len))
+
+    def _unshared(self, s):
+        return s.history - (self.prefix_len if s.shares_prefix else 0)
+
+    def _required(self, s):
+        need = ceil_div(self._unshared(s), self.bm.block_size) + 1
+        if s.fork_child >= 0 and not s.forked:
+            need += 1
+        return need
+
+    def _admit(self, s, rec):
+        bm = self.bm
+        if s.shares_prefix:
+            bm.fork(self.prefix_seq, s.seq_id)
+            for pos in range(self.prefix_len, s.history):
+                slot, src, dst = bm.append_slot(s.seq_id)
+                if src >= 0:
+                    rec.copy(src, dst)
+                rec.write(s.seq_id, pos, slot)
+        else:
+            bm.allocate(s.seq_id, s.history)
+            for pos, slot in enumerate(bm.slots(s.seq_id, 0, s.history)):
+                rec.write(s.seq_id, pos, slot)
+        self.running.append(s)
+        rec.admitted.append(s.seq_id)
+        if s.fork_child >= 0 and not s.forked:
+            s.forked = True
+            bm.fork(s.seq_id, s.fork_child)
+            child = _Seq(s.fork_child, s.fork_output_len, s.shares_prefix,
+                         s.history, 0, is_child=True)
+            self.running.append(child)
+            rec.admitted.append(child.seq_id)
+
+    def _preempt_last(self, rec):
+        victim = self.running.pop()
+        self.bm.free(victim.seq_id)
+        self.waiting.insert(0, victim)
+        rec.preempted.append(victim.seq_id)
+        return victim
+
+    def step(self):
+        rec = StepRecord()
+        bm = self.bm
+        # 1. finish
+        keep = []
+        for s in self.running:
+            if s.generated >= s.output_len:
+                bm.free(s.seq_id)
+                rec.finished.append(s.seq_id)
+            else:
+                keep.append(s)
+        self.running = keep
+        # 2. admit (FCFS, stop at the first request that does not fit)
+        budget = bm.num_free
+        while self.waiting and budget > 0 and len(self.running) < self.max_running:
+            s = self.waiting[0]
+            need = self._required(s)
+            if need > budget:
+                break
+            extra = 1 if (s.fork_child >= 0 and not s.forked) else 0
+            if len(self.running) + 1 + extra > self.max_running:
+                break
+            self.waiting.pop(0)
+            budget -= need
+            self._admit(s, rec)
+        # 3. reserve the next token's slot for every running sequence
+        i = 0
+        while i < len(self.running):
+            s = self.running[i]
+            try:
+                slot, src, dst = bm.append_slot(s.seq_id)
+            except NoBlocks:
+                victim = self._preempt_last(rec)
+                if victim is s:
+                    continue          # the sequence itself was preempted
+                continue              # retry the same sequence
+            if src >= 0:
+                rec.copy(src, dst)
+            rec.write(s.seq_id, s.history, slot)
+            s.history += 1
+            s.generated += 1
+            i += 1
+        rec.running = [s.seq_id for s in self.running]
+        rec.context_lens = [s.history for s in self.running]
+        return rec
