@@ -1,0 +1,407 @@
+"""Benchmark of the paged decode step (cache write of one new token per
+sequence + decode attention over the block tables) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 70b|7b|long|tiny]
+    python bench.py --impl reference ...      # the CPU oracle, same workload
+
+Prints one JSON line.  ``value`` is KV bytes read per second over the whole
+step (cache write + plan + decode + reduce), inputs resident in HBM, L2
+flushed between steps (the flush is outside the per-step events).  ``e2e`` is
+the same metric through ``pa_step`` with pinned host buffers, host<->device
+copies inside the timed region.  ``roofline`` is the decode kernel's achieved
+bandwidth (algorithmic bytes / its average event-timed duration) against the
+measured HBM copy bandwidth.  N > 1 runs independent replicas (one per GPU,
+no data-path collective; weak scaling).
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_381_b200 import workloads as wl  # noqa: E402
+
+WORKLOAD_NAMES = {
+    "70b": "llama3-70b-shaped decode layer: bf16, 64 q / 8 kv heads (GQA 8), head_dim 128, block 16, "
+           "256 seqs, contexts ~ Zipf(1.2) on [16, 8192], shuffled physical blocks",
+    "7b": "llama2-7b-shaped decode layer: fp16, 32 q / 32 kv heads, head_dim 128, block 16, 64 seqs, "
+          "contexts ~ U[128, 2048]",
+    "long": "long-context split-K: bf16, 64 q / 8 kv heads, head_dim 128, block 16, 8 seqs x 32768 tokens, "
+            "512-token partitions, 1% of K rows x8",
+    "tiny": "tiny fp32 paged decode: 4 seqs {1,16,17,90}, 4/4 heads, head_dim 64, block 16, 32-block pool",
+}
+METRIC = "paged decode attention: KV GB/s read (% of B200 HBM peak); decode tokens/s"
+KERNEL_SOURCES = ["paged_kv_cache_381_b200/csrc/device/decode.cuh",
+                  "paged_kv_cache_381_b200/csrc/device/common.cuh"]
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--workload", default="70b", choices=list(WORKLOAD_NAMES))
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"decode_{workload}_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        j = json.load(f)
+    if j.get("kernel_source_sha256_16") != kernel_hash():
+        return None
+    return j.get("dram_bytes_per_launch")
+
+
+def elt_bytes(dtype):
+    return wl.ELEMENT_BYTES[dtype]
+
+
+def kv_bytes(cfg, lens):
+    return int(np.sum(lens)) * 2 * cfg.num_kv_heads * cfg.head_dim * elt_bytes(cfg.dtype)
+
+
+def decode_kernel_bytes(cfg, lens, partition):
+    """Algorithmic bytes one decode-kernel launch must move: live K/V rows, q,
+    the final rows of one-partition sequences, the fp32 partials (o, m, l) of
+    split sequences, and the block-table entries each kv head reads."""
+    e = elt_bytes(cfg.dtype)
+    S, Hq, Hkv, D, bs = len(lens), cfg.num_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
+    P = partition or 512
+    maxc = int(np.max(lens)) if S else 0
+    nparts = np.where(lens <= P, 1, -(-lens // P)) if maxc > P else np.ones(S, dtype=np.int64)
+    single = nparts == 1
+    b = kv_bytes(cfg, lens)
+    b += S * Hq * D * e                                   # q
+    b += int(single.sum()) * Hq * D * e                   # final rows
+    b += int(nparts[~single].sum()) * Hq * (D + 2) * 4    # partials
+    b += int(np.sum(-(-lens // bs))) * Hkv * 4            # block-table entries
+    return int(b)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(cfg, seed, seqs, lens):
+    """Host histories for the sampled sequences (numpy draws of the same shape)."""
+    r = np.random.default_rng([seed, 7])
+    Hq, Hkv, D = cfg.num_heads, cfg.num_kv_heads, cfg.head_dim
+    items = []
+    for s in seqs:
+        n = int(lens[s])
+        q = wl.normal_storage(r, (Hq, D), cfg.dtype)
+        k = wl.normal_storage(r, (n, Hkv, D), cfg.dtype)
+        v = wl.normal_storage(r, (n, Hkv, D), cfg.dtype)
+        items.append((q, k, v))
+    return items
+
+
+def _time_oracle(cfg, items):
+    from oracle import attention as oa
+    from oracle.numerics import widen
+    t0 = time.perf_counter()
+    for q, k, v in items:
+        oa.decode_history(widen(q, cfg.dtype), widen(k, cfg.dtype), widen(v, cfg.dtype), cfg.scale)
+    return time.perf_counter() - t0
+
+
+def _single_thread():
+    """Context manager limiting BLAS to one thread (no-op if unavailable)."""
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=1)
+    except ImportError:
+        import contextlib
+        return contextlib.nullcontext()
+
+
+def cpu_baseline(cfg, seed, lens, unit_scale):
+    """The oracle, as it stands, on every 4th sequence of the workload."""
+    seqs = list(range(0, len(lens), 4)) or [0]
+    items = _oracle_sample(cfg, seed, seqs, lens)
+    with _single_thread():
+        secs = _time_oracle(cfg, items)
+    b = kv_bytes(cfg, lens[seqs])
+    return {"value": b / secs / unit_scale, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(seqs)} of {len(lens)} sequences (every 4th), all {cfg.num_heads} query heads, "
+                      f"float64 numpy, 1 BLAS thread, {secs:.2f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = wl.CONFIGS[args.workload]
+    lens = wl.context_lengths(cfg, wl.rng(args.seed))
+    seqs = list(range(0, len(lens), 4)) or [0]
+    items = _oracle_sample(cfg, args.seed, seqs, lens)
+    sample_bytes = kv_bytes(cfg, lens[seqs])
+    with _single_thread():
+        for _ in range(args.warmup):
+            _time_oracle(cfg, items[:1])
+        times = [_time_oracle(cfg, items) for _ in range(args.steps)]
+    secs = sum(times) / len(times)
+    value = sample_bytes / secs / 1e9
+    sample = (f"{len(seqs)} of {len(lens)} sequences (every 4th) per step, all {cfg.num_heads} query heads, "
+              f"float64 numpy, 1 BLAS thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAMES[args.workload], "num_seqs": len(lens),
+                       "kv_bytes_per_step": sample_bytes, "parallelism": "replicas"},
+            "tokens_per_s": len(seqs) / secs,
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# native arm
+# ---------------------------------------------------------------------------
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    from paged_kv_cache_381_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    import paged_kv_cache_381_b200 as pa
+    from paged_kv_cache_381_b200.batch import PagedBatch
+
+    cfg = wl.CONFIGS[args.workload]
+    seed = args.seed + rank                       # independent replica per rank
+    d = wl.draw_device(cfg, seed, device=dev)
+    batch = PagedBatch(d.k_hist, d.v_hist, d.offsets, d.context_lens, d.num_blocks, cfg.block_size, d.free_order)
+    lens = d.context_lens
+    q = d.q
+    out = torch.empty_like(q)
+    P = cfg.partition_size
+    batch.ensure_workspace(cfg.num_heads, P)
+    step_kv = kv_bytes(cfg, lens)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    del d.k_hist, d.v_hist
+    torch.cuda.synchronize()
+    pa.pa_get_device_error()
+
+    def step():
+        batch.write_new_tokens()
+        batch.decode(out, q, cfg.scale, partition_size=P)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = pa.launch_count()
+    pa.profile_begin()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+        flush.zero_()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    prof = pa.profile_end()
+    launches = pa.launch_count() - launches0
+    clk = clocks.stop()
+    err = pa.pa_get_device_error()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = sum(step_ms) / len(step_ms)
+    dec_ms = prof["decode"][0] / max(1, prof["decode"][1])
+    if world > 1:
+        t = torch.tensor([ms, dec_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, dec_ms = float(t[0]), float(t[1])
+
+    # ---- e2e: the same step from pinned host buffers through pa_step
+    e2e = None
+    if not args.no_e2e:
+        S, Hq, D = q.shape
+        host = {"q": q.cpu().pin_memory(), "k": batch.k_new.cpu().pin_memory(), "v": batch.v_new.cpu().pin_memory(),
+                "slot_mapping": batch.slot_mapping.cpu().pin_memory(),
+                "block_tables": batch.block_tables.cpu().pin_memory(),
+                "context_lens": batch.context_lens.cpu().pin_memory(),
+                "out": torch.empty_like(q, device="cpu").pin_memory()}
+        devb = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+        devb["workspace"] = batch.workspace
+        h2d = sum(host[k].numel() * host[k].element_size() for k in host if k != "out")
+        d2h = host["out"].numel() * host["out"].element_size()
+
+        def e2e_step():
+            pa.pa_step(host, devb, batch.k_cache, batch.v_cache, cfg.scale, batch.max_context_len, P)
+
+        for _ in range(3):
+            e2e_step()
+            flush.zero_()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(args.steps):
+            ev2[i][0].record()
+            e2e_step()
+            ev2[i][1].record()
+            flush.zero_()
+        torch.cuda.synchronize()
+        ems = sum(a.elapsed_time(b) for a, b in ev2) / args.steps
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t[0])
+        e2e = {"value": world * step_kv / (ems * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": ems,
+               "tokens_per_s": world * len(lens) / (ems * 1e-3)}
+
+    peak, peak_kind = measured_peaks()
+    dec_bytes = decode_kernel_bytes(cfg, lens, P)
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(args.workload)
+    value = world * step_kv / (ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES[args.workload], "num_seqs": len(lens),
+                   "context_tokens": int(lens.sum()), "kv_bytes_per_step": step_kv,
+                   "partition_size": P or 512, "l2": "flushed between steps (256 MiB write, outside step events)",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "pct_of_hbm_peak": value / world / peak,
+        "tokens_per_s": world * len(lens) / (ms * 1e-3),
+        "kernel_ms": {k: v[0] / max(1, v[1]) for k, v in prof.items() if v[1]},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "kernel": "decode_kernel", "algorithmic_bytes": dec_bytes,
+                     "peak_source": peak_kind},
+        "gpu_launches": int(launches), "device_error_flags": err, "wall_s": wall,
+        "e2e": e2e, "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cfg, args.seed, lens, 1e9)
+    if rank == 0:
+        print(json.dumps(result))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,326 @@
+/*
+ * pa.h -- C ABI of the paged KV-cache decode library (libpa.so, sm_100a).
+ *
+ * Pages this interface follows (cited by title and section):
+ *   [P1] "大模型推理引擎高频优化：连续批处理、PagedAttention 与 KV Cache 实战拆解"
+ *        section 2.2 (iteration-level scheduler), 3.2 (fixed-size blocks, block
+ *        table, a new block only when the current one is full), 3.3 (allocate /
+ *        append_token).
+ *   [P2] "vLLM推理加速框架：PagedAttention与连续批处理技术解析"
+ *        section 2.1 (Block: ref_count, data of shape (BLOCK_SIZE, NUM_HEADS,
+ *        HEAD_SIZE)), 2.2 (memory pool, copy-on-write, block-level kernel
+ *        scheduling), 3.2 (preemptive scheduling), 6.2 (kernel signature
+ *        paged_attention_kernel(out, q, k, v, block_tables)).
+ *   [P3] "大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置"
+ *        section "PagedAttention分页注意力机制原理" (block table lookup inside the
+ *        attention kernel over non-contiguous blocks, prefix sharing by
+ *        reference, free-block pool) and "连续批处理Continuous Batching配置".
+ *
+ * Conventions for every call below
+ * --------------------------------
+ * Ownership.  All tensors are owned by the caller.  Device pointers must point
+ *   to memory of the current CUDA device; host pointers to ordinary (ideally
+ *   pinned) host memory.  The library never allocates device memory: scratch
+ *   space for the split-K path is passed in (pa_decode_workspace_size).  The
+ *   host block manager and scheduler own only host memory.
+ * Layouts (all row-major, contiguous):
+ *   q, out          [num_seqs, num_heads, head_dim]
+ *   k, v (new rows) [num_tokens, num_kv_heads, head_dim]
+ *   k_cache,v_cache [num_blocks, block_size, num_kv_heads, head_dim]   (one
+ *                   pool for K, one for V; [P2] 2.1's block data shape)
+ *   block_tables    int32 [num_seqs, max_blocks_per_seq]; entry j of row s is
+ *                   the physical block holding logical tokens
+ *                   [j*block_size, (j+1)*block_size) of sequence s.  Entries
+ *                   at or past ceil(context_len/block_size) are never read.
+ *   context_lens    int32 [num_seqs]; tokens held by each sequence, the
+ *                   current step's new token included.
+ *   slot_mapping    int64 [num_tokens]; slot = block*block_size + offset;
+ *                   negative = padding token, not written.
+ * Supported shapes.  dtype in {PA_F32, PA_F16, PA_BF16}; head_dim in {64, 128};
+ *   block_size in {8, 16, 32}; num_heads % num_kv_heads == 0; base pointers
+ *   16-byte aligned.  Anything else returns PA_ERR_UNSUPPORTED or
+ *   PA_ERR_INVALID_ARG before any launch.
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Device calls are asynchronous on that stream.
+ * Errors.  Argument errors are reported synchronously before any launch.
+ *   A failed launch returns PA_ERR_CUDA.  Device-side data (block ids, slots,
+ *   context lengths) are preconditions; the kernels check them anyway, clamp
+ *   or skip the bad access (never faulting), and set bits in a device error
+ *   word read by pa_get_device_error.
+ * Threads.  Calls on different streams may run concurrently; a pa_bm or
+ *   pa_sched object must not be used from two threads at once.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* malformed argument, unknown sequence id */
+    PA_ERR_UNSUPPORTED = 2,   /* shape / dtype outside the supported set */
+    PA_ERR_NO_BLOCKS = 3,     /* free list cannot satisfy the request */
+    PA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    PA_ERR_DEVICE = 5         /* a kernel flagged bad device data or a timeout */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+/* Geometry of one K or V pool. */
+typedef struct {
+    int num_blocks;
+    int block_size;
+    int num_kv_heads;
+    int head_dim;
+    pa_dtype dtype;
+} pa_cache_desc;
+
+/* Bits of the device error word. */
+#define PA_DEVERR_SLOT        0x1u  /* cache write: slot >= num_blocks*block_size (skipped) */
+#define PA_DEVERR_BLOCK_ID    0x2u  /* decode / copy: block id outside [0, num_blocks) (clamped / skipped) */
+#define PA_DEVERR_CONTEXT_LEN 0x4u  /* decode: context_len < 0, > max_context_len or > table width (clamped) */
+#define PA_DEVERR_TIMEOUT     0x8u  /* decode: a bounded wait on a staging barrier expired (CTA abandoned its work) */
+
+/* ------------------------------------------------------------------------ */
+/* Device hot path                                                           */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * pa_cache_write -- append each new token's K/V to its slot ([P1] 3.2-3.3: the
+ * new token is written at the end of the sequence's current block, or at the
+ * start of a freshly taken block).
+ *   k, v            device, [num_tokens, Hkv, D] of cache->dtype
+ *   k_cache,v_cache device pools described by `cache`
+ *   slot_mapping    device int64 [num_tokens]
+ * For every t with slot_mapping[t] >= 0:
+ *   k_cache[slot / bs][slot % bs][:][:] = k[t][:][:]   (same for v), bit-exact.
+ * num_tokens == 0 is a no-op.
+ */
+pa_status pa_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens,
+                         const pa_cache_desc* cache, void* stream);
+
+/*
+ * Scratch bytes pa_decode needs for a batch of this shape.  Zero when the
+ * whole batch fits one partition (max_context_len <= partition size) -- the
+ * single-pass path uses no scratch.  partition_size 0 = library default (512).
+ */
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim,
+                                int max_context_len, int partition_size);
+
+/*
+ * pa_decode -- one decode step of paged attention over a continuous batch
+ * ([P3] "PagedAttention分页注意力机制原理": the kernel resolves each logical block
+ * through the block table and runs attention over non-contiguous physical
+ * blocks; [P2] 6.2: out, q, k, v, block_tables).
+ *   out             device [num_seqs, num_heads, head_dim] (written)
+ *   q               device [num_seqs, num_heads, head_dim]
+ *   k_cache,v_cache device pools [num_blocks, block_size, num_kv_heads, head_dim]
+ *   block_tables    device int32 [num_seqs, max_blocks_per_seq]
+ *   context_lens    device int32 [num_seqs]
+ *   scale           softmax scale applied to the fp32 dot products
+ * For sequence s with n = context_lens[s] tokens and query head h, kv head
+ * g = h / (num_heads / num_kv_heads):
+ *   out[s][h] = sum_t softmax_t(scale * q[s][h] . K_s[t][g]) * V_s[t][g]
+ * with fp32 accumulation and an fp32 softmax; n == 0 writes a zero row.
+ * Contexts longer than the partition size (partition_size, 0 = 512 tokens)
+ * are split into partitions whose partial results are merged by a
+ * log-sum-exp reduction; the workspace (device, >= pa_decode_workspace_size
+ * bytes, 256-byte aligned, contents undefined on entry) holds the partials.
+ * max_context_len must bound every context_lens[s]; larger values are clamped
+ * and flagged (PA_DEVERR_CONTEXT_LEN).
+ */
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, float scale,
+                    int block_size, int num_kv_heads,
+                    int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                    int max_context_len, int num_blocks, pa_dtype dtype,
+                    int partition_size, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write support ([P2] 2.2: a shared block is copied
+ * before it is written).  pairs: device int32 [num_pairs][2] of (src, dst)
+ * physical block ids; copies the whole block (all block_size slots, all heads)
+ * in both pools.  Destinations must be distinct and must not appear as a
+ * source in the same call.  Out-of-range ids are skipped and flagged.
+ */
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int num_pairs,
+                         const pa_cache_desc* cache, void* stream);
+
+/*
+ * pa_step -- one layer-step driven from HOST buffers: copies the step's inputs
+ * host->device (one cudaMemcpyAsync per buffer), runs pa_copy_blocks (when
+ * num_cow > 0), pa_cache_write and pa_decode, and copies `out` back
+ * device->host.  The caller provides the device staging buffers (no
+ * allocation here).  Returns once the work is enqueued; the host output is
+ * valid after the stream synchronizes.
+ */
+typedef struct {
+    /* host inputs */
+    const void* q;               /* [num_seqs, num_heads, head_dim] */
+    const void* k;               /* [num_tokens, num_kv_heads, head_dim] */
+    const void* v;
+    const int64_t* slot_mapping; /* [num_tokens] */
+    const int32_t* block_tables; /* [num_seqs, max_blocks_per_seq] */
+    const int32_t* context_lens; /* [num_seqs] */
+    const int32_t* cow_pairs;    /* [num_cow][2], may be NULL when num_cow == 0 */
+    /* host output */
+    void* out;                   /* [num_seqs, num_heads, head_dim] */
+} pa_step_host;
+
+typedef struct {
+    /* device staging buffers of the same shapes as pa_step_host's */
+    void* q; void* k; void* v;
+    int64_t* slot_mapping; int32_t* block_tables; int32_t* context_lens;
+    int32_t* cow_pairs; void* out;
+    void* workspace; size_t workspace_bytes;
+} pa_step_device;
+
+typedef struct {
+    int num_seqs, num_heads, num_kv_heads, head_dim;
+    int block_size, num_blocks, max_blocks_per_seq, max_context_len;
+    int num_tokens, num_cow;
+    pa_dtype dtype;
+    float scale;
+    int partition_size;
+} pa_step_shape;
+
+pa_status pa_step(const pa_step_host* host, const pa_step_device* dev, void* k_cache,
+                  void* v_cache, const pa_step_shape* shape, void* stream);
+
+/* Reads and clears the device error word (synchronizes `stream`).  Returns
+ * PA_ERR_DEVICE when any bit was set, PA_OK otherwise. */
+pa_status pa_get_device_error(uint32_t* flags, void* stream);
+
+const char* pa_status_string(pa_status status);
+
+/* ------------------------------------------------------------------------ */
+/* Launch accounting and per-kernel device time                              */
+/* ------------------------------------------------------------------------ */
+
+typedef enum {
+    PA_KERNEL_CACHE_WRITE = 0,
+    PA_KERNEL_DECODE = 1,        /* single-pass or partition kernel */
+    PA_KERNEL_REDUCE = 2,        /* log-sum-exp merge of partitions */
+    PA_KERNEL_PLAN = 3,          /* orders partitions longest-first */
+    PA_KERNEL_COPY_BLOCKS = 4,
+    PA_KERNEL_COUNT = 5
+} pa_kernel_id;
+
+/* Number of kernels this library has launched in the process so far. */
+int64_t pa_launch_count(void);
+
+/* Start recording a CUDA event pair around every launch (on its stream);
+ * clears earlier records. */
+pa_status pa_profile_begin(void);
+
+/* Stop recording, wait for the recorded events, and return per kernel id the
+ * summed device milliseconds and launch counts (arrays of PA_KERNEL_COUNT). */
+pa_status pa_profile_end(double* total_ms, int64_t* launches);
+
+/* ------------------------------------------------------------------------ */
+/* Host block manager (no CUDA calls)                                        */
+/* ------------------------------------------------------------------------ */
+
+typedef struct pa_bm pa_bm;
+
+/* Pool of num_blocks blocks of block_size tokens.  initial_free_order (may be
+ * NULL = 0..num_blocks-1) is the free list's initial content; blocks are taken
+ * from its END ([P1] 3.3, free_blocks.pop()). */
+pa_status pa_bm_create(int num_blocks, int block_size, const int32_t* initial_free_order,
+                       pa_bm** out);
+void pa_bm_destroy(pa_bm* bm);
+
+/* New sequence holding num_tokens tokens: takes ceil(num_tokens/block_size)
+ * blocks in logical order ([P1] 3.3 allocate). */
+pa_status pa_bm_allocate(pa_bm* bm, int64_t seq_id, int num_tokens);
+
+/* child shares every block of parent by reference (ref_count + 1 each;
+ * prefix sharing [P3], parallel sampling [P2] 1.1). */
+pa_status pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child);
+
+/* Reserve the slot of the sequence's next token.  Takes a fresh block only when
+ * the last one is full ([P1] 3.3 append_token); copies a shared last block
+ * first ([P2] 2.2): then cow_src and cow_dst receive the block pair to copy,
+ * otherwise both are -1.  On PA_ERR_NO_BLOCKS nothing changes. */
+pa_status pa_bm_append_slot(pa_bm* bm, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                            int32_t* cow_dst);
+
+/* Release a sequence: walk its table in logical order, decrement, and push
+ * blocks reaching zero onto the free list. */
+pa_status pa_bm_free(pa_bm* bm, int64_t seq_id);
+
+/* Copy the sequence's block table (logical order) into out[0..cap); *n = its
+ * length (also when cap is too small, which returns PA_ERR_INVALID_ARG). */
+pa_status pa_bm_block_table(const pa_bm* bm, int64_t seq_id, int32_t* out, int cap, int* n);
+
+/* Slots of logical positions [start, start+count) of a sequence. */
+pa_status pa_bm_slots(const pa_bm* bm, int64_t seq_id, int start, int count, int64_t* out);
+
+/* Pool statistics; context_len receives the sequence's token count, or -1
+ * when seq_id is unknown (pass seq_id < 0 to skip). */
+pa_status pa_bm_stats(const pa_bm* bm, int64_t seq_id, int* num_free, int* num_used,
+                      int* context_len);
+
+/* Reference count of one physical block, and the free list from bottom to top
+ * (the next block taken is free_list[n-1]). */
+pa_status pa_bm_ref_count(const pa_bm* bm, int32_t block, int* count);
+pa_status pa_bm_free_list(const pa_bm* bm, int32_t* out, int cap, int* n);
+
+/* Pack the tables and context lengths of a batch into the device layout:
+ * tables [n][width] padded with -1, context_lens [n]. */
+pa_status pa_bm_pack(const pa_bm* bm, const int64_t* seq_ids, int n, int width,
+                     int32_t* tables, int32_t* context_lens);
+
+/* ------------------------------------------------------------------------ */
+/* Host scheduler: iteration-level (continuous) batching                     */
+/* ------------------------------------------------------------------------ */
+
+typedef struct pa_sched pa_sched;
+
+/* Scheduler over `bm` (not owned) with at most max_running running sequences.
+ * prefix_seq >= 0 names a sequence already resident in bm whose blocks
+ * prefix-sharing requests fork. */
+pa_status pa_sched_create(pa_bm* bm, int max_running, int64_t prefix_seq, pa_sched** out);
+void pa_sched_destroy(pa_sched* s);
+
+/* Queue a request (FCFS).  prompt_len counts the request's own tokens (the
+ * shared prefix excluded).  fork_child >= 0 forks a parallel-sampling child
+ * with that id right after the prompt is placed. */
+pa_status pa_sched_add_request(pa_sched* s, int64_t seq_id, int prompt_len, int output_len,
+                               int shares_prefix, int64_t fork_child, int fork_output_len);
+
+/* Run one iteration ([P1] 2.2): finish, admit (FCFS, stop at the first request
+ * that does not fit the free-block budget), then reserve every running
+ * sequence's next slot, preempting the most recently admitted sequence when
+ * the pool is exhausted.  The step's record is kept until the next call. */
+pa_status pa_sched_step(pa_sched* s);
+
+/* Sizes of the last step's record. */
+typedef struct {
+    int num_finished, num_admitted, num_preempted, num_ops, num_running, num_waiting;
+} pa_sched_counts;
+pa_status pa_sched_counts_get(const pa_sched* s, pa_sched_counts* c);
+
+/* The last step's record.  Any pointer may be NULL to skip that array.
+ *   finished/admitted/preempted: sequence ids in event order.
+ *   ops: num_ops entries in issue order; op_kind[i] = 0 for a cache write
+ *        (a = seq, b = position, c = slot) or 1 for a copy-on-write block copy
+ *        (a = src block, b = dst block, c = -1).  A copy must be applied after
+ *        every earlier write and before every later one.
+ *   running/context_lens: the batch to decode, in admission order. */
+pa_status pa_sched_record(const pa_sched* s, int64_t* finished, int64_t* admitted,
+                          int64_t* preempted, int32_t* op_kind, int64_t* op_a, int64_t* op_b,
+                          int64_t* op_c, int64_t* running, int32_t* context_lens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

@@ -1,0 +1,324 @@
+"""Paged KV-cache decode for B200 (sm_100a): Python binding of libpa.so.
+
+Argument marshalling only -- every step of the path runs in the library's CUDA
+kernels or its native host code.  PyTorch supplies device memory and streams.
+The names follow the C ABI in include/pa.h:
+
+    pa_cache_write(k, v, k_cache, v_cache, slot_mapping)
+    pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, ...)
+    pa_copy_blocks(k_cache, v_cache, pairs)
+    pa_step(...)                  one layer-step from host buffers
+    BlockManager / Scheduler      host bookkeeping (pa_bm_*, pa_sched_*)
+"""
+
+import ctypes
+
+import numpy as np
+
+from . import _native
+
+PA_OK = 0
+STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_NO_BLOCKS",
+                4: "PA_ERR_CUDA", 5: "PA_ERR_DEVICE"}
+PA_ERR_NO_BLOCKS = 3
+DEVERR_SLOT, DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+KERNELS = ("cache_write", "decode", "reduce", "plan", "copy_blocks")
+DEFAULT_PARTITION = 512
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class NoBlocksError(PagedAttentionError):
+    pass
+
+
+def _check(status, what):
+    if status != PA_OK:
+        if status == PA_ERR_NO_BLOCKS:
+            raise NoBlocksError(status, what)
+        raise PagedAttentionError(status, what)
+
+
+def lib():
+    return _native.load()
+
+
+# ---------------------------------------------------------------------------
+# device path
+# ---------------------------------------------------------------------------
+
+def _dtype_code(t):
+    import torch
+    codes = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def _stream(t, stream=None):
+    import torch
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _dev(t, name):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _cache_desc(k_cache):
+    nb, bs, hkv, d = k_cache.shape
+    return _native.CacheDesc(nb, bs, hkv, d, _dtype_code(k_cache))
+
+
+def pa_cache_write(k, v, k_cache, v_cache, slot_mapping, stream=None):
+    """Scatter new-token rows k, v [T, Hkv, D] into the pools through int64 slots."""
+    import torch
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    desc = _cache_desc(k_cache)
+    T = int(slot_mapping.numel())
+    st = lib().pa_cache_write(_dev(k, "k"), _dev(v, "v"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                              _dev(slot_mapping, "slot_mapping"), T, ctypes.byref(desc), _stream(k_cache, stream))
+    _check(st, "pa_cache_write")
+
+
+def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
+    """Copy whole blocks src -> dst in both pools; pairs: int32 [n, 2] on the device."""
+    import torch
+    if pairs.dtype != torch.int32:
+        raise TypeError("pairs must be int32")
+    desc = _cache_desc(k_cache)
+    n = int(pairs.numel() // 2)
+    st = lib().pa_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(pairs, "pairs"), n,
+                              ctypes.byref(desc), _stream(k_cache, stream))
+    _check(st, "pa_copy_blocks")
+
+
+def pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len, partition_size=0):
+    return int(lib().pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len, partition_size))
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size=None, num_kv_heads=None,
+              max_context_len=None, partition_size=0, workspace=None, stream=None):
+    """One paged decode-attention step.
+
+    q, out: [S, Hq, D]; caches [NB, bs, Hkv, D]; block_tables int32 [S, max_blocks];
+    context_lens int32 [S].  ``max_context_len`` bounds every context length
+    (default: the table capacity).  ``workspace``: a uint8 CUDA tensor of at
+    least pa_decode_workspace_size bytes, allocated here when omitted.
+    """
+    import torch
+    nb, bs, hkv, d = k_cache.shape
+    block_size = bs if block_size is None else block_size
+    num_kv_heads = hkv if num_kv_heads is None else num_kv_heads
+    S, Hq, D = q.shape
+    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 1
+    if max_context_len is None:
+        max_context_len = maxb * block_size
+    need = pa_decode_workspace_size(S, Hq, D, max_context_len, partition_size)
+    ws_ptr, ws_bytes = ctypes.c_void_p(0), 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        if workspace.numel() < need:
+            raise ValueError(f"workspace needs {need} bytes")
+        ws_ptr, ws_bytes = ctypes.c_void_p(workspace.data_ptr()), int(workspace.numel())
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    st = lib().pa_decode(_dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                         _dev(block_tables, "block_tables"), _dev(context_lens, "context_lens"), float(scale),
+                         int(block_size), int(num_kv_heads), S, Hq, D, maxb, int(max_context_len), nb,
+                         _dtype_code(q), int(partition_size), ws_ptr, ws_bytes, _stream(q, stream))
+    _check(st, "pa_decode")
+    return out
+
+
+def pa_step(host, dev, k_cache, v_cache, scale, max_context_len, partition_size=0, stream=None):
+    """One layer-step from host buffers (see include/pa.h, pa_step).
+
+    host: dict of pinned CPU tensors q, k, v, slot_mapping, block_tables,
+    context_lens, out (and optionally cow_pairs); dev: dict of CUDA tensors of
+    the same shapes plus ``workspace``.
+    """
+    nb, bs, hkv, d = k_cache.shape
+    S, Hq, D = host["q"].shape
+    T = int(host["slot_mapping"].numel())
+    cow = host.get("cow_pairs")
+    ncow = 0 if cow is None else int(cow.numel() // 2)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+    h = _native.StepHost(ptr(host["q"]), ptr(host["k"]), ptr(host["v"]), ptr(host["slot_mapping"]),
+                         ptr(host["block_tables"]), ptr(host["context_lens"]), ptr(cow), ptr(host["out"]))
+    ws = dev.get("workspace")
+    dv = _native.StepDevice(ptr(dev["q"]), ptr(dev["k"]), ptr(dev["v"]), ptr(dev["slot_mapping"]),
+                            ptr(dev["block_tables"]), ptr(dev["context_lens"]), ptr(dev.get("cow_pairs")),
+                            ptr(dev["out"]), ptr(ws), 0 if ws is None else int(ws.numel()))
+    shape = _native.StepShape(S, Hq, hkv, D, bs, nb, int(host["block_tables"].shape[1]), int(max_context_len), T,
+                              ncow, _dtype_code(k_cache), float(scale), int(partition_size))
+    st = lib().pa_step(ctypes.byref(h), ctypes.byref(dv), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                       ctypes.byref(shape), _stream(k_cache, stream))
+    _check(st, "pa_step")
+
+
+def pa_get_device_error(stream=None):
+    """Read and clear the device error word; returns the PA_DEVERR_* bits."""
+    import torch
+    flags = ctypes.c_uint32(0)
+    s = ctypes.c_void_p(stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream)
+    st = lib().pa_get_device_error(ctypes.byref(flags), s)
+    if st not in (PA_OK, 5):
+        _check(st, "pa_get_device_error")
+    return int(flags.value)
+
+
+def launch_count():
+    return int(lib().pa_launch_count())
+
+
+def profile_begin():
+    _check(lib().pa_profile_begin(), "pa_profile_begin")
+
+
+def profile_end():
+    """Stop recording; returns {kernel name: (total_ms, launches)}."""
+    ms = (ctypes.c_double * len(KERNELS))()
+    n = (ctypes.c_int64 * len(KERNELS))()
+    _check(lib().pa_profile_end(ms, n), "pa_profile_end")
+    return {k: (float(ms[i]), int(n[i])) for i, k in enumerate(KERNELS)}
+
+
+# ---------------------------------------------------------------------------
+# host block manager and scheduler
+# ---------------------------------------------------------------------------
+
+def _i32(a):
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None and a.size else ctypes.c_void_p(0)
+
+
+class BlockManager:
+    """Free list, reference counts and block tables (pa_bm_*)."""
+
+    def __init__(self, num_blocks, block_size, initial_free_order=None):
+        self._h = ctypes.c_void_p()
+        order = None if initial_free_order is None else _i32(initial_free_order)
+        _check(lib().pa_bm_create(num_blocks, block_size, _ptr(order), ctypes.byref(self._h)), "pa_bm_create")
+        self.num_blocks, self.block_size = num_blocks, block_size
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            lib().pa_bm_destroy(h)
+            self._h = None
+
+    @property
+    def handle(self):
+        return self._h
+
+    def allocate(self, seq, num_tokens):
+        _check(lib().pa_bm_allocate(self._h, seq, num_tokens), "pa_bm_allocate")
+
+    def fork(self, parent, child):
+        _check(lib().pa_bm_fork(self._h, parent, child), "pa_bm_fork")
+
+    def append_slot(self, seq):
+        slot, src, dst = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().pa_bm_append_slot(self._h, seq, ctypes.byref(slot), ctypes.byref(src), ctypes.byref(dst)),
+               "pa_bm_append_slot")
+        return slot.value, src.value, dst.value
+
+    def free(self, seq):
+        _check(lib().pa_bm_free(self._h, seq), "pa_bm_free")
+
+    def block_table(self, seq):
+        n = ctypes.c_int()
+        lib().pa_bm_block_table(self._h, seq, ctypes.c_void_p(0), 0, ctypes.byref(n))
+        out = np.zeros(max(n.value, 1), dtype=np.int32)
+        _check(lib().pa_bm_block_table(self._h, seq, _ptr(out), out.size, ctypes.byref(n)), "pa_bm_block_table")
+        return out[:n.value].tolist()
+
+    def slots(self, seq, start, count):
+        out = np.zeros(max(count, 1), dtype=np.int64)
+        _check(lib().pa_bm_slots(self._h, seq, start, count, _ptr(out)), "pa_bm_slots")
+        return out[:count]
+
+    def stats(self, seq=-1):
+        f, u, c = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        _check(lib().pa_bm_stats(self._h, seq, ctypes.byref(f), ctypes.byref(u), ctypes.byref(c)), "pa_bm_stats")
+        return f.value, u.value, c.value
+
+    @property
+    def num_free(self):
+        return self.stats()[0]
+
+    def context_len(self, seq):
+        c = self.stats(seq)[2]
+        if c < 0:
+            raise PagedAttentionError(1, "unknown sequence")
+        return c
+
+    def ref_count(self, block):
+        c = ctypes.c_int()
+        _check(lib().pa_bm_ref_count(self._h, block, ctypes.byref(c)), "pa_bm_ref_count")
+        return c.value
+
+    def free_list(self):
+        out = np.zeros(self.num_blocks, dtype=np.int32)
+        n = ctypes.c_int()
+        _check(lib().pa_bm_free_list(self._h, _ptr(out), out.size, ctypes.byref(n)), "pa_bm_free_list")
+        return out[:n.value].tolist()
+
+    def pack(self, seq_ids, width):
+        """Device-layout tables [n, width] (-1 padded) and context lengths [n]."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        tables = np.full((len(ids), max(width, 1)), -1, dtype=np.int32)
+        lens = np.zeros(len(ids), dtype=np.int32)
+        _check(lib().pa_bm_pack(self._h, _ptr(ids), len(ids), width, _ptr(tables), _ptr(lens)), "pa_bm_pack")
+        return tables[:, :width], lens
+
+
+class Scheduler:
+    """Iteration-level batching over a BlockManager (pa_sched_*)."""
+
+    def __init__(self, bm, max_running, prefix_seq=-1):
+        self.bm = bm           # keeps the block manager alive
+        self._h = ctypes.c_void_p()
+        _check(lib().pa_sched_create(bm.handle, max_running, prefix_seq, ctypes.byref(self._h)), "pa_sched_create")
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            lib().pa_sched_destroy(h)
+            self._h = None
+
+    def add_request(self, seq_id, prompt_len, output_len, shares_prefix=False, fork_child=-1, fork_output_len=0):
+        _check(lib().pa_sched_add_request(self._h, seq_id, prompt_len, output_len, int(bool(shares_prefix)),
+                                          fork_child, fork_output_len), "pa_sched_add_request")
+
+    def step(self):
+        """Run one iteration; returns the step record as a dict of lists."""
+        _check(lib().pa_sched_step(self._h), "pa_sched_step")
+        c = _native.SchedCounts()
+        _check(lib().pa_sched_counts_get(self._h, ctypes.byref(c)), "pa_sched_counts_get")
+        fin = np.zeros(c.num_finished, np.int64)
+        adm = np.zeros(c.num_admitted, np.int64)
+        pre = np.zeros(c.num_preempted, np.int64)
+        kind = np.zeros(c.num_ops, np.int32)
+        oa, ob, oc = (np.zeros(c.num_ops, np.int64) for _ in range(3))
+        run = np.zeros(c.num_running, np.int64)
+        ctx = np.zeros(c.num_running, np.int32)
+        _check(lib().pa_sched_record(self._h, _ptr(fin), _ptr(adm), _ptr(pre), _ptr(kind), _ptr(oa), _ptr(ob),
+                                     _ptr(oc), _ptr(run), _ptr(ctx)), "pa_sched_record")
+        ops = [("w", int(a), int(b), int(cc)) if k == 0 else ("c", int(a), int(b))
+               for k, a, b, cc in zip(kind.tolist(), oa.tolist(), ob.tolist(), oc.tolist())]
+        return {"finished": fin.tolist(), "admitted": adm.tolist(), "preempted": pre.tolist(), "ops": ops,
+                "running": run.tolist(), "context_lens": ctx.tolist(), "num_waiting": c.num_waiting}

@@ -1,0 +1,65 @@
+// KV-cache scatter (append new-token rows through the slot mapping) and
+// whole-block copy for copy-on-write.
+//
+// Slot addressing ("大模型推理引擎高频优化：连续批处理、PagedAttention 与 KV Cache 实战拆解"
+// 3.2-3.3): a new token goes to the end of the sequence's current block, or to
+// a fresh block when the current one is full; the host resolves that to
+// slot = block * block_size + offset.  In the pool layout
+// [num_blocks, block_size, num_kv_heads, head_dim] the row of one slot (all kv
+// heads) is contiguous, and so is a token's row of the new K / V, so each
+// token is one contiguous copy of num_kv_heads * head_dim elements.
+// Copy-on-write ("vLLM推理加速框架：PagedAttention与连续批处理技术解析" 2.2) copies a
+// whole block (block_size * num_kv_heads * head_dim elements) in both pools.
+#pragma once
+
+#include "common.cuh"
+
+namespace pa_dev {
+
+// One warp per token; 16-byte vectors.  row_vecs = 16-byte vectors per token row.
+__global__ void __launch_bounds__(256) cache_write_kernel(const uint4* __restrict__ k,
+                                                          const uint4* __restrict__ v,
+                                                          uint4* __restrict__ k_cache,
+                                                          uint4* __restrict__ v_cache,
+                                                          const int64_t* __restrict__ slot_mapping,
+                                                          int num_tokens, int row_vecs, int64_t num_slots) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= num_tokens) return;
+    const int64_t slot = slot_mapping[warp];
+    if (slot < 0) return;                       // padding token
+    if (slot >= num_slots) {
+        if (lane == 0) flag_error(PA_DEVERR_SLOT);
+        return;
+    }
+    const uint4* ks = k + (int64_t)warp * row_vecs;
+    const uint4* vs = v + (int64_t)warp * row_vecs;
+    uint4* kd = k_cache + slot * row_vecs;
+    uint4* vd = v_cache + slot * row_vecs;
+    for (int i = lane; i < row_vecs; i += 32) {
+        uint4 a = __ldg(ks + i);
+        uint4 b = __ldg(vs + i);
+        kd[i] = a;
+        vd[i] = b;
+    }
+}
+
+// grid (num_pairs, 2): blockIdx.y selects the K or V pool.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_cache,
+                                                          uint4* __restrict__ v_cache,
+                                                          const int32_t* __restrict__ pairs,
+                                                          int64_t block_vecs, int num_blocks) {
+    const int pair = blockIdx.x;
+    const int32_t src = pairs[2 * pair];
+    const int32_t dst = pairs[2 * pair + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) flag_error(PA_DEVERR_BLOCK_ID);
+        return;
+    }
+    uint4* pool = blockIdx.y == 0 ? k_cache : v_cache;
+    const uint4* s = pool + (int64_t)src * block_vecs;
+    uint4* d = pool + (int64_t)dst * block_vecs;
+    for (int64_t i = threadIdx.x; i < block_vecs; i += blockDim.x) d[i] = s[i];
+}
+
+}  // namespace pa_dev

@@ -1,0 +1,531 @@
+// Paged decode attention for sm_100a: single pass, split-K partitions and the
+// log-sum-exp merge.
+//
+// What is computed ("大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置",
+// section "PagedAttention分页注意力机制原理": the kernel resolves every logical block
+// through the block table and runs attention over the non-contiguous physical
+// blocks; "vLLM推理加速框架：PagedAttention与连续批处理技术解析" 2.2: the kernel works
+// block by block; 6.2: out, q, k, v, block_tables): for sequence s, query
+// head h and kv head g = h / group,
+//     out[s][h] = sum_t softmax_t(scale * q[s][h] . K_s[t][g]) V_s[t][g].
+//
+// Design (B200):
+//  * Work item = (sequence, context partition, kv head, query-head chunk).  A
+//    CTA handles all query heads of a kv-head group that share the K/V rows it
+//    streams, so each K/V byte leaves HBM once.  Contexts longer than the
+//    partition size are split; items are ordered longest-first by a small
+//    planning kernel and a persistent grid (a multiple of the SM count) walks
+//    them with a fixed stride.
+//  * One producer warp resolves block ids through the block table (staged in
+//    shared memory) and issues one bulk copy per token row (the row of one kv
+//    head is contiguous: head_dim * elt bytes) into a ring of shared-memory
+//    stages of 32 rows, each stage completed on an mbarrier with transaction
+//    counts.  Rows are stored with a 16-byte pad so stride-row reads spread
+//    over all banks.
+//  * Four consumer warps: phase 1 computes the scaled scores of every token of
+//    the partition into shared memory (16-byte vector reads, fp32 FMAs, a
+//    transposing butterfly that reduces G partial dot products over the lanes
+//    of a row with G-1 shuffles); phase 2 takes the exact max and the
+//    exponentials (fp32, base 2 with log2(e) folded into the scale) and their
+//    sum; phase 3 accumulates p * V in fp32 registers; an epilogue merges the
+//    warps in a fixed order and either writes the normalised row (one
+//    partition) or the partition's unnormalised output, max and sum.
+//  * Every reduction order depends only on logical token positions, so the
+//    result is bitwise independent of the physical placement of blocks.
+//  * All waits are bounded: on expiry the CTA records PA_DEVERR_TIMEOUT and
+//    runs through its remaining work without touching the stages.
+#pragma once
+
+#include "common.cuh"
+
+namespace pa_dev {
+
+struct DecodeArgs {
+    void* out;
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    float scale_log2;          // softmax scale * log2(e)
+    int num_seqs;
+    int num_heads;
+    int num_kv_heads;
+    int group;                 // num_heads / num_kv_heads
+    int n_gchunks;             // query-head chunks per kv head
+    int log2_bs;
+    int max_blocks_per_seq;
+    int ctx_cap;               // min(max_context_len, max_blocks_per_seq * block_size)
+    int num_blocks;
+    int partition_size;        // tokens per partition (multiple of 32)
+    int max_partitions;        // 1: single pass, no plan / partials
+    const int2* plan;          // split mode: (seq, partition), longest first
+    const int* plan_count;
+    float* part_m;             // [num_seqs * num_heads, max_partitions] (log2 units)
+    float* part_l;             // [num_seqs * num_heads, max_partitions]
+    float* part_o;             // [num_seqs * num_heads, max_partitions, head_dim]
+};
+
+struct WorkItem {
+    int s, p, h, gc, t0, n, np;
+};
+
+__device__ __forceinline__ int clamp_context(const DecodeArgs& a, int s, bool report) {
+    int c = a.context_lens[s];
+    if (c < 0 || c > a.ctx_cap) {
+        if (report) flag_error(PA_DEVERR_CONTEXT_LEN);
+        c = c < 0 ? 0 : a.ctx_cap;
+    }
+    return c;
+}
+
+__device__ __forceinline__ int partitions_of(const DecodeArgs& a, int ctx) {
+    return ctx == 0 ? 1 : (ctx + a.partition_size - 1) / a.partition_size;
+}
+
+__device__ __forceinline__ WorkItem decode_item(const DecodeArgs& a, int i, bool report) {
+    const int per = a.num_kv_heads * a.n_gchunks;
+    const int pair = i / per;
+    const int rem = i - pair * per;
+    WorkItem w;
+    w.h = rem / a.n_gchunks;
+    w.gc = rem - w.h * a.n_gchunks;
+    if (a.max_partitions == 1) {
+        w.s = pair;
+        w.p = 0;
+    } else {
+        const int2 e = a.plan[pair];
+        w.s = e.x;
+        w.p = e.y;
+    }
+    const int ctx = clamp_context(a, w.s, report);
+    w.np = partitions_of(a, ctx);
+    w.t0 = w.p * a.partition_size;
+    w.n = min(max(ctx - w.t0, 0), a.partition_size);
+    return w;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Reduce GC partial dot products held by each of the LPT lanes of a row.  Each
+// halving step trades half of the values with the partner lane, so after the
+// loop lane c of the row holds the complete sum for query c / (LPT / GC).
+template <int GC, int LPT>
+__device__ __forceinline__ float reduce_row_dots(float (&v)[GC], int lane) {
+    constexpr int STEPS = ilog2(LPT);
+#pragma unroll
+    for (int step = 0; step < STEPS; ++step) {
+        const int o = LPT >> (step + 1);
+        const int n = GC >> step;
+        if (n >= 2) {
+            const int h = n >> 1;
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < GC / 2; ++i) {
+                if (i < h) {
+                    const float send = upper ? v[i] : v[i + h];
+                    const float keep = upper ? v[i + h] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
+            }
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+        }
+    }
+    return v[0];
+}
+
+template <typename T, int D, int GC>
+struct DecodeCfg {
+    using Tr = ElemTraits<T>;
+    static constexpr int ELT = (int)sizeof(T);
+    static constexpr int VEC = Tr::VEC;             // elements per 16-byte vector
+    static constexpr int LPT = D / VEC;             // lanes per token row
+    static constexpr int RPI = 32 / LPT;            // rows per warp instruction
+    static constexpr int ROW_BYTES = D * ELT;
+    static constexpr int PITCH = ROW_BYTES + 16;    // padded shared-memory row
+    static constexpr int STAGE_ROWS = 32;
+    static constexpr int STAGE_BYTES = STAGE_ROWS * PITCH;
+    static constexpr int NSTAGES = 8;
+    static constexpr int NCW = 4;                   // consumer warps
+    static constexpr int THREADS = (NCW + 1) * 32;
+    static constexpr int MAX_PARTITION = 1024;
+    static constexpr int MAX_TABLE = MAX_PARTITION / 8;
+    static constexpr int OFF_FULL = NSTAGES * STAGE_BYTES;
+    static constexpr int OFF_EMPTY = OFF_FULL + NSTAGES * 8;
+    static constexpr int OFF_TABLE = OFF_EMPTY + NSTAGES * 8;
+    static constexpr int OFF_STATS = OFF_TABLE + MAX_TABLE * 4;
+    static constexpr int OFF_RED = ((OFF_STATS + (2 * GC + 4) * 4) + 127) / 128 * 128;
+    static constexpr int RED_BYTES = NCW * GC * D * 4;
+    static constexpr int OFF_LOGITS = OFF_RED + RED_BYTES;
+    static_assert(GC <= LPT, "query chunk wider than the lanes of a row");
+    static_assert(LPT >= 1 && LPT <= 32 && (32 % LPT) == 0, "row must span a divisor of the warp");
+    static_assert(PITCH % 16 == 0, "bulk copies need 16-byte aligned rows");
+    static size_t smem_bytes(int partition) { return (size_t)OFF_LOGITS + (size_t)partition * GC * 4; }
+};
+
+template <typename T, int D, int GC>
+__global__ void __launch_bounds__(DecodeCfg<T, D, GC>::THREADS, 2) decode_kernel(const DecodeArgs a) {
+    using C = DecodeCfg<T, D, GC>;
+    using Tr = ElemTraits<T>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_FULL);
+    uint64_t* empty = reinterpret_cast<uint64_t*>(smem + C::OFF_EMPTY);
+    int32_t* tbl = reinterpret_cast<int32_t*>(smem + C::OFF_TABLE);
+    float* stat_m = reinterpret_cast<float*>(smem + C::OFF_STATS);
+    float* stat_l = stat_m + GC;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(stat_l + GC);
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+    float* logits = reinterpret_cast<float*>(smem + C::OFF_LOGITS);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NSTAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    const int pairs = a.max_partitions == 1 ? a.num_seqs : *a.plan_count;
+    const int total = pairs * a.num_kv_heads * a.n_gchunks;
+    const int bs = 1 << a.log2_bs;
+
+    if (warp == C::NCW) {
+        // ------------------------------------------------------------ producer
+        const unsigned char* kbase = static_cast<const unsigned char*>(a.k_cache);
+        const unsigned char* vbase = static_cast<const unsigned char*>(a.v_cache);
+        const int64_t slot_stride = (int64_t)a.num_kv_heads * C::ROW_BYTES;
+        const uint64_t policy = l2_policy_evict_first();
+        uint32_t stage = 0;
+        bool ok = true;
+        for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+            const WorkItem w = decode_item(a, i, lane == 0);
+            if (w.n == 0) continue;
+            const int nst = (w.n + C::STAGE_ROWS - 1) / C::STAGE_ROWS;
+            const int nblk = (w.n + bs - 1) >> a.log2_bs;
+            const int32_t* trow = a.block_tables + (int64_t)w.s * a.max_blocks_per_seq + (w.t0 >> a.log2_bs);
+            for (int j = lane; j < nblk; j += 32) {
+                int32_t id = trow[j];
+                if (id < 0 || id >= a.num_blocks) {
+                    flag_error(PA_DEVERR_BLOCK_ID);
+                    id = 0;
+                }
+                tbl[j] = id;
+            }
+            __syncwarp();
+            for (int pass = 0; pass < 2 && ok; ++pass) {
+                const unsigned char* base = (pass ? vbase : kbase) + (int64_t)w.h * C::ROW_BYTES;
+                for (int st = 0; st < nst; ++st, ++stage) {
+                    const int slot = stage % C::NSTAGES;
+                    const uint32_t parity = ((stage / C::NSTAGES) & 1u) ^ 1u;
+                    if (!mbar_wait(&empty[slot], parity, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
+                    if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(rows * C::ROW_BYTES));
+                    __syncwarp();
+                    if (lane < rows) {
+                        const int tok = st * C::STAGE_ROWS + lane;
+                        const int64_t phys = (int64_t)tbl[tok >> a.log2_bs] * bs + (tok & (bs - 1));
+                        bulk_copy_g2s_hint(smem + slot * C::STAGE_BYTES + lane * C::PITCH, base + phys * slot_stride,
+                                           (uint32_t)C::ROW_BYTES, &full[slot], policy);
+                    }
+                }
+            }
+        }
+        if (!ok) {
+            if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            // let copies already issued land before the CTA can retire
+            const uint32_t issued = stage;
+            for (int slot = lane; slot < C::NSTAGES; slot += 32) {
+                if ((uint32_t)slot < issued) {
+                    const uint32_t last = issued - 1 - ((issued - 1 - slot) % C::NSTAGES);
+                    const volatile int never = 0;
+                    mbar_wait(&full[slot], (last / C::NSTAGES) & 1u, &never);
+                }
+            }
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    constexpr int NCT = C::NCW * 32;
+    const int ctid = threadIdx.x;
+    const int row_in = lane / C::LPT;                 // row within a warp instruction
+    const int chunk = lane % C::LPT;                  // 16-byte chunk within the row
+    const int gsel = chunk / (C::LPT / GC);           // query owned after the row reduction
+    const bool gwriter = (chunk % (C::LPT / GC)) == 0;
+    const T* qg = static_cast<const T*>(a.q);
+    T* outg = static_cast<T*>(a.out);
+    uint32_t stage = 0;
+
+    for (int i = blockIdx.x; i < total; i += gridDim.x) {
+        const WorkItem w = decode_item(a, i, false);
+        const int gq = min(GC, a.group - w.gc * GC);
+        const int hq0 = w.h * a.group + w.gc * GC;
+        const int64_t row0 = (int64_t)w.s * a.num_heads + hq0;
+        if (w.n == 0) {
+            for (int e = ctid; e < gq * D; e += NCT) outg[row0 * D + e] = Tr::from_float(0.f);
+            continue;
+        }
+        const int nst = (w.n + C::STAGE_ROWS - 1) / C::STAGE_ROWS;
+
+        // ---- phase 1: scores z' = (q . k) * scale * log2(e) for every token
+        {
+            float qf[GC][C::VEC];
+#pragma unroll
+            for (int g = 0; g < GC; ++g) {
+                if (g < gq) {
+                    const uint4 u = __ldg(reinterpret_cast<const uint4*>(qg + (row0 + g) * D + chunk * C::VEC));
+                    Tr::unpack(u, qf[g]);
+                } else {
+#pragma unroll
+                    for (int v = 0; v < C::VEC; ++v) qf[g][v] = 0.f;
+                }
+            }
+            for (int st = warp; st < nst; st += C::NCW) {
+                const uint32_t c = stage + st;
+                const int slot = c % C::NSTAGES;
+                if (*abort_flag || !mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag)) {
+                    *abort_flag = 1;
+                    continue;
+                }
+                const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
+                const unsigned char* sb = smem + slot * C::STAGE_BYTES;
+                for (int r0 = 0; r0 < rows; r0 += C::RPI) {
+                    const int r = r0 + row_in;
+                    const uint4 u = *reinterpret_cast<const uint4*>(sb + r * C::PITCH + chunk * 16);
+                    float kf[C::VEC];
+                    Tr::unpack(u, kf);
+                    float part[GC];
+#pragma unroll
+                    for (int g = 0; g < GC; ++g) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int v = 0; v < C::VEC; ++v) acc = fmaf(qf[g][v], kf[v], acc);
+                        part[g] = acc;
+                    }
+                    const float z = reduce_row_dots<GC, C::LPT>(part, lane);
+                    if (gwriter && r < rows) logits[(st * C::STAGE_ROWS + r) * GC + gsel] = z * a.scale_log2;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);
+            }
+            stage += nst;
+        }
+        named_barrier(1, NCT);
+
+        // ---- phase 2: exact max, exponentials and their sum per query
+        for (int g = warp; g < GC; g += C::NCW) {
+            float m = -INFINITY;
+            for (int t = lane; t < w.n; t += 32) m = fmaxf(m, logits[t * GC + g]);
+            m = warp_max(m);
+            float l = 0.f;
+            for (int t = lane; t < w.n; t += 32) {
+                const float p = exp2f(logits[t * GC + g] - m);
+                logits[t * GC + g] = p;
+                l += p;
+            }
+            l = warp_sum(l);
+            if (lane == 0) {
+                stat_m[g] = m;
+                stat_l[g] = l;
+            }
+        }
+        named_barrier(1, NCT);
+
+        // ---- phase 3: o = sum_t p_t v_t
+        float acc[GC][C::VEC];
+#pragma unroll
+        for (int g = 0; g < GC; ++g)
+#pragma unroll
+            for (int v = 0; v < C::VEC; ++v) acc[g][v] = 0.f;
+        for (int st = warp; st < nst; st += C::NCW) {
+            const uint32_t c = stage + st;
+            const int slot = c % C::NSTAGES;
+            if (*abort_flag || !mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag)) {
+                *abort_flag = 1;
+                continue;
+            }
+            const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
+            const unsigned char* sb = smem + slot * C::STAGE_BYTES;
+            for (int r0 = 0; r0 < rows; r0 += C::RPI) {
+                const int r = r0 + row_in;
+                if (r < rows) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(sb + r * C::PITCH + chunk * 16);
+                    float vf[C::VEC];
+                    Tr::unpack(u, vf);
+                    const float* pr = logits + (st * C::STAGE_ROWS + r) * GC;
+                    float p[GC];
+                    if constexpr (GC % 4 == 0) {
+#pragma unroll
+                        for (int g = 0; g < GC; g += 4) {
+                            const float4 x = *reinterpret_cast<const float4*>(pr + g);
+                            p[g] = x.x; p[g + 1] = x.y; p[g + 2] = x.z; p[g + 3] = x.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < GC; ++g) p[g] = pr[g];
+                    }
+#pragma unroll
+                    for (int g = 0; g < GC; ++g)
+#pragma unroll
+                        for (int v = 0; v < C::VEC; ++v) acc[g][v] = fmaf(p[g], vf[v], acc[g][v]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        }
+        stage += nst;
+
+        // ---- epilogue: merge rows of a warp, then warps in a fixed order
+#pragma unroll
+        for (int o = C::LPT; o < 32; o <<= 1)
+#pragma unroll
+            for (int g = 0; g < GC; ++g)
+#pragma unroll
+                for (int v = 0; v < C::VEC; ++v) acc[g][v] += __shfl_xor_sync(0xffffffffu, acc[g][v], o);
+        if (row_in == 0) {
+#pragma unroll
+            for (int g = 0; g < GC; ++g) {
+                float* dst = red + (warp * GC + g) * D + chunk * C::VEC;
+#pragma unroll
+                for (int v = 0; v < C::VEC; v += 4)
+                    *reinterpret_cast<float4*>(dst + v) = make_float4(acc[g][v], acc[g][v + 1], acc[g][v + 2], acc[g][v + 3]);
+            }
+        }
+        named_barrier(1, NCT);
+        const bool single = (w.np == 1);
+        for (int e = ctid; e < gq * D; e += NCT) {
+            const int g = e / D;
+            const int d = e - g * D;
+            float o = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < C::NCW; ++ww) o += red[(ww * GC + g) * D + d];
+            const int64_t row = row0 + g;
+            if (single) {
+                outg[row * D + d] = Tr::from_float(o / stat_l[g]);
+            } else {
+                const int64_t pidx = row * a.max_partitions + w.p;
+                a.part_o[pidx * D + d] = o;
+                if (d == 0) {
+                    a.part_m[pidx] = stat_m[g];
+                    a.part_l[pidx] = stat_l[g];
+                }
+            }
+        }
+        named_barrier(1, NCT);
+    }
+}
+
+// Orders (sequence, partition) pairs longest-first: all pairs of the highest
+// partition index first, then the next, so the long sequences' full partitions
+// start early and the short tails fill in at the end.  One CTA.
+__global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, int2* plan, int* count) {
+    __shared__ int warp_incl[32];
+    __shared__ int s_base;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int nw = blockDim.x >> 5;
+    if (tid == 0) s_base = 0;
+    __syncthreads();
+    for (int p = a.max_partitions - 1; p >= 0; --p) {
+        for (int s0 = 0; s0 < a.num_seqs; s0 += blockDim.x) {
+            const int s = s0 + tid;
+            int flag = 0;
+            if (s < a.num_seqs) {
+                const int ctx = clamp_context(a, s, p == a.max_partitions - 1);
+                flag = partitions_of(a, ctx) > p ? 1 : 0;
+            }
+            int x = flag;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane == 31) warp_incl[warp] = x;
+            __syncthreads();
+            if (warp == 0) {
+                int t = lane < nw ? warp_incl[lane] : 0;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, t, o);
+                    if (lane >= o) t += y;
+                }
+                if (lane < nw) warp_incl[lane] = t;
+            }
+            __syncthreads();
+            const int base = s_base + (warp == 0 ? 0 : warp_incl[warp - 1]);
+            if (flag) plan[base + x - 1] = make_int2(s, p);
+            __syncthreads();
+            if (tid == 0) s_base += warp_incl[nw - 1];
+            __syncthreads();
+        }
+    }
+    if (tid == 0) *count = s_base;
+}
+
+// Log-sum-exp merge of a sequence's partitions (base-2 units): with
+// M = max_i m_i, w_i = 2^(m_i - M):  out = sum_i w_i o_i / sum_i w_i l_i.
+// One warp per (sequence, query head); sequences with one partition were
+// finished by the decode kernel.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) reduce_kernel(const DecodeArgs a) {
+    using Tr = ElemTraits<T>;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 4 + warp;
+    if (row >= (int64_t)a.num_seqs * a.num_heads) return;
+    const int s = (int)(row / a.num_heads);
+    const int np = partitions_of(a, clamp_context(a, s, false));
+    if (np <= 1) return;
+    const float* pm = a.part_m + row * a.max_partitions;
+    const float* pl = a.part_l + row * a.max_partitions;
+    float M = -INFINITY;
+    for (int i = lane; i < np; i += 32) M = fmaxf(M, pm[i]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int i = lane; i < np; i += 32) L += exp2f(pm[i] - M) * pl[i];
+    L = warp_sum(L);
+    constexpr int PER = D / 32;
+    float o[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) o[j] = 0.f;
+    const float* po = a.part_o + row * a.max_partitions * D + lane * PER;
+    for (int i = 0; i < np; ++i) {
+        const float wgt = exp2f(pm[i] - M);
+        if constexpr (PER == 4) {
+            const float4 x = *reinterpret_cast<const float4*>(po + (int64_t)i * D);
+            o[0] = fmaf(wgt, x.x, o[0]);
+            o[1] = fmaf(wgt, x.y, o[1]);
+            o[2] = fmaf(wgt, x.z, o[2]);
+            o[3] = fmaf(wgt, x.w, o[3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < PER; ++j) o[j] = fmaf(wgt, po[(int64_t)i * D + j], o[j]);
+        }
+    }
+    T* out = static_cast<T*>(a.out) + row * D + lane * PER;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) out[j] = Tr::from_float(o[j] / L);
+}
+
+}  // namespace pa_dev

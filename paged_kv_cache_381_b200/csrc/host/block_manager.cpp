@@ -1,0 +1,224 @@
+// Host block manager: free list, per-block reference counts, block tables,
+// copy-on-write.  Plain C++17, no CUDA calls.
+//
+// Rules (pages cited by title and section):
+//  * "大模型推理引擎高频优化：连续批处理、PagedAttention 与 KV Cache 实战拆解" 3.3:
+//    blocks are taken from the end of the free list; allocate takes
+//    ceil_div(num_tokens, block_size) blocks; append_token takes a new block
+//    only when the last one is full, otherwise writes at the end of it.
+//  * "vLLM推理加速框架：PagedAttention与连续批处理技术解析" 2.1-2.2: a per-block
+//    ref_count; blocks shared by several sequences are copied before a write
+//    (copy-on-write).
+//  * "大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置", section
+//    "PagedAttention分页注意力机制原理": sequences share prefix blocks by
+//    reference; finished requests return their blocks to the free pool.
+//  Free pushes blocks whose count reaches zero in logical table order.
+
+#include "block_manager.hpp"
+
+#include <new>
+
+namespace pa_host {
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+BlockManager::BlockManager(int num_blocks, int block_size, const int32_t* initial_free_order)
+    : num_blocks_(num_blocks), block_size_(block_size), ref_(num_blocks, 0) {
+    free_.reserve(num_blocks);
+    for (int i = 0; i < num_blocks; ++i)
+        free_.push_back(initial_free_order ? initial_free_order[i] : i);
+}
+
+bool BlockManager::valid_order(int num_blocks, const int32_t* order) {
+    if (!order) return true;
+    std::vector<char> seen(num_blocks, 0);
+    for (int i = 0; i < num_blocks; ++i) {
+        int32_t b = order[i];
+        if (b < 0 || b >= num_blocks || seen[b]) return false;
+        seen[b] = 1;
+    }
+    return true;
+}
+
+pa_status BlockManager::allocate(int64_t seq, int num_tokens) {
+    if (num_tokens < 0 || seqs_.count(seq)) return PA_ERR_INVALID_ARG;
+    int64_t need = ceil_div(num_tokens, block_size_);
+    if (need > (int64_t)free_.size()) return PA_ERR_NO_BLOCKS;
+    Seq s;
+    s.ctx = num_tokens;
+    s.table.reserve(need);
+    for (int64_t i = 0; i < need; ++i) {
+        int32_t b = free_.back();
+        free_.pop_back();
+        ref_[b] = 1;
+        s.table.push_back(b);
+    }
+    seqs_.emplace(seq, std::move(s));
+    return PA_OK;
+}
+
+pa_status BlockManager::fork(int64_t parent, int64_t child) {
+    auto it = seqs_.find(parent);
+    if (it == seqs_.end() || seqs_.count(child)) return PA_ERR_INVALID_ARG;
+    Seq c = it->second;
+    for (int32_t b : c.table) ref_[b] += 1;
+    seqs_.emplace(child, std::move(c));
+    return PA_OK;
+}
+
+pa_status BlockManager::append_slot(int64_t seq, int64_t* slot, int32_t* cow_src, int32_t* cow_dst) {
+    auto it = seqs_.find(seq);
+    if (it == seqs_.end()) return PA_ERR_INVALID_ARG;
+    Seq& s = it->second;
+    const int64_t pos = s.ctx;
+    int32_t src = -1, dst = -1;
+    if (pos % block_size_ == 0) {
+        // the last block is full (or there is none): open a fresh block
+        if (free_.empty()) return PA_ERR_NO_BLOCKS;
+        int32_t b = free_.back();
+        free_.pop_back();
+        ref_[b] = 1;
+        s.table.push_back(b);
+    } else {
+        int32_t last = s.table.back();
+        if (ref_[last] > 1) {
+            // shared partly filled block: give this sequence a private copy
+            if (free_.empty()) return PA_ERR_NO_BLOCKS;
+            int32_t b = free_.back();
+            free_.pop_back();
+            ref_[b] = 1;
+            ref_[last] -= 1;
+            s.table.back() = b;
+            src = last;
+            dst = b;
+        }
+    }
+    s.ctx = pos + 1;
+    if (slot) *slot = (int64_t)s.table[pos / block_size_] * block_size_ + pos % block_size_;
+    if (cow_src) *cow_src = src;
+    if (cow_dst) *cow_dst = dst;
+    return PA_OK;
+}
+
+pa_status BlockManager::free_seq(int64_t seq) {
+    auto it = seqs_.find(seq);
+    if (it == seqs_.end()) return PA_ERR_INVALID_ARG;
+    for (int32_t b : it->second.table) {
+        if (ref_[b] <= 0) return PA_ERR_INVALID_ARG;  // corrupted counts; never expected
+        if (--ref_[b] == 0) free_.push_back(b);
+    }
+    seqs_.erase(it);
+    return PA_OK;
+}
+
+const BlockManager::Seq* BlockManager::find(int64_t seq) const {
+    auto it = seqs_.find(seq);
+    return it == seqs_.end() ? nullptr : &it->second;
+}
+
+pa_status BlockManager::slots(int64_t seq, int64_t start, int64_t count, int64_t* out) const {
+    const Seq* s = find(seq);
+    if (!s || start < 0 || count < 0) return PA_ERR_INVALID_ARG;
+    if (start + count > (int64_t)s->table.size() * block_size_) return PA_ERR_INVALID_ARG;
+    for (int64_t p = start; p < start + count; ++p)
+        out[p - start] = (int64_t)s->table[p / block_size_] * block_size_ + p % block_size_;
+    return PA_OK;
+}
+
+}  // namespace pa_host
+
+using pa_host::BlockManager;
+
+struct pa_bm {
+    BlockManager impl;
+    pa_bm(int nb, int bs, const int32_t* order) : impl(nb, bs, order) {}
+};
+
+extern "C" {
+
+pa_status pa_bm_create(int num_blocks, int block_size, const int32_t* initial_free_order, pa_bm** out) {
+    if (!out || num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+    if (!BlockManager::valid_order(num_blocks, initial_free_order)) return PA_ERR_INVALID_ARG;
+    *out = new (std::nothrow) pa_bm(num_blocks, block_size, initial_free_order);
+    return *out ? PA_OK : PA_ERR_INVALID_ARG;
+}
+
+void pa_bm_destroy(pa_bm* bm) { delete bm; }
+
+pa_status pa_bm_allocate(pa_bm* bm, int64_t seq_id, int num_tokens) {
+    return bm ? bm->impl.allocate(seq_id, num_tokens) : PA_ERR_INVALID_ARG;
+}
+
+pa_status pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child) {
+    return bm ? bm->impl.fork(parent, child) : PA_ERR_INVALID_ARG;
+}
+
+pa_status pa_bm_append_slot(pa_bm* bm, int64_t seq_id, int64_t* slot, int32_t* cow_src, int32_t* cow_dst) {
+    return bm ? bm->impl.append_slot(seq_id, slot, cow_src, cow_dst) : PA_ERR_INVALID_ARG;
+}
+
+pa_status pa_bm_free(pa_bm* bm, int64_t seq_id) {
+    return bm ? bm->impl.free_seq(seq_id) : PA_ERR_INVALID_ARG;
+}
+
+pa_status pa_bm_block_table(const pa_bm* bm, int64_t seq_id, int32_t* out, int cap, int* n) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    const BlockManager::Seq* s = bm->impl.find(seq_id);
+    if (!s) return PA_ERR_INVALID_ARG;
+    int len = (int)s->table.size();
+    if (n) *n = len;
+    if (len > cap || (len > 0 && !out)) return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < len; ++i) out[i] = s->table[i];
+    return PA_OK;
+}
+
+pa_status pa_bm_slots(const pa_bm* bm, int64_t seq_id, int start, int count, int64_t* out) {
+    if (!bm || (count > 0 && !out)) return PA_ERR_INVALID_ARG;
+    return bm->impl.slots(seq_id, start, count, out);
+}
+
+pa_status pa_bm_stats(const pa_bm* bm, int64_t seq_id, int* num_free, int* num_used, int* context_len) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    if (num_free) *num_free = bm->impl.num_free();
+    if (num_used) *num_used = bm->impl.num_blocks() - bm->impl.num_free();
+    if (context_len) {
+        const BlockManager::Seq* s = seq_id >= 0 ? bm->impl.find(seq_id) : nullptr;
+        *context_len = s ? (int)s->ctx : -1;
+    }
+    return PA_OK;
+}
+
+pa_status pa_bm_ref_count(const pa_bm* bm, int32_t block, int* count) {
+    if (!bm || !count || block < 0 || block >= bm->impl.num_blocks()) return PA_ERR_INVALID_ARG;
+    *count = bm->impl.ref(block);
+    return PA_OK;
+}
+
+pa_status pa_bm_free_list(const pa_bm* bm, int32_t* out, int cap, int* n) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    const auto& fl = bm->impl.free_list();
+    int len = (int)fl.size();
+    if (n) *n = len;
+    if (len > cap || (len > 0 && !out)) return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < len; ++i) out[i] = fl[i];
+    return PA_OK;
+}
+
+pa_status pa_bm_pack(const pa_bm* bm, const int64_t* seq_ids, int n, int width, int32_t* tables,
+                     int32_t* context_lens) {
+    if (!bm || n < 0 || width < 0 || (n > 0 && (!seq_ids || !tables || !context_lens)))
+        return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        const BlockManager::Seq* s = bm->impl.find(seq_ids[i]);
+        if (!s || (int)s->table.size() > width) return PA_ERR_INVALID_ARG;
+        int32_t* row = tables + (int64_t)i * width;
+        int len = (int)s->table.size();
+        for (int j = 0; j < width; ++j) row[j] = j < len ? s->table[j] : -1;
+        context_lens[i] = (int32_t)s->ctx;
+    }
+    return PA_OK;
+}
+
+}  // extern "C"
+
+pa_host::BlockManager* pa_bm_impl(pa_bm* bm) { return bm ? &bm->impl : nullptr; }

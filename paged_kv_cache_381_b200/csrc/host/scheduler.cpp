@@ -1,0 +1,233 @@
+// Host scheduler: iteration-level (continuous) batching over the block
+// manager.  Plain C++17, no CUDA calls.
+//
+// One step ("大模型推理引擎高频优化：连续批处理、PagedAttention 与 KV Cache 实战拆解" 2.2,
+// Scheduler.schedule; "大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置",
+// section "连续批处理Continuous Batching配置"):
+//  1. sequences that generated their output length leave and free their blocks;
+//  2. admission, first-come first-served, against a free-block budget that each
+//     admitted request charges with ceil(own_tokens / block_size) + 1 (+1 when it
+//     forks a parallel-sampling child); the first request that does not fit
+//     stops admission and stays at the head of the queue; the running count is
+//     capped (max-num-seqs);
+//  3. every running sequence reserves the slot of its next token; when the pool
+//     is exhausted the most recently admitted running sequence is preempted
+//     ("vLLM推理加速框架：PagedAttention与连续批处理技术解析" 3.2 names preemptive
+//     scheduling; recompute-style preemption is the reading adopted): its blocks
+//     are freed and it returns to the front of the queue with its progress, and
+//     its whole history is written again when it is re-admitted.
+// The step's record lists cache writes and copy-on-write copies in issue order.
+
+#include <deque>
+#include <new>
+#include <vector>
+
+#include "block_manager.hpp"
+
+namespace {
+
+struct SeqState {
+    int64_t id = -1;
+    int64_t output_len = 0;
+    bool shares_prefix = false;
+    int64_t history = 0;     // tokens held (shared prefix included)
+    int64_t generated = 0;
+    int64_t fork_child = -1;
+    int64_t fork_output_len = 0;
+    bool forked = false;
+};
+
+}  // namespace
+
+struct pa_sched {
+    pa_host::BlockManager* bm = nullptr;
+    int max_running = 0;
+    int64_t prefix_seq = -1;
+    int64_t prefix_len = 0;
+    std::deque<SeqState> waiting;
+    std::vector<SeqState> running;
+    // record of the last step
+    std::vector<int64_t> finished, admitted, preempted;
+    std::vector<int32_t> op_kind;
+    std::vector<int64_t> op_a, op_b, op_c;
+    std::vector<int64_t> run_ids;
+    std::vector<int32_t> run_ctx;
+
+    void rec_write(int64_t seq, int64_t pos, int64_t slot) {
+        op_kind.push_back(0); op_a.push_back(seq); op_b.push_back(pos); op_c.push_back(slot);
+    }
+    void rec_copy(int32_t src, int32_t dst) {
+        op_kind.push_back(1); op_a.push_back(src); op_b.push_back(dst); op_c.push_back(-1);
+    }
+    int64_t own_tokens(const SeqState& s) const { return s.history - (s.shares_prefix ? prefix_len : 0); }
+    int64_t required(const SeqState& s) const {
+        int64_t need = pa_host::ceil_div(own_tokens(s), bm->block_size()) + 1;
+        if (s.fork_child >= 0 && !s.forked) need += 1;
+        return need;
+    }
+    pa_status admit(SeqState s);
+    pa_status step();
+};
+
+pa_status pa_sched::admit(SeqState s) {
+    pa_status st;
+    if (s.shares_prefix) {
+        if ((st = bm->fork(prefix_seq, s.id)) != PA_OK) return st;
+        for (int64_t pos = prefix_len; pos < s.history; ++pos) {
+            int64_t slot; int32_t src, dst;
+            if ((st = bm->append_slot(s.id, &slot, &src, &dst)) != PA_OK) return st;
+            if (src >= 0) rec_copy(src, dst);
+            rec_write(s.id, pos, slot);
+        }
+    } else {
+        if ((st = bm->allocate(s.id, (int)s.history)) != PA_OK) return st;
+        std::vector<int64_t> slots(s.history);
+        if (s.history > 0 && (st = bm->slots(s.id, 0, s.history, slots.data())) != PA_OK) return st;
+        for (int64_t pos = 0; pos < s.history; ++pos) rec_write(s.id, pos, slots[pos]);
+    }
+    admitted.push_back(s.id);
+    const bool spawn = s.fork_child >= 0 && !s.forked;
+    if (spawn) s.forked = true;
+    running.push_back(s);
+    if (spawn) {
+        if ((st = bm->fork(s.id, s.fork_child)) != PA_OK) return st;
+        SeqState c;
+        c.id = s.fork_child;
+        c.output_len = s.fork_output_len;
+        c.shares_prefix = s.shares_prefix;
+        c.history = s.history;
+        running.push_back(c);
+        admitted.push_back(c.id);
+    }
+    return PA_OK;
+}
+
+pa_status pa_sched::step() {
+    finished.clear(); admitted.clear(); preempted.clear();
+    op_kind.clear(); op_a.clear(); op_b.clear(); op_c.clear();
+    run_ids.clear(); run_ctx.clear();
+    pa_status st;
+    // 1. finish
+    std::vector<SeqState> keep;
+    keep.reserve(running.size());
+    for (const SeqState& s : running) {
+        if (s.generated >= s.output_len) {
+            if ((st = bm->free_seq(s.id)) != PA_OK) return st;
+            finished.push_back(s.id);
+        } else {
+            keep.push_back(s);
+        }
+    }
+    running.swap(keep);
+    // 2. admit, FCFS against the free-block budget
+    int64_t budget = bm->num_free();
+    while (!waiting.empty() && budget > 0 && (int)running.size() < max_running) {
+        const SeqState& head = waiting.front();
+        int64_t need = required(head);
+        if (need > budget) break;
+        int extra = (head.fork_child >= 0 && !head.forked) ? 1 : 0;
+        if ((int)running.size() + 1 + extra > max_running) break;
+        SeqState s = head;
+        waiting.pop_front();
+        budget -= need;
+        if ((st = admit(s)) != PA_OK) return st;
+    }
+    // 3. reserve every running sequence's next slot, preempting when exhausted
+    size_t i = 0;
+    while (i < running.size()) {
+        SeqState& s = running[i];
+        int64_t slot; int32_t src, dst;
+        st = bm->append_slot(s.id, &slot, &src, &dst);
+        if (st == PA_ERR_NO_BLOCKS) {
+            SeqState victim = running.back();
+            running.pop_back();
+            if ((st = bm->free_seq(victim.id)) != PA_OK) return st;
+            preempted.push_back(victim.id);
+            waiting.push_front(victim);
+            continue;   // retry the same index (or stop if the victim was this one)
+        }
+        if (st != PA_OK) return st;
+        if (src >= 0) rec_copy(src, dst);
+        rec_write(s.id, s.history, slot);
+        s.history += 1;
+        s.generated += 1;
+        ++i;
+    }
+    for (const SeqState& s : running) {
+        run_ids.push_back(s.id);
+        run_ctx.push_back((int32_t)s.history);
+    }
+    return PA_OK;
+}
+
+extern "C" {
+
+pa_status pa_sched_create(pa_bm* bm, int max_running, int64_t prefix_seq, pa_sched** out) {
+    pa_host::BlockManager* impl = pa_bm_impl(bm);
+    if (!impl || !out || max_running <= 0) return PA_ERR_INVALID_ARG;
+    int64_t plen = 0;
+    if (prefix_seq >= 0) {
+        const pa_host::BlockManager::Seq* p = impl->find(prefix_seq);
+        if (!p) return PA_ERR_INVALID_ARG;
+        plen = p->ctx;
+    }
+    pa_sched* s = new (std::nothrow) pa_sched();
+    if (!s) return PA_ERR_INVALID_ARG;
+    s->bm = impl;
+    s->max_running = max_running;
+    s->prefix_seq = prefix_seq;
+    s->prefix_len = plen;
+    *out = s;
+    return PA_OK;
+}
+
+void pa_sched_destroy(pa_sched* s) { delete s; }
+
+pa_status pa_sched_add_request(pa_sched* s, int64_t seq_id, int prompt_len, int output_len,
+                               int shares_prefix, int64_t fork_child, int fork_output_len) {
+    if (!s || prompt_len < 0 || output_len < 0 || fork_output_len < 0) return PA_ERR_INVALID_ARG;
+    if (shares_prefix && s->prefix_seq < 0) return PA_ERR_INVALID_ARG;
+    SeqState q;
+    q.id = seq_id;
+    q.output_len = output_len;
+    q.shares_prefix = shares_prefix != 0;
+    q.history = (q.shares_prefix ? s->prefix_len : 0) + prompt_len;
+    q.fork_child = fork_child;
+    q.fork_output_len = fork_output_len;
+    s->waiting.push_back(q);
+    return PA_OK;
+}
+
+pa_status pa_sched_step(pa_sched* s) { return s ? s->step() : PA_ERR_INVALID_ARG; }
+
+pa_status pa_sched_counts_get(const pa_sched* s, pa_sched_counts* c) {
+    if (!s || !c) return PA_ERR_INVALID_ARG;
+    c->num_finished = (int)s->finished.size();
+    c->num_admitted = (int)s->admitted.size();
+    c->num_preempted = (int)s->preempted.size();
+    c->num_ops = (int)s->op_kind.size();
+    c->num_running = (int)s->run_ids.size();
+    c->num_waiting = (int)s->waiting.size();
+    return PA_OK;
+}
+
+pa_status pa_sched_record(const pa_sched* s, int64_t* finished, int64_t* admitted, int64_t* preempted,
+                          int32_t* op_kind, int64_t* op_a, int64_t* op_b, int64_t* op_c,
+                          int64_t* running, int32_t* context_lens) {
+    if (!s) return PA_ERR_INVALID_ARG;
+    auto put64 = [](int64_t* dst, const std::vector<int64_t>& src) {
+        if (dst) for (size_t i = 0; i < src.size(); ++i) dst[i] = src[i];
+    };
+    put64(finished, s->finished);
+    put64(admitted, s->admitted);
+    put64(preempted, s->preempted);
+    if (op_kind) for (size_t i = 0; i < s->op_kind.size(); ++i) op_kind[i] = s->op_kind[i];
+    put64(op_a, s->op_a);
+    put64(op_b, s->op_b);
+    put64(op_c, s->op_c);
+    put64(running, s->run_ids);
+    if (context_lens) for (size_t i = 0; i < s->run_ctx.size(); ++i) context_lens[i] = s->run_ctx[i];
+    return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,423 @@
+// C ABI of the paged KV-cache decode library: argument checks, kernel
+// dispatch, launch accounting, the host-buffer step and the device error word.
+// Declarations and contracts: include/pa.h.
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "device/cache_ops.cuh"
+#include "device/decode.cuh"
+#include "pa.h"
+
+namespace {
+
+constexpr int kDefaultPartition = 512;
+constexpr int kMaxDevices = 64;
+
+// ---------------------------------------------------------------- accounting
+std::atomic<int64_t> g_launches{0};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+struct ProfRecord {
+    int kernel;
+    cudaEvent_t start, stop;
+};
+std::vector<ProfRecord> g_prof_records;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Counts one launch and, while profiling, brackets it with an event pair on
+// its stream.
+class LaunchScope {
+  public:
+    LaunchScope(int kernel, cudaStream_t stream) : kernel_(kernel), stream_(stream) {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        if (g_prof_on) {
+            start_ = take_event();
+            stop_ = take_event();
+            if (start_ && stop_) cudaEventRecord(start_, stream_);
+        }
+    }
+    ~LaunchScope() {
+        if (!start_ || !stop_) return;
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        cudaEventRecord(stop_, stream_);
+        g_prof_records.push_back({kernel_, start_, stop_});
+    }
+
+  private:
+    int kernel_;
+    cudaStream_t stream_;
+    cudaEvent_t start_ = nullptr, stop_ = nullptr;
+};
+
+pa_status launch_status() { return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+// ------------------------------------------------------------- device info
+int device_sms(int dev) {
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cache[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_bytes(pa_dtype t) { return t == PA_F32 ? 4 : 2; }
+
+bool valid_dtype(int t) { return t == PA_F32 || t == PA_F16 || t == PA_BF16; }
+
+bool supported_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32; }
+
+bool supported_head_dim(int d) { return d == 64 || d == 128; }
+
+pa_status check_cache_desc(const pa_cache_desc* c) {
+    if (!c || c->num_blocks <= 0 || c->num_kv_heads <= 0 || !valid_dtype(c->dtype)) return PA_ERR_INVALID_ARG;
+    if (!supported_block_size(c->block_size) || !supported_head_dim(c->head_dim)) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+// ------------------------------------------------------------ workspace
+struct WsLayout {
+    size_t plan, count, m, l, o, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t maxP) {
+    WsLayout w{};
+    size_t off = 0;
+    w.plan = off;
+    off = align256(off + (size_t)(S * maxP) * sizeof(int2));
+    w.count = off;
+    off = align256(off + sizeof(int));
+    w.m = off;
+    off = align256(off + (size_t)(S * Hq * maxP) * sizeof(float));
+    w.l = off;
+    off = align256(off + (size_t)(S * Hq * maxP) * sizeof(float));
+    w.o = off;
+    off = align256(off + (size_t)(S * Hq * maxP * D) * sizeof(float));
+    w.total = off;
+    return w;
+}
+
+int resolve_partition(int partition_size) { return partition_size == 0 ? kDefaultPartition : partition_size; }
+
+bool valid_partition(int p) { return p >= 32 && p <= 1024 && p % 32 == 0; }
+
+int64_t partitions_for(int64_t ctx, int64_t P) { return ctx <= P ? 1 : (ctx + P - 1) / P; }
+
+// ------------------------------------------------------------ decode launch
+template <typename T, int D, int GC>
+pa_status launch_decode(const pa_dev::DecodeArgs& a, int64_t pair_upper, cudaStream_t stream) {
+    using C = pa_dev::DecodeCfg<T, D, GC>;
+    auto kern = pa_dev::decode_kernel<T, D, GC>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    static std::atomic<uint64_t> configured{0};
+    const uint64_t bit = 1ull << (dev & 63);
+    const size_t smem_max = C::smem_bytes(C::MAX_PARTITION);
+    if (!(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max) != cudaSuccess)
+            return PA_ERR_CUDA;
+        configured.fetch_or(bit);
+    }
+    const size_t smem = C::smem_bytes(a.partition_size);
+    static std::atomic<int64_t> occ_cache{0};   // (dev << 40) | (smem << 8) | blocks
+    int occ = 0;
+    const int64_t key = ((int64_t)dev << 40) | ((int64_t)smem << 8);
+    const int64_t cached = occ_cache.load();
+    if ((cached & ~int64_t(255)) == key && (cached & 255) > 0) {
+        occ = (int)(cached & 255);
+    } else {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, C::THREADS, smem) != cudaSuccess || occ <= 0)
+            return PA_ERR_CUDA;
+        occ_cache.store(key | std::min(occ, 255));
+    }
+    const int64_t items_upper = pair_upper * a.num_kv_heads * a.n_gchunks;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items_upper, (int64_t)device_sms(dev) * occ));
+    LaunchScope scope(PA_KERNEL_DECODE, stream);
+    kern<<<(unsigned)grid, C::THREADS, smem, stream>>>(a);
+    return launch_status();
+}
+
+template <typename T, int D>
+pa_status dispatch_group(const pa_dev::DecodeArgs& a, int gc, int64_t pair_upper, cudaStream_t st) {
+    switch (gc) {
+        case 1: return launch_decode<T, D, 1>(a, pair_upper, st);
+        case 2: return launch_decode<T, D, 2>(a, pair_upper, st);
+        case 4: return launch_decode<T, D, 4>(a, pair_upper, st);
+        case 8: return launch_decode<T, D, 8>(a, pair_upper, st);
+        default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T>
+pa_status dispatch_head_dim(const pa_dev::DecodeArgs& a, int D, int gc, int64_t pair_upper, cudaStream_t st) {
+    return D == 64 ? dispatch_group<T, 64>(a, gc, pair_upper, st) : dispatch_group<T, 128>(a, gc, pair_upper, st);
+}
+
+template <typename T>
+pa_status launch_reduce(const pa_dev::DecodeArgs& a, int D, cudaStream_t stream) {
+    const int64_t rows = (int64_t)a.num_seqs * a.num_heads;
+    const unsigned grid = (unsigned)((rows + 3) / 4);
+    LaunchScope scope(PA_KERNEL_REDUCE, stream);
+    if (D == 64)
+        pa_dev::reduce_kernel<T, 64><<<grid, 128, 0, stream>>>(a);
+    else
+        pa_dev::reduce_kernel<T, 128><<<grid, 128, 0, stream>>>(a);
+    return launch_status();
+}
+
+int query_chunk(int group) {
+    int g = std::min(group, 8);
+    int c = 1;
+    while (c < g) c <<= 1;
+    return c;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(pa_status s) {
+    switch (s) {
+        case PA_OK: return "ok";
+        case PA_ERR_INVALID_ARG: return "invalid argument";
+        case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case PA_ERR_NO_BLOCKS: return "no free blocks";
+        case PA_ERR_CUDA: return "CUDA error";
+        case PA_ERR_DEVICE: return "device-side error flagged";
+    }
+    return "unknown status";
+}
+
+int64_t pa_launch_count(void) { return g_launches.load(); }
+
+pa_status pa_profile_begin(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (auto& r : g_prof_records) {
+        g_event_pool.push_back(r.start);
+        g_event_pool.push_back(r.stop);
+    }
+    g_prof_records.clear();
+    g_prof_on = true;
+    return PA_OK;
+}
+
+pa_status pa_profile_end(double* total_ms, int64_t* launches) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_on = false;
+    for (int k = 0; k < PA_KERNEL_COUNT; ++k) {
+        if (total_ms) total_ms[k] = 0.0;
+        if (launches) launches[k] = 0;
+    }
+    pa_status st = PA_OK;
+    for (auto& r : g_prof_records) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+            st = PA_ERR_CUDA;
+        } else if (r.kernel >= 0 && r.kernel < PA_KERNEL_COUNT) {
+            if (total_ms) total_ms[r.kernel] += ms;
+            if (launches) launches[r.kernel] += 1;
+        }
+        g_event_pool.push_back(r.start);
+        g_event_pool.push_back(r.stop);
+    }
+    g_prof_records.clear();
+    return st;
+}
+
+pa_status pa_cache_write(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                         int num_tokens, const pa_cache_desc* cache, void* stream) {
+    pa_status st = check_cache_desc(cache);
+    if (st != PA_OK) return st;
+    if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+    const int64_t row_bytes = (int64_t)cache->num_kv_heads * cache->head_dim * elem_bytes(cache->dtype);
+    const int row_vecs = (int)(row_bytes / 16);
+    const int64_t num_slots = (int64_t)cache->num_blocks * cache->block_size;
+    const int64_t threads = (int64_t)num_tokens * 32;
+    const unsigned grid = (unsigned)((threads + 255) / 256);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    LaunchScope scope(PA_KERNEL_CACHE_WRITE, s);
+    pa_dev::cache_write_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+                                                     static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                                                     slot_mapping, num_tokens, row_vecs, num_slots);
+    return launch_status();
+}
+
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int num_pairs, const pa_cache_desc* cache,
+                         void* stream) {
+    pa_status st = check_cache_desc(cache);
+    if (st != PA_OK) return st;
+    if (num_pairs < 0) return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !pairs || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+    const int64_t block_vecs =
+        (int64_t)cache->block_size * cache->num_kv_heads * cache->head_dim * elem_bytes(cache->dtype) / 16;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    LaunchScope scope(PA_KERNEL_COPY_BLOCKS, s);
+    pa_dev::copy_blocks_kernel<<<dim3((unsigned)num_pairs, 2), 256, 0, s>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, block_vecs, cache->num_blocks);
+    return launch_status();
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_context_len, int partition_size) {
+    const int P = resolve_partition(partition_size);
+    if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 || !valid_partition(P)) return 0;
+    const int64_t maxP = partitions_for(max_context_len, P);
+    if (maxP <= 1) return 0;
+    return ws_layout(num_seqs, num_heads, head_dim, maxP).total;
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                    const int32_t* context_lens, float scale, int block_size, int num_kv_heads, int num_seqs,
+                    int num_heads, int head_dim, int max_blocks_per_seq, int max_context_len, int num_blocks,
+                    pa_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes, void* stream) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+        max_context_len < 0 || !valid_dtype(dtype) || !std::isfinite(scale))
+        return PA_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    const int P = resolve_partition(partition_size);
+    if (!valid_partition(P)) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+
+    const int64_t table_cap = (int64_t)max_blocks_per_seq * block_size;
+    const int64_t cap = std::min<int64_t>(max_context_len, table_cap);
+    if (cap > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
+    const int64_t maxP = partitions_for(cap, P);
+    const int group = num_heads / num_kv_heads;
+    const int gc = query_chunk(group);
+    const int n_gchunks = (group + gc - 1) / gc;
+    if ((int64_t)num_seqs * maxP * num_kv_heads * n_gchunks > INT32_MAX) return PA_ERR_INVALID_ARG;
+
+    pa_dev::DecodeArgs a{};
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.num_seqs = num_seqs;
+    a.num_heads = num_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.group = group;
+    a.n_gchunks = n_gchunks;
+    a.log2_bs = block_size == 8 ? 3 : block_size == 16 ? 4 : 5;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.ctx_cap = (int)cap;
+    a.num_blocks = num_blocks;
+    a.partition_size = P;
+    a.max_partitions = (int)maxP;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (maxP > 1) {
+        const WsLayout L = ws_layout(num_seqs, num_heads, head_dim, maxP);
+        if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return PA_ERR_INVALID_ARG;
+        char* ws = static_cast<char*>(workspace);
+        a.plan = reinterpret_cast<const int2*>(ws + L.plan);
+        a.plan_count = reinterpret_cast<const int*>(ws + L.count);
+        a.part_m = reinterpret_cast<float*>(ws + L.m);
+        a.part_l = reinterpret_cast<float*>(ws + L.l);
+        a.part_o = reinterpret_cast<float*>(ws + L.o);
+        {
+            LaunchScope scope(PA_KERNEL_PLAN, s);
+            const int threads = std::min(1024, std::max(32, (num_seqs + 31) / 32 * 32));
+            pa_dev::plan_kernel<<<1, threads, 0, s>>>(a, reinterpret_cast<int2*>(ws + L.plan),
+                                                      reinterpret_cast<int*>(ws + L.count));
+            if (launch_status() != PA_OK) return PA_ERR_CUDA;
+        }
+    }
+    const int64_t pair_upper = (int64_t)num_seqs * maxP;
+    pa_status st;
+    switch (dtype) {
+        case PA_F32: st = dispatch_head_dim<float>(a, head_dim, gc, pair_upper, s); break;
+        case PA_F16: st = dispatch_head_dim<__half>(a, head_dim, gc, pair_upper, s); break;
+        default: st = dispatch_head_dim<__nv_bfloat16>(a, head_dim, gc, pair_upper, s); break;
+    }
+    if (st != PA_OK || maxP <= 1) return st;
+    switch (dtype) {
+        case PA_F32: return launch_reduce<float>(a, head_dim, s);
+        case PA_F16: return launch_reduce<__half>(a, head_dim, s);
+        default: return launch_reduce<__nv_bfloat16>(a, head_dim, s);
+    }
+}
+
+pa_status pa_step(const pa_step_host* h, const pa_step_device* d, void* k_cache, void* v_cache,
+                  const pa_step_shape* sh, void* stream) {
+    if (!h || !d || !sh || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+    if (sh->num_seqs < 0 || sh->num_tokens < 0 || sh->num_cow < 0 || !valid_dtype(sh->dtype)) return PA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t e = elem_bytes(sh->dtype);
+    const size_t qbytes = (size_t)sh->num_seqs * sh->num_heads * sh->head_dim * e;
+    const size_t kvbytes = (size_t)sh->num_tokens * sh->num_kv_heads * sh->head_dim * e;
+    auto h2d = [&](void* dst, const void* src, size_t n) -> bool {
+        if (n == 0) return true;
+        if (!dst || !src) return false;
+        return cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    };
+    if (!h2d(d->q, h->q, qbytes) || !h2d(d->k, h->k, kvbytes) || !h2d(d->v, h->v, kvbytes) ||
+        !h2d(d->slot_mapping, h->slot_mapping, (size_t)sh->num_tokens * sizeof(int64_t)) ||
+        !h2d(d->block_tables, h->block_tables, (size_t)sh->num_seqs * sh->max_blocks_per_seq * sizeof(int32_t)) ||
+        !h2d(d->context_lens, h->context_lens, (size_t)sh->num_seqs * sizeof(int32_t)) ||
+        !h2d(d->cow_pairs, h->cow_pairs, (size_t)sh->num_cow * 2 * sizeof(int32_t)))
+        return PA_ERR_CUDA;
+    pa_cache_desc cd{sh->num_blocks, sh->block_size, sh->num_kv_heads, sh->head_dim, sh->dtype};
+    pa_status st = PA_OK;
+    if (sh->num_cow > 0 && (st = pa_copy_blocks(k_cache, v_cache, d->cow_pairs, sh->num_cow, &cd, stream)) != PA_OK)
+        return st;
+    if ((st = pa_cache_write(d->k, d->v, k_cache, v_cache, d->slot_mapping, sh->num_tokens, &cd, stream)) != PA_OK)
+        return st;
+    if ((st = pa_decode(d->out, d->q, k_cache, v_cache, d->block_tables, d->context_lens, sh->scale, sh->block_size,
+                        sh->num_kv_heads, sh->num_seqs, sh->num_heads, sh->head_dim, sh->max_blocks_per_seq,
+                        sh->max_context_len, sh->num_blocks, sh->dtype, sh->partition_size, d->workspace,
+                        d->workspace_bytes, stream)) != PA_OK)
+        return st;
+    if (qbytes && (!h->out || !d->out || cudaMemcpyAsync(h->out, d->out, qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess))
+        return PA_ERR_CUDA;
+    return PA_OK;
+}
+
+pa_status pa_get_device_error(uint32_t* flags, void* stream) {
+    if (!flags) return PA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int v = 0;
+    const unsigned int zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, pa_dev::g_error, sizeof(v), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaMemcpyToSymbolAsync(pa_dev::g_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+    *flags = v;
+    return v ? PA_ERR_DEVICE : PA_OK;
+}
+
+}  // extern "C"

@@ -250,3 +250,53 @@ def token_values(seed, stream, pos, shape, dtype, salt=0):
     """
     r = np.random.default_rng([int(seed), int(stream) & 0xFFFFFFFF, int(stream) >> 32, int(pos), int(salt)])
     return to_storage(r.standard_normal(shape, dtype=np.float32), dtype)
+
+
+# ---------------------------------------------------------------------------
+# Device-side draws for full-size workloads (torch RNG on the GPU)
+# ---------------------------------------------------------------------------
+
+@dataclass
+class DeviceDraw:
+    cfg: DecodeConfig
+    context_lens: np.ndarray      # int64 [S]
+    offsets: np.ndarray           # int64 [S + 1]: sequence s owns history rows [off[s], off[s+1])
+    num_blocks: int
+    free_order: np.ndarray        # int32 permutation of the pool (blocks are taken from its end)
+    q: object                     # torch [S, Hq, D]
+    k_hist: object                # torch [sum(ctx), Hkv, D]
+    v_hist: object
+
+
+def draw_device(cfg, seed, device="cuda", context_lens=None, block_size=None):
+    """Draw one decode step's inputs directly on the GPU.
+
+    Lengths, the pool size and its shuffled free order come from numpy's
+    seeded generator; values are standard normal from a seeded torch CUDA
+    generator, rounded to the dtype (1% of K rows scaled by 8 first when the
+    config asks for outliers).
+    """
+    import torch
+    r = rng(seed)
+    bs = block_size or cfg.block_size
+    lens = np.asarray(context_lens if context_lens is not None else context_lengths(cfg, r), dtype=np.int64)
+    need = sum(blocks_for(lens, bs))
+    nb = cfg.num_blocks if cfg.num_blocks else int(math.ceil(need * (1.0 + cfg.spare)))
+    order = r.permutation(nb).astype(np.int32)
+    offsets = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    total = int(offsets[-1])
+    S, Hq, Hkv, D = len(lens), cfg.num_heads, cfg.num_kv_heads, cfg.head_dim
+    tt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[cfg.dtype]
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 1000003 + 17)
+    q = torch.randn((S, Hq, D), generator=g, device=device, dtype=torch.float32).to(tt)
+    k32 = torch.randn((total, Hkv, D), generator=g, device=device, dtype=torch.float32)
+    if cfg.outlier_frac > 0:
+        rows = outlier_rows(r, total * Hkv, cfg.outlier_frac)
+        idx = torch.from_numpy(rows).to(device)
+        flat = k32.view(total * Hkv, D)
+        flat[idx] *= cfg.outlier_scale
+    k = k32.to(tt)
+    del k32
+    v = torch.randn((total, Hkv, D), generator=g, device=device, dtype=torch.float32).to(tt)
+    return DeviceDraw(cfg, lens, offsets, nb, order, q, k, v)

@@ -1,0 +1,218 @@
+"""CPU tests of libpa.so: it loads without a GPU, exports every function that
+include/pa.h declares, and its host block manager and scheduler agree
+bit-exactly with the oracle's Python models (golden traces and random op
+streams).  No CUDA call is made here."""
+
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import block_manager as obm
+from oracle import scheduler as osch
+from paged_kv_cache_381_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from paged_kv_cache_381_b200 import build
+    build.build()
+    import paged_kv_cache_381_b200 as pa
+    return pa
+
+
+def _declared_functions():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if not f.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(pa_\w+)\s*\(", src):
+            names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol(pa):
+    names = _declared_functions()
+    assert len(names) >= 20
+    lib = pa.lib()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    from paged_kv_cache_381_b200 import _native
+    assert names == set(_native.SIGNATURES), names ^ set(_native.SIGNATURES)
+
+
+def test_status_strings(pa):
+    assert pa.lib().pa_status_string(0) == b"ok"
+    assert pa.lib().pa_status_string(3) == b"no free blocks"
+
+
+def test_workspace_size_rules(pa):
+    assert pa.pa_decode_workspace_size(8, 64, 128, 512, 512) == 0      # one partition: no scratch
+    n = pa.pa_decode_workspace_size(8, 64, 128, 32768, 512)
+    parts = 8 * 64 * 64
+    assert n >= parts * 128 * 4 + 2 * parts * 4 + 8 * 64 * 8
+    assert n % 256 == 0
+    assert pa.pa_decode_workspace_size(8, 64, 128, 32768, 100) == 0    # invalid partition size
+
+
+class _Native:
+    """Adapter giving the C++ manager the oracle model's interface."""
+
+    def __init__(self, pa, nb, bs, order):
+        self.bm = pa.BlockManager(nb, bs, order)
+        self.pa = pa
+
+    def apply(self, op):
+        k = op["op"]
+        if k == "allocate":
+            return self.bm.allocate(op["seq"], op["tokens"])
+        if k == "fork":
+            return self.bm.fork(op["parent"], op["child"])
+        if k == "append":
+            return self.bm.append_slot(op["seq"])
+        return self.bm.free(op["seq"])
+
+
+def test_block_manager_golden_trace(pa):
+    with open(os.path.join(GOLDEN, "block_manager_trace.json")) as f:
+        g = json.load(f)
+    nat = _Native(pa, g["num_blocks"], g["block_size"], g["initial_free_order"])
+    for op in g["ops"]:
+        exp = op["expect"]
+        seq = op.get("seq", op.get("child"))
+        if "error" in exp:
+            with pytest.raises(pa.PagedAttentionError) as ei:
+                nat.apply(op)
+            assert ei.value.status == {"no_blocks": 3, "invalid_arg": 1}[exp["error"]]
+        else:
+            res = nat.apply(op)
+            if "slot" in exp:
+                assert res[0] == exp["slot"] and [res[1], res[2]] == exp["cow"], op
+        if "table" in exp:
+            assert nat.bm.block_table(seq) == exp["table"], op
+        if "free" in exp:
+            assert nat.bm.free_list() == exp["free"], op
+        if "ref" in exp:
+            for b, c in exp["ref"].items():
+                assert nat.bm.ref_count(int(b)) == c
+        if "ctx" in exp:
+            assert nat.bm.context_len(seq) == exp["ctx"]
+
+
+def test_block_manager_matches_model_on_random_streams(pa):
+    r = np.random.default_rng(12)
+    for trial in range(25):
+        nb, bs = int(r.integers(3, 50)), int(r.choice([1, 2, 4, 8, 16]))
+        order = r.permutation(nb).tolist()
+        model = obm.BlockManager(nb, bs, order)
+        nat = pa.BlockManager(nb, bs, order)
+        live, nid = [], 0
+        for _ in range(400):
+            c = r.random()
+            if c < 0.2 or not live:
+                op = ("allocate", nid, int(r.integers(0, 4 * bs)))
+            elif c < 0.35:
+                op = ("fork", live[int(r.integers(len(live)))], nid)
+            elif c < 0.85:
+                op = ("append", live[int(r.integers(len(live)))])
+            else:
+                op = ("free", live[int(r.integers(len(live)))])
+            m_err = n_err = None
+            m_res = n_res = None
+            try:
+                m_res = getattr(model, {"append": "append_slot"}.get(op[0], op[0]))(*op[1:])
+            except (obm.NoBlocks, obm.InvalidArg) as e:
+                m_err = type(e).__name__
+            try:
+                n_res = getattr(nat, {"append": "append_slot"}.get(op[0], op[0]))(*op[1:])
+            except pa.PagedAttentionError as e:
+                n_err = {3: "NoBlocks", 1: "InvalidArg"}[e.status]
+            assert m_err == n_err, (op, m_err, n_err)
+            if op[0] == "append" and m_err is None:
+                assert tuple(m_res) == tuple(n_res), op
+            if m_err is None:
+                if op[0] in ("allocate", "fork"):
+                    live.append(op[-1] if op[0] == "fork" else op[1])
+                    nid += 1
+                elif op[0] == "free":
+                    live.remove(op[1])
+            assert model.free_list == nat.free_list(), op
+        for s in live:
+            assert model.block_table(s) == nat.block_table(s)
+            assert model.context_len(s) == nat.context_len(s)
+        assert [model.ref[b] for b in range(nb)] == [nat.ref_count(b) for b in range(nb)]
+
+
+def test_pack_layout(pa):
+    bm = pa.BlockManager(10, 4, list(range(10)))
+    bm.allocate(1, 9)
+    bm.allocate(2, 0)
+    bm.allocate(3, 4)
+    tables, lens = bm.pack([3, 1, 2], 4)
+    assert lens.tolist() == [4, 9, 0]
+    assert tables.tolist() == [[6, -1, -1, -1], [9, 8, 7, -1], [-1, -1, -1, -1]]
+    with pytest.raises(pa.PagedAttentionError):
+        bm.pack([1], 2)          # table wider than the requested width
+
+
+def _load_traces():
+    with open(os.path.join(GOLDEN, "scheduler_traces.json")) as f:
+        return json.load(f)["traces"]
+
+
+@pytest.mark.parametrize("tr", _load_traces(), ids=lambda t: t["name"])
+def test_scheduler_golden_traces(pa, tr):
+    bm = pa.BlockManager(tr["num_blocks"], tr["block_size"], tr["initial_free_order"])
+    prefix = -1
+    if tr["prefix"]:
+        prefix = tr["prefix"]["seq"]
+        bm.allocate(prefix, tr["prefix"]["tokens"])
+    sch = pa.Scheduler(bm, tr["max_running"], prefix)
+    for q in tr["requests"]:
+        sch.add_request(q["seq"], q["prompt"], q["output"], q.get("shares_prefix", False),
+                        q.get("fork_child", -1), q.get("fork_output", 0))
+    for i, exp in enumerate(tr["steps"]):
+        rec = sch.step()
+        for key in ("finished", "admitted", "preempted", "running", "context_lens"):
+            assert rec[key] == exp[key], (i, key, rec[key])
+        assert [list(o) for o in rec["ops"]] == exp["ops"], (i, rec["ops"])
+
+
+def test_scheduler_matches_model_on_trace(pa):
+    """Scaled-down continuous-batching trace: C++ and Python agree every step."""
+    tc = wl.TraceConfig(block_size=8, max_running=32, num_requests=80, steps=150, prefix_len=36,
+                        prompt_hi=100, output_mean=30.0, fork_every=5)
+    reqs = wl.make_trace_requests(tc, 3)
+    nb = 160
+    order = np.random.default_rng(4).permutation(nb).tolist()
+    mb = obm.BlockManager(nb, tc.block_size, order)
+    nbm = pa.BlockManager(nb, tc.block_size, order)
+    mb.allocate(wl.PREFIX_SEQ, tc.prefix_len)
+    nbm.allocate(wl.PREFIX_SEQ, tc.prefix_len)
+    ms = osch.Scheduler(mb, tc.max_running, wl.PREFIX_SEQ)
+    ns = pa.Scheduler(nbm, tc.max_running, wl.PREFIX_SEQ)
+    for q in reqs:
+        ms.add_request(osch.Request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child,
+                                    q.fork_output_len))
+        ns.add_request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child, q.fork_output_len)
+    seen = set()
+    for step in range(tc.steps):
+        a = ms.step()
+        b = ns.step()
+        assert a.finished == b["finished"], step
+        assert a.admitted == b["admitted"], step
+        assert a.preempted == b["preempted"], step
+        assert [tuple(o) for o in a.ops] == b["ops"], step
+        assert a.running == b["running"] and a.context_lens == b["context_lens"], step
+        assert mb.free_list == nbm.free_list(), step
+        seen |= {"preempt"} if a.preempted else set()
+        seen |= {"cow"} if a.cow else set()
+        seen |= {"finish"} if a.finished else set()
+    assert seen == {"preempt", "cow", "finish"}
