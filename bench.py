@@ -49,13 +49,17 @@ KERNEL_SOURCES = ["paged_kv_cache_381_b200/csrc/device/decode.cuh",
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--workload", default="70b", choices=list(WORKLOAD_NAMES))
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--math", default="auto", choices=["auto", "simt"],
+                   help="decode arithmetic: tensor cores for fp16/bf16 (auto) or CUDA cores (simt)")
+    p.add_argument("--num-seqs", type=int, default=0,
+                   help="keep only the first N sequences (smaller cases for profiling)")
     return p.parse_args()
 
 
@@ -267,10 +271,14 @@ def run_native(args):
         dist.barrier()
     import paged_kv_cache_381_b200 as pa
     from paged_kv_cache_381_b200.batch import PagedBatch
+    pa.set_decode_math(pa.MATH_AUTO if args.math == "auto" else pa.MATH_SIMT)
 
     cfg = wl.CONFIGS[args.workload]
     seed = args.seed + rank                       # independent replica per rank
-    d = wl.draw_device(cfg, seed, device=dev)
+    lens_override = None
+    if args.num_seqs:
+        lens_override = wl.context_lengths(cfg, wl.rng(seed))[:args.num_seqs]
+    d = wl.draw_device(cfg, seed, device=dev, context_lens=lens_override)
     batch = PagedBatch(d.k_hist, d.v_hist, d.offsets, d.context_lens, d.num_blocks, cfg.block_size, d.free_order)
     lens = d.context_lens
     q = d.q
@@ -376,7 +384,7 @@ def run_native(args):
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
         "config": {"workload": WORKLOAD_NAMES[args.workload], "num_seqs": len(lens),
                    "context_tokens": int(lens.sum()), "kv_bytes_per_step": step_kv,
-                   "partition_size": P or 512, "l2": "flushed between steps (256 MiB write, outside step events)",
+                   "partition_size": P or 512, "decode_math": args.math, "l2": "flushed between steps (256 MiB write, outside step events)",
                    "parallelism": "replicas" if world > 1 else "single"},
         "pct_of_hbm_peak": value / world / peak,
         "tokens_per_s": world * len(lens) / (ms * 1e-3),

@@ -99,6 +99,8 @@ typedef struct {
  *   slot_mapping    device int64 [num_tokens]
  * For every t with slot_mapping[t] >= 0:
  *   k_cache[slot / bs][slot % bs][:][:] = k[t][:][:]   (same for v), bit-exact.
+ * Non-negative slots must be distinct within one call (tokens are written in
+ * parallel; for a repeated slot it is unspecified which row remains).
  * num_tokens == 0 is a no-op.
  */
 pa_status pa_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
@@ -193,6 +195,20 @@ typedef struct {
 
 pa_status pa_step(const pa_step_host* host, const pa_step_device* dev, void* k_cache,
                   void* v_cache, const pa_step_shape* shape, void* stream);
+
+/*
+ * Arithmetic used by pa_decode's score and output contractions (process-wide):
+ *   PA_MATH_AUTO   tensor cores (mma m16n8k16, fp32 accumulate) for fp16 / bf16,
+ *                  CUDA-core fp32 FMAs for fp32 -- the default;
+ *   PA_MATH_SIMT   CUDA-core fp32 FMAs for every dtype;
+ *   PA_MATH_TENSOR same as AUTO (fp32 always uses CUDA cores).
+ * Both paths give results within the same tolerance of the exact attention;
+ * bits differ between them.  Not to be changed while a decode is being
+ * enqueued on another thread.
+ */
+typedef enum { PA_MATH_AUTO = 0, PA_MATH_SIMT = 1, PA_MATH_TENSOR = 2 } pa_decode_math;
+pa_status pa_set_decode_math(int mode);
+int pa_get_decode_math(void);
 
 /* Reads and clears the device error word (synchronizes `stream`).  Returns
  * PA_ERR_DEVICE when any bit was set, PA_OK otherwise. */
@@ -313,7 +329,8 @@ pa_status pa_sched_counts_get(const pa_sched* s, pa_sched_counts* c);
  *   ops: num_ops entries in issue order; op_kind[i] = 0 for a cache write
  *        (a = seq, b = position, c = slot) or 1 for a copy-on-write block copy
  *        (a = src block, b = dst block, c = -1).  A copy must be applied after
- *        every earlier write and before every later one.
+ *        every earlier write and before every later one.  Ops made dead by a
+ *        preemption in the same step are not listed, so no slot appears twice.
  *   running/context_lens: the batch to decode, in admission order. */
 pa_status pa_sched_record(const pa_sched* s, int64_t* finished, int64_t* admitted,
                           int64_t* preempted, int32_t* op_kind, int64_t* op_a, int64_t* op_b,

@@ -33,7 +33,11 @@ checker compares: cache writes (seq, position, slot) in issue order, CoW
 pairs, admitted / preempted / finished ids, and the running batch with its
 context lengths.  ``ops`` holds the writes and CoW copies interleaved in
 issue order: a copy must see every earlier write to its source block and none
-of the later ones, so the device has to apply them in that order.
+of the later ones, so the device has to apply them in that order.  When a
+preemption frees blocks, every op of the step that targets a freed block (a
+write into it, a copy into it) is dropped from the record: that work is dead,
+and a freed block can be taken again later in the same step, so keeping it
+would list one slot twice.  Within a step every slot is written at most once.
 """
 
 from dataclasses import dataclass, field
@@ -82,6 +86,14 @@ class StepRecord:
     def copy(self, src, dst):
         self.cow.append((src, dst))
         self.ops.append(("c", src, dst))
+
+    def drop_dead(self, bm):
+        """Remove ops whose target block is back on the free list."""
+        bs = bm.block_size
+        live = lambda op: bm.ref[op[3] // bs if op[0] == "w" else op[2]] > 0
+        self.ops = [op for op in self.ops if live(op)]
+        self.writes = [(o[1], o[2], o[3]) for o in self.ops if o[0] == "w"]
+        self.cow = [(o[1], o[2]) for o in self.ops if o[0] == "c"]
 
 
 class Scheduler:
@@ -136,6 +148,7 @@ class Scheduler:
     def _preempt_last(self, rec):
         victim = self.running.pop()
         self.bm.free(victim.seq_id)
+        rec.drop_dead(self.bm)
         self.waiting.insert(0, victim)
         rec.preempted.append(victim.seq_id)
         return victim

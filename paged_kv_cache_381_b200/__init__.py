@@ -177,6 +177,18 @@ def pa_get_device_error(stream=None):
     return int(flags.value)
 
 
+MATH_AUTO, MATH_SIMT, MATH_TENSOR = 0, 1, 2
+
+
+def set_decode_math(mode):
+    """Choose tensor-core (default for fp16/bf16) or CUDA-core decode arithmetic."""
+    _check(lib().pa_set_decode_math(int(mode)), "pa_set_decode_math")
+
+
+def get_decode_math():
+    return int(lib().pa_get_decode_math())
+
+
 def launch_count():
     return int(lib().pa_launch_count())
 

@@ -52,6 +52,8 @@ SIGNATURES = {
     "pa_get_device_error": (c_int, [P(c_uint32), c_void_p]),
     "pa_status_string": (ctypes.c_char_p, [c_int]),
     "pa_launch_count": (c_int64, []),
+    "pa_set_decode_math": (c_int, [c_int]),
+    "pa_get_decode_math": (c_int, []),
     "pa_profile_begin": (c_int, []),
     "pa_profile_end": (c_int, [P(c_double), P(c_int64)]),
     "pa_bm_create": (c_int, [c_int, c_int, c_void_p, P(c_void_p)]),

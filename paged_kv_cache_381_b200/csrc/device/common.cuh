@@ -163,3 +163,79 @@ struct ElemTraits<__half> {
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x >> 1); }
 
 }  // namespace pa_dev
+
+namespace pa_dev {
+
+// ---------------------------------------------------------------------------
+// Warp-level tensor-core helpers (mma.sync m16n8k16, fp32 accumulate) and
+// shared-memory matrix loads.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+template <typename T>
+struct MmaOps;
+
+template <>
+struct MmaOps<__nv_bfloat16> {
+    __device__ __forceinline__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    // two values -> one register, first value in the low half
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ __forceinline__ static float2 unpack(uint32_t r) {
+        return make_float2(__uint_as_float(r << 16), __uint_as_float(r & 0xffff0000u));
+    }
+};
+
+template <>
+struct MmaOps<__half> {
+    __device__ __forceinline__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+        __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ __forceinline__ static float2 unpack(uint32_t r) {
+        return __half22float2(*reinterpret_cast<const __half2*>(&r));
+    }
+};
+
+// Split two fp32 values into a rounded 16-bit pair and the 16-bit pair of
+// what rounding left over: hi + lo carries about twice the mantissa bits.
+template <typename M>
+__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    hi = M::pack(x0, x1);
+    const float2 h = M::unpack(hi);
+    lo = M::pack(x0 - h.x, x1 - h.y);
+}
+
+// Keep the elements of a two-element register whose index (first = 0) is
+// below `valid`: 0 -> none, 1 -> low half only, >= 2 -> both.
+__device__ __forceinline__ uint32_t keep_pair(uint32_t r, int valid) {
+    return valid >= 2 ? r : (valid == 1 ? (r & 0x0000ffffu) : 0u);
+}
+
+}  // namespace pa_dev

@@ -145,15 +145,15 @@ __device__ __forceinline__ float reduce_row_dots(float (&v)[GC], int lane) {
     return v[0];
 }
 
-template <typename T, int D, int GC>
+template <typename T, int D, int GC, bool TENSOR>
 struct DecodeCfg {
     using Tr = ElemTraits<T>;
     static constexpr int ELT = (int)sizeof(T);
     static constexpr int VEC = Tr::VEC;             // elements per 16-byte vector
-    static constexpr int LPT = D / VEC;             // lanes per token row
-    static constexpr int RPI = 32 / LPT;            // rows per warp instruction
+    static constexpr int LPT = D / VEC;             // lanes per token row (SIMT path)
+    static constexpr int RPI = 32 / LPT;            // rows per warp instruction (SIMT path)
     static constexpr int ROW_BYTES = D * ELT;
-    static constexpr int PITCH = ROW_BYTES + 16;    // padded shared-memory row
+    static constexpr int PITCH = ROW_BYTES + 16;    // padded row: stride-row reads hit distinct banks
     static constexpr int STAGE_ROWS = 32;
     static constexpr int STAGE_BYTES = STAGE_ROWS * PITCH;
     static constexpr int NSTAGES = 8;
@@ -161,29 +161,44 @@ struct DecodeCfg {
     static constexpr int THREADS = (NCW + 1) * 32;
     static constexpr int MAX_PARTITION = 1024;
     static constexpr int MAX_TABLE = MAX_PARTITION / 8;
+    // scores row stride (floats): the tensor path reads 8-query rows as pairs;
+    // the SIMT path pads to GC + 1 so per-query column walks avoid bank conflicts
+    static constexpr int LSTRIDE = TENSOR ? GC : (GC == 1 ? 1 : GC + 1);
     static constexpr int OFF_FULL = NSTAGES * STAGE_BYTES;
     static constexpr int OFF_EMPTY = OFF_FULL + NSTAGES * 8;
     static constexpr int OFF_TABLE = OFF_EMPTY + NSTAGES * 8;
-    static constexpr int OFF_STATS = OFF_TABLE + MAX_TABLE * 4;
-    static constexpr int OFF_RED = ((OFF_STATS + (2 * GC + 4) * 4) + 127) / 128 * 128;
+    static constexpr int OFF_STATS = OFF_TABLE + MAX_TABLE * 4;     // wmax, wsum [NCW][GC], m, l [GC], abort
+    static constexpr int STATS_FLOATS = 2 * NCW * GC + 2 * GC + 4;
+    static constexpr int OFF_RED = ((OFF_STATS + STATS_FLOATS * 4) + 127) / 128 * 128;
     static constexpr int RED_BYTES = NCW * GC * D * 4;
     static constexpr int OFF_LOGITS = OFF_RED + RED_BYTES;
-    static_assert(GC <= LPT, "query chunk wider than the lanes of a row");
+    static_assert(TENSOR ? (GC == 8 && ELT == 2) : (GC <= LPT), "unsupported query chunk");
     static_assert(LPT >= 1 && LPT <= 32 && (32 % LPT) == 0, "row must span a divisor of the warp");
     static_assert(PITCH % 16 == 0, "bulk copies need 16-byte aligned rows");
-    static size_t smem_bytes(int partition) { return (size_t)OFF_LOGITS + (size_t)partition * GC * 4; }
+    static size_t smem_bytes(int partition) { return (size_t)OFF_LOGITS + (size_t)partition * LSTRIDE * 4; }
 };
 
-template <typename T, int D, int GC>
-__global__ void __launch_bounds__(DecodeCfg<T, D, GC>::THREADS, 2) decode_kernel(const DecodeArgs a) {
-    using C = DecodeCfg<T, D, GC>;
+// Tensor path (fp16 / bf16), per warp and per 16-token tile, with G <= 8
+// queries of one kv head padded to the n = 8 of mma.m16n8k16:
+//   scores   S^T[16 tok x 8 q]  = K[16 x D] . Q^T[D x 8]    (A = K via ldmatrix, B = q in registers)
+//   output   O^T[D x 8 q]      += V^T[D x 16 tok] . P^T[16 tok x 8 q]
+//                                                (A = V via ldmatrix.trans, B = p built in registers,
+//                                                 p split into a 16-bit value and its remainder)
+// Fragment layouts (PTX m16n8k16): A regs {rows 0-7 | 8-15} x {cols 0-7 | 8-15},
+// B reg0 = (k = 2*tig, 2*tig+1; n = gid), reg1 = same k + 8, C = (gid | gid+8, 2*tig | 2*tig+1),
+// where gid = lane / 4 and tig = lane % 4.
+template <typename T, int D, int GC, bool TENSOR>
+__global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decode_kernel(const DecodeArgs a) {
+    using C = DecodeCfg<T, D, GC, TENSOR>;
     using Tr = ElemTraits<T>;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_FULL);
     uint64_t* empty = reinterpret_cast<uint64_t*>(smem + C::OFF_EMPTY);
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + C::OFF_TABLE);
-    float* stat_m = reinterpret_cast<float*>(smem + C::OFF_STATS);
-    float* stat_l = stat_m + GC;
+    float* wmax = reinterpret_cast<float*>(smem + C::OFF_STATS);   // [NCW][GC]
+    float* wsum = wmax + C::NCW * GC;                                // [NCW][GC]
+    float* stat_m = wsum + C::NCW * GC;                              // [GC]
+    float* stat_l = stat_m + GC;                                     // [GC]
     volatile int* abort_flag = reinterpret_cast<volatile int*>(stat_l + GC);
     float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
     float* logits = reinterpret_cast<float*>(smem + C::OFF_LOGITS);
@@ -268,13 +283,23 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC>::THREADS, 2) decode_kernel
     // -------------------------------------------------------------- consumers
     constexpr int NCT = C::NCW * 32;
     const int ctid = threadIdx.x;
-    const int row_in = lane / C::LPT;                 // row within a warp instruction
-    const int chunk = lane % C::LPT;                  // 16-byte chunk within the row
-    const int gsel = chunk / (C::LPT / GC);           // query owned after the row reduction
-    const bool gwriter = (chunk % (C::LPT / GC)) == 0;
     const T* qg = static_cast<const T*>(a.q);
     T* outg = static_cast<T*>(a.out);
     uint32_t stage = 0;
+
+    // Wait for a stage this warp owns; false once the CTA has given up.
+    auto acquire = [&](uint32_t c) -> bool {
+        const int slot = c % C::NSTAGES;
+        if (*abort_flag || !mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag)) {
+            *abort_flag = 1;
+            return false;
+        }
+        return true;
+    };
+    auto release = [&](uint32_t c) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[c % C::NSTAGES]);
+    };
 
     for (int i = blockIdx.x; i < total; i += gridDim.x) {
         const WorkItem w = decode_item(a, i, false);
@@ -287,131 +312,268 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC>::THREADS, 2) decode_kernel
         }
         const int nst = (w.n + C::STAGE_ROWS - 1) / C::STAGE_ROWS;
 
-        // ---- phase 1: scores z' = (q . k) * scale * log2(e) for every token
-        {
-            float qf[GC][C::VEC];
+        if constexpr (TENSOR) {
+            using M = MmaOps<T>;
+            constexpr int KS = D / 16;                 // k-steps over head_dim
+            const int gid = lane >> 2;
+            const int tig = lane & 3;
+            // ---- phase 1: S^T tiles, scaled to base-2 units, with a running max
+            uint32_t qb[KS][2];
 #pragma unroll
-            for (int g = 0; g < GC; ++g) {
-                if (g < gq) {
-                    const uint4 u = __ldg(reinterpret_cast<const uint4*>(qg + (row0 + g) * D + chunk * C::VEC));
-                    Tr::unpack(u, qf[g]);
+            for (int kk = 0; kk < KS; ++kk) {
+                if (gid < gq) {
+                    const T* qrow = qg + (row0 + gid) * D + kk * 16 + tig * 2;
+                    qb[kk][0] = __ldg(reinterpret_cast<const unsigned int*>(qrow));
+                    qb[kk][1] = __ldg(reinterpret_cast<const unsigned int*>(qrow + 8));
                 } else {
-#pragma unroll
-                    for (int v = 0; v < C::VEC; ++v) qf[g][v] = 0.f;
+                    qb[kk][0] = qb[kk][1] = 0u;
                 }
             }
+            float mlo = -INFINITY, mhi = -INFINITY;      // queries 2*tig, 2*tig+1
             for (int st = warp; st < nst; st += C::NCW) {
                 const uint32_t c = stage + st;
-                const int slot = c % C::NSTAGES;
-                if (*abort_flag || !mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag)) {
-                    *abort_flag = 1;
-                    continue;
-                }
+                if (!acquire(c)) continue;
                 const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
-                const unsigned char* sb = smem + slot * C::STAGE_BYTES;
-                for (int r0 = 0; r0 < rows; r0 += C::RPI) {
-                    const int r = r0 + row_in;
-                    const uint4 u = *reinterpret_cast<const uint4*>(sb + r * C::PITCH + chunk * 16);
-                    float kf[C::VEC];
-                    Tr::unpack(u, kf);
-                    float part[GC];
+                const uint32_t sb = smem_addr(smem + (c % C::NSTAGES) * C::STAGE_BYTES);
+                // ldmatrix row address of this lane: matrix lane/8 -> (+8 rows if odd, +8 cols if >= 2)
+                const uint32_t lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+                const uint32_t lcol = (lane >> 4) * 8;
 #pragma unroll
-                    for (int g = 0; g < GC; ++g) {
-                        float acc = 0.f;
+                for (int mt = 0; mt < 2; ++mt) {
+                    if (mt * 16 >= rows) break;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    const uint32_t base = sb + (mt * 16 + lrow) * C::PITCH + lcol * 2;
 #pragma unroll
-                        for (int v = 0; v < C::VEC; ++v) acc = fmaf(qf[g][v], kf[v], acc);
-                        part[g] = acc;
+                    for (int kk = 0; kk < KS; ++kk) {
+                        uint32_t af[4];
+                        ldsm_x4(base + kk * 32, af[0], af[1], af[2], af[3]);
+                        M::mma(acc, af, qb[kk][0], qb[kk][1]);
                     }
-                    const float z = reduce_row_dots<GC, C::LPT>(part, lane);
-                    if (gwriter && r < rows) logits[(st * C::STAGE_ROWS + r) * GC + gsel] = z * a.scale_log2;
+                    const int t_lo = mt * 16 + gid;            // stage-relative token of acc[0..1]
+                    float* lrow_lo = logits + (st * C::STAGE_ROWS + t_lo) * GC + tig * 2;
+                    if (t_lo < rows) {
+                        const float z0 = acc[0] * a.scale_log2, z1 = acc[1] * a.scale_log2;
+                        *reinterpret_cast<float2*>(lrow_lo) = make_float2(z0, z1);
+                        mlo = fmaxf(mlo, z0);
+                        mhi = fmaxf(mhi, z1);
+                    }
+                    if (t_lo + 8 < rows) {
+                        const float z2 = acc[2] * a.scale_log2, z3 = acc[3] * a.scale_log2;
+                        *reinterpret_cast<float2*>(lrow_lo + 8 * GC) = make_float2(z2, z3);
+                        mlo = fmaxf(mlo, z2);
+                        mhi = fmaxf(mhi, z3);
+                    }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[slot]);
+                release(c);
             }
             stage += nst;
-        }
-        named_barrier(1, NCT);
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, o));
+                mhi = fmaxf(mhi, __shfl_xor_sync(0xffffffffu, mhi, o));
+            }
+            if (gid == 0) {
+                wmax[warp * GC + tig * 2] = mlo;
+                wmax[warp * GC + tig * 2 + 1] = mhi;
+            }
+            named_barrier(1, NCT);
 
-        // ---- phase 2: exact max, exponentials and their sum per query
-        for (int g = warp; g < GC; g += C::NCW) {
-            float m = -INFINITY;
-            for (int t = lane; t < w.n; t += 32) m = fmaxf(m, logits[t * GC + g]);
-            m = warp_max(m);
-            float l = 0.f;
-            for (int t = lane; t < w.n; t += 32) {
-                const float p = exp2f(logits[t * GC + g] - m);
-                logits[t * GC + g] = p;
-                l += p;
-            }
-            l = warp_sum(l);
-            if (lane == 0) {
-                stat_m[g] = m;
-                stat_l[g] = l;
-            }
-        }
-        named_barrier(1, NCT);
-
-        // ---- phase 3: o = sum_t p_t v_t
-        float acc[GC][C::VEC];
+            // ---- phase 3: p = 2^(z - max) built straight into B fragments; O^T += V^T P^T
+            float mg = wmax[gid];
 #pragma unroll
-        for (int g = 0; g < GC; ++g)
+            for (int ww = 1; ww < C::NCW; ++ww) mg = fmaxf(mg, wmax[ww * GC + gid]);
+            float oacc[KS][4];
 #pragma unroll
-            for (int v = 0; v < C::VEC; ++v) acc[g][v] = 0.f;
-        for (int st = warp; st < nst; st += C::NCW) {
-            const uint32_t c = stage + st;
-            const int slot = c % C::NSTAGES;
-            if (*abort_flag || !mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag)) {
-                *abort_flag = 1;
-                continue;
-            }
-            const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
-            const unsigned char* sb = smem + slot * C::STAGE_BYTES;
-            for (int r0 = 0; r0 < rows; r0 += C::RPI) {
-                const int r = r0 + row_in;
-                if (r < rows) {
-                    const uint4 u = *reinterpret_cast<const uint4*>(sb + r * C::PITCH + chunk * 16);
-                    float vf[C::VEC];
-                    Tr::unpack(u, vf);
-                    const float* pr = logits + (st * C::STAGE_ROWS + r) * GC;
-                    float p[GC];
-                    if constexpr (GC % 4 == 0) {
+            for (int dm = 0; dm < KS; ++dm) oacc[dm][0] = oacc[dm][1] = oacc[dm][2] = oacc[dm][3] = 0.f;
+            float lsum = 0.f;
+            // ldmatrix.trans row address: matrix lane/8 -> (+8 tokens if >= 2, +8 head-dim cols if odd)
+            const uint32_t vrow = (lane & 7) + (lane >> 4) * 8;
+            const uint32_t vcol = ((lane >> 3) & 1) * 8;
+            for (int st = warp; st < nst; st += C::NCW) {
+                const uint32_t c = stage + st;
+                if (!acquire(c)) continue;
+                const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
+                const uint32_t sb = smem_addr(smem + (c % C::NSTAGES) * C::STAGE_BYTES);
 #pragma unroll
-                        for (int g = 0; g < GC; g += 4) {
-                            const float4 x = *reinterpret_cast<const float4*>(pr + g);
-                            p[g] = x.x; p[g + 1] = x.y; p[g + 2] = x.z; p[g + 3] = x.w;
+                for (int mt = 0; mt < 2; ++mt) {
+                    if (mt * 16 >= rows) break;
+                    const int k0 = mt * 16 + tig * 2;       // stage-relative tokens of b0; b1 is k0 + 8
+                    const float* lz = logits + (st * C::STAGE_ROWS + k0) * GC + gid;
+                    const float p00 = k0 < rows ? exp2f(lz[0] - mg) : 0.f;
+                    const float p01 = k0 + 1 < rows ? exp2f(lz[GC] - mg) : 0.f;
+                    const float p10 = k0 + 8 < rows ? exp2f(lz[8 * GC] - mg) : 0.f;
+                    const float p11 = k0 + 9 < rows ? exp2f(lz[9 * GC] - mg) : 0.f;
+                    lsum += (p00 + p01) + (p10 + p11);
+                    // p as a 16-bit pair (hi) plus its rounding remainder (lo): two mma per
+                    // tile keep ~16 mantissa bits of p instead of 8 (bf16) or 11 (fp16)
+                    uint32_t b0, b1, b0l, b1l;
+                    split_pack<M>(p00, p01, b0, b0l);
+                    split_pack<M>(p10, p11, b1, b1l);
+                    const bool whole = mt * 16 + 16 <= rows;
+                    const int vlo = rows - k0;              // valid tokens from k0 on (for masking)
+                    const uint32_t base = sb + (mt * 16 + vrow) * C::PITCH + vcol * 2;
+#pragma unroll
+                    for (int dm = 0; dm < KS; ++dm) {
+                        uint32_t af[4];
+                        ldsm_x4_trans(base + dm * 32, af[0], af[1], af[2], af[3]);
+                        if (!whole) {   // rows past the context may hold stale bits (even NaN)
+                            af[0] = keep_pair(af[0], vlo);
+                            af[1] = keep_pair(af[1], vlo);
+                            af[2] = keep_pair(af[2], vlo - 8);
+                            af[3] = keep_pair(af[3], vlo - 8);
                         }
+                        M::mma(oacc[dm], af, b0, b1);
+                        M::mma(oacc[dm], af, b0l, b1l);
+                    }
+                }
+                release(c);
+            }
+            stage += nst;
+            // sum of p for query gid over the lanes holding it (tig = 0..3)
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+            if (tig == 0) wsum[warp * GC + gid] = lsum;
+            // O^T fragment: (d = 16*dm + gid [+8], query 2*tig [+1])
+            float* rw = red + warp * GC * D;
+#pragma unroll
+            for (int dm = 0; dm < KS; ++dm) {
+                const int d0 = dm * 16 + gid;
+                rw[(tig * 2) * D + d0] = oacc[dm][0];
+                rw[(tig * 2 + 1) * D + d0] = oacc[dm][1];
+                rw[(tig * 2) * D + d0 + 8] = oacc[dm][2];
+                rw[(tig * 2 + 1) * D + d0 + 8] = oacc[dm][3];
+            }
+            named_barrier(1, NCT);
+            if (ctid < GC) {
+                float m = wmax[ctid], l = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < C::NCW; ++ww) {
+                    m = fmaxf(m, wmax[ww * GC + ctid]);
+                    l += wsum[ww * GC + ctid];
+                }
+                stat_m[ctid] = m;
+                stat_l[ctid] = l;
+            }
+            named_barrier(1, NCT);
+        } else {
+            constexpr int LS = C::LSTRIDE;
+            const int row_in = lane / C::LPT;                 // row within a warp instruction
+            const int chunk = lane % C::LPT;                  // 16-byte chunk within the row
+            const int gsel = chunk / (C::LPT / GC);           // query owned after the row reduction
+            const bool gwriter = (chunk % (C::LPT / GC)) == 0;
+            // ---- phase 1: z' = (q . k) * scale * log2(e) for every token
+            {
+                float qf[GC][C::VEC];
+#pragma unroll
+                for (int g = 0; g < GC; ++g) {
+                    if (g < gq) {
+                        const uint4 u = __ldg(reinterpret_cast<const uint4*>(qg + (row0 + g) * D + chunk * C::VEC));
+                        Tr::unpack(u, qf[g]);
                     } else {
 #pragma unroll
-                        for (int g = 0; g < GC; ++g) p[g] = pr[g];
+                        for (int v = 0; v < C::VEC; ++v) qf[g][v] = 0.f;
                     }
+                }
+                for (int st = warp; st < nst; st += C::NCW) {
+                    const uint32_t c = stage + st;
+                    if (!acquire(c)) continue;
+                    const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
+                    const unsigned char* sb = smem + (c % C::NSTAGES) * C::STAGE_BYTES;
+#pragma unroll 2
+                    for (int r0 = 0; r0 < rows; r0 += C::RPI) {
+                        const int r = r0 + row_in;
+                        const uint4 u = *reinterpret_cast<const uint4*>(sb + r * C::PITCH + chunk * 16);
+                        float kf[C::VEC];
+                        Tr::unpack(u, kf);
+                        float part[GC];
 #pragma unroll
-                    for (int g = 0; g < GC; ++g)
+                        for (int g = 0; g < GC; ++g) {
+                            float acc = 0.f;
 #pragma unroll
-                        for (int v = 0; v < C::VEC; ++v) acc[g][v] = fmaf(p[g], vf[v], acc[g][v]);
+                            for (int v = 0; v < C::VEC; ++v) acc = fmaf(qf[g][v], kf[v], acc);
+                            part[g] = acc;
+                        }
+                        const float z = reduce_row_dots<GC, C::LPT>(part, lane);
+                        if (gwriter && r < rows) logits[(st * C::STAGE_ROWS + r) * LS + gsel] = z * a.scale_log2;
+                    }
+                    release(c);
+                }
+                stage += nst;
+            }
+            named_barrier(1, NCT);
+
+            // ---- phase 2: exact max, exponentials and their sum per query
+            for (int g = warp; g < GC; g += C::NCW) {
+                float m = -INFINITY;
+                for (int t = lane; t < w.n; t += 32) m = fmaxf(m, logits[t * LS + g]);
+                m = warp_max(m);
+                float l = 0.f;
+                for (int t = lane; t < w.n; t += 32) {
+                    const float p = exp2f(logits[t * LS + g] - m);
+                    logits[t * LS + g] = p;
+                    l += p;
+                }
+                l = warp_sum(l);
+                if (lane == 0) {
+                    stat_m[g] = m;
+                    stat_l[g] = l;
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-        }
-        stage += nst;
+            named_barrier(1, NCT);
 
-        // ---- epilogue: merge rows of a warp, then warps in a fixed order
-#pragma unroll
-        for (int o = C::LPT; o < 32; o <<= 1)
+            // ---- phase 3: o = sum_t p_t v_t
+            float acc[GC][C::VEC];
 #pragma unroll
             for (int g = 0; g < GC; ++g)
 #pragma unroll
-                for (int v = 0; v < C::VEC; ++v) acc[g][v] += __shfl_xor_sync(0xffffffffu, acc[g][v], o);
-        if (row_in == 0) {
+                for (int v = 0; v < C::VEC; ++v) acc[g][v] = 0.f;
+            for (int st = warp; st < nst; st += C::NCW) {
+                const uint32_t c = stage + st;
+                if (!acquire(c)) continue;
+                const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
+                const unsigned char* sb = smem + (c % C::NSTAGES) * C::STAGE_BYTES;
+#pragma unroll 2
+                for (int r0 = 0; r0 < rows; r0 += C::RPI) {
+                    const int r = r0 + row_in;
+                    if (r < rows) {
+                        const uint4 u = *reinterpret_cast<const uint4*>(sb + r * C::PITCH + chunk * 16);
+                        float vf[C::VEC];
+                        Tr::unpack(u, vf);
+                        const float* pr = logits + (st * C::STAGE_ROWS + r) * LS;
+                        float p[GC];
 #pragma unroll
-            for (int g = 0; g < GC; ++g) {
-                float* dst = red + (warp * GC + g) * D + chunk * C::VEC;
+                        for (int g = 0; g < GC; ++g) p[g] = pr[g];
 #pragma unroll
-                for (int v = 0; v < C::VEC; v += 4)
-                    *reinterpret_cast<float4*>(dst + v) = make_float4(acc[g][v], acc[g][v + 1], acc[g][v + 2], acc[g][v + 3]);
+                        for (int g = 0; g < GC; ++g)
+#pragma unroll
+                            for (int v = 0; v < C::VEC; ++v) acc[g][v] = fmaf(p[g], vf[v], acc[g][v]);
+                    }
+                }
+                release(c);
             }
+            stage += nst;
+
+            // merge the rows of a warp, then hand the warp's partial to the epilogue
+#pragma unroll
+            for (int o = C::LPT; o < 32; o <<= 1)
+#pragma unroll
+                for (int g = 0; g < GC; ++g)
+#pragma unroll
+                    for (int v = 0; v < C::VEC; ++v) acc[g][v] += __shfl_xor_sync(0xffffffffu, acc[g][v], o);
+            if (row_in == 0) {
+#pragma unroll
+                for (int g = 0; g < GC; ++g) {
+                    float* dst = red + (warp * GC + g) * D + chunk * C::VEC;
+#pragma unroll
+                    for (int v = 0; v < C::VEC; v += 4)
+                        *reinterpret_cast<float4*>(dst + v) =
+                            make_float4(acc[g][v], acc[g][v + 1], acc[g][v + 2], acc[g][v + 3]);
+                }
+            }
+            named_barrier(1, NCT);
         }
-        named_barrier(1, NCT);
+
+        // ---- epilogue: warps merged in a fixed order; final row or partition partials
         const bool single = (w.np == 1);
         for (int e = ctid; e < gq * D; e += NCT) {
             const int g = e / D;

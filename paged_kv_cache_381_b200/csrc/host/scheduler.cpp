@@ -17,6 +17,9 @@
 //     are freed and it returns to the front of the queue with its progress, and
 //     its whole history is written again when it is re-admitted.
 // The step's record lists cache writes and copy-on-write copies in issue order.
+// A preemption drops from it every op whose target block the preemption
+// returned to the free list (dead work; the block may be taken again later in
+// the same step), so within a step every slot is written at most once.
 
 #include <deque>
 #include <new>
@@ -58,6 +61,18 @@ struct pa_sched {
     }
     void rec_copy(int32_t src, int32_t dst) {
         op_kind.push_back(1); op_a.push_back(src); op_b.push_back(dst); op_c.push_back(-1);
+    }
+    // Remove ops (writes into, copies into) whose target block is free again.
+    void drop_dead_ops() {
+        const int bs = bm->block_size();
+        size_t w = 0;
+        for (size_t i = 0; i < op_kind.size(); ++i) {
+            const int64_t block = op_kind[i] == 0 ? op_c[i] / bs : op_b[i];
+            if (bm->ref((int32_t)block) == 0) continue;
+            op_kind[w] = op_kind[i]; op_a[w] = op_a[i]; op_b[w] = op_b[i]; op_c[w] = op_c[i];
+            ++w;
+        }
+        op_kind.resize(w); op_a.resize(w); op_b.resize(w); op_c.resize(w);
     }
     int64_t own_tokens(const SeqState& s) const { return s.history - (s.shares_prefix ? prefix_len : 0); }
     int64_t required(const SeqState& s) const {
@@ -142,6 +157,7 @@ pa_status pa_sched::step() {
             SeqState victim = running.back();
             running.pop_back();
             if ((st = bm->free_seq(victim.id)) != PA_OK) return st;
+            drop_dead_ops();
             preempted.push_back(victim.id);
             waiting.push_front(victim);
             continue;   // retry the same index (or stop if the victim was this one)

@@ -127,10 +127,12 @@ bool valid_partition(int p) { return p >= 32 && p <= 1024 && p % 32 == 0; }
 int64_t partitions_for(int64_t ctx, int64_t P) { return ctx <= P ? 1 : (ctx + P - 1) / P; }
 
 // ------------------------------------------------------------ decode launch
-template <typename T, int D, int GC>
+std::atomic<int> g_decode_math{PA_MATH_AUTO};
+
+template <typename T, int D, int GC, bool TENSOR>
 pa_status launch_decode(const pa_dev::DecodeArgs& a, int64_t pair_upper, cudaStream_t stream) {
-    using C = pa_dev::DecodeCfg<T, D, GC>;
-    auto kern = pa_dev::decode_kernel<T, D, GC>;
+    using C = pa_dev::DecodeCfg<T, D, GC, TENSOR>;
+    auto kern = pa_dev::decode_kernel<T, D, GC, TENSOR>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
     static std::atomic<uint64_t> configured{0};
@@ -161,19 +163,24 @@ pa_status launch_decode(const pa_dev::DecodeArgs& a, int64_t pair_upper, cudaStr
 }
 
 template <typename T, int D>
-pa_status dispatch_group(const pa_dev::DecodeArgs& a, int gc, int64_t pair_upper, cudaStream_t st) {
+pa_status dispatch_group(const pa_dev::DecodeArgs& a, int gc, bool tensor, int64_t pair_upper, cudaStream_t st) {
+    if constexpr (sizeof(T) == 2) {
+        if (tensor) return launch_decode<T, D, 8, true>(a, pair_upper, st);
+    }
     switch (gc) {
-        case 1: return launch_decode<T, D, 1>(a, pair_upper, st);
-        case 2: return launch_decode<T, D, 2>(a, pair_upper, st);
-        case 4: return launch_decode<T, D, 4>(a, pair_upper, st);
-        case 8: return launch_decode<T, D, 8>(a, pair_upper, st);
+        case 1: return launch_decode<T, D, 1, false>(a, pair_upper, st);
+        case 2: return launch_decode<T, D, 2, false>(a, pair_upper, st);
+        case 4: return launch_decode<T, D, 4, false>(a, pair_upper, st);
+        case 8: return launch_decode<T, D, 8, false>(a, pair_upper, st);
         default: return PA_ERR_UNSUPPORTED;
     }
 }
 
 template <typename T>
-pa_status dispatch_head_dim(const pa_dev::DecodeArgs& a, int D, int gc, int64_t pair_upper, cudaStream_t st) {
-    return D == 64 ? dispatch_group<T, 64>(a, gc, pair_upper, st) : dispatch_group<T, 128>(a, gc, pair_upper, st);
+pa_status dispatch_head_dim(const pa_dev::DecodeArgs& a, int D, int gc, bool tensor, int64_t pair_upper,
+                            cudaStream_t st) {
+    return D == 64 ? dispatch_group<T, 64>(a, gc, tensor, pair_upper, st)
+                   : dispatch_group<T, 128>(a, gc, tensor, pair_upper, st);
 }
 
 template <typename T>
@@ -188,7 +195,8 @@ pa_status launch_reduce(const pa_dev::DecodeArgs& a, int D, cudaStream_t stream)
     return launch_status();
 }
 
-int query_chunk(int group) {
+int query_chunk(int group, bool tensor) {
+    if (tensor) return 8;                  // mma n = 8: one tile holds up to 8 queries
     int g = std::min(group, 8);
     int c = 1;
     while (c < g) c <<= 1;
@@ -212,6 +220,14 @@ const char* pa_status_string(pa_status s) {
 }
 
 int64_t pa_launch_count(void) { return g_launches.load(); }
+
+pa_status pa_set_decode_math(int mode) {
+    if (mode != PA_MATH_AUTO && mode != PA_MATH_SIMT && mode != PA_MATH_TENSOR) return PA_ERR_INVALID_ARG;
+    g_decode_math.store(mode);
+    return PA_OK;
+}
+
+int pa_get_decode_math(void) { return g_decode_math.load(); }
 
 pa_status pa_profile_begin(void) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -312,7 +328,9 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     if (cap > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
     const int64_t maxP = partitions_for(cap, P);
     const int group = num_heads / num_kv_heads;
-    const int gc = query_chunk(group);
+    const int math = g_decode_math.load(std::memory_order_relaxed);
+    const bool tensor = dtype != PA_F32 && math != PA_MATH_SIMT;
+    const int gc = query_chunk(group, tensor);
     const int n_gchunks = (group + gc - 1) / gc;
     if ((int64_t)num_seqs * maxP * num_kv_heads * n_gchunks > INT32_MAX) return PA_ERR_INVALID_ARG;
 
@@ -358,9 +376,9 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     const int64_t pair_upper = (int64_t)num_seqs * maxP;
     pa_status st;
     switch (dtype) {
-        case PA_F32: st = dispatch_head_dim<float>(a, head_dim, gc, pair_upper, s); break;
-        case PA_F16: st = dispatch_head_dim<__half>(a, head_dim, gc, pair_upper, s); break;
-        default: st = dispatch_head_dim<__nv_bfloat16>(a, head_dim, gc, pair_upper, s); break;
+        case PA_F32: st = dispatch_head_dim<float>(a, head_dim, gc, false, pair_upper, s); break;
+        case PA_F16: st = dispatch_head_dim<__half>(a, head_dim, gc, tensor, pair_upper, s); break;
+        default: st = dispatch_head_dim<__nv_bfloat16>(a, head_dim, gc, tensor, pair_upper, s); break;
     }
     if (st != PA_OK || maxP <= 1) return st;
     switch (dtype) {

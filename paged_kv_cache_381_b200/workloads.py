@@ -300,3 +300,54 @@ def draw_device(cfg, seed, device="cuda", context_lens=None, block_size=None):
     del k32
     v = torch.randn((total, Hkv, D), generator=g, device=device, dtype=torch.float32).to(tt)
     return DeviceDraw(cfg, lens, offsets, nb, order, q, k, v)
+
+
+# ---------------------------------------------------------------------------
+# Counter-based rows for traces: any (stream, position) can be regenerated
+# ---------------------------------------------------------------------------
+
+_M64 = np.uint64(0xFFFFFFFFFFFFFFFF)
+
+
+def _splitmix64(x):
+    """SplitMix64 finaliser (Steele, Lea, Flood 2014) on uint64 arrays."""
+    x = np.asarray(x, dtype=np.uint64)
+    z = x + np.uint64(0x9E3779B97F4A7C15)
+    z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+    z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+    return z ^ (z >> np.uint64(31))
+
+
+_ROW_TABLES = {}
+
+
+def _row_tables(seed, width):
+    key = (int(seed), int(width))
+    if key not in _ROW_TABLES:
+        r = np.random.default_rng([int(seed) & 0xFFFFFFFF, 0x5EED, width])
+        _ROW_TABLES[key] = (r.standard_normal((4096, width), dtype=np.float32),
+                            r.standard_normal((4096, width), dtype=np.float32))
+    return _ROW_TABLES[key]
+
+
+def token_rows(seed, stream, positions, heads, head_dim, dtype, salt=0):
+    """Standard-normal rows [len(positions), heads, head_dim] in storage form,
+    keyed by (seed, stream, position, salt) so any row can be drawn again.
+
+    Two tables A, B of 4096 standard-normal rows are drawn once per seed; a
+    row is (A[i] + B[j]) / sqrt(2) with (i, j) taken from a SplitMix64 hash of
+    the key -- 16.7M distinct rows, each element N(0, 1).  salt separates K (0),
+    V (1) and queries (2).
+    """
+    pos = np.asarray(positions, dtype=np.uint64).reshape(-1)
+    with np.errstate(over="ignore"):
+        h = _splitmix64(np.uint64(int(seed) & 0xFFFFFFFFFFFFFFFF) ^ _splitmix64(
+            np.uint64(int(stream) & 0xFFFFFFFFFFFFFFFF) ^ _splitmix64(np.uint64(int(salt) + 1))))
+        h = _splitmix64(h ^ _splitmix64(pos + np.uint64(0x632BE59BD9B4E019)))
+    i = (h & np.uint64(4095)).astype(np.int64)
+    j = ((h >> np.uint64(12)) & np.uint64(4095)).astype(np.int64)
+    A, B = _row_tables(seed, heads * head_dim)
+    z = A[i]
+    z += B[j]
+    z *= np.float32(0.7071067811865476)
+    return to_storage(z.reshape(len(pos), heads, head_dim), dtype)

@@ -31,6 +31,14 @@ def _gpu():
     yield
 
 
+@pytest.fixture(params=["auto", "simt"])
+def math_path(request):
+    """Run a test with the tensor-core (auto) and the CUDA-core decode path."""
+    pa.set_decode_math(pa.MATH_AUTO if request.param == "auto" else pa.MATH_SIMT)
+    yield request.param
+    pa.set_decode_math(pa.MATH_AUTO)
+
+
 def _no_device_error():
     assert pa.pa_get_device_error() == 0
 
@@ -54,6 +62,17 @@ def test_tiny_config_fp32():
     _no_device_error()
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_single_token_context_returns_value_exactly(dtype, math_path):
+    cfg = _grid_cfg(dtype, 128, 16, 8)
+    inp = wl.make_decode_inputs(cfg, 40, context_lens=(1, 1, 300))
+    b, got = _run(inp)
+    G = cfg.num_heads // cfg.num_kv_heads
+    for s in (0, 1):
+        for h in range(cfg.num_heads):
+            assert np.array_equal(got[s, h], inp.v_hist[s][0, h // G]), (s, h)
+
+
 def _grid_cfg(dtype, D, bs, G, hkv=2):
     return wl.DecodeConfig("grid", dtype, 0, G * hkv, hkv, D, bs, "fixed")
 
@@ -65,7 +84,9 @@ GRID_LENS = (0, 1, 2, 31, 32, 33, 100, 511, 512, 513, 1100)
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("bs", [8, 16, 32])
 @pytest.mark.parametrize("G", [1, 4, 8])
-def test_shape_grid(dtype, D, bs, G):
+def test_shape_grid(dtype, D, bs, G, math_path):
+    if dtype == "f32" and math_path != "auto":
+        pytest.skip("fp32 always uses the CUDA-core path")
     cfg = _grid_cfg(dtype, D, bs, G)
     inp = wl.make_decode_inputs(cfg, 1000 + D + bs + G, context_lens=GRID_LENS)
     b, got = _run(inp)
@@ -74,7 +95,7 @@ def test_shape_grid(dtype, D, bs, G):
 
 
 @pytest.mark.parametrize("G", [3, 6, 12, 16])
-def test_uneven_and_wide_groups(G):
+def test_uneven_and_wide_groups(G, math_path):
     """Groups that are not a power of two, or wider than one query chunk."""
     cfg = _grid_cfg("bf16", 128, 16, G)
     inp = wl.make_decode_inputs(cfg, 77 + G, context_lens=(5, 700, 64, 1))
@@ -84,7 +105,7 @@ def test_uneven_and_wide_groups(G):
 
 
 @pytest.mark.parametrize("P", [32, 64, 96, 512, 1024])
-def test_partition_sizes(P):
+def test_partition_sizes(P, math_path):
     cfg = _grid_cfg("f16", 128, 16, 4)
     inp = wl.make_decode_inputs(cfg, 5, context_lens=(1, 95, 96, 97, 1023, 1024, 1025, 2500))
     b, got = _run(inp, partition_size=P)
@@ -92,7 +113,7 @@ def test_partition_sizes(P):
     _no_device_error()
 
 
-def test_split_vs_single_pass():
+def test_split_vs_single_pass(math_path):
     cfg = _grid_cfg("bf16", 128, 16, 8)
     inp = wl.make_decode_inputs(cfg, 6, context_lens=(1000, 17, 640, 1024))
     ref = oracle_outputs(inp)
@@ -116,7 +137,7 @@ def test_cache_write_bit_exact_all_dtypes():
     _no_device_error()
 
 
-def test_block_permutation_is_bitwise_invariant():
+def test_block_permutation_is_bitwise_invariant(math_path):
     cfg = _grid_cfg("bf16", 128, 16, 8)
     lens = (3, 200, 777, 1500)
     inp = wl.make_decode_inputs(cfg, 10, context_lens=lens)
@@ -131,7 +152,7 @@ def test_block_permutation_is_bitwise_invariant():
     assert_close(outs[0], oracle_outputs(inp), "bf16")
 
 
-def test_shared_prefix_matches_private_copies_bitwise():
+def test_shared_prefix_matches_private_copies_bitwise(math_path):
     """Sequences that fork a prefix holder (shared blocks, copy-on-write on the
     first divergent write) give the same bits as sequences holding copies."""
     cfg = _grid_cfg("f16", 128, 16, 4)
@@ -205,7 +226,7 @@ def test_copy_blocks_bit_exact():
     _no_device_error()
 
 
-def test_long_context_with_outlier_keys():
+def test_long_context_with_outlier_keys(math_path):
     """Two 8192-token sequences, 1% of K rows scaled by 8, 512-token partitions."""
     cfg = wl.DecodeConfig("longsmall", "bf16", 2, 64, 8, 128, 16, "const", len_lo=8192, len_hi=8192,
                           partition_size=512, outlier_frac=0.01)
@@ -249,11 +270,12 @@ def test_argument_errors_are_synchronous():
     inp = wl.make_decode_inputs(cfg, 13, context_lens=(10,))
     b = DeviceBatch(inp)
     out = torch.empty_like(b.q)
+    wide = torch.zeros((1, 400), dtype=torch.int32, device="cuda")    # valid ids, wide enough for 5000 tokens
     ptrs = (out.data_ptr(), b.q.data_ptr(), b.k_cache.data_ptr(), b.v_cache.data_ptr(),
-            b.block_tables.data_ptr(), b.context_lens.data_ptr())
+            wide.data_ptr(), b.context_lens.data_ptr())
 
     def call(bs=16, hkv=2, hq=16, D=128, mcl=10):
-        return pa.lib().pa_decode(*ptrs, 0.1, bs, hkv, 1, hq, D, 1, mcl, b.nb, 2, 0, None, 0, None)
+        return pa.lib().pa_decode(*ptrs, 0.1, bs, hkv, 1, hq, D, 400, mcl, b.nb, 2, 0, None, 0, None)
 
     assert call(D=96) == 2           # head_dim 96 unsupported
     assert call(hkv=3) == 1          # 16 query heads are not a multiple of 3 kv heads
@@ -317,7 +339,7 @@ def _sample_rows(lens, Hq, k, seed):
 
 
 @pytest.mark.parametrize("name", ["7b", "70b", "long"])
-def test_full_size_sampled(name):
+def test_full_size_sampled(name, math_path):
     cfg = wl.CONFIGS[name]
     d = wl.draw_device(cfg, 0)
     batch = PagedBatch(d.k_hist, d.v_hist, d.offsets, d.context_lens, d.num_blocks, cfg.block_size,

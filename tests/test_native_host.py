@@ -216,3 +216,43 @@ def test_scheduler_matches_model_on_trace(pa):
         seen |= {"cow"} if a.cow else set()
         seen |= {"finish"} if a.finished else set()
     assert seen == {"preempt", "cow", "finish"}
+
+
+def test_full_trace_host_side_lockstep(pa):
+    """The full-size continuous-batching trace's bookkeeping (no device work):
+    native scheduler == oracle model every step, slots unique within a step."""
+    import math
+    tc = wl.TRACE
+    reqs = wl.make_trace_requests(tc, 5)
+    big = pa.BlockManager(1 << 20, tc.block_size)
+    big.allocate(wl.PREFIX_SEQ, tc.prefix_len)
+    dry = pa.Scheduler(big, tc.max_running, wl.PREFIX_SEQ)
+    for q in reqs:
+        dry.add_request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child, q.fork_output_len)
+    peak = 0
+    for _ in range(tc.steps):
+        dry.step()
+        peak = max(peak, big.stats()[1])
+    nb = int(math.ceil(tc.pool_frac * peak))
+    order = np.random.default_rng(5).permutation(nb).tolist()
+    mb = obm.BlockManager(nb, tc.block_size, order)
+    nbm = pa.BlockManager(nb, tc.block_size, order)
+    mb.allocate(wl.PREFIX_SEQ, tc.prefix_len)
+    nbm.allocate(wl.PREFIX_SEQ, tc.prefix_len)
+    ms = osch.Scheduler(mb, tc.max_running, wl.PREFIX_SEQ)
+    ns = pa.Scheduler(nbm, tc.max_running, wl.PREFIX_SEQ)
+    for q in reqs:
+        ms.add_request(osch.Request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child,
+                                    q.fork_output_len))
+        ns.add_request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child, q.fork_output_len)
+    preempted = 0
+    for step in range(tc.steps):
+        a = ms.step()
+        b = ns.step()
+        assert [tuple(o) for o in a.ops] == b["ops"] and a.running == b["running"], step
+        assert a.context_lens == b["context_lens"] and a.preempted == b["preempted"], step
+        slots = [w[2] for w in a.writes]
+        assert len(slots) == len(set(slots)), step
+        preempted += len(a.preempted)
+        mb.check()
+    assert preempted > 0

@@ -271,6 +271,8 @@ def test_scheduler_random_trace_invariants():
             else:
                 _, seq, pos, slot = op
                 shadow[slot] = (stream_of(seq, pos), pos)
+        slots = [w[2] for w in rec.writes]
+        assert len(slots) == len(set(slots)), "a slot written twice in one step"
         saw_preempt |= bool(rec.preempted)
         for a in rec.admitted:
             if a < tc.num_requests and a not in first_admit:
