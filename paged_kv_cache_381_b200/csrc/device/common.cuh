@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>          // CUtensorMap (type only; no driver library is linked)
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -236,6 +237,26 @@ __device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uin
 // below `valid`: 0 -> none, 1 -> low half only, >= 2 -> both.
 __device__ __forceinline__ uint32_t keep_pair(uint32_t r, int valid) {
     return valid >= 2 ? r : (valid == 1 ? (r & 0x0000ffffu) : 0u);
+}
+
+}  // namespace pa_dev
+
+namespace pa_dev {
+
+// Tiled TMA load of one 3-D box (coordinates innermost first) into shared
+// memory, completion counted on `bar`, with an L2 eviction-priority policy.
+// The tensor map lives in kernel parameter space (__grid_constant__).
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int c0, int c1, int c2, uint64_t* bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void* tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
 }  // namespace pa_dev

@@ -17,11 +17,16 @@
 //    planning kernel and a persistent grid (a multiple of the SM count) walks
 //    them with a fixed stride.
 //  * One producer warp resolves block ids through the block table (staged in
-//    shared memory) and issues one bulk copy per token row (the row of one kv
-//    head is contiguous: head_dim * elt bytes) into a ring of shared-memory
-//    stages of 32 rows, each stage completed on an mbarrier with transaction
-//    counts.  Rows are stored with a 16-byte pad so stride-row reads spread
-//    over all banks.
+//    shared memory) and issues tiled TMA loads into a ring of shared-memory
+//    stages of 32 token rows, each stage completed on an mbarrier with
+//    transaction counts.  The pool is seen by the TMA unit as a 3-D tensor
+//    [num_blocks * block_size rows][num_kv_heads][head_dim]; one box is the
+//    block_size rows of one kv head and one 128-byte slice of head_dim, so a
+//    16-token block of a 128-wide bf16 head arrives in two 2 KiB loads (per-row
+//    256-byte bulk copies were measured to cap a producer warp near 7 GB/s).
+//    Boxes land with the 128-byte swizzle (16-byte chunk index XOR row % 8),
+//    which keeps 8-row ldmatrix and 16-byte vector reads free of bank
+//    conflicts; consumers apply the same XOR when they address a row.
 //  * Four consumer warps: phase 1 computes the scaled scores of every token of
 //    the partition into shared memory (16-byte vector reads, fp32 FMAs, a
 //    transposing butterfly that reduces G partial dot products over the lanes
@@ -153,9 +158,10 @@ struct DecodeCfg {
     static constexpr int LPT = D / VEC;             // lanes per token row (SIMT path)
     static constexpr int RPI = 32 / LPT;            // rows per warp instruction (SIMT path)
     static constexpr int ROW_BYTES = D * ELT;
-    static constexpr int PITCH = ROW_BYTES + 16;    // padded row: stride-row reads hit distinct banks
+    static constexpr int NH = ROW_BYTES / 128;      // 128-byte slices of a row (one TMA box each)
+    static constexpr int BOX_ELEMS = 128 / ELT;     // head_dim elements per slice
     static constexpr int STAGE_ROWS = 32;
-    static constexpr int STAGE_BYTES = STAGE_ROWS * PITCH;
+    static constexpr int STAGE_BYTES = STAGE_ROWS * ROW_BYTES;
     static constexpr int NSTAGES = 8;
     static constexpr int NCW = 4;                   // consumer warps
     static constexpr int THREADS = (NCW + 1) * 32;
@@ -164,7 +170,7 @@ struct DecodeCfg {
     // scores row stride (floats): the tensor path reads 8-query rows as pairs;
     // the SIMT path pads to GC + 1 so per-query column walks avoid bank conflicts
     static constexpr int LSTRIDE = TENSOR ? GC : (GC == 1 ? 1 : GC + 1);
-    static constexpr int OFF_FULL = NSTAGES * STAGE_BYTES;
+    static constexpr int OFF_FULL = NSTAGES * STAGE_BYTES;   // ring at a 1024-byte aligned base
     static constexpr int OFF_EMPTY = OFF_FULL + NSTAGES * 8;
     static constexpr int OFF_TABLE = OFF_EMPTY + NSTAGES * 8;
     static constexpr int OFF_STATS = OFF_TABLE + MAX_TABLE * 4;     // wmax, wsum [NCW][GC], m, l [GC], abort
@@ -174,8 +180,11 @@ struct DecodeCfg {
     static constexpr int OFF_LOGITS = OFF_RED + RED_BYTES;
     static_assert(TENSOR ? (GC == 8 && ELT == 2) : (GC <= LPT), "unsupported query chunk");
     static_assert(LPT >= 1 && LPT <= 32 && (32 % LPT) == 0, "row must span a divisor of the warp");
-    static_assert(PITCH % 16 == 0, "bulk copies need 16-byte aligned rows");
-    static size_t smem_bytes(int partition) { return (size_t)OFF_LOGITS + (size_t)partition * LSTRIDE * 4; }
+    static_assert(ROW_BYTES % 128 == 0 && STAGE_BYTES % 1024 == 0, "swizzled boxes need 1024-byte alignment");
+    // + 1024: the dynamic shared-memory base is rounded up to 1024 bytes in the kernel
+    static size_t smem_bytes(int partition) {
+        return 1024 + (size_t)OFF_LOGITS + (size_t)partition * LSTRIDE * 4;
+    }
 };
 
 // Tensor path (fp16 / bf16), per warp and per 16-token tile, with G <= 8
@@ -188,10 +197,14 @@ struct DecodeCfg {
 // B reg0 = (k = 2*tig, 2*tig+1; n = gid), reg1 = same k + 8, C = (gid | gid+8, 2*tig | 2*tig+1),
 // where gid = lane / 4 and tig = lane % 4.
 template <typename T, int D, int GC, bool TENSOR>
-__global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2)
+    decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_v) {
     using C = DecodeCfg<T, D, GC, TENSOR>;
     using Tr = ElemTraits<T>;
-    extern __shared__ __align__(128) unsigned char smem[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_FULL);
     uint64_t* empty = reinterpret_cast<uint64_t*>(smem + C::OFF_EMPTY);
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + C::OFF_TABLE);
@@ -219,12 +232,21 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decod
     const int pairs = a.max_partitions == 1 ? a.num_seqs : *a.plan_count;
     const int total = pairs * a.num_kv_heads * a.n_gchunks;
     const int bs = 1 << a.log2_bs;
+    const int box_bytes = bs * 128;
+    // byte offset, within a stage, of 16-byte chunk c of stage row r
+    auto row_base = [&](int r) -> int {
+        return ((r >> a.log2_bs) * C::NH) * box_bytes + (r & (bs - 1)) * 128;
+    };
+    auto chunk_off = [&](int r, int c) -> int {
+        return row_base(r) + (c >> 3) * box_bytes + (((c & 7) ^ (r & 7)) << 4);
+    };
 
     if (warp == C::NCW) {
         // ------------------------------------------------------------ producer
-        const unsigned char* kbase = static_cast<const unsigned char*>(a.k_cache);
-        const unsigned char* vbase = static_cast<const unsigned char*>(a.v_cache);
-        const int64_t slot_stride = (int64_t)a.num_kv_heads * C::ROW_BYTES;
+        if (lane == 0) {
+            prefetch_tmap(&tmap_k);
+            prefetch_tmap(&tmap_v);
+        }
         const uint64_t policy = l2_policy_evict_first();
         uint32_t stage = 0;
         bool ok = true;
@@ -244,7 +266,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decod
             }
             __syncwarp();
             for (int pass = 0; pass < 2 && ok; ++pass) {
-                const unsigned char* base = (pass ? vbase : kbase) + (int64_t)w.h * C::ROW_BYTES;
+                const void* tmap = pass ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
                 for (int st = 0; st < nst; ++st, ++stage) {
                     const int slot = stage % C::NSTAGES;
                     const uint32_t parity = ((stage / C::NSTAGES) & 1u) ^ 1u;
@@ -253,13 +275,16 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decod
                         break;
                     }
                     const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
-                    if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(rows * C::ROW_BYTES));
+                    const int nblk_st = (rows + bs - 1) >> a.log2_bs;      // whole blocks are loaded
+                    const int nbox = nblk_st * C::NH;
+                    if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbox * box_bytes));
                     __syncwarp();
-                    if (lane < rows) {
-                        const int tok = st * C::STAGE_ROWS + lane;
-                        const int64_t phys = (int64_t)tbl[tok >> a.log2_bs] * bs + (tok & (bs - 1));
-                        bulk_copy_g2s_hint(smem + slot * C::STAGE_BYTES + lane * C::PITCH, base + phys * slot_stride,
-                                           (uint32_t)C::ROW_BYTES, &full[slot], policy);
+                    if (lane < nbox) {
+                        const int b = lane / C::NH;
+                        const int half = lane - b * C::NH;
+                        const int phys = tbl[((st * C::STAGE_ROWS) >> a.log2_bs) + b];
+                        tma_load_3d(smem + slot * C::STAGE_BYTES + (b * C::NH + half) * box_bytes, tmap,
+                                    half * C::BOX_ELEMS, w.h, phys * bs, &full[slot], policy);
                     }
                 }
             }
@@ -335,18 +360,21 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decod
                 if (!acquire(c)) continue;
                 const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
                 const uint32_t sb = smem_addr(smem + (c % C::NSTAGES) * C::STAGE_BYTES);
-                // ldmatrix row address of this lane: matrix lane/8 -> (+8 rows if odd, +8 cols if >= 2)
-                const uint32_t lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
-                const uint32_t lcol = (lane >> 4) * 8;
+                // ldmatrix row address of this lane: matrix lane/8 -> (+8 rows if odd, +8 cols if >= 2);
+                // row % 8 == lane % 8, the swizzle key
+                const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int hi = lane >> 4;
+                const int x = lane & 7;
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
                     if (mt * 16 >= rows) break;
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    const uint32_t base = sb + (mt * 16 + lrow) * C::PITCH + lcol * 2;
+                    const uint32_t base = sb + row_base(mt * 16 + lrow);
 #pragma unroll
                     for (int kk = 0; kk < KS; ++kk) {
                         uint32_t af[4];
-                        ldsm_x4(base + kk * 32, af[0], af[1], af[2], af[3]);
+                        const int cc = ((kk * 2) & 7) + hi;         // 16-byte chunk within the slice
+                        ldsm_x4(base + (kk >> 2) * box_bytes + ((cc ^ x) << 4), af[0], af[1], af[2], af[3]);
                         M::mma(acc, af, qb[kk][0], qb[kk][1]);
                     }
                     const int t_lo = mt * 16 + gid;            // stage-relative token of acc[0..1]
@@ -387,8 +415,9 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decod
             for (int dm = 0; dm < KS; ++dm) oacc[dm][0] = oacc[dm][1] = oacc[dm][2] = oacc[dm][3] = 0.f;
             float lsum = 0.f;
             // ldmatrix.trans row address: matrix lane/8 -> (+8 tokens if >= 2, +8 head-dim cols if odd)
-            const uint32_t vrow = (lane & 7) + (lane >> 4) * 8;
-            const uint32_t vcol = ((lane >> 3) & 1) * 8;
+            const int vrow = (lane & 7) + (lane >> 4) * 8;
+            const int vhi = (lane >> 3) & 1;
+            const int vx = lane & 7;
             for (int st = warp; st < nst; st += C::NCW) {
                 const uint32_t c = stage + st;
                 if (!acquire(c)) continue;
@@ -411,11 +440,12 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decod
                     split_pack<M>(p10, p11, b1, b1l);
                     const bool whole = mt * 16 + 16 <= rows;
                     const int vlo = rows - k0;              // valid tokens from k0 on (for masking)
-                    const uint32_t base = sb + (mt * 16 + vrow) * C::PITCH + vcol * 2;
+                    const uint32_t base = sb + row_base(mt * 16 + vrow);
 #pragma unroll
                     for (int dm = 0; dm < KS; ++dm) {
                         uint32_t af[4];
-                        ldsm_x4_trans(base + dm * 32, af[0], af[1], af[2], af[3]);
+                        const int cc = ((dm * 2) & 7) + vhi;
+                        ldsm_x4_trans(base + (dm >> 2) * box_bytes + ((cc ^ vx) << 4), af[0], af[1], af[2], af[3]);
                         if (!whole) {   // rows past the context may hold stale bits (even NaN)
                             af[0] = keep_pair(af[0], vlo);
                             af[1] = keep_pair(af[1], vlo);
@@ -482,7 +512,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decod
 #pragma unroll 2
                     for (int r0 = 0; r0 < rows; r0 += C::RPI) {
                         const int r = r0 + row_in;
-                        const uint4 u = *reinterpret_cast<const uint4*>(sb + r * C::PITCH + chunk * 16);
+                        const uint4 u = *reinterpret_cast<const uint4*>(sb + chunk_off(r, chunk));
                         float kf[C::VEC];
                         Tr::unpack(u, kf);
                         float part[GC];
@@ -536,7 +566,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2) decod
                 for (int r0 = 0; r0 < rows; r0 += C::RPI) {
                     const int r = r0 + row_in;
                     if (r < rows) {
-                        const uint4 u = *reinterpret_cast<const uint4*>(sb + r * C::PITCH + chunk * 16);
+                        const uint4 u = *reinterpret_cast<const uint4*>(sb + chunk_off(r, chunk));
                         float vf[C::VEC];
                         Tr::unpack(u, vf);
                         const float* pr = logits + (st * C::STAGE_ROWS + r) * LS;

@@ -4,6 +4,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cudaTypedefs.h>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -129,8 +130,48 @@ int64_t partitions_for(int64_t ctx, int64_t P) { return ctx <= P ? 1 : (ctx + P 
 // ------------------------------------------------------------ decode launch
 std::atomic<int> g_decode_math{PA_MATH_AUTO};
 
+// ---------------------------------------------------------------- TMA maps
+// cuTensorMapEncodeTiled is reached through the runtime's driver entry point,
+// so no driver library is linked.  Encoding is pure host work.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// The pool [num_blocks, block_size, num_kv_heads, head_dim] as the 3-D tensor
+// (head_dim, num_kv_heads, num_blocks * block_size), innermost first; one box
+// is one 128-byte slice of head_dim for one kv head and block_size rows,
+// landing with the 128-byte swizzle.
+bool encode_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, int head_dim, int num_kv_heads,
+                     int num_blocks, int block_size) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t elt = dtype == PA_F32 ? 4 : 2;
+    const CUtensorMapDataType t = dtype == PA_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                  : dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
+                          (cuuint64_t)num_blocks * (cuuint64_t)block_size};
+    cuuint64_t strides[2] = {(cuuint64_t)head_dim * elt, (cuuint64_t)num_kv_heads * head_dim * elt};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / elt), 1u, (cuuint32_t)block_size};
+    cuuint32_t estride[3] = {1u, 1u, 1u};
+    CUresult r = enc(map, t, 3, const_cast<void*>(pool), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <typename T, int D, int GC, bool TENSOR>
-pa_status launch_decode(const pa_dev::DecodeArgs& a, int64_t pair_upper, cudaStream_t stream) {
+pa_status launch_decode(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                        int64_t pair_upper, cudaStream_t stream) {
     using C = pa_dev::DecodeCfg<T, D, GC, TENSOR>;
     auto kern = pa_dev::decode_kernel<T, D, GC, TENSOR>;
     int dev = 0;
@@ -158,29 +199,30 @@ pa_status launch_decode(const pa_dev::DecodeArgs& a, int64_t pair_upper, cudaStr
     const int64_t items_upper = pair_upper * a.num_kv_heads * a.n_gchunks;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items_upper, (int64_t)device_sms(dev) * occ));
     LaunchScope scope(PA_KERNEL_DECODE, stream);
-    kern<<<(unsigned)grid, C::THREADS, smem, stream>>>(a);
+    kern<<<(unsigned)grid, C::THREADS, smem, stream>>>(a, tk, tv);
     return launch_status();
 }
 
 template <typename T, int D>
-pa_status dispatch_group(const pa_dev::DecodeArgs& a, int gc, bool tensor, int64_t pair_upper, cudaStream_t st) {
+pa_status dispatch_group(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int gc,
+                         bool tensor, int64_t pair_upper, cudaStream_t st) {
     if constexpr (sizeof(T) == 2) {
-        if (tensor) return launch_decode<T, D, 8, true>(a, pair_upper, st);
+        if (tensor) return launch_decode<T, D, 8, true>(a, tk, tv, pair_upper, st);
     }
     switch (gc) {
-        case 1: return launch_decode<T, D, 1, false>(a, pair_upper, st);
-        case 2: return launch_decode<T, D, 2, false>(a, pair_upper, st);
-        case 4: return launch_decode<T, D, 4, false>(a, pair_upper, st);
-        case 8: return launch_decode<T, D, 8, false>(a, pair_upper, st);
+        case 1: return launch_decode<T, D, 1, false>(a, tk, tv, pair_upper, st);
+        case 2: return launch_decode<T, D, 2, false>(a, tk, tv, pair_upper, st);
+        case 4: return launch_decode<T, D, 4, false>(a, tk, tv, pair_upper, st);
+        case 8: return launch_decode<T, D, 8, false>(a, tk, tv, pair_upper, st);
         default: return PA_ERR_UNSUPPORTED;
     }
 }
 
 template <typename T>
-pa_status dispatch_head_dim(const pa_dev::DecodeArgs& a, int D, int gc, bool tensor, int64_t pair_upper,
-                            cudaStream_t st) {
-    return D == 64 ? dispatch_group<T, 64>(a, gc, tensor, pair_upper, st)
-                   : dispatch_group<T, 128>(a, gc, tensor, pair_upper, st);
+pa_status dispatch_head_dim(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int D, int gc,
+                            bool tensor, int64_t pair_upper, cudaStream_t st) {
+    return D == 64 ? dispatch_group<T, 64>(a, tk, tv, gc, tensor, pair_upper, st)
+                   : dispatch_group<T, 128>(a, tk, tv, gc, tensor, pair_upper, st);
 }
 
 template <typename T>
@@ -323,6 +365,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
 
+    if ((int64_t)num_blocks * block_size > INT32_MAX) return PA_ERR_UNSUPPORTED;
     const int64_t table_cap = (int64_t)max_blocks_per_seq * block_size;
     const int64_t cap = std::min<int64_t>(max_context_len, table_cap);
     if (cap > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
@@ -373,12 +416,16 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
             if (launch_status() != PA_OK) return PA_ERR_CUDA;
         }
     }
+    CUtensorMap tk, tv;
+    if (!encode_pool_map(&tk, k_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size) ||
+        !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size))
+        return PA_ERR_CUDA;
     const int64_t pair_upper = (int64_t)num_seqs * maxP;
     pa_status st;
     switch (dtype) {
-        case PA_F32: st = dispatch_head_dim<float>(a, head_dim, gc, false, pair_upper, s); break;
-        case PA_F16: st = dispatch_head_dim<__half>(a, head_dim, gc, tensor, pair_upper, s); break;
-        default: st = dispatch_head_dim<__nv_bfloat16>(a, head_dim, gc, tensor, pair_upper, s); break;
+        case PA_F32: st = dispatch_head_dim<float>(a, tk, tv, head_dim, gc, false, pair_upper, s); break;
+        case PA_F16: st = dispatch_head_dim<__half>(a, tk, tv, head_dim, gc, tensor, pair_upper, s); break;
+        default: st = dispatch_head_dim<__nv_bfloat16>(a, tk, tv, head_dim, gc, tensor, pair_upper, s); break;
     }
     if (st != PA_OK || maxP <= 1) return st;
     switch (dtype) {
