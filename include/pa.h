@@ -146,6 +146,32 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     void* stream);
 
 /*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this call: it exists for users of
+ * this library whose device memory is already spoken for (a serving engine
+ * that gives nearly all of it to the KV block pool and allocates nothing
+ * afterwards) or who may not call cudaMalloc on their path (an allocation can
+ * synchronise the device).  Same inputs, outputs and result as pa_decode; the
+ * split-K scratch is a fixed device array of PA_NOALLOC_SCRATCH_BYTES inside
+ * the library instead of a caller-supplied workspace.
+ *   - Every GPU on which the library is loaded holds that array until exit.
+ *   - A batch needing more scratch than that (pa_decode_workspace_size) is
+ *     rejected with PA_ERR_UNSUPPORTED before any launch.
+ *   - The first call on a device looks up the array's device address for that
+ *     device; make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents (no part
+ *     of it needs to start at zero); calls that overlap on the GPU race on it.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens, float scale,
+                            int block_size, int num_kv_heads,
+                            int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                            int max_context_len, int num_blocks, pa_dtype dtype,
+                            int partition_size, void* stream);
+
+/*
  * pa_copy_blocks -- copy-on-write support ([P2] 2.2: a shared block is copied
  * before it is written).  pairs: device int32 [num_pairs][2] of (src, dst)
  * physical block ids; copies the whole block (all block_size slots, all heads)

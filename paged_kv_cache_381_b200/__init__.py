@@ -140,6 +140,29 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block
     return out
 
 
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size=None,
+                      num_kv_heads=None, max_context_len=None, partition_size=0, stream=None):
+    """pa_decode without a workspace: the library's fixed scratch array is used
+    (for callers that cannot allocate device memory; see include/pa.h)."""
+    import torch
+    nb, bs, hkv, d = k_cache.shape
+    block_size = bs if block_size is None else block_size
+    num_kv_heads = hkv if num_kv_heads is None else num_kv_heads
+    S, Hq, D = q.shape
+    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 1
+    if max_context_len is None:
+        max_context_len = maxb * block_size
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    st = lib().pa_decode_noalloc(_dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
+                                 _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables"),
+                                 _dev(context_lens, "context_lens"), float(scale), int(block_size),
+                                 int(num_kv_heads), S, Hq, D, maxb, int(max_context_len), nb, _dtype_code(q),
+                                 int(partition_size), _stream(q, stream))
+    _check(st, "pa_decode_noalloc")
+    return out
+
+
 def pa_step(host, dev, k_cache, v_cache, scale, max_context_len, partition_size=0, stream=None):
     """One layer-step from host buffers (see include/pa.h, pa_step).
 

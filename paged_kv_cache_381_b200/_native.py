@@ -47,6 +47,8 @@ SIGNATURES = {
     "pa_decode_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "pa_decode": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int, c_int,
                           c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "pa_decode_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int,
+                                  c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p]),
     "pa_copy_blocks": (c_int, [c_void_p, c_void_p, c_void_p, c_int, P(CacheDesc), c_void_p]),
     "pa_step": (c_int, [P(StepHost), P(StepDevice), c_void_p, c_void_p, P(StepShape), c_void_p]),
     "pa_get_device_error": (c_int, [P(c_uint32), c_void_p]),

@@ -19,6 +19,7 @@ LIB = os.path.join(PKG, "libpa.so")
 
 SOURCES = [
     os.path.join(CSRC, "pa_api.cu"),
+    os.path.join(CSRC, "pa_noalloc.cu"),
     os.path.join(CSRC, "host", "block_manager.cpp"),
     os.path.join(CSRC, "host", "scheduler.cpp"),
 ]
