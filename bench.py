@@ -58,6 +58,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--math", default="auto", choices=["auto", "simt"],
                    help="decode arithmetic: tensor cores for fp16/bf16 (auto) or CUDA cores (simt)")
+    p.add_argument("--merge", default="kernel", choices=["kernel", "fused"],
+                   help="merge split partitions with the reduce kernel or inside the decode kernel")
     p.add_argument("--num-seqs", type=int, default=0,
                    help="keep only the first N sequences (smaller cases for profiling)")
     return p.parse_args()
@@ -101,10 +103,12 @@ def kv_bytes(cfg, lens):
     return int(np.sum(lens)) * 2 * cfg.num_kv_heads * cfg.head_dim * elt_bytes(cfg.dtype)
 
 
-def decode_kernel_bytes(cfg, lens, partition):
+def decode_kernel_bytes(cfg, lens, partition, fused=False):
     """Algorithmic bytes one decode-kernel launch must move: live K/V rows, q,
-    the final rows of one-partition sequences, the fp32 partials (o, m, l) of
-    split sequences, and the block-table entries each kv head reads."""
+    the final rows it writes (all of them when partitions are merged in the
+    kernel, else those of one-partition sequences), the fp32 partials (o, m, l)
+    of split sequences (written, and read back when merged in the kernel), and
+    the block-table entries each kv head reads."""
     e = elt_bytes(cfg.dtype)
     S, Hq, Hkv, D, bs = len(lens), cfg.num_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
     P = partition or 512
@@ -113,8 +117,8 @@ def decode_kernel_bytes(cfg, lens, partition):
     single = nparts == 1
     b = kv_bytes(cfg, lens)
     b += S * Hq * D * e                                   # q
-    b += int(single.sum()) * Hq * D * e                   # final rows
-    b += int(nparts[~single].sum()) * Hq * (D + 2) * 4    # partials
+    b += (S * Hq * D * e if fused else int(single.sum()) * Hq * D * e)   # final rows
+    b += (2 if fused else 1) * int(nparts[~single].sum()) * Hq * (D + 2) * 4   # partials (+ read back when fused)
     b += int(np.sum(-(-lens // bs))) * Hkv * 4            # block-table entries
     return int(b)
 
@@ -205,16 +209,20 @@ def _single_thread():
         return contextlib.nullcontext()
 
 
-def cpu_baseline(cfg, seed, lens, unit_scale):
-    """The oracle, as it stands, on every 4th sequence of the workload."""
+def cpu_baseline(cfg, seed, lens, unit_scale, min_seconds=10.0, max_rounds=200):
+    """The oracle, as it stands, on every 4th sequence of the workload, repeated
+    until at least ``min_seconds`` of CPU work have been timed."""
     seqs = list(range(0, len(lens), 4)) or [0]
     items = _oracle_sample(cfg, seed, seqs, lens)
+    secs, rounds = 0.0, 0
     with _single_thread():
-        secs = _time_oracle(cfg, items)
-    b = kv_bytes(cfg, lens[seqs])
+        while secs < min_seconds and rounds < max_rounds:
+            secs += _time_oracle(cfg, items)
+            rounds += 1
+    b = kv_bytes(cfg, lens[seqs]) * rounds
     return {"value": b / secs / unit_scale, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"{len(seqs)} of {len(lens)} sequences (every 4th), all {cfg.num_heads} query heads, "
-                      f"float64 numpy, 1 BLAS thread, {secs:.2f} s"}
+                      f"{rounds} rounds, float64 numpy, 1 BLAS thread, {secs:.1f} s"}
 
 
 def run_reference(args):
@@ -272,6 +280,7 @@ def run_native(args):
     import paged_kv_cache_381_b200 as pa
     from paged_kv_cache_381_b200.batch import PagedBatch
     pa.set_decode_math(pa.MATH_AUTO if args.math == "auto" else pa.MATH_SIMT)
+    pa.set_split_merge(pa.MERGE_KERNEL if args.merge == "kernel" else pa.MERGE_FUSED)
 
     cfg = wl.CONFIGS[args.workload]
     seed = args.seed + rank                       # independent replica per rank
@@ -374,7 +383,7 @@ def run_native(args):
                "tokens_per_s": world * len(lens) / (ems * 1e-3)}
 
     peak, peak_kind = measured_peaks()
-    dec_bytes = decode_kernel_bytes(cfg, lens, P)
+    dec_bytes = decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused")
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     traffic = recorded_traffic(args.workload)
     value = world * step_kv / (ms * 1e-3) / 1e9
@@ -384,7 +393,7 @@ def run_native(args):
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
         "config": {"workload": WORKLOAD_NAMES[args.workload], "num_seqs": len(lens),
                    "context_tokens": int(lens.sum()), "kv_bytes_per_step": step_kv,
-                   "partition_size": P or 512, "decode_math": args.math, "l2": "flushed between steps (256 MiB write, outside step events)",
+                   "partition_size": P or 512, "decode_math": args.math, "split_merge": args.merge, "l2": "flushed between steps (256 MiB write, outside step events)",
                    "parallelism": "replicas" if world > 1 else "single"},
         "pct_of_hbm_peak": value / world / peak,
         "tokens_per_s": world * len(lens) / (ms * 1e-3),

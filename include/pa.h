@@ -135,7 +135,8 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim,
  * log-sum-exp reduction; the workspace (device, >= pa_decode_workspace_size
  * bytes, 256-byte aligned, contents undefined on entry) holds the partials.
  * max_context_len must bound every context_lens[s]; larger values are clamped
- * and flagged (PA_DEVERR_CONTEXT_LEN).
+ * and flagged (PA_DEVERR_CONTEXT_LEN).  At most 4096 partitions per sequence
+ * (PA_ERR_UNSUPPORTED beyond).
  */
 pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, const int32_t* context_lens, float scale,
@@ -235,6 +236,19 @@ pa_status pa_step(const pa_step_host* host, const pa_step_device* dev, void* k_c
 typedef enum { PA_MATH_AUTO = 0, PA_MATH_SIMT = 1, PA_MATH_TENSOR = 2 } pa_decode_math;
 pa_status pa_set_decode_math(int mode);
 int pa_get_decode_math(void);
+
+/*
+ * How pa_decode merges the partitions of split sequences (process-wide):
+ *   PA_MERGE_KERNEL  a separate log-sum-exp reduce kernel runs after decode
+ *                    -- the default (measured faster on B200);
+ *   PA_MERGE_FUSED   the decode kernel's CTA that finishes a sequence's last
+ *                    partition merges them (no extra launch).
+ * Both compute M = max_i m_i, o = sum_i 2^(m_i-M) o_i / sum_i 2^(m_i-M) l_i in
+ * partition order; bits may differ in the last place between the two.
+ */
+typedef enum { PA_MERGE_FUSED = 0, PA_MERGE_KERNEL = 1 } pa_split_merge;
+pa_status pa_set_split_merge(int mode);
+int pa_get_split_merge(void);
 
 /* Reads and clears the device error word (synchronizes `stream`).  Returns
  * PA_ERR_DEVICE when any bit was set, PA_OK otherwise. */

@@ -212,6 +212,19 @@ def get_decode_math():
     return int(lib().pa_get_decode_math())
 
 
+MERGE_FUSED, MERGE_KERNEL = 0, 1
+
+
+def set_split_merge(mode):
+    """Merge split partitions with the separate log-sum-exp reduce kernel
+    (default) or inside the decode kernel."""
+    _check(lib().pa_set_split_merge(int(mode)), "pa_set_split_merge")
+
+
+def get_split_merge():
+    return int(lib().pa_get_split_merge())
+
+
 def launch_count():
     return int(lib().pa_launch_count())
 

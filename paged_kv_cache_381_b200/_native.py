@@ -56,6 +56,8 @@ SIGNATURES = {
     "pa_launch_count": (c_int64, []),
     "pa_set_decode_math": (c_int, [c_int]),
     "pa_get_decode_math": (c_int, []),
+    "pa_set_split_merge": (c_int, [c_int]),
+    "pa_get_split_merge": (c_int, []),
     "pa_profile_begin": (c_int, []),
     "pa_profile_end": (c_int, [P(c_double), P(c_int64)]),
     "pa_bm_create": (c_int, [c_int, c_int, c_void_p, P(c_void_p)]),

@@ -16,31 +16,30 @@
 
 namespace pa_dev {
 
-// One warp per token; 16-byte vectors.  row_vecs = 16-byte vectors per token row.
+// One thread per 16-byte vector of a token row (K and V), grid-stride; many
+// independent loads in flight keep this short kernel from being latency-bound.
+// row_vecs = 16-byte vectors per token row.
 __global__ void __launch_bounds__(256) cache_write_kernel(const uint4* __restrict__ k,
                                                           const uint4* __restrict__ v,
                                                           uint4* __restrict__ k_cache,
                                                           uint4* __restrict__ v_cache,
                                                           const int64_t* __restrict__ slot_mapping,
                                                           int num_tokens, int row_vecs, int64_t num_slots) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (warp >= num_tokens) return;
-    const int64_t slot = slot_mapping[warp];
-    if (slot < 0) return;                       // padding token
-    if (slot >= num_slots) {
-        if (lane == 0) flag_error(PA_DEVERR_SLOT);
-        return;
-    }
-    const uint4* ks = k + (int64_t)warp * row_vecs;
-    const uint4* vs = v + (int64_t)warp * row_vecs;
-    uint4* kd = k_cache + slot * row_vecs;
-    uint4* vd = v_cache + slot * row_vecs;
-    for (int i = lane; i < row_vecs; i += 32) {
-        uint4 a = __ldg(ks + i);
-        uint4 b = __ldg(vs + i);
-        kd[i] = a;
-        vd[i] = b;
+    const int64_t total = (int64_t)num_tokens * row_vecs;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / row_vecs;
+        const int64_t j = i - t * row_vecs;
+        const int64_t slot = __ldg(slot_mapping + t);
+        if (slot < 0) continue;                 // padding token
+        if (slot >= num_slots) {
+            if (j == 0) flag_error(PA_DEVERR_SLOT);
+            continue;
+        }
+        const uint4 a = __ldg(k + i);
+        const uint4 b = __ldg(v + i);
+        k_cache[slot * row_vecs + j] = a;
+        v_cache[slot * row_vecs + j] = b;
     }
 }
 

@@ -69,6 +69,8 @@ struct DecodeArgs {
     float* part_m;             // [num_seqs * num_heads, max_partitions] (log2 units)
     float* part_l;             // [num_seqs * num_heads, max_partitions]
     float* part_o;             // [num_seqs * num_heads, max_partitions, head_dim]
+    int* merge_count;          // split mode, fused merge: finished partitions per (seq, kv head, chunk);
+                               // nullptr: partitions are merged by reduce_kernel instead
 };
 
 struct WorkItem {
@@ -150,6 +152,15 @@ __device__ __forceinline__ float reduce_row_dots(float (&v)[GC], int lane) {
     return v[0];
 }
 
+// Ring depth (stages of 32 token rows) and the CTAs per SM the launch bounds
+// aim for; build-time tuning knobs.
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 8
+#endif
+#ifndef PA_DECODE_MIN_CTAS
+#define PA_DECODE_MIN_CTAS 2
+#endif
+
 template <typename T, int D, int GC, bool TENSOR>
 struct DecodeCfg {
     using Tr = ElemTraits<T>;
@@ -162,7 +173,7 @@ struct DecodeCfg {
     static constexpr int BOX_ELEMS = 128 / ELT;     // head_dim elements per slice
     static constexpr int STAGE_ROWS = 32;
     static constexpr int STAGE_BYTES = STAGE_ROWS * ROW_BYTES;
-    static constexpr int NSTAGES = 8;
+    static constexpr int NSTAGES = PA_DECODE_STAGES;
     static constexpr int NCW = 4;                   // consumer warps
     static constexpr int THREADS = (NCW + 1) * 32;
     static constexpr int MAX_PARTITION = 1024;
@@ -181,6 +192,13 @@ struct DecodeCfg {
     static_assert(TENSOR ? (GC == 8 && ELT == 2) : (GC <= LPT), "unsupported query chunk");
     static_assert(LPT >= 1 && LPT <= 32 && (32 % LPT) == 0, "row must span a divisor of the warp");
     static_assert(ROW_BYTES % 128 == 0 && STAGE_BYTES % 1024 == 0, "swizzled boxes need 1024-byte alignment");
+    // Consumer warp w takes the stages st = w, w + NCW, ... of a phase, and a
+    // ring slot is reused every NSTAGES stages.  Only when NSTAGES is a multiple
+    // of NCW does one warp own every use of a slot within a phase; otherwise a
+    // warp could test a slot's full barrier for its next use while the previous
+    // use (another warp's) is still in flight, and the parity test would answer
+    // "complete" for the wrong phase.
+    static_assert(NSTAGES % NCW == 0, "ring depth must be a multiple of the consumer warps");
     // + 1024: the dynamic shared-memory base is rounded up to 1024 bytes in the kernel
     static size_t smem_bytes(int partition) {
         return 1024 + (size_t)OFF_LOGITS + (size_t)partition * LSTRIDE * 4;
@@ -197,7 +215,7 @@ struct DecodeCfg {
 // B reg0 = (k = 2*tig, 2*tig+1; n = gid), reg1 = same k + 8, C = (gid | gid+8, 2*tig | 2*tig+1),
 // where gid = lane / 4 and tig = lane % 4.
 template <typename T, int D, int GC, bool TENSOR>
-__global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2)
+__global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, PA_DECODE_MIN_CTAS)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
     using C = DecodeCfg<T, D, GC, TENSOR>;
@@ -605,6 +623,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2)
 
         // ---- epilogue: warps merged in a fixed order; final row or partition partials
         const bool single = (w.np == 1);
+        volatile int* last_flag = abort_flag + 1;
         for (int e = ctid; e < gq * D; e += NCT) {
             const int g = e / D;
             const int d = e - g * D;
@@ -623,56 +642,176 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, 2)
                 }
             }
         }
+        if (!single && a.merge_count != nullptr) {
+            // The CTA that finishes the last partition of this (sequence, kv head,
+            // chunk) merges all of them: partials are published with a fence
+            // before the counter increment; the last arriver fences and reads
+            // them from L2.  Nothing waits; the merge order is fixed (partition 0
+            // first), so the bits do not depend on which CTA ends up merging.
+            __threadfence();
+            named_barrier(1, NCT);
+            if (ctid == 0) {
+                const int64_t cidx = ((int64_t)w.s * a.num_kv_heads + w.h) * a.n_gchunks + w.gc;
+                const int prev = atomicAdd(a.merge_count + cidx, 1);
+                *last_flag = (prev == w.np - 1) ? 1 : 0;
+            }
+            named_barrier(1, NCT);
+            if (*last_flag) {
+                __threadfence();
+                for (int g = warp; g < gq; g += C::NCW) {       // one warp per query, lanes over partitions
+                    const float* pm = a.part_m + (row0 + g) * a.max_partitions;
+                    const float* pl = a.part_l + (row0 + g) * a.max_partitions;
+                    float M = -INFINITY;
+                    for (int i = lane; i < w.np; i += 32) M = fmaxf(M, __ldcg(pm + i));
+                    M = warp_max(M);
+                    float L = 0.f;
+                    for (int i = lane; i < w.np; i += 32) L += exp2f(__ldcg(pm + i) - M) * __ldcg(pl + i);
+                    L = warp_sum(L);
+                    if (lane == 0) {
+                        stat_m[g] = M;
+                        stat_l[g] = L;
+                    }
+                }
+                named_barrier(1, NCT);
+                // four consecutive head-dim elements per thread and step
+                for (int e = ctid * 4; e < gq * D; e += NCT * 4) {
+                    const int g = e / D;
+                    const int d = e - g * D;
+                    const int64_t base = (row0 + g) * a.max_partitions;
+                    const float Mg = stat_m[g];
+                    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+                    int i = 0;
+                    for (; i + 8 <= w.np; i += 8) {
+                        float4 x[8];
+                        float wt[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            x[j] = __ldcg(reinterpret_cast<const float4*>(a.part_o + (base + i + j) * D + d));
+                            wt[j] = exp2f(__ldcg(a.part_m + base + i + j) - Mg);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            o.x = fmaf(wt[j], x[j].x, o.x);
+                            o.y = fmaf(wt[j], x[j].y, o.y);
+                            o.z = fmaf(wt[j], x[j].z, o.z);
+                            o.w = fmaf(wt[j], x[j].w, o.w);
+                        }
+                    }
+                    for (; i < w.np; ++i) {
+                        const float4 x = __ldcg(reinterpret_cast<const float4*>(a.part_o + (base + i) * D + d));
+                        const float wt = exp2f(__ldcg(a.part_m + base + i) - Mg);
+                        o.x = fmaf(wt, x.x, o.x);
+                        o.y = fmaf(wt, x.y, o.y);
+                        o.z = fmaf(wt, x.z, o.z);
+                        o.w = fmaf(wt, x.w, o.w);
+                    }
+                    const float Lg = stat_l[g];
+                    T* dst = outg + (row0 + g) * D + d;
+                    dst[0] = Tr::from_float(o.x / Lg);
+                    dst[1] = Tr::from_float(o.y / Lg);
+                    dst[2] = Tr::from_float(o.z / Lg);
+                    dst[3] = Tr::from_float(o.w / Lg);
+                }
+            }
+        }
         named_barrier(1, NCT);
     }
 }
 
 // Orders (sequence, partition) pairs longest-first: all pairs of the highest
-// partition index first, then the next, so the long sequences' full partitions
-// start early and the short tails fill in at the end.  One CTA.
-__global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, int2* plan, int* count) {
-    __shared__ int warp_incl[32];
-    __shared__ int s_base;
+// partition index come first, then the next level, so the full partitions of
+// long sequences start early and the short tails fill in at the end.  The
+// order inside a level does not matter (results never depend on which CTA
+// takes an item).  One CTA: a histogram of partition counts, a suffix scan that
+// places the levels, then one atomic slot reservation per pair.  It also clears
+// the fused-merge counters for this call.
+// Dynamic shared memory: 2 * (max_partitions + 1) ints.
+__global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, int2* plan, int* count, int* merge_count,
+                                                    int num_counters) {
+    extern __shared__ int plan_smem[];
+    const int L = a.max_partitions;
+    int* hist = plan_smem;                       // hist[k]: sequences with k partitions, k = 1 .. L
+    int* cur = plan_smem + L + 1;                // first plan slot of level p, then its cursor
+    __shared__ int warp_tot[32];
+    __shared__ int carry;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int nw = blockDim.x >> 5;
-    if (tid == 0) s_base = 0;
+    for (int i = tid; i <= L; i += blockDim.x) hist[i] = 0;
+    for (int i = tid; i < num_counters; i += blockDim.x) merge_count[i] = 0;
+    if (tid == 0) carry = 0;
     __syncthreads();
-    for (int p = a.max_partitions - 1; p >= 0; --p) {
-        for (int s0 = 0; s0 < a.num_seqs; s0 += blockDim.x) {
-            const int s = s0 + tid;
-            int flag = 0;
-            if (s < a.num_seqs) {
-                const int ctx = clamp_context(a, s, p == a.max_partitions - 1);
-                flag = partitions_of(a, ctx) > p ? 1 : 0;
-            }
-            int x = flag;
+    for (int s = tid; s < a.num_seqs; s += blockDim.x)
+        atomicAdd(&hist[partitions_of(a, clamp_context(a, s, true))], 1);
+    __syncthreads();
+    // level p holds the sequences with more than p partitions: size(p) = sum_{k > p} hist[k];
+    // cur[p] = sum of size(p') over p' > p.  Scan k = L .. 1 (a running suffix of hist)
+    // and levels p = L-1 .. 0 in the same descending pass.
+    for (int c0 = 0; c0 < L; c0 += blockDim.x) {
+        const int p = L - 1 - (c0 + tid);
+        // size(p) = number of sequences with partitions > p, from a suffix scan of hist
+        int x = p >= 0 ? hist[p + 1] : 0;
+        int incl = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int t = lane < nw ? warp_tot[lane] : 0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
+                const int y = __shfl_up_sync(0xffffffffu, t, o);
+                if (lane >= o) t += y;
             }
-            if (lane == 31) warp_incl[warp] = x;
-            __syncthreads();
-            if (warp == 0) {
-                int t = lane < nw ? warp_incl[lane] : 0;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int y = __shfl_up_sync(0xffffffffu, t, o);
-                    if (lane >= o) t += y;
-                }
-                if (lane < nw) warp_incl[lane] = t;
-            }
-            __syncthreads();
-            const int base = s_base + (warp == 0 ? 0 : warp_incl[warp - 1]);
-            if (flag) plan[base + x - 1] = make_int2(s, p);
-            __syncthreads();
-            if (tid == 0) s_base += warp_incl[nw - 1];
-            __syncthreads();
+            if (lane < nw) warp_tot[lane] = t;
         }
+        __syncthreads();
+        // running suffix count of sequences with > p partitions
+        const int size_p = carry + (warp ? warp_tot[warp - 1] : 0) + incl;
+        if (p >= 0) cur[p] = size_p;              // sizes first; turned into offsets below
+        __syncthreads();
+        if (tid == 0) carry += warp_tot[nw - 1];
+        __syncthreads();
     }
-    if (tid == 0) *count = s_base;
+    // offsets: cur[p] = sum_{p' > p} size(p'), a second descending scan over the sizes
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int c0 = 0; c0 < L; c0 += blockDim.x) {
+        const int p = L - 1 - (c0 + tid);
+        const int x = p >= 0 ? cur[p] : 0;
+        int incl = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int t = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, t, o);
+                if (lane >= o) t += y;
+            }
+            if (lane < nw) warp_tot[lane] = t;
+        }
+        __syncthreads();
+        if (p >= 0) cur[p] = carry + (warp ? warp_tot[warp - 1] : 0) + incl - x;
+        __syncthreads();
+        if (tid == 0) carry += warp_tot[nw - 1];
+        __syncthreads();
+    }
+    for (int s = tid; s < a.num_seqs; s += blockDim.x) {
+        const int np = partitions_of(a, clamp_context(a, s, false));
+        for (int p = 0; p < np; ++p) plan[atomicAdd(&cur[p], 1)] = make_int2(s, p);
+    }
+    __syncthreads();
+    if (tid == 0) *count = carry;
 }
 
 // Log-sum-exp merge of a sequence's partitions (base-2 units): with

@@ -99,7 +99,7 @@ pa_status check_cache_desc(const pa_cache_desc* c) {
 
 // ------------------------------------------------------------ workspace
 struct WsLayout {
-    size_t plan, count, m, l, o, total;
+    size_t plan, count, counters, m, l, o, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -111,6 +111,8 @@ WsLayout ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t maxP) {
     off = align256(off + (size_t)(S * maxP) * sizeof(int2));
     w.count = off;
     off = align256(off + sizeof(int));
+    w.counters = off;                                   // fused-merge counters, <= S * Hq of them
+    off = align256(off + (size_t)(S * Hq) * sizeof(int));
     w.m = off;
     off = align256(off + (size_t)(S * Hq * maxP) * sizeof(float));
     w.l = off;
@@ -129,6 +131,8 @@ int64_t partitions_for(int64_t ctx, int64_t P) { return ctx <= P ? 1 : (ctx + P 
 
 // ------------------------------------------------------------ decode launch
 std::atomic<int> g_decode_math{PA_MATH_AUTO};
+std::atomic<int> g_split_merge{PA_MERGE_KERNEL};
+constexpr int kMaxPartitions = 4096;    // plan kernel: 2 * kMaxPartitions ints of shared memory
 
 // ---------------------------------------------------------------- TMA maps
 // cuTensorMapEncodeTiled is reached through the runtime's driver entry point,
@@ -271,6 +275,14 @@ pa_status pa_set_decode_math(int mode) {
 
 int pa_get_decode_math(void) { return g_decode_math.load(); }
 
+pa_status pa_set_split_merge(int mode) {
+    if (mode != PA_MERGE_FUSED && mode != PA_MERGE_KERNEL) return PA_ERR_INVALID_ARG;
+    g_split_merge.store(mode);
+    return PA_OK;
+}
+
+int pa_get_split_merge(void) { return g_split_merge.load(); }
+
 pa_status pa_profile_begin(void) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     for (auto& r : g_prof_records) {
@@ -316,8 +328,8 @@ pa_status pa_cache_write(const void* k, const void* v, void* k_cache, void* v_ca
     const int64_t row_bytes = (int64_t)cache->num_kv_heads * cache->head_dim * elem_bytes(cache->dtype);
     const int row_vecs = (int)(row_bytes / 16);
     const int64_t num_slots = (int64_t)cache->num_blocks * cache->block_size;
-    const int64_t threads = (int64_t)num_tokens * 32;
-    const unsigned grid = (unsigned)((threads + 255) / 256);
+    const int64_t threads = (int64_t)num_tokens * row_vecs;
+    const unsigned grid = (unsigned)std::min<int64_t>((threads + 255) / 256, 65535);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     LaunchScope scope(PA_KERNEL_CACHE_WRITE, s);
     pa_dev::cache_write_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
@@ -370,6 +382,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     const int64_t cap = std::min<int64_t>(max_context_len, table_cap);
     if (cap > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
     const int64_t maxP = partitions_for(cap, P);
+    if (maxP > kMaxPartitions) return PA_ERR_UNSUPPORTED;
     const int group = num_heads / num_kv_heads;
     const int math = g_decode_math.load(std::memory_order_relaxed);
     const bool tensor = dtype != PA_F32 && math != PA_MATH_SIMT;
@@ -408,11 +421,16 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
         a.part_m = reinterpret_cast<float*>(ws + L.m);
         a.part_l = reinterpret_cast<float*>(ws + L.l);
         a.part_o = reinterpret_cast<float*>(ws + L.o);
+        const bool fused = g_split_merge.load(std::memory_order_relaxed) == PA_MERGE_FUSED;
+        int* counters = reinterpret_cast<int*>(ws + L.counters);
+        a.merge_count = fused ? counters : nullptr;
         {
             LaunchScope scope(PA_KERNEL_PLAN, s);
             const int threads = std::min(1024, std::max(32, (num_seqs + 31) / 32 * 32));
-            pa_dev::plan_kernel<<<1, threads, 0, s>>>(a, reinterpret_cast<int2*>(ws + L.plan),
-                                                      reinterpret_cast<int*>(ws + L.count));
+            const int num_counters = fused ? num_seqs * num_kv_heads * n_gchunks : 0;
+            pa_dev::plan_kernel<<<1, threads, 2 * (maxP + 1) * sizeof(int), s>>>(
+                a, reinterpret_cast<int2*>(ws + L.plan), reinterpret_cast<int*>(ws + L.count), counters,
+                num_counters);
             if (launch_status() != PA_OK) return PA_ERR_CUDA;
         }
     }
@@ -427,7 +445,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
         case PA_F16: st = dispatch_head_dim<__half>(a, tk, tv, head_dim, gc, tensor, pair_upper, s); break;
         default: st = dispatch_head_dim<__nv_bfloat16>(a, tk, tv, head_dim, gc, tensor, pair_upper, s); break;
     }
-    if (st != PA_OK || maxP <= 1) return st;
+    if (st != PA_OK || maxP <= 1 || a.merge_count != nullptr) return st;
     switch (dtype) {
         case PA_F32: return launch_reduce<float>(a, head_dim, s);
         case PA_F16: return launch_reduce<__half>(a, head_dim, s);

@@ -39,6 +39,14 @@ def math_path(request):
     pa.set_decode_math(pa.MATH_AUTO)
 
 
+@pytest.fixture(params=["fused", "kernel"])
+def merge_mode(request):
+    """Merge split partitions in the decode kernel (fused) or in the reduce kernel."""
+    pa.set_split_merge(pa.MERGE_FUSED if request.param == "fused" else pa.MERGE_KERNEL)
+    yield request.param
+    pa.set_split_merge(pa.MERGE_KERNEL)
+
+
 def _no_device_error():
     assert pa.pa_get_device_error() == 0
 
@@ -105,7 +113,7 @@ def test_uneven_and_wide_groups(G, math_path):
 
 
 @pytest.mark.parametrize("P", [32, 64, 96, 512, 1024])
-def test_partition_sizes(P, math_path):
+def test_partition_sizes(P, math_path, merge_mode):
     cfg = _grid_cfg("f16", 128, 16, 4)
     inp = wl.make_decode_inputs(cfg, 5, context_lens=(1, 95, 96, 97, 1023, 1024, 1025, 2500))
     b, got = _run(inp, partition_size=P)
@@ -113,7 +121,7 @@ def test_partition_sizes(P, math_path):
     _no_device_error()
 
 
-def test_split_vs_single_pass(math_path):
+def test_split_vs_single_pass(math_path, merge_mode):
     cfg = _grid_cfg("bf16", 128, 16, 8)
     inp = wl.make_decode_inputs(cfg, 6, context_lens=(1000, 17, 640, 1024))
     ref = oracle_outputs(inp)
@@ -226,7 +234,7 @@ def test_copy_blocks_bit_exact():
     _no_device_error()
 
 
-def test_long_context_with_outlier_keys(math_path):
+def test_long_context_with_outlier_keys(math_path, merge_mode):
     """Two 8192-token sequences, 1% of K rows scaled by 8, 512-token partitions."""
     cfg = wl.DecodeConfig("longsmall", "bf16", 2, 64, 8, 128, 16, "const", len_lo=8192, len_hi=8192,
                           partition_size=512, outlier_frac=0.01)
@@ -313,7 +321,7 @@ def test_pa_step_from_host_buffers_matches_device_path():
     _no_device_error()
 
 
-def test_launch_count_and_profile():
+def test_launch_count_and_profile(merge_mode):
     cfg = _grid_cfg("bf16", 128, 16, 8)
     inp = wl.make_decode_inputs(cfg, 14, context_lens=(2000, 30))
     b = DeviceBatch(inp)
@@ -322,9 +330,12 @@ def test_launch_count_and_profile():
     b.step_write()
     b.decode()
     prof = pa.profile_end()
-    assert pa.launch_count() - n0 == 4           # cache write, plan, decode, reduce
+    fused = merge_mode == "fused"
+    # cache write, plan, decode (+ reduce when partitions are merged by their own kernel)
+    assert pa.launch_count() - n0 == (3 if fused else 4)
     assert prof["decode"][1] == 1 and prof["decode"][0] > 0
-    assert prof["plan"][1] == 1 and prof["reduce"][1] == 1 and prof["cache_write"][1] == 1
+    assert prof["plan"][1] == 1 and prof["cache_write"][1] == 1
+    assert prof["reduce"][1] == (0 if fused else 1)
 
 
 # -- full-size workloads, sampled rows, in the bench's launch configuration -------
@@ -339,7 +350,7 @@ def _sample_rows(lens, Hq, k, seed):
 
 
 @pytest.mark.parametrize("name", ["7b", "70b", "long"])
-def test_full_size_sampled(name, math_path):
+def test_full_size_sampled(name, math_path, merge_mode):
     cfg = wl.CONFIGS[name]
     d = wl.draw_device(cfg, 0)
     batch = PagedBatch(d.k_hist, d.v_hist, d.offsets, d.context_lens, d.num_blocks, cfg.block_size,
