@@ -57,7 +57,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--math", default="auto", choices=["auto", "simt"],
-                   help="decode arithmetic: tensor cores for fp16/bf16 (auto) or CUDA cores (simt)")
+                   help="decode arithmetic: tensor cores for fp16/bf16 (auto), CUDA cores (simt)")
     p.add_argument("--merge", default="kernel", choices=["kernel", "fused"],
                    help="merge split partitions with the reduce kernel or inside the decode kernel")
     p.add_argument("--num-seqs", type=int, default=0,

@@ -152,13 +152,82 @@ __device__ __forceinline__ float reduce_row_dots(float (&v)[GC], int lane) {
     return v[0];
 }
 
+// Merge the partitions of one (sequence, kv head, query chunk) in partition
+// order: M = max_i m_i, out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
+// Called by the CTA that finished the last of them, after a fence; reads the
+// partials from L2.  Uses `stat_m` / `stat_l` (>= gq floats of shared memory)
+// and named barrier 1 over the ncw consumer warps.
+template <typename T, int D>
+__device__ __forceinline__ void merge_partitions(const DecodeArgs& a, int64_t row0, int gq, int np, float* stat_m,
+                                                 float* stat_l, int warp, int lane, int ctid, int ncw) {
+    using Tr = ElemTraits<T>;
+    T* outg = static_cast<T*>(a.out);
+    for (int g = warp; g < gq; g += ncw) {       // one warp per query, lanes over partitions
+        const float* pm = a.part_m + (row0 + g) * a.max_partitions;
+        const float* pl = a.part_l + (row0 + g) * a.max_partitions;
+        float M = -INFINITY;
+        for (int i = lane; i < np; i += 32) M = fmaxf(M, __ldcg(pm + i));
+        M = warp_max(M);
+        float L = 0.f;
+        for (int i = lane; i < np; i += 32) L += exp2f(__ldcg(pm + i) - M) * __ldcg(pl + i);
+        L = warp_sum(L);
+        if (lane == 0) {
+            stat_m[g] = M;
+            stat_l[g] = L;
+        }
+    }
+    named_barrier(1, ncw * 32);
+    // four consecutive head-dim elements per thread and step
+    for (int e = ctid * 4; e < gq * D; e += ncw * 32 * 4) {
+        const int g = e / D;
+        const int d = e - g * D;
+        const int64_t base = (row0 + g) * a.max_partitions;
+        const float Mg = stat_m[g];
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        int i = 0;
+        for (; i + 8 <= np; i += 8) {
+            float4 x[8];
+            float wt[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                x[j] = __ldcg(reinterpret_cast<const float4*>(a.part_o + (base + i + j) * D + d));
+                wt[j] = exp2f(__ldcg(a.part_m + base + i + j) - Mg);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                o.x = fmaf(wt[j], x[j].x, o.x);
+                o.y = fmaf(wt[j], x[j].y, o.y);
+                o.z = fmaf(wt[j], x[j].z, o.z);
+                o.w = fmaf(wt[j], x[j].w, o.w);
+            }
+        }
+        for (; i < np; ++i) {
+            const float4 xv = __ldcg(reinterpret_cast<const float4*>(a.part_o + (base + i) * D + d));
+            const float wt = exp2f(__ldcg(a.part_m + base + i) - Mg);
+            o.x = fmaf(wt, xv.x, o.x);
+            o.y = fmaf(wt, xv.y, o.y);
+            o.z = fmaf(wt, xv.z, o.z);
+            o.w = fmaf(wt, xv.w, o.w);
+        }
+        const float Lg = stat_l[g];
+        T* dst = outg + (row0 + g) * D + d;
+        dst[0] = Tr::from_float(o.x / Lg);
+        dst[1] = Tr::from_float(o.y / Lg);
+        dst[2] = Tr::from_float(o.z / Lg);
+        dst[3] = Tr::from_float(o.w / Lg);
+    }
+}
+
 // Ring depth (stages of 32 token rows) and the CTAs per SM the launch bounds
-// aim for; build-time tuning knobs.
+// aim for (tensor-core path; the CUDA-core path holds more registers and aims
+// for 2); build-time tuning knobs.  Measured on B200 (70B-shaped batch): 4
+// stages at 4 CTAs per SM beat 8 stages at 2 (more independent items per SM
+// hide the per-item phase barriers of short sequences).
 #ifndef PA_DECODE_STAGES
-#define PA_DECODE_STAGES 8
+#define PA_DECODE_STAGES 4
 #endif
 #ifndef PA_DECODE_MIN_CTAS
-#define PA_DECODE_MIN_CTAS 2
+#define PA_DECODE_MIN_CTAS 4
 #endif
 
 template <typename T, int D, int GC, bool TENSOR>
@@ -186,9 +255,12 @@ struct DecodeCfg {
     static constexpr int OFF_TABLE = OFF_EMPTY + NSTAGES * 8;
     static constexpr int OFF_STATS = OFF_TABLE + MAX_TABLE * 4;     // wmax, wsum [NCW][GC], m, l [GC], abort
     static constexpr int STATS_FLOATS = 2 * NCW * GC + 2 * GC + 4;
-    static constexpr int OFF_RED = ((OFF_STATS + STATS_FLOATS * 4) + 127) / 128 * 128;
+    // The scores (phases 1-3) and the warps' output partials (epilogue) share
+    // one region: a barrier separates the last score read from the first
+    // partial write.
+    static constexpr int OFF_LOGITS = ((OFF_STATS + STATS_FLOATS * 4) + 127) / 128 * 128;
+    static constexpr int OFF_RED = OFF_LOGITS;
     static constexpr int RED_BYTES = NCW * GC * D * 4;
-    static constexpr int OFF_LOGITS = OFF_RED + RED_BYTES;
     static_assert(TENSOR ? (GC == 8 && ELT == 2) : (GC <= LPT), "unsupported query chunk");
     static_assert(LPT >= 1 && LPT <= 32 && (32 % LPT) == 0, "row must span a divisor of the warp");
     static_assert(ROW_BYTES % 128 == 0 && STAGE_BYTES % 1024 == 0, "swizzled boxes need 1024-byte alignment");
@@ -201,7 +273,8 @@ struct DecodeCfg {
     static_assert(NSTAGES % NCW == 0, "ring depth must be a multiple of the consumer warps");
     // + 1024: the dynamic shared-memory base is rounded up to 1024 bytes in the kernel
     static size_t smem_bytes(int partition) {
-        return 1024 + (size_t)OFF_LOGITS + (size_t)partition * LSTRIDE * 4;
+        const size_t scores = (size_t)partition * LSTRIDE * 4;
+        return 1024 + (size_t)OFF_LOGITS + (scores > (size_t)RED_BYTES ? scores : (size_t)RED_BYTES);
     }
 };
 
@@ -215,7 +288,7 @@ struct DecodeCfg {
 // B reg0 = (k = 2*tig, 2*tig+1; n = gid), reg1 = same k + 8, C = (gid | gid+8, 2*tig | 2*tig+1),
 // where gid = lane / 4 and tig = lane % 4.
 template <typename T, int D, int GC, bool TENSOR>
-__global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, PA_DECODE_MIN_CTAS)
+__global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ? PA_DECODE_MIN_CTAS : 2)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
     using C = DecodeCfg<T, D, GC, TENSOR>;
@@ -481,6 +554,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, PA_DECOD
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
             if (tig == 0) wsum[warp * GC + gid] = lsum;
+            named_barrier(1, NCT);            // every warp is done with the scores: reuse them as `red`
             // O^T fragment: (d = 16*dm + gid [+8], query 2*tig [+1])
             float* rw = red + warp * GC * D;
 #pragma unroll
@@ -608,6 +682,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, PA_DECOD
                 for (int g = 0; g < GC; ++g)
 #pragma unroll
                     for (int v = 0; v < C::VEC; ++v) acc[g][v] += __shfl_xor_sync(0xffffffffu, acc[g][v], o);
+            named_barrier(1, NCT);            // every warp is done with the scores: reuse them as `red`
             if (row_in == 0) {
 #pragma unroll
                 for (int g = 0; g < GC; ++g) {
@@ -658,60 +733,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, PA_DECOD
             named_barrier(1, NCT);
             if (*last_flag) {
                 __threadfence();
-                for (int g = warp; g < gq; g += C::NCW) {       // one warp per query, lanes over partitions
-                    const float* pm = a.part_m + (row0 + g) * a.max_partitions;
-                    const float* pl = a.part_l + (row0 + g) * a.max_partitions;
-                    float M = -INFINITY;
-                    for (int i = lane; i < w.np; i += 32) M = fmaxf(M, __ldcg(pm + i));
-                    M = warp_max(M);
-                    float L = 0.f;
-                    for (int i = lane; i < w.np; i += 32) L += exp2f(__ldcg(pm + i) - M) * __ldcg(pl + i);
-                    L = warp_sum(L);
-                    if (lane == 0) {
-                        stat_m[g] = M;
-                        stat_l[g] = L;
-                    }
-                }
-                named_barrier(1, NCT);
-                // four consecutive head-dim elements per thread and step
-                for (int e = ctid * 4; e < gq * D; e += NCT * 4) {
-                    const int g = e / D;
-                    const int d = e - g * D;
-                    const int64_t base = (row0 + g) * a.max_partitions;
-                    const float Mg = stat_m[g];
-                    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-                    int i = 0;
-                    for (; i + 8 <= w.np; i += 8) {
-                        float4 x[8];
-                        float wt[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            x[j] = __ldcg(reinterpret_cast<const float4*>(a.part_o + (base + i + j) * D + d));
-                            wt[j] = exp2f(__ldcg(a.part_m + base + i + j) - Mg);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            o.x = fmaf(wt[j], x[j].x, o.x);
-                            o.y = fmaf(wt[j], x[j].y, o.y);
-                            o.z = fmaf(wt[j], x[j].z, o.z);
-                            o.w = fmaf(wt[j], x[j].w, o.w);
-                        }
-                    }
-                    for (; i < w.np; ++i) {
-                        const float4 x = __ldcg(reinterpret_cast<const float4*>(a.part_o + (base + i) * D + d));
-                        const float wt = exp2f(__ldcg(a.part_m + base + i) - Mg);
-                        o.x = fmaf(wt, x.x, o.x);
-                        o.y = fmaf(wt, x.y, o.y);
-                        o.z = fmaf(wt, x.z, o.z);
-                        o.w = fmaf(wt, x.w, o.w);
-                    }
-                    const float Lg = stat_l[g];
-                    T* dst = outg + (row0 + g) * D + d;
-                    dst[0] = Tr::from_float(o.x / Lg);
-                    dst[1] = Tr::from_float(o.y / Lg);
-                    dst[2] = Tr::from_float(o.z / Lg);
-                    dst[3] = Tr::from_float(o.w / Lg);
-                }
+                merge_partitions<T, D>(a, row0, gq, w.np, stat_m, stat_l, warp, lane, ctid, C::NCW);
             }
         }
         named_barrier(1, NCT);

@@ -155,7 +155,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // is one 128-byte slice of head_dim for one kv head and block_size rows,
 // landing with the 128-byte swizzle.
 bool encode_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, int head_dim, int num_kv_heads,
-                     int num_blocks, int block_size) {
+                     int num_blocks, int block_size, int box_rows) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t elt = dtype == PA_F32 ? 4 : 2;
@@ -165,7 +165,7 @@ bool encode_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, int hea
     cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
                           (cuuint64_t)num_blocks * (cuuint64_t)block_size};
     cuuint64_t strides[2] = {(cuuint64_t)head_dim * elt, (cuuint64_t)num_kv_heads * head_dim * elt};
-    cuuint32_t box[3] = {(cuuint32_t)(128 / elt), 1u, (cuuint32_t)block_size};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / elt), 1u, (cuuint32_t)box_rows};
     cuuint32_t estride[3] = {1u, 1u, 1u};
     CUresult r = enc(map, t, 3, const_cast<void*>(pool), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -434,9 +434,10 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
             if (launch_status() != PA_OK) return PA_ERR_CUDA;
         }
     }
+    const int box_rows = block_size;          // one TMA box = one block of one kv head, one 128-byte slice
     CUtensorMap tk, tv;
-    if (!encode_pool_map(&tk, k_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size) ||
-        !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size))
+    if (!encode_pool_map(&tk, k_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, box_rows) ||
+        !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, box_rows))
         return PA_ERR_CUDA;
     const int64_t pair_upper = (int64_t)num_seqs * maxP;
     pa_status st;
