@@ -316,7 +316,7 @@ def run_native(args):
     clocks.start()
     time.sleep(0.3)
     launches0 = pa.launch_count()
-    pa.profile_begin()
+    pa.profile_begin(["decode"])          # events around the decode kernel only
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()

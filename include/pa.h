@@ -276,6 +276,10 @@ int64_t pa_launch_count(void);
  * clears earlier records. */
 pa_status pa_profile_begin(void);
 
+/* Same, recording only the kernels whose bit (1 << pa_kernel_id) is set in
+ * kernel_mask; fewer event pairs disturb the timed stream less. */
+pa_status pa_profile_begin_mask(uint32_t kernel_mask);
+
 /* Stop recording, wait for the recorded events, and return per kernel id the
  * summed device milliseconds and launch counts (arrays of PA_KERNEL_COUNT). */
 pa_status pa_profile_end(double* total_ms, int64_t* launches);

@@ -229,8 +229,15 @@ def launch_count():
     return int(lib().pa_launch_count())
 
 
-def profile_begin():
-    _check(lib().pa_profile_begin(), "pa_profile_begin")
+def profile_begin(kernels=None):
+    """Start per-launch event timing, for all kernels or the named ones."""
+    if kernels is None:
+        _check(lib().pa_profile_begin(), "pa_profile_begin")
+    else:
+        mask = 0
+        for k in kernels:
+            mask |= 1 << KERNELS.index(k)
+        _check(lib().pa_profile_begin_mask(mask), "pa_profile_begin_mask")
 
 
 def profile_end():

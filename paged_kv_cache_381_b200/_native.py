@@ -59,6 +59,7 @@ SIGNATURES = {
     "pa_set_split_merge": (c_int, [c_int]),
     "pa_get_split_merge": (c_int, []),
     "pa_profile_begin": (c_int, []),
+    "pa_profile_begin_mask": (c_int, [c_uint32]),
     "pa_profile_end": (c_int, [P(c_double), P(c_int64)]),
     "pa_bm_create": (c_int, [c_int, c_int, c_void_p, P(c_void_p)]),
     "pa_bm_destroy": (None, [c_void_p]),

@@ -260,3 +260,12 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 }
 
 }  // namespace pa_dev
+
+namespace pa_dev {
+
+// Programmatic dependent launch: wait until the grids this one depends on have
+// completed and their memory is visible; let dependents start launching.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+}  // namespace pa_dev

@@ -320,6 +320,9 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
     }
     __syncthreads();
 
+    // launched as a programmatic dependent of the plan kernel (or of whatever
+    // precedes it): nothing written by earlier kernels is read before this
+    grid_dependency_wait();
     const int pairs = a.max_partitions == 1 ? a.num_seqs : *a.plan_count;
     const int total = pairs * a.num_kv_heads * a.n_gchunks;
     const int bs = 1 << a.log2_bs;
@@ -738,6 +741,9 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
         }
         named_barrier(1, NCT);
     }
+    // this CTA's work is done: a dependent kernel (the reduce) may start launching;
+    // it still waits for this grid's completion before reading anything
+    grid_launch_dependents();
 }
 
 // Orders (sequence, partition) pairs longest-first: all pairs of the highest
@@ -751,6 +757,8 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
 __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, int2* plan, int* count, int* merge_count,
                                                     int num_counters) {
     extern __shared__ int plan_smem[];
+    grid_dependency_wait();        // earlier kernels done before the plan and counters are rewritten
+    grid_launch_dependents();      // the decode kernel may start its prologue meanwhile
     const int L = a.max_partitions;
     int* hist = plan_smem;                       // hist[k]: sequences with k partitions, k = 1 .. L
     int* cur = plan_smem + L + 1;                // first plan slot of level p, then its cursor
@@ -843,6 +851,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, int2* pl
 template <typename T, int D>
 __global__ void __launch_bounds__(128) reduce_kernel(const DecodeArgs a) {
     using Tr = ElemTraits<T>;
+    grid_dependency_wait();                       // the decode kernel's partials must be complete
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 4 + warp;
@@ -863,17 +872,37 @@ __global__ void __launch_bounds__(128) reduce_kernel(const DecodeArgs a) {
 #pragma unroll
     for (int j = 0; j < PER; ++j) o[j] = 0.f;
     const float* po = a.part_o + row * a.max_partitions * D + lane * PER;
-    for (int i = 0; i < np; ++i) {
-        const float wgt = exp2f(pm[i] - M);
-        if constexpr (PER == 4) {
-            const float4 x = *reinterpret_cast<const float4*>(po + (int64_t)i * D);
-            o[0] = fmaf(wgt, x.x, o[0]);
-            o[1] = fmaf(wgt, x.y, o[1]);
-            o[2] = fmaf(wgt, x.z, o[2]);
-            o[3] = fmaf(wgt, x.w, o[3]);
-        } else {
+    // partitions in order; each lane computes one weight per 32 partitions and
+    // the loads of 8 partitions are issued before their FMAs
+    for (int b = 0; b < np; b += 32) {
+        const float wl = b + lane < np ? exp2f(pm[b + lane] - M) : 0.f;
+        const int cnt = min(32, np - b);
+        int i = 0;
+        for (; i + 8 <= cnt; i += 8) {
+            float x[8][PER];
 #pragma unroll
-            for (int j = 0; j < PER; ++j) o[j] = fmaf(wgt, po[(int64_t)i * D + j], o[j]);
+            for (int j = 0; j < 8; ++j) {
+                const float* src = po + (int64_t)(b + i + j) * D;
+                if constexpr (PER == 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(src);
+                    x[j][0] = v.x; x[j][1] = v.y; x[j][2] = v.z; x[j][3] = v.w;
+                } else {
+                    const float2 v = *reinterpret_cast<const float2*>(src);
+                    x[j][0] = v.x; x[j][1] = v.y;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float wgt = __shfl_sync(0xffffffffu, wl, i + j);
+#pragma unroll
+                for (int k = 0; k < PER; ++k) o[k] = fmaf(wgt, x[j][k], o[k]);
+            }
+        }
+        for (; i < cnt; ++i) {
+            const float wgt = __shfl_sync(0xffffffffu, wl, i);
+            const float* src = po + (int64_t)(b + i) * D;
+#pragma unroll
+            for (int k = 0; k < PER; ++k) o[k] = fmaf(wgt, src[k], o[k]);
         }
     }
     T* out = static_cast<T*>(a.out) + row * D + lane * PER;

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "device/cache_ops.cuh"
@@ -23,6 +24,7 @@ constexpr int kMaxDevices = 64;
 std::atomic<int64_t> g_launches{0};
 std::mutex g_prof_mu;
 bool g_prof_on = false;
+uint32_t g_prof_mask = 0;
 struct ProfRecord {
     int kernel;
     cudaEvent_t start, stop;
@@ -48,7 +50,7 @@ class LaunchScope {
     LaunchScope(int kernel, cudaStream_t stream) : kernel_(kernel), stream_(stream) {
         g_launches.fetch_add(1, std::memory_order_relaxed);
         std::lock_guard<std::mutex> lk(g_prof_mu);
-        if (g_prof_on) {
+        if (g_prof_on && (g_prof_mask & (1u << kernel))) {
             start_ = take_event();
             stop_ = take_event();
             if (start_ && stop_) cudaEventRecord(start_, stream_);
@@ -68,6 +70,26 @@ class LaunchScope {
 };
 
 pa_status launch_status() { return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+// Launch as a programmatic dependent of the previous kernel in the stream: the
+// launch may overlap that kernel's tail.  Every kernel launched this way
+// executes griddepcontrol.wait before it reads anything earlier kernels wrote
+// (and before it exits), so completion stays ordered along the stream.
+template <typename... Params, typename... Args>
+pa_status launch_dependent(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                           Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
 
 // ------------------------------------------------------------- device info
 int device_sms(int dev) {
@@ -203,8 +225,7 @@ pa_status launch_decode(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, cons
     const int64_t items_upper = pair_upper * a.num_kv_heads * a.n_gchunks;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items_upper, (int64_t)device_sms(dev) * occ));
     LaunchScope scope(PA_KERNEL_DECODE, stream);
-    kern<<<(unsigned)grid, C::THREADS, smem, stream>>>(a, tk, tv);
-    return launch_status();
+    return launch_dependent(kern, dim3((unsigned)grid), dim3(C::THREADS), smem, stream, a, tk, tv);
 }
 
 template <typename T, int D>
@@ -234,11 +255,8 @@ pa_status launch_reduce(const pa_dev::DecodeArgs& a, int D, cudaStream_t stream)
     const int64_t rows = (int64_t)a.num_seqs * a.num_heads;
     const unsigned grid = (unsigned)((rows + 3) / 4);
     LaunchScope scope(PA_KERNEL_REDUCE, stream);
-    if (D == 64)
-        pa_dev::reduce_kernel<T, 64><<<grid, 128, 0, stream>>>(a);
-    else
-        pa_dev::reduce_kernel<T, 128><<<grid, 128, 0, stream>>>(a);
-    return launch_status();
+    if (D == 64) return launch_dependent(pa_dev::reduce_kernel<T, 64>, dim3(grid), dim3(128), 0, stream, a);
+    return launch_dependent(pa_dev::reduce_kernel<T, 128>, dim3(grid), dim3(128), 0, stream, a);
 }
 
 int query_chunk(int group, bool tensor) {
@@ -283,8 +301,11 @@ pa_status pa_set_split_merge(int mode) {
 
 int pa_get_split_merge(void) { return g_split_merge.load(); }
 
-pa_status pa_profile_begin(void) {
+pa_status pa_profile_begin(void) { return pa_profile_begin_mask(0xffffffffu); }
+
+pa_status pa_profile_begin_mask(uint32_t kernel_mask) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_mask = kernel_mask;
     for (auto& r : g_prof_records) {
         g_event_pool.push_back(r.start);
         g_event_pool.push_back(r.stop);
@@ -428,10 +449,10 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
             LaunchScope scope(PA_KERNEL_PLAN, s);
             const int threads = std::min(1024, std::max(32, (num_seqs + 31) / 32 * 32));
             const int num_counters = fused ? num_seqs * num_kv_heads * n_gchunks : 0;
-            pa_dev::plan_kernel<<<1, threads, 2 * (maxP + 1) * sizeof(int), s>>>(
-                a, reinterpret_cast<int2*>(ws + L.plan), reinterpret_cast<int*>(ws + L.count), counters,
-                num_counters);
-            if (launch_status() != PA_OK) return PA_ERR_CUDA;
+            if (launch_dependent(pa_dev::plan_kernel, dim3(1), dim3(threads), 2 * (maxP + 1) * sizeof(int), s, a,
+                                 reinterpret_cast<int2*>(ws + L.plan), reinterpret_cast<int*>(ws + L.count),
+                                 counters, num_counters) != PA_OK)
+                return PA_ERR_CUDA;
         }
     }
     const int box_rows = block_size;          // one TMA box = one block of one kv head, one 128-byte slice
