@@ -338,6 +338,45 @@ pa_status pa_bm_free_list(const pa_bm* bm, int32_t* out, int cap, int* n);
 pa_status pa_bm_pack(const pa_bm* bm, const int64_t* seq_ids, int n, int width,
                      int32_t* tables, int32_t* context_lens);
 
+/* ---- prefix cache ([P3] "Prefix Caching前缀复用优化": a request whose prompt
+ * starts with cached KV references those blocks and skips their prefill) ----
+ *
+ * Off by default; with it off every call below behaves like its plain
+ * counterpart and the pool behaves exactly as described above.  With it on, a
+ * FULL block is cached under the exact key (parent block, its block_size token
+ * ids), where parent is the previous block of the same table or -1 for the
+ * first block; the key therefore names the whole token prefix up to the end of
+ * that block.  A cached block whose count reaches zero is not put on the free
+ * list: it waits on an LRU list (counted as free by pa_bm_stats) and is evicted
+ * (its key dropped, the block reused) only when the free list is empty.
+ * Partly filled blocks are never shared through the cache. */
+pa_status pa_bm_enable_prefix_cache(pa_bm* bm, int enable);
+
+/* New sequence with the prompt tokens[0..num_tokens): references the longest
+ * run of cached full blocks that starts the prompt (ref_count + 1 each) and
+ * takes fresh blocks for the rest, registering the new full ones.
+ * *cached_tokens (may be NULL) = block_size x the blocks found: the caller
+ * writes K/V only for positions >= *cached_tokens.  On PA_ERR_NO_BLOCKS nothing
+ * changes (the hit/lookup counters included). */
+pa_status pa_bm_allocate_prefix(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int num_tokens,
+                                int* cached_tokens);
+
+/* pa_bm_append_slot that also records the token id, so that the block it
+ * fills can be cached.  A sequence made by pa_bm_allocate, or that got a slot
+ * from pa_bm_append_slot, has unknown tokens: its later blocks are not cached. */
+pa_status pa_bm_append_token(pa_bm* bm, int64_t seq_id, int32_t token, int64_t* slot,
+                             int32_t* cow_src, int32_t* cow_dst);
+
+/* Cached blocks (in use or not), evictable blocks (cached, count zero),
+ * full blocks found and full blocks probed by pa_bm_allocate_prefix so far;
+ * any pointer may be NULL. */
+pa_status pa_bm_cache_stats(const pa_bm* bm, int* cached_blocks, int* evictable_blocks,
+                            int64_t* hits, int64_t* lookups);
+
+/* The evictable blocks, next victim first; *n = their number (also when cap is
+ * too small, which returns PA_ERR_INVALID_ARG). */
+pa_status pa_bm_evictable(const pa_bm* bm, int32_t* out, int cap, int* n);
+
 /* ------------------------------------------------------------------------ */
 /* Host scheduler: iteration-level (continuous) batching                     */
 /* ------------------------------------------------------------------------ */

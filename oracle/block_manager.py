@@ -166,3 +166,205 @@ class BlockManager:
         assert free.isdisjoint(held.keys()), "block both free and held"
         assert free | set(held.keys()) == set(range(self.num_blocks)), "block lost"
         assert sum(self.ref) == sum(len(t) for t in self.tables.values())
+
+
+class PrefixCachingBlockManager(BlockManager):
+    """Block manager with a prefix cache (oracle; test infrastructure only).
+
+    [P3] "大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置", section
+    "Prefix Caching前缀复用优化": when a new request begins with a prefix whose KV
+    is already cached, it references those blocks instead of computing them
+    again.  Readings adopted where the page is silent:
+
+    * Only FULL blocks are cached, each under the whole token prefix that ends
+      with it: block j of a table is named by ``tuple(tokens[:(j + 1) * bs])``.
+      Two requests hit the same block exactly when their first (j + 1) * bs
+      tokens agree, so a hit never reuses KV computed for other tokens.
+    * A block is named only if every earlier block of its table is the block
+      the cache names for that earlier prefix (the cache is a tree grown from
+      the first block), and only if its prefix and the block are not named yet.
+    * ``allocate_prefix`` walks the prompt's full blocks from the first and
+      stops at the first prefix the cache does not hold; it references the
+      blocks found and takes fresh ones for the rest.  Partly filled blocks are
+      never shared through the cache.
+    * A named block whose count reaches zero is not put on the free list; it
+      waits on an evictable list, oldest first, still counted as free.  A
+      fresh block comes from the free list while it has one, else the oldest
+      evictable block is taken and its name dropped (least recently used).
+    * ``free`` walks the table as the plain manager does; the named blocks that
+      reach zero join the evictable list last block first, so a deeper block
+      is always evicted before the block it extends.
+    * ``allocate`` and ``append_slot`` give no token ids: such a sequence
+      names no further blocks.  ``append_token`` gives the id and names the
+      block it fills.
+    """
+
+    def __init__(self, num_blocks, block_size, initial_free_order=None):
+        super().__init__(num_blocks, block_size, initial_free_order)
+        self.cache = {}          # token prefix (tuple) -> block
+        self.name = {}           # block -> token prefix
+        self.evictable = []      # named blocks with count zero, oldest first
+        self.tokens = {}         # seq id -> token ids held, or None when unknown
+        self.hits = 0
+        self.lookups = 0
+
+    @property
+    def num_free(self):
+        return len(self.free_list) + len(self.evictable)
+
+    @property
+    def num_used(self):
+        return self.num_blocks - self.num_free
+
+    @property
+    def num_cached(self):
+        return len(self.name)
+
+    def _take(self):
+        if self.free_list:
+            return self.free_list.pop()
+        b = self.evictable.pop(0)
+        del self.cache[self.name.pop(b)]
+        return b
+
+    def _key(self, toks, j):
+        """Name of block j of a table holding ``toks``: the whole prefix ending with it."""
+        return tuple(toks[:(j + 1) * self.block_size])
+
+    def _name(self, seq, j):
+        """Name block j of seq's table, if the rules above allow it."""
+        table, toks = self.tables[seq], self.tokens[seq]
+        bs = self.block_size
+        if toks is None or len(toks) < (j + 1) * bs:
+            return
+        for i in range(j):
+            if self.cache.get(self._key(toks, i)) != table[i]:
+                return
+        key = self._key(toks, j)
+        if key in self.cache or table[j] in self.name:
+            return
+        self.cache[key] = table[j]
+        self.name[table[j]] = key
+
+    def allocate(self, seq, num_tokens):
+        if seq in self.tables:
+            raise InvalidArg(f"sequence {seq} already exists")
+        if num_tokens < 0:
+            raise InvalidArg("negative token count")
+        need = ceil_div(num_tokens, self.block_size)
+        if need > self.num_free:
+            raise NoBlocks(f"need {need} blocks, {self.num_free} free")
+        blocks = [self._take() for _ in range(need)]
+        for b in blocks:
+            self.ref[b] = 1
+        self.tables[seq] = blocks
+        self.ctx[seq] = int(num_tokens)
+        self.tokens[seq] = [] if num_tokens == 0 else None
+        return list(blocks)
+
+    def allocate_prefix(self, seq, tokens):
+        """New sequence holding ``tokens``; returns how many leading tokens are cached."""
+        if seq in self.tables:
+            raise InvalidArg(f"sequence {seq} already exists")
+        toks = [int(t) for t in tokens]
+        bs = self.block_size
+        nfull = len(toks) // bs
+        found, probed = [], 0
+        for j in range(nfull):
+            probed += 1
+            b = self.cache.get(self._key(toks, j))
+            if b is None:
+                break
+            found.append(b)
+        need = ceil_div(len(toks), bs) - len(found)
+        if need > self.num_free - sum(1 for b in found if b in self.evictable):
+            raise NoBlocks(f"need {need} blocks")
+        self.lookups += probed
+        self.hits += len(found)
+        for b in found:
+            if b in self.evictable:
+                self.evictable.remove(b)
+            self.ref[b] += 1
+        table = list(found)
+        self.tables[seq] = table
+        self.ctx[seq] = len(toks)
+        self.tokens[seq] = toks
+        for j in range(len(found), ceil_div(len(toks), bs)):
+            b = self._take()
+            self.ref[b] = 1
+            table.append(b)
+            self._name(seq, j)
+        return len(found) * bs
+
+    def fork(self, parent, child):
+        super().fork(parent, child)
+        t = self.tokens[parent]
+        self.tokens[child] = None if t is None else list(t)
+
+    def _append(self, seq, token):
+        if seq not in self.tables:
+            raise InvalidArg(f"unknown sequence {seq}")
+        table = self.tables[seq]
+        bs = self.block_size
+        pos = self.ctx[seq]
+        cow_src = cow_dst = -1
+        if pos % bs == 0 or self.ref[table[-1]] > 1:
+            if self.num_free == 0:
+                raise NoBlocks("no block for the next token")
+            b = self._take()
+            self.ref[b] = 1
+            if pos % bs == 0:
+                table.append(b)
+            else:                                   # copy-on-write of a shared last block
+                cow_src, cow_dst = table[-1], b
+                self.ref[table[-1]] -= 1
+                table[-1] = b
+        self.ctx[seq] = pos + 1
+        toks = self.tokens[seq]
+        if toks is not None and token is not None:
+            toks.append(int(token))
+        else:
+            self.tokens[seq] = None
+        if (pos + 1) % bs == 0:
+            self._name(seq, pos // bs)
+        return table[pos // bs] * bs + pos % bs, cow_src, cow_dst
+
+    def append_slot(self, seq):
+        return self._append(seq, None)
+
+    def append_token(self, seq, token):
+        return self._append(seq, token)
+
+    def free(self, seq):
+        if seq not in self.tables:
+            raise InvalidArg(f"unknown sequence {seq}")
+        named = []
+        for b in self.tables[seq]:
+            if self.ref[b] <= 0:
+                raise AssertionError("reference count underflow")
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                if b in self.name:
+                    named.append(b)
+                else:
+                    self.free_list.append(b)
+        self.evictable.extend(reversed(named))
+        del self.tables[seq], self.ctx[seq], self.tokens[seq]
+
+    def check(self):
+        held = {}
+        for seq, table in self.tables.items():
+            assert len(table) == ceil_div(self.ctx[seq], self.block_size), seq
+            for b in table:
+                held[b] = held.get(b, 0) + 1
+        for b in range(self.num_blocks):
+            assert self.ref[b] == held.get(b, 0), (b, self.ref[b], held.get(b, 0))
+        free, ev = set(self.free_list), set(self.evictable)
+        assert len(free) == len(self.free_list) and len(ev) == len(self.evictable), "duplicate"
+        assert not (free & ev) and not (free & held.keys()) and not (ev & held.keys()), "block in two places"
+        assert free | ev | set(held) == set(range(self.num_blocks)), "block lost"
+        assert ev <= set(self.name), "evictable block without a name"
+        assert not (free & set(self.name)), "named block on the free list"
+        assert {self.cache[k]: k for k in self.cache} == self.name, "cache and names disagree"
+        for key, b in self.cache.items():
+            assert len(key) % self.block_size == 0 and len(key) > 0

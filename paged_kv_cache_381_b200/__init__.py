@@ -340,6 +340,40 @@ class BlockManager:
         _check(lib().pa_bm_pack(self._h, _ptr(ids), len(ids), width, _ptr(tables), _ptr(lens)), "pa_bm_pack")
         return tables[:, :width], lens
 
+    # ---- prefix cache (pa_bm_enable_prefix_cache and friends) ----
+
+    def enable_prefix_cache(self, enable=True):
+        _check(lib().pa_bm_enable_prefix_cache(self._h, int(bool(enable))), "pa_bm_enable_prefix_cache")
+
+    def allocate_prefix(self, seq, tokens):
+        """New sequence holding the prompt `tokens`; returns the number of leading
+        tokens whose K/V is already cached (a multiple of block_size)."""
+        toks = np.ascontiguousarray(tokens, dtype=np.int32)
+        cached = ctypes.c_int()
+        _check(lib().pa_bm_allocate_prefix(self._h, seq, _ptr(toks), toks.size, ctypes.byref(cached)),
+               "pa_bm_allocate_prefix")
+        return cached.value
+
+    def append_token(self, seq, token):
+        slot, src, dst = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().pa_bm_append_token(self._h, seq, int(token), ctypes.byref(slot), ctypes.byref(src),
+                                        ctypes.byref(dst)), "pa_bm_append_token")
+        return slot.value, src.value, dst.value
+
+    def cache_stats(self):
+        """(cached blocks, evictable blocks, block hits, block lookups)."""
+        c, e, h, l = ctypes.c_int(), ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64()
+        _check(lib().pa_bm_cache_stats(self._h, ctypes.byref(c), ctypes.byref(e), ctypes.byref(h), ctypes.byref(l)),
+               "pa_bm_cache_stats")
+        return c.value, e.value, h.value, l.value
+
+    def evictable(self):
+        """Evictable cached blocks, next victim first."""
+        out = np.zeros(self.num_blocks, dtype=np.int32)
+        n = ctypes.c_int()
+        _check(lib().pa_bm_evictable(self._h, _ptr(out), out.size, ctypes.byref(n)), "pa_bm_evictable")
+        return out[:n.value].tolist()
+
 
 class Scheduler:
     """Iteration-level batching over a BlockManager (pa_sched_*)."""

@@ -73,6 +73,11 @@ SIGNATURES = {
     "pa_bm_ref_count": (c_int, [c_void_p, c_int32, P(c_int)]),
     "pa_bm_free_list": (c_int, [c_void_p, c_void_p, c_int, P(c_int)]),
     "pa_bm_pack": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
+    "pa_bm_enable_prefix_cache": (c_int, [c_void_p, c_int]),
+    "pa_bm_allocate_prefix": (c_int, [c_void_p, c_int64, c_void_p, c_int, P(c_int)]),
+    "pa_bm_append_token": (c_int, [c_void_p, c_int64, c_int32, P(c_int64), P(c_int32), P(c_int32)]),
+    "pa_bm_cache_stats": (c_int, [c_void_p, P(c_int), P(c_int), P(c_int64), P(c_int64)]),
+    "pa_bm_evictable": (c_int, [c_void_p, c_void_p, c_int, P(c_int)]),
     "pa_sched_create": (c_int, [c_void_p, c_int, c_int64, P(c_void_p)]),
     "pa_sched_destroy": (None, [c_void_p]),
     "pa_sched_add_request": (c_int, [c_void_p, c_int64, c_int, c_int, c_int, c_int64, c_int]),

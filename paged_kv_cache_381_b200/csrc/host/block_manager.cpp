@@ -13,9 +13,25 @@
 //    "PagedAttention分页注意力机制原理": sequences share prefix blocks by
 //    reference; finished requests return their blocks to the free pool.
 //  Free pushes blocks whose count reaches zero in logical table order.
+//
+//  Prefix cache ("大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置",
+//  section "Prefix Caching前缀复用优化": a new request whose prefix matches
+//  cached KV references those blocks and skips their prefill), when enabled:
+//  a full block is keyed by (parent block, its token ids), which names the
+//  whole prefix exactly (no hash collisions); allocate_prefix references the
+//  longest cached run of full prompt blocks and allocates the rest; blocks
+//  filled by allocate_prefix or append_token are registered; a registered
+//  block whose count reaches zero stays cached on an LRU list and is evicted
+//  (unregistered and reused) only when the free list is empty.  A partly
+//  filled block is never shared through the cache.  A block is registered
+//  only under a registered parent (or as a first block), and free_seq puts a
+//  sequence's cached blocks on the LRU list last block first, so a child is
+//  always evicted before its parent and no key can name a reused parent.
 
 #include "block_manager.hpp"
 
+#include <cstring>
+#include <iterator>
 #include <new>
 
 namespace pa_host {
@@ -23,7 +39,8 @@ namespace pa_host {
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 BlockManager::BlockManager(int num_blocks, int block_size, const int32_t* initial_free_order)
-    : num_blocks_(num_blocks), block_size_(block_size), ref_(num_blocks, 0) {
+    : num_blocks_(num_blocks), block_size_(block_size), ref_(num_blocks, 0), lru_pos_(num_blocks),
+      in_lru_(num_blocks, 0) {
     free_.reserve(num_blocks);
     for (int i = 0; i < num_blocks; ++i)
         free_.push_back(initial_free_order ? initial_free_order[i] : i);
@@ -40,20 +57,115 @@ bool BlockManager::valid_order(int num_blocks, const int32_t* order) {
     return true;
 }
 
+int32_t BlockManager::take_block() {
+    if (!free_.empty()) {
+        int32_t b = free_.back();
+        free_.pop_back();
+        return b;
+    }
+    if (!lru_.empty()) {                 // evict the least recently released cached block
+        int32_t b = lru_.front();
+        lru_.pop_front();
+        in_lru_[b] = 0;
+        auto it = key_of_.find(b);
+        if (it != key_of_.end()) {
+            block_of_.erase(it->second);
+            key_of_.erase(it);
+        }
+        return b;
+    }
+    return -1;
+}
+
+void BlockManager::release_block(int32_t b) {
+    if (key_of_.count(b)) {
+        lru_.push_back(b);
+        lru_pos_[b] = std::prev(lru_.end());
+        in_lru_[b] = 1;
+    } else {
+        free_.push_back(b);
+    }
+}
+
+std::string BlockManager::make_key(int32_t parent, const int32_t* tokens) const {
+    std::string k(sizeof(int32_t) * (1 + block_size_), '\0');
+    std::memcpy(&k[0], &parent, sizeof(int32_t));
+    std::memcpy(&k[sizeof(int32_t)], tokens, sizeof(int32_t) * block_size_);
+    return k;
+}
+
+void BlockManager::register_block(int32_t block, int32_t parent, const int32_t* tokens) {
+    if (parent >= 0 && !key_of_.count(parent)) return;         // prefix not named by the cache
+    std::string k = make_key(parent, tokens);
+    if (block_of_.count(k) || key_of_.count(block)) return;   // identical content already cached
+    block_of_.emplace(k, block);
+    key_of_.emplace(block, std::move(k));
+}
+
 pa_status BlockManager::allocate(int64_t seq, int num_tokens) {
     if (num_tokens < 0 || seqs_.count(seq)) return PA_ERR_INVALID_ARG;
     int64_t need = ceil_div(num_tokens, block_size_);
-    if (need > (int64_t)free_.size()) return PA_ERR_NO_BLOCKS;
+    if (need > (int64_t)num_free()) return PA_ERR_NO_BLOCKS;
     Seq s;
     s.ctx = num_tokens;
+    s.tail_known = num_tokens == 0;
     s.table.reserve(need);
     for (int64_t i = 0; i < need; ++i) {
-        int32_t b = free_.back();
-        free_.pop_back();
+        int32_t b = take_block();
         ref_[b] = 1;
         s.table.push_back(b);
     }
     seqs_.emplace(seq, std::move(s));
+    return PA_OK;
+}
+
+pa_status BlockManager::allocate_prefix(int64_t seq, const int32_t* tokens, int num_tokens, int* cached_tokens) {
+    if (num_tokens < 0 || seqs_.count(seq) || (num_tokens > 0 && !tokens)) return PA_ERR_INVALID_ARG;
+    const int bs = block_size_;
+    const int nfull = num_tokens / bs;
+    // longest run of cached full blocks, probed before anything changes
+    std::vector<int32_t> hit;
+    int32_t parent = -1;
+    int probed = 0;
+    if (prefix_cache_) {
+        for (int j = 0; j < nfull; ++j) {
+            ++probed;
+            auto it = block_of_.find(make_key(parent, tokens + (int64_t)j * bs));
+            if (it == block_of_.end()) break;
+            hit.push_back(it->second);
+            parent = it->second;
+        }
+    }
+    int64_t hits_in_lru = 0;
+    for (int32_t b : hit) hits_in_lru += in_lru_[b];
+    const int64_t need = ceil_div(num_tokens, bs) - (int64_t)hit.size();
+    if (need > (int64_t)num_free() - hits_in_lru) return PA_ERR_NO_BLOCKS;
+    lookups_ += probed;
+    hits_ += (int64_t)hit.size();
+    Seq s;
+    s.ctx = num_tokens;
+    for (int32_t b : hit) {
+        if (in_lru_[b]) {
+            lru_.erase(lru_pos_[b]);
+            in_lru_[b] = 0;
+        }
+        ref_[b] += 1;
+        s.table.push_back(b);
+    }
+    parent = hit.empty() ? -1 : hit.back();
+    for (int64_t j = (int64_t)hit.size(); j < ceil_div(num_tokens, bs); ++j) {
+        int32_t b = take_block();
+        ref_[b] = 1;
+        s.table.push_back(b);
+        if (prefix_cache_ && j < nfull) {
+            register_block(b, parent, tokens + j * bs);
+            parent = b;
+        }
+    }
+    s.tail.assign(tokens + (int64_t)nfull * bs, tokens + num_tokens);
+    s.tail_known = true;
+    seqs_.emplace(seq, std::move(s));
+    if (cached_tokens) *cached_tokens = (int)hit.size() * bs;
     return PA_OK;
 }
 
@@ -67,6 +179,15 @@ pa_status BlockManager::fork(int64_t parent, int64_t child) {
 }
 
 pa_status BlockManager::append_slot(int64_t seq, int64_t* slot, int32_t* cow_src, int32_t* cow_dst) {
+    return append(seq, 0, false, slot, cow_src, cow_dst);
+}
+
+pa_status BlockManager::append_token(int64_t seq, int32_t token, int64_t* slot, int32_t* cow_src, int32_t* cow_dst) {
+    return append(seq, token, true, slot, cow_src, cow_dst);
+}
+
+pa_status BlockManager::append(int64_t seq, int32_t token, bool known, int64_t* slot, int32_t* cow_src,
+                               int32_t* cow_dst) {
     auto it = seqs_.find(seq);
     if (it == seqs_.end()) return PA_ERR_INVALID_ARG;
     Seq& s = it->second;
@@ -74,18 +195,17 @@ pa_status BlockManager::append_slot(int64_t seq, int64_t* slot, int32_t* cow_src
     int32_t src = -1, dst = -1;
     if (pos % block_size_ == 0) {
         // the last block is full (or there is none): open a fresh block
-        if (free_.empty()) return PA_ERR_NO_BLOCKS;
-        int32_t b = free_.back();
-        free_.pop_back();
+        if (num_free() == 0) return PA_ERR_NO_BLOCKS;
+        int32_t b = take_block();
         ref_[b] = 1;
         s.table.push_back(b);
+        s.tail.clear();
     } else {
         int32_t last = s.table.back();
         if (ref_[last] > 1) {
             // shared partly filled block: give this sequence a private copy
-            if (free_.empty()) return PA_ERR_NO_BLOCKS;
-            int32_t b = free_.back();
-            free_.pop_back();
+            if (num_free() == 0) return PA_ERR_NO_BLOCKS;
+            int32_t b = take_block();
             ref_[b] = 1;
             ref_[last] -= 1;
             s.table.back() = b;
@@ -94,6 +214,12 @@ pa_status BlockManager::append_slot(int64_t seq, int64_t* slot, int32_t* cow_src
         }
     }
     s.ctx = pos + 1;
+    s.tail.push_back(token);
+    s.tail_known = s.tail_known && known;
+    if (prefix_cache_ && s.tail_known && (int)s.tail.size() == block_size_) {
+        const size_t n = s.table.size();
+        register_block(s.table[n - 1], n >= 2 ? s.table[n - 2] : -1, s.tail.data());
+    }
     if (slot) *slot = (int64_t)s.table[pos / block_size_] * block_size_ + pos % block_size_;
     if (cow_src) *cow_src = src;
     if (cow_dst) *cow_dst = dst;
@@ -103,10 +229,17 @@ pa_status BlockManager::append_slot(int64_t seq, int64_t* slot, int32_t* cow_src
 pa_status BlockManager::free_seq(int64_t seq) {
     auto it = seqs_.find(seq);
     if (it == seqs_.end()) return PA_ERR_INVALID_ARG;
+    std::vector<int32_t> cached;
     for (int32_t b : it->second.table) {
         if (ref_[b] <= 0) return PA_ERR_INVALID_ARG;  // corrupted counts; never expected
-        if (--ref_[b] == 0) free_.push_back(b);
+        if (--ref_[b] == 0) {
+            if (key_of_.count(b))
+                cached.push_back(b);
+            else
+                free_.push_back(b);
+        }
     }
+    for (auto r = cached.rbegin(); r != cached.rend(); ++r) release_block(*r);   // last block first
     seqs_.erase(it);
     return PA_OK;
 }
@@ -222,3 +355,44 @@ pa_status pa_bm_pack(const pa_bm* bm, const int64_t* seq_ids, int n, int width, 
 }  // extern "C"
 
 pa_host::BlockManager* pa_bm_impl(pa_bm* bm) { return bm ? &bm->impl : nullptr; }
+
+extern "C" {
+
+pa_status pa_bm_enable_prefix_cache(pa_bm* bm, int enable) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    bm->impl.enable_prefix_cache(enable != 0);
+    return PA_OK;
+}
+
+pa_status pa_bm_allocate_prefix(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int num_tokens,
+                                int* cached_tokens) {
+    return bm ? bm->impl.allocate_prefix(seq_id, tokens, num_tokens, cached_tokens) : PA_ERR_INVALID_ARG;
+}
+
+pa_status pa_bm_append_token(pa_bm* bm, int64_t seq_id, int32_t token, int64_t* slot, int32_t* cow_src,
+                             int32_t* cow_dst) {
+    return bm ? bm->impl.append_token(seq_id, token, slot, cow_src, cow_dst) : PA_ERR_INVALID_ARG;
+}
+
+pa_status pa_bm_cache_stats(const pa_bm* bm, int* cached_blocks, int* evictable_blocks, int64_t* hits,
+                            int64_t* lookups) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    if (cached_blocks) *cached_blocks = bm->impl.num_cached();
+    if (evictable_blocks) *evictable_blocks = bm->impl.num_evictable();
+    if (hits) *hits = bm->impl.hits();
+    if (lookups) *lookups = bm->impl.lookups();
+    return PA_OK;
+}
+
+pa_status pa_bm_evictable(const pa_bm* bm, int32_t* out, int cap, int* n) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    const auto& l = bm->impl.evictable();
+    int len = (int)l.size();
+    if (n) *n = len;
+    if (len > cap || (len > 0 && !out)) return PA_ERR_INVALID_ARG;
+    int i = 0;
+    for (int32_t b : l) out[i++] = b;
+    return PA_OK;
+}
+
+}  // extern "C"

@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cstdint>
+#include <list>
+#include <string>
 #include <unordered_map>
 #include <vector>
 
@@ -16,6 +18,8 @@ class BlockManager {
     struct Seq {
         std::vector<int32_t> table;   // physical ids, logical order
         int64_t ctx = 0;              // tokens held
+        std::vector<int32_t> tail;    // token ids of the partly filled last block (prefix cache)
+        bool tail_known = true;       // false once a token was appended without its id
     };
 
     BlockManager(int num_blocks, int block_size, const int32_t* initial_free_order);
@@ -27,19 +31,45 @@ class BlockManager {
     pa_status free_seq(int64_t seq);
     pa_status slots(int64_t seq, int64_t start, int64_t count, int64_t* out) const;
 
+    // prefix cache
+    void enable_prefix_cache(bool on) { prefix_cache_ = on; }
+    bool prefix_cache() const { return prefix_cache_; }
+    pa_status allocate_prefix(int64_t seq, const int32_t* tokens, int num_tokens, int* cached_tokens);
+    pa_status append_token(int64_t seq, int32_t token, int64_t* slot, int32_t* cow_src, int32_t* cow_dst);
+    int num_cached() const { return (int)key_of_.size(); }
+    int num_evictable() const { return (int)lru_.size(); }
+    int64_t hits() const { return hits_; }
+    int64_t lookups() const { return lookups_; }
+    const std::list<int32_t>& evictable() const { return lru_; }
+
     const Seq* find(int64_t seq) const;
-    int num_free() const { return (int)free_.size(); }
+    int num_free() const { return (int)(free_.size() + lru_.size()); }
     int num_blocks() const { return num_blocks_; }
     int block_size() const { return block_size_; }
     int ref(int32_t b) const { return ref_[b]; }
     const std::vector<int32_t>& free_list() const { return free_; }
 
   private:
+    pa_status append(int64_t seq, int32_t token, bool known, int64_t* slot, int32_t* cow_src,
+                     int32_t* cow_dst);
+    int32_t take_block();                                   // free list first, then evict LRU
+    std::string make_key(int32_t parent, const int32_t* tokens) const;
+    void register_block(int32_t block, int32_t parent, const int32_t* tokens);
+    void release_block(int32_t block);                      // ref reached zero
+
     int num_blocks_;
     int block_size_;
     std::vector<int32_t> free_;   // back() is taken next
     std::vector<int32_t> ref_;
     std::unordered_map<int64_t, Seq> seqs_;
+    // prefix cache: (parent block, token ids) of a full block -> block, and back
+    bool prefix_cache_ = false;
+    std::unordered_map<std::string, int32_t> block_of_;
+    std::unordered_map<int32_t, std::string> key_of_;
+    std::list<int32_t> lru_;                                  // cached blocks with ref 0, oldest first
+    std::vector<std::list<int32_t>::iterator> lru_pos_;
+    std::vector<char> in_lru_;
+    int64_t hits_ = 0, lookups_ = 0;
 };
 
 }  // namespace pa_host
