@@ -338,6 +338,16 @@ pa_status pa_bm_free_list(const pa_bm* bm, int32_t* out, int cap, int* n);
 pa_status pa_bm_pack(const pa_bm* bm, const int64_t* seq_ids, int n, int width,
                      int32_t* tables, int32_t* context_lens);
 
+/* Memory actually used by the pool's live sequences ([P3] "大模型推理显存优化
+ * 实战：PagedAttention机制原理与vLLM连续批处理配置", sections on the memory
+ * bottleneck and on paged attention: contiguous per-request reservation wastes
+ * memory, paging wastes at most the tail of each sequence's last block).
+ * *held_blocks = blocks whose count is above zero; *filled_slots = their slots
+ * below the context length of at least one holder (a shared block is counted
+ * once).  Reserved-but-unused share = 1 - filled / (held x block_size).
+ * Either pointer may be NULL. */
+pa_status pa_bm_usage(const pa_bm* bm, int64_t* held_blocks, int64_t* filled_slots);
+
 /* ---- prefix cache ([P3] "Prefix Caching前缀复用优化": a request whose prompt
  * starts with cached KV references those blocks and skips their prefill) ----
  *

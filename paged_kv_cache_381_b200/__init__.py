@@ -340,6 +340,12 @@ class BlockManager:
         _check(lib().pa_bm_pack(self._h, _ptr(ids), len(ids), width, _ptr(tables), _ptr(lens)), "pa_bm_pack")
         return tables[:, :width], lens
 
+    def usage(self):
+        """(blocks held by live sequences, their slots holding a token)."""
+        h, f = ctypes.c_int64(), ctypes.c_int64()
+        _check(lib().pa_bm_usage(self._h, ctypes.byref(h), ctypes.byref(f)), "pa_bm_usage")
+        return h.value, f.value
+
     # ---- prefix cache (pa_bm_enable_prefix_cache and friends) ----
 
     def enable_prefix_cache(self, enable=True):

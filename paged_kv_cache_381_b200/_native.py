@@ -73,6 +73,7 @@ SIGNATURES = {
     "pa_bm_ref_count": (c_int, [c_void_p, c_int32, P(c_int)]),
     "pa_bm_free_list": (c_int, [c_void_p, c_void_p, c_int, P(c_int)]),
     "pa_bm_pack": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
+    "pa_bm_usage": (c_int, [c_void_p, P(c_int64), P(c_int64)]),
     "pa_bm_enable_prefix_cache": (c_int, [c_void_p, c_int]),
     "pa_bm_allocate_prefix": (c_int, [c_void_p, c_int64, c_void_p, c_int, P(c_int)]),
     "pa_bm_append_token": (c_int, [c_void_p, c_int64, c_int32, P(c_int64), P(c_int32), P(c_int32)]),

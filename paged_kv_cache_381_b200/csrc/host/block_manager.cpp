@@ -244,6 +244,28 @@ pa_status BlockManager::free_seq(int64_t seq) {
     return PA_OK;
 }
 
+void BlockManager::usage(int64_t* held_blocks, int64_t* filled_slots) const {
+    // a shared block is counted once, filled up to the furthest of its holders
+    std::vector<int32_t> fill(num_blocks_, 0);
+    for (const auto& kv : seqs_) {
+        const Seq& s = kv.second;
+        for (size_t j = 0; j < s.table.size(); ++j) {
+            int64_t f = s.ctx - (int64_t)j * block_size_;
+            int32_t n = (int32_t)(f < block_size_ ? f : block_size_);
+            if (n > fill[s.table[j]]) fill[s.table[j]] = n;
+        }
+    }
+    int64_t held = 0, filled = 0;
+    for (int b = 0; b < num_blocks_; ++b) {
+        if (ref_[b] > 0) {
+            ++held;
+            filled += fill[b];
+        }
+    }
+    if (held_blocks) *held_blocks = held;
+    if (filled_slots) *filled_slots = filled;
+}
+
 const BlockManager::Seq* BlockManager::find(int64_t seq) const {
     auto it = seqs_.find(seq);
     return it == seqs_.end() ? nullptr : &it->second;
@@ -381,6 +403,12 @@ pa_status pa_bm_cache_stats(const pa_bm* bm, int* cached_blocks, int* evictable_
     if (evictable_blocks) *evictable_blocks = bm->impl.num_evictable();
     if (hits) *hits = bm->impl.hits();
     if (lookups) *lookups = bm->impl.lookups();
+    return PA_OK;
+}
+
+pa_status pa_bm_usage(const pa_bm* bm, int64_t* held_blocks, int64_t* filled_slots) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    bm->impl.usage(held_blocks, filled_slots);
     return PA_OK;
 }
 

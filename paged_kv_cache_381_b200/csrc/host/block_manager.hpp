@@ -42,6 +42,9 @@ class BlockManager {
     int64_t lookups() const { return lookups_; }
     const std::list<int32_t>& evictable() const { return lru_; }
 
+    // blocks held by live sequences, and their slots holding a token of some holder
+    void usage(int64_t* held_blocks, int64_t* filled_slots) const;
+
     const Seq* find(int64_t seq) const;
     int num_free() const { return (int)(free_.size() + lru_.size()); }
     int num_blocks() const { return num_blocks_; }

@@ -351,3 +351,29 @@ def token_rows(seed, stream, positions, heads, head_dim, dtype, salt=0):
     z += B[j]
     z *= np.float32(0.7071067811865476)
     return to_storage(z.reshape(len(pos), heads, head_dim), dtype)
+
+
+def prefix_keys(tokens):
+    """uint64 key of every prefix tokens[:p+1], p = 0..n-1 (a SplitMix64 chain),
+    so the K/V rows drawn from these keys depend on the whole prefix, as a
+    model's K/V at a position does."""
+    toks = np.asarray(tokens, dtype=np.int64).astype(np.uint64)
+    with np.errstate(over="ignore"):
+        mixed = _splitmix64(toks + np.uint64(0x13198A2E03707344)).tolist()
+    m = 0xFFFFFFFFFFFFFFFF
+    keys = []
+    h = 0x243F6A8885A308D3
+    for x in mixed:                      # the chain itself, in Python integers
+        z = ((h ^ x) + 0x9E3779B97F4A7C15) & m
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & m
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & m
+        h = z ^ (z >> 31)
+        keys.append(h)
+    return np.array(keys, dtype=np.uint64)
+
+
+def prefix_rows(seed, tokens, start, heads, head_dim, dtype, salt=0):
+    """Rows [n - start, heads, head_dim] for positions start..n-1 of the token
+    sequence, each keyed by its whole prefix (prefix_keys) and salt (K 0, V 1)."""
+    keys = prefix_keys(tokens)[start:]
+    return token_rows(seed, 0x9F, keys, heads, head_dim, dtype, salt)

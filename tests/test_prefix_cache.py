@@ -437,3 +437,14 @@ def test_native_matches_model_op_by_op(pa, seed):
     for s in model.toks:
         assert model.m.table(s) == nat.m.table(s)
     assert [model.m.ref(b) for b in range(nb)] == [nat.m.ref(b) for b in range(nb)]
+
+
+def test_conversation_workload_host_side(pa):
+    """The multi-turn workload the GPU test runs, host side only: it reuses
+    most K/V rows and some continued conversations lose blocks to eviction."""
+    import sys
+    sys.path.insert(0, ROOT)
+    from tests.prefix_workload import NullDevice, run_conversations
+    st = run_conversations(NullDevice())
+    assert st["written"] + st["cached"] == st["total"]
+    assert st["cached"] > 0.4 * st["total"] and st["short"] > 0, st
