@@ -119,3 +119,39 @@ def paged_decode_rows(q, k_cache, v_cache, block_tables, context_lens, scale,
         V = widen(gather(v_cache[:, :, g:g + 1, :], block_tables[s], n, block_size), dtype)[:, 0, :]
         res.append(attend(widen(q[s, h], dtype), K, V, scale))
     return np.stack(res) if res else np.zeros((0, q.shape[2]))
+
+
+def paged_verify(q, k_cache, v_cache, block_tables, context_lens, scale,
+                 block_size, dtype):
+    """Multi-query paged attention: the target model's verification pass of
+    speculative decoding ([P1] "大模型推理引擎高频优化：连续批处理、PagedAttention 与
+    KV Cache 实战拆解", section 5: a draft model proposes 5-6 candidate tokens and
+    the target model checks them in one parallel pass).
+
+    q: [S, Q, Hq, D] storage form; the K/V of the Q candidate tokens are the
+    last Q positions of each sequence's context (written before the call).
+    Query i of sequence s sits at position p = context_lens[s] - Q + i and
+    attends causally to positions 0..p of its own sequence:
+
+        out[s, i, h] = attend(q[s, i, h], K_s[0..p, h // G], V_s[0..p, h // G])
+
+    (Q = 1 is plain decode.)  A row with p < 0 (context shorter than Q) is a
+    zero row, as an empty context is in decode.  Returns float64 [S, Q, Hq, D].
+    """
+    q = np.asarray(q)
+    S, Q, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((S, Q, Hq, D), dtype=np.float64)
+    for s in range(S):
+        n = int(context_lens[s])
+        K = widen(gather(k_cache, block_tables[s], n, block_size), dtype)
+        V = widen(gather(v_cache, block_tables[s], n, block_size), dtype)
+        for i in range(Q):
+            p = n - Q + i
+            if p < 0:
+                continue
+            qi = widen(q[s, i], dtype)
+            for h in range(Hq):
+                out[s, i, h] = attend(qi[h], K[:p + 1, h // G], V[:p + 1, h // G], scale)
+    return out
