@@ -368,3 +368,120 @@ class PrefixCachingBlockManager(BlockManager):
         assert {self.cache[k]: k for k in self.cache} == self.name, "cache and names disagree"
         for key, b in self.cache.items():
             assert len(key) % self.block_size == 0 and len(key) > 0
+
+
+class SwappingBlockManager(BlockManager):
+    """Block manager with a host (CPU) swap pool (oracle; test infrastructure only).
+
+    [P3] "大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置", section
+    "生产部署注意事项": when GPU memory runs short, the KV cache of some requests
+    is moved out to CPU memory and moved back once GPU memory is free again.
+    Readings adopted where the page is silent:
+
+    * The host pool holds ``num_cpu_blocks`` blocks of the same shape, on its
+      own free list (taken from the end, like the GPU list).
+    * ``swap_out(seq)`` moves every block the sequence holds ALONE (count 1)
+      to a host block, in logical order, and returns the GPU block it leaves
+      to the free list (logical order); blocks it shares (count > 1) stay on
+      the GPU and the sequence keeps its reference, since their contents
+      remain resident for the other holders.  Returns the (gpu, cpu) copies
+      to run BEFORE the freed GPU blocks are reused.  All or nothing: with too
+      few host blocks, NoBlocks and no change.
+    * ``swap_in(seq)`` takes a fresh GPU block for each host block of the
+      sequence, in logical order, returns the host blocks to their list, and
+      returns the (cpu, gpu) copies.  All or nothing on GPU blocks.
+    * A swapped-out sequence cannot append or fork; ``free`` releases its host
+      blocks (logical order) and its shared GPU references.
+    """
+
+    def __init__(self, num_blocks, block_size, num_cpu_blocks, initial_free_order=None):
+        super().__init__(num_blocks, block_size, initial_free_order)
+        self.num_cpu_blocks = int(num_cpu_blocks)
+        self.cpu_free = list(range(self.num_cpu_blocks))
+        self.on_cpu = {}                 # seq id -> list of bools per logical block (swapped sequences)
+
+    def swapped(self, seq):
+        return seq in self.on_cpu
+
+    def swap_out(self, seq):
+        if seq not in self.tables or seq in self.on_cpu:
+            raise InvalidArg(f"sequence {seq} is not resident")
+        table = self.tables[seq]
+        alone = [j for j, b in enumerate(table) if self.ref[b] == 1]
+        if len(alone) > len(self.cpu_free):
+            raise NoBlocks(f"need {len(alone)} host blocks, {len(self.cpu_free)} free")
+        loc = [False] * len(table)
+        pairs = []
+        for j in alone:
+            g = table[j]
+            c = self.cpu_free.pop()
+            pairs.append((g, c))
+            self.ref[g] = 0
+            self.free_list.append(g)
+            table[j] = c
+            loc[j] = True
+        self.on_cpu[seq] = loc
+        return pairs
+
+    def swap_in(self, seq):
+        if seq not in self.on_cpu:
+            raise InvalidArg(f"sequence {seq} is not swapped out")
+        table, loc = self.tables[seq], self.on_cpu[seq]
+        need = sum(loc)
+        if need > len(self.free_list):
+            raise NoBlocks(f"need {need} blocks, {len(self.free_list)} free")
+        pairs = []
+        for j, here in enumerate(loc):
+            if here:
+                c = table[j]
+                g = self.free_list.pop()
+                self.ref[g] = 1
+                pairs.append((c, g))
+                self.cpu_free.append(c)
+                table[j] = g
+        del self.on_cpu[seq]
+        return pairs
+
+    def fork(self, parent, child):
+        if parent in self.on_cpu:
+            raise InvalidArg(f"sequence {parent} is swapped out")
+        super().fork(parent, child)
+
+    def append_slot(self, seq):
+        if seq in self.on_cpu:
+            raise InvalidArg(f"sequence {seq} is swapped out")
+        return super().append_slot(seq)
+
+    def free(self, seq):
+        if seq not in self.on_cpu:
+            return super().free(seq)
+        for b, here in zip(self.tables[seq], self.on_cpu[seq]):
+            if here:
+                self.cpu_free.append(b)
+            else:
+                if self.ref[b] <= 0:
+                    raise AssertionError("reference count underflow")
+                self.ref[b] -= 1
+                if self.ref[b] == 0:
+                    self.free_list.append(b)
+        del self.tables[seq], self.ctx[seq], self.on_cpu[seq]
+
+    def check(self):
+        held, cpu_held = {}, []
+        for seq, table in self.tables.items():
+            assert len(table) == ceil_div(self.ctx[seq], self.block_size), seq
+            loc = self.on_cpu.get(seq, [False] * len(table))
+            for b, here in zip(table, loc):
+                if here:
+                    cpu_held.append(b)
+                else:
+                    held[b] = held.get(b, 0) + 1
+        for b in range(self.num_blocks):
+            assert self.ref[b] == held.get(b, 0), (b, self.ref[b], held.get(b, 0))
+        free = set(self.free_list)
+        assert len(free) == len(self.free_list) and free.isdisjoint(held)
+        assert free | set(held) == set(range(self.num_blocks)), "block lost"
+        assert len(set(cpu_held)) == len(cpu_held), "host block held twice"
+        cf = set(self.cpu_free)
+        assert len(cf) == len(self.cpu_free) and cf.isdisjoint(cpu_held)
+        assert cf | set(cpu_held) == set(range(self.num_cpu_blocks)), "host block lost"
