@@ -42,6 +42,7 @@ WORKLOAD_NAMES = {
     "tiny": "tiny fp32 paged decode: 4 seqs {1,16,17,90}, 4/4 heads, head_dim 64, block 16, 32-block pool",
 }
 METRIC = "paged decode attention: KV GB/s read (% of B200 HBM peak); decode tokens/s"
+VERIFY_METRIC = "paged verification attention (speculative decoding): KV GB/s read; verified tokens/s"
 KERNEL_SOURCES = ["paged_kv_cache_381_b200/csrc/device/decode.cuh",
                   "paged_kv_cache_381_b200/csrc/device/common.cuh"]
 
@@ -62,6 +63,9 @@ def parse():
                    help="merge split partitions with the reduce kernel or inside the decode kernel")
     p.add_argument("--num-seqs", type=int, default=0,
                    help="keep only the first N sequences (smaller cases for profiling)")
+    p.add_argument("--queries", type=int, default=1,
+                   help="candidate tokens per sequence: > 1 times the verification pass (pa_verify) "
+                        "of speculative decoding instead of decode")
     return p.parse_args()
 
 
@@ -121,6 +125,38 @@ def decode_kernel_bytes(cfg, lens, partition, fused=False):
     b += (2 if fused else 1) * int(nparts[~single].sum()) * Hq * (D + 2) * 4   # partials (+ read back when fused)
     b += int(np.sum(-(-lens // bs))) * Hkv * 4            # block-table entries
     return int(b)
+
+
+def verify_kernel_bytes(cfg, lens, partition, Q):
+    """decode_kernel_bytes for the verification pass: Q query and output rows
+    per sequence and head (partials likewise)."""
+    e = elt_bytes(cfg.dtype)
+    S, Hq, Hkv, D, bs = len(lens), cfg.num_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
+    P = partition or 512
+    maxc = int(np.max(lens)) if S else 0
+    nparts = np.where(lens <= P, 1, -(-lens // P)) if maxc > P else np.ones(S, dtype=np.int64)
+    single = nparts == 1
+    b = kv_bytes(cfg, lens)
+    b += S * Q * Hq * D * e
+    b += int(single.sum()) * Q * Hq * D * e
+    b += int(nparts[~single].sum()) * Q * Hq * (D + 2) * 4
+    b += int(np.sum(-(-lens // bs))) * Hkv * 4
+    return int(b)
+
+
+def verify_flops(cfg, lens, Q):
+    """Multiply-adds x 2 of S = QK^T and O = PV over the causal prefix of every
+    query row: 4 * D * Hq * sum_s sum_i (ctx_s - Q + i + 1)."""
+    seen = sum(max(0, int(n) - Q + i + 1) for n in lens for i in range(Q))
+    return 4.0 * cfg.head_dim * cfg.num_heads * seen
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
 
 
 class ClockSampler:
@@ -288,9 +324,15 @@ def run_native(args):
     if args.num_seqs:
         lens_override = wl.context_lengths(cfg, wl.rng(seed))[:args.num_seqs]
     d = wl.draw_device(cfg, seed, device=dev, context_lens=lens_override)
-    batch = PagedBatch(d.k_hist, d.v_hist, d.offsets, d.context_lens, d.num_blocks, cfg.block_size, d.free_order)
+    Q = args.queries
+    batch = PagedBatch(d.k_hist, d.v_hist, d.offsets, d.context_lens, d.num_blocks, cfg.block_size, d.free_order,
+                       new_tokens=Q)
     lens = d.context_lens
     q = d.q
+    if Q > 1:
+        gq = torch.Generator(device=dev).manual_seed(seed * 7919 + Q)
+        q = torch.randn((len(lens), Q, cfg.num_heads, cfg.head_dim), generator=gq, device=dev,
+                        dtype=torch.float32).to(d.q.dtype)
     out = torch.empty_like(q)
     P = cfg.partition_size
     batch.ensure_workspace(cfg.num_heads, P)
@@ -300,9 +342,14 @@ def run_native(args):
     torch.cuda.synchronize()
     pa.pa_get_device_error()
 
+    kernel = "verify" if Q > 1 else "decode"
+
     def step():
         batch.write_new_tokens()
-        batch.decode(out, q, cfg.scale, partition_size=P)
+        if Q > 1:
+            batch.verify(out, q, cfg.scale, partition_size=P)
+        else:
+            batch.decode(out, q, cfg.scale, partition_size=P)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -316,7 +363,7 @@ def run_native(args):
     clocks.start()
     time.sleep(0.3)
     launches0 = pa.launch_count()
-    pa.profile_begin(["decode"])          # events around the decode kernel only
+    pa.profile_begin([kernel])            # events around the attention kernel only
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -336,7 +383,7 @@ def run_native(args):
     err = pa.pa_get_device_error()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     ms = sum(step_ms) / len(step_ms)
-    dec_ms = prof["decode"][0] / max(1, prof["decode"][1])
+    dec_ms = prof[kernel][0] / max(1, prof[kernel][1])
     if world > 1:
         t = torch.tensor([ms, dec_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -344,7 +391,7 @@ def run_native(args):
 
     # ---- e2e: the same step from pinned host buffers through pa_step
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and Q == 1:
         S, Hq, D = q.shape
         host = {"q": q.cpu().pin_memory(), "k": batch.k_new.cpu().pin_memory(), "v": batch.v_new.cpu().pin_memory(),
                 "slot_mapping": batch.slot_mapping.cpu().pin_memory(),
@@ -383,9 +430,13 @@ def run_native(args):
                "tokens_per_s": world * len(lens) / (ems * 1e-3)}
 
     peak, peak_kind = measured_peaks()
-    dec_bytes = decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused")
+    if Q > 1:
+        dec_bytes = verify_kernel_bytes(cfg, lens, P, Q)
+        traffic = None
+    else:
+        dec_bytes = decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused")
+        traffic = recorded_traffic(args.workload)
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(args.workload)
     value = world * step_kv / (ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -399,12 +450,21 @@ def run_native(args):
         "tokens_per_s": world * len(lens) / (ms * 1e-3),
         "kernel_ms": {k: v[0] / max(1, v[1]) for k, v in prof.items() if v[1]},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": "decode_kernel", "algorithmic_bytes": dec_bytes,
+                     "traffic": traffic, "kernel": f"{kernel}_kernel", "algorithmic_bytes": dec_bytes,
                      "peak_source": peak_kind},
         "gpu_launches": int(launches), "device_error_flags": err, "wall_s": wall,
         "e2e": e2e, "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if Q > 1:
+        tpeak, tkind = measured_tensor_peak()
+        fl = verify_flops(cfg, lens, Q)
+        result["metric"] = VERIFY_METRIC
+        result["tokens_per_s"] = world * len(lens) * Q / (ms * 1e-3)
+        result["config"]["queries_per_seq"] = Q
+        result["tensor"] = {"flops_per_launch": fl, "achieved_tflops": fl / (dec_ms * 1e-3) / 1e12,
+                            "peak_tflops": tpeak, "frac": fl / (dec_ms * 1e-3) / 1e12 / tpeak,
+                            "peak_source": tkind, "note": "plain flops; P.V runs as two mma (16-bit value + remainder)"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and Q == 1:
         result["cpu_baseline"] = cpu_baseline(cfg, args.seed, lens, 1e9)
     if rank == 0:
         print(json.dumps(result))

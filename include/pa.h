@@ -147,6 +147,41 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     void* stream);
 
 /*
+ * Scratch bytes pa_verify needs (zero when every context fits one partition).
+ */
+size_t pa_verify_workspace_size(int num_seqs, int num_queries, int num_heads, int head_dim,
+                                int max_context_len, int partition_size);
+
+/*
+ * pa_verify -- multi-query paged attention: the target model's verification
+ * pass of speculative decoding ([P1] "大模型推理引擎高频优化：连续批处理、
+ * PagedAttention 与 KV Cache 实战拆解", section 5: a draft model proposes a
+ * handful of candidate tokens and the target model checks them in one
+ * parallel pass).  Every sequence brings num_queries (Q) query rows per head;
+ * their K/V must already be the last Q positions of its paged context (write
+ * them with pa_cache_write first).
+ *   out   device [num_seqs, Q, num_heads, head_dim] (written)
+ *   q     device [num_seqs, Q, num_heads, head_dim]
+ *   other arguments as for pa_decode.
+ * Query i of sequence s with n = context_lens[s] sits at position
+ * p = n - Q + i and attends to positions 0..p of its own sequence:
+ *   out[s][i][h] = sum_{t <= p} softmax_t(scale * q[s][i][h] . K_s[t][g]) V_s[t][g],
+ *   g = h / (num_heads / num_kv_heads)
+ * (Q = 1 is pa_decode).  A row with p < 0 (a context shorter than Q) is a zero
+ * row.  fp16 and bf16 only (tensor cores; fp32 returns PA_ERR_UNSUPPORTED);
+ * 1 <= Q <= 64.  Long contexts are split and merged as in pa_decode; the
+ * workspace (>= pa_verify_workspace_size bytes, 256-byte aligned) holds the
+ * partials.
+ */
+pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, float scale,
+                    int block_size, int num_kv_heads,
+                    int num_seqs, int num_queries, int num_heads, int head_dim, int max_blocks_per_seq,
+                    int max_context_len, int num_blocks, pa_dtype dtype,
+                    int partition_size, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
  * memory.  The pages have no counterpart to this call: it exists for users of
  * this library whose device memory is already spoken for (a serving engine
@@ -181,6 +216,28 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const
  */
 pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int num_pairs,
                          const pa_cache_desc* cache, void* stream);
+
+/*
+ * pa_swap_blocks -- move whole blocks between two pools of the same block
+ * shape (cache->block_size, num_kv_heads, head_dim, dtype), K and V alike
+ * ([P3] "大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置",
+ * section "生产部署注意事项": KV cache swapped out to CPU memory when GPU memory
+ * runs short and back in later).  Either pool may be device memory or PINNED
+ * host memory (cudaHostAlloc / cudaHostRegister; pageable host memory is
+ * rejected with PA_ERR_INVALID_ARG); a host pool is read or written in place
+ * by one kernel launch over the host link.
+ *   dst_k, dst_v   pools of dst_blocks blocks
+ *   src_k, src_v   pools of src_blocks blocks
+ *   pairs          int32 [num_pairs][2] of (source block, destination block),
+ *                  device or pinned host memory
+ * Destinations must be distinct and must not be read as sources in the same
+ * call.  Out-of-range ids are skipped and flagged (PA_DEVERR_BLOCK_ID).  The
+ * copy is asynchronous on `stream`; keep the host pool alive and unmodified
+ * until it completes.  cache->num_blocks is ignored.
+ */
+pa_status pa_swap_blocks(void* dst_k, void* dst_v, int dst_blocks, const void* src_k, const void* src_v,
+                         int src_blocks, const int32_t* pairs, int num_pairs, const pa_cache_desc* cache,
+                         void* stream);
 
 /*
  * pa_step -- one layer-step driven from HOST buffers: copies the step's inputs
@@ -266,7 +323,9 @@ typedef enum {
     PA_KERNEL_REDUCE = 2,        /* log-sum-exp merge of partitions */
     PA_KERNEL_PLAN = 3,          /* orders partitions longest-first */
     PA_KERNEL_COPY_BLOCKS = 4,
-    PA_KERNEL_COUNT = 5
+    PA_KERNEL_VERIFY = 5,        /* multi-query (verification) kernel */
+    PA_KERNEL_SWAP = 6,          /* block moves between device and host pools */
+    PA_KERNEL_COUNT = 7
 } pa_kernel_id;
 
 /* Number of kernels this library has launched in the process so far. */
@@ -376,6 +435,34 @@ pa_status pa_bm_allocate_prefix(pa_bm* bm, int64_t seq_id, const int32_t* tokens
  * from pa_bm_append_slot, has unknown tokens: its later blocks are not cached. */
 pa_status pa_bm_append_token(pa_bm* bm, int64_t seq_id, int32_t token, int64_t* slot,
                              int32_t* cow_src, int32_t* cow_dst);
+
+/* ---- host swap pool ([P3] "生产部署注意事项": KV cache moved out to CPU memory
+ * when GPU memory runs short, back in when it frees up) ----
+ *
+ * Size the host pool (block ids 0..num_cpu_blocks-1 on a LIFO free list, like
+ * the GPU list); not while a sequence is swapped out. */
+pa_status pa_bm_set_cpu_blocks(pa_bm* bm, int num_cpu_blocks);
+
+/* Swap a resident sequence out: every block it holds ALONE (count 1) moves to
+ * a host block, in logical order, and the GPU block goes back to the free
+ * list; shared blocks stay resident and referenced.  pairs receives
+ * *n (gpu, cpu) pairs ([n][2], cap pairs of room) for pa_swap_blocks, which
+ * must run before the freed GPU blocks are written again.  All or nothing:
+ * PA_ERR_NO_BLOCKS when the host pool is short, PA_ERR_INVALID_ARG when cap
+ * is short (nothing changes; *n tells the need); PA_ERR_UNSUPPORTED with the
+ * prefix cache on.  A swapped-out sequence cannot append, fork, pack or give
+ * slots until it is swapped in; pa_bm_free releases it. */
+pa_status pa_bm_swap_out(pa_bm* bm, int64_t seq_id, int32_t* pairs, int cap, int* n);
+
+/* Swap a sequence back in: a fresh GPU block (taken from the free list) for
+ * each of its host blocks, in logical order; pairs receives the (cpu, gpu)
+ * copies.  All or nothing, as for pa_bm_swap_out. */
+pa_status pa_bm_swap_in(pa_bm* bm, int64_t seq_id, int32_t* pairs, int cap, int* n);
+
+/* *swapped = 1 while the sequence is swapped out; the host free list from
+ * bottom to top. */
+pa_status pa_bm_swapped(const pa_bm* bm, int64_t seq_id, int* swapped);
+pa_status pa_bm_cpu_free_list(const pa_bm* bm, int32_t* out, int cap, int* n);
 
 /* Cached blocks (in use or not), evictable blocks (cached, count zero),
  * full blocks found and full blocks probed by pa_bm_allocate_prefix so far;

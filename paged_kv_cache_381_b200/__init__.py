@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3:
                 4: "PA_ERR_CUDA", 5: "PA_ERR_DEVICE"}
 PA_ERR_NO_BLOCKS = 3
 DEVERR_SLOT, DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
-KERNELS = ("cache_write", "decode", "reduce", "plan", "copy_blocks")
+KERNELS = ("cache_write", "decode", "reduce", "plan", "copy_blocks", "verify", "swap")
 DEFAULT_PARTITION = 512
 
 
@@ -101,6 +101,31 @@ def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
     _check(st, "pa_copy_blocks")
 
 
+def _reachable(t, name):
+    """Device tensor or pinned host tensor (both reachable from kernels)."""
+    if not t.is_contiguous() or not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor or pinned host tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, pairs, stream=None):
+    """Copy whole blocks between pools of one block shape (device or pinned
+    host memory); pairs: int32 [n, 2] of (source, destination) block ids on
+    the device or in pinned host memory."""
+    import torch
+    if pairs.dtype != torch.int32:
+        raise TypeError("pairs must be int32")
+    n = int(pairs.numel() // 2)
+    if n == 0:
+        return
+    dev = dst_k if dst_k.is_cuda else src_k
+    desc = _native.CacheDesc(0, dst_k.shape[1], dst_k.shape[2], dst_k.shape[3], _dtype_code(dst_k))
+    st = lib().pa_swap_blocks(_reachable(dst_k, "dst_k"), _reachable(dst_v, "dst_v"), int(dst_k.shape[0]),
+                              _reachable(src_k, "src_k"), _reachable(src_v, "src_v"), int(src_k.shape[0]),
+                              _reachable(pairs, "pairs"), n, ctypes.byref(desc), _stream(dev, stream))
+    _check(st, "pa_swap_blocks")
+
+
 def pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len, partition_size=0):
     return int(lib().pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len, partition_size))
 
@@ -137,6 +162,44 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block
                          int(block_size), int(num_kv_heads), S, Hq, D, maxb, int(max_context_len), nb,
                          _dtype_code(q), int(partition_size), ws_ptr, ws_bytes, _stream(q, stream))
     _check(st, "pa_decode")
+    return out
+
+
+def pa_verify_workspace_size(num_seqs, num_queries, num_heads, head_dim, max_context_len, partition_size=0):
+    return int(lib().pa_verify_workspace_size(num_seqs, num_queries, num_heads, head_dim, max_context_len,
+                                              partition_size))
+
+
+def pa_verify(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size=None, num_kv_heads=None,
+              max_context_len=None, partition_size=0, workspace=None, stream=None):
+    """Multi-query paged attention (speculative verification pass).
+
+    q, out: [S, Q, Hq, D]; the K/V of the Q query tokens are the last Q
+    positions of each context.  Other arguments as for pa_decode.
+    """
+    import torch
+    nb, bs, hkv, d = k_cache.shape
+    block_size = bs if block_size is None else block_size
+    num_kv_heads = hkv if num_kv_heads is None else num_kv_heads
+    S, Q, Hq, D = q.shape
+    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 1
+    if max_context_len is None:
+        max_context_len = maxb * block_size
+    need = pa_verify_workspace_size(S, Q, Hq, D, max_context_len, partition_size)
+    ws_ptr, ws_bytes = ctypes.c_void_p(0), 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        if workspace.numel() < need:
+            raise ValueError(f"workspace needs {need} bytes")
+        ws_ptr, ws_bytes = ctypes.c_void_p(workspace.data_ptr()), int(workspace.numel())
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    st = lib().pa_verify(_dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                         _dev(block_tables, "block_tables"), _dev(context_lens, "context_lens"), float(scale),
+                         int(block_size), int(num_kv_heads), S, Q, Hq, D, maxb, int(max_context_len), nb,
+                         _dtype_code(q), int(partition_size), ws_ptr, ws_bytes, _stream(q, stream))
+    _check(st, "pa_verify")
     return out
 
 
@@ -345,6 +408,42 @@ class BlockManager:
         h, f = ctypes.c_int64(), ctypes.c_int64()
         _check(lib().pa_bm_usage(self._h, ctypes.byref(h), ctypes.byref(f)), "pa_bm_usage")
         return h.value, f.value
+
+    # ---- host swap pool (pa_bm_set_cpu_blocks and friends) ----
+
+    def set_cpu_blocks(self, n):
+        _check(lib().pa_bm_set_cpu_blocks(self._h, int(n)), "pa_bm_set_cpu_blocks")
+
+    def _swap(self, fn, seq, what):
+        n = ctypes.c_int()
+        st = fn(self._h, seq, ctypes.c_void_p(0), 0, ctypes.byref(n))
+        if st == 0:                       # nothing to move
+            return np.zeros((0, 2), dtype=np.int32)
+        if n.value <= 0:
+            _check(st, what)
+        out = np.zeros((n.value, 2), dtype=np.int32)
+        _check(fn(self._h, seq, _ptr(out), n.value, ctypes.byref(n)), what)
+        return out
+
+    def swap_out(self, seq):
+        """(gpu, cpu) block pairs [n, 2] to copy device -> host."""
+        return self._swap(lib().pa_bm_swap_out, seq, "pa_bm_swap_out")
+
+    def swap_in(self, seq):
+        """(cpu, gpu) block pairs [n, 2] to copy host -> device."""
+        return self._swap(lib().pa_bm_swap_in, seq, "pa_bm_swap_in")
+
+    def swapped(self, seq):
+        f = ctypes.c_int()
+        _check(lib().pa_bm_swapped(self._h, seq, ctypes.byref(f)), "pa_bm_swapped")
+        return bool(f.value)
+
+    def cpu_free_list(self):
+        n = ctypes.c_int()
+        lib().pa_bm_cpu_free_list(self._h, ctypes.c_void_p(0), 0, ctypes.byref(n))
+        out = np.zeros(max(n.value, 1), dtype=np.int32)
+        _check(lib().pa_bm_cpu_free_list(self._h, _ptr(out), out.size, ctypes.byref(n)), "pa_bm_cpu_free_list")
+        return out[:n.value].tolist()
 
     # ---- prefix cache (pa_bm_enable_prefix_cache and friends) ----
 

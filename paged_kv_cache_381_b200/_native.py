@@ -47,6 +47,10 @@ SIGNATURES = {
     "pa_decode_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "pa_decode": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int, c_int,
                           c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "pa_verify_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
+    "pa_verify": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int, c_int,
+                          c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_size_t,
+                          c_void_p]),
     "pa_decode_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int,
                                   c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p]),
     "pa_copy_blocks": (c_int, [c_void_p, c_void_p, c_void_p, c_int, P(CacheDesc), c_void_p]),
@@ -74,6 +78,13 @@ SIGNATURES = {
     "pa_bm_free_list": (c_int, [c_void_p, c_void_p, c_int, P(c_int)]),
     "pa_bm_pack": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
     "pa_bm_usage": (c_int, [c_void_p, P(c_int64), P(c_int64)]),
+    "pa_bm_set_cpu_blocks": (c_int, [c_void_p, c_int]),
+    "pa_bm_swap_out": (c_int, [c_void_p, c_int64, c_void_p, c_int, P(c_int)]),
+    "pa_bm_swap_in": (c_int, [c_void_p, c_int64, c_void_p, c_int, P(c_int)]),
+    "pa_bm_swapped": (c_int, [c_void_p, c_int64, P(c_int)]),
+    "pa_bm_cpu_free_list": (c_int, [c_void_p, c_void_p, c_int, P(c_int)]),
+    "pa_swap_blocks": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_int, P(CacheDesc),
+                               c_void_p]),
     "pa_bm_enable_prefix_cache": (c_int, [c_void_p, c_int]),
     "pa_bm_allocate_prefix": (c_int, [c_void_p, c_int64, c_void_p, c_int, P(c_int)]),
     "pa_bm_append_token": (c_int, [c_void_p, c_int64, c_int32, P(c_int64), P(c_int32), P(c_int32)]),

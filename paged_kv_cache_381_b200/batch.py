@@ -8,17 +8,22 @@ their slots for the decode step, which writes them and then decodes:
 
     batch.write_new_tokens()      # pa_cache_write of one token per sequence
     batch.decode(out)             # pa_decode over the block tables
+
+With ``new_tokens = Q > 1`` the last Q rows of each history are held back
+instead (a speculative step's candidate tokens), written together by
+``write_new_tokens`` and attended by ``verify`` (pa_verify).
 """
 
 import numpy as np
 import torch
 
-from . import BlockManager, pa_cache_write, pa_decode, pa_decode_workspace_size
+from . import (BlockManager, pa_cache_write, pa_decode, pa_decode_workspace_size, pa_verify,
+               pa_verify_workspace_size)
 
 
 class PagedBatch:
     def __init__(self, k_hist, v_hist, offsets, context_lens, num_blocks, block_size, free_order=None,
-                 table_width=None, fill=None):
+                 table_width=None, fill=None, new_tokens=1):
         dev = k_hist.device
         self.lens = np.asarray(context_lens, dtype=np.int64)
         self.offsets = np.asarray(offsets, dtype=np.int64)
@@ -37,20 +42,22 @@ class PagedBatch:
             self.v_cache = torch.empty(shape, dtype=k_hist.dtype, device=dev)
         else:
             self.k_cache, self.v_cache = fill(shape)
-        # prefill: every history row except each sequence's newest one
+        # prefill: every history row except each sequence's newest Q ones, which the
+        # step writes (rows ordered [sequence][i]; slot -1 where a context is shorter than Q)
+        Q = self.new_tokens = int(new_tokens)
         rows, slots = [], []
         newest_rows, newest_slots = [], []
         for s in range(S):
             n = int(self.lens[s])
-            if n == 0:
-                newest_rows.append(-1)
-                newest_slots.append(-1)
-                continue
-            sl = self.bm.slots(s, 0, n)
-            rows.append(np.arange(self.offsets[s], self.offsets[s] + n - 1))
-            slots.append(sl[:-1])
-            newest_rows.append(int(self.offsets[s] + n - 1))
-            newest_slots.append(int(sl[-1]))
+            sl = self.bm.slots(s, 0, n) if n else np.zeros(0, np.int64)
+            k = min(n, Q)
+            if n > k:
+                rows.append(np.arange(self.offsets[s], self.offsets[s] + n - k))
+                slots.append(sl[:n - k])
+            for i in range(Q):
+                p = n - Q + i
+                newest_rows.append(int(self.offsets[s] + p) if p >= 0 else -1)
+                newest_slots.append(int(sl[p]) if p >= 0 else -1)
         if rows:
             r = torch.from_numpy(np.concatenate(rows)).to(dev)
             sm = torch.from_numpy(np.concatenate(slots).astype(np.int64)).to(dev)
@@ -75,7 +82,12 @@ class PagedBatch:
         pa_cache_write(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping, stream=stream)
 
     def ensure_workspace(self, num_heads, partition_size=0):
-        need = pa_decode_workspace_size(self.num_seqs, num_heads, self.head_dim, self.max_context_len, partition_size)
+        if self.new_tokens > 1:
+            need = pa_verify_workspace_size(self.num_seqs, self.new_tokens, num_heads, self.head_dim,
+                                            self.max_context_len, partition_size)
+        else:
+            need = pa_decode_workspace_size(self.num_seqs, num_heads, self.head_dim, self.max_context_len,
+                                            partition_size)
         if need and (self.workspace is None or self.workspace.numel() < need):
             self.workspace = torch.empty(need, dtype=torch.uint8, device=self.k_cache.device)
         return self.workspace
@@ -83,5 +95,12 @@ class PagedBatch:
     def decode(self, out, q, scale, partition_size=0, stream=None):
         ws = self.ensure_workspace(q.shape[1], partition_size)
         return pa_decode(out, q, self.k_cache, self.v_cache, self.block_tables, self.context_lens, scale,
+                         self.block_size, self.num_kv_heads, max_context_len=self.max_context_len,
+                         partition_size=partition_size, workspace=ws, stream=stream)
+
+    def verify(self, out, q, scale, partition_size=0, stream=None):
+        """q, out: [S, Q, Hq, D] with Q = new_tokens."""
+        ws = self.ensure_workspace(q.shape[2], partition_size)
+        return pa_verify(out, q, self.k_cache, self.v_cache, self.block_tables, self.context_lens, scale,
                          self.block_size, self.num_kv_heads, max_context_len=self.max_context_len,
                          partition_size=partition_size, workspace=ws, stream=stream)

@@ -61,4 +61,34 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_
     for (int64_t i = threadIdx.x; i < block_vecs; i += blockDim.x) d[i] = s[i];
 }
 
+// Swap copies between two pools of the same block shape, either of which may
+// be pinned host memory reached over the host link (the kernel reads or writes
+// it in place, so one launch moves every block of a swap; many 16-byte
+// accesses in flight per thread keep the link busy).  grid (num_pairs, 2):
+// blockIdx.y selects the K or V pool; pairs[i] = (source block, destination
+// block); ids outside their pool are skipped and flagged.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(uint4* __restrict__ dst_k, uint4* __restrict__ dst_v,
+                                                          int dst_blocks, const uint4* __restrict__ src_k,
+                                                          const uint4* __restrict__ src_v, int src_blocks,
+                                                          const int32_t* __restrict__ pairs, int64_t block_vecs) {
+    const int pair = blockIdx.x;
+    const int32_t src = pairs[2 * pair];
+    const int32_t dst = pairs[2 * pair + 1];
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) flag_error(PA_DEVERR_BLOCK_ID);
+        return;
+    }
+    const uint4* s = (blockIdx.y == 0 ? src_k : src_v) + (int64_t)src * block_vecs;
+    uint4* d = (blockIdx.y == 0 ? dst_k : dst_v) + (int64_t)dst * block_vecs;
+    int64_t i = threadIdx.x;
+    for (; i + 3 * 256 < block_vecs; i += 4 * 256) {
+        const uint4 a = s[i], b = s[i + 256], c = s[i + 512], e = s[i + 768];
+        d[i] = a;
+        d[i + 256] = b;
+        d[i + 512] = c;
+        d[i + 768] = e;
+    }
+    for (; i < block_vecs; i += 256) d[i] = s[i];
+}
+
 }  // namespace pa_dev

@@ -71,6 +71,7 @@ struct DecodeArgs {
     float* part_o;             // [num_seqs * num_heads, max_partitions, head_dim]
     int* merge_count;          // split mode, fused merge: finished partitions per (seq, kv head, chunk);
                                // nullptr: partitions are merged by reduce_kernel instead
+    int num_queries;           // query rows per sequence and head (1: decode; > 1: verification pass)
 };
 
 struct WorkItem {
@@ -846,8 +847,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, int2* pl
 
 // Log-sum-exp merge of a sequence's partitions (base-2 units): with
 // M = max_i m_i, w_i = 2^(m_i - M):  out = sum_i w_i o_i / sum_i w_i l_i.
-// One warp per (sequence, query head); sequences with one partition were
-// finished by the decode kernel.
+// One warp per (sequence, query head) -- for the verification pass, per
+// (sequence, query row, head) with num_heads = rows x heads; sequences with one
+// partition were finished by the attention kernel.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) reduce_kernel(const DecodeArgs a) {
     using Tr = ElemTraits<T>;
@@ -906,8 +908,10 @@ __global__ void __launch_bounds__(128) reduce_kernel(const DecodeArgs a) {
         }
     }
     T* out = static_cast<T*>(a.out) + row * D + lane * PER;
+    // L == 0 only for a verification row that sees no token (context shorter
+    // than the query rows): a zero row, as for an empty context
 #pragma unroll
-    for (int j = 0; j < PER; ++j) out[j] = Tr::from_float(o[j] / L);
+    for (int j = 0; j < PER; ++j) out[j] = Tr::from_float(L > 0.f ? o[j] / L : 0.f);
 }
 
 }  // namespace pa_dev

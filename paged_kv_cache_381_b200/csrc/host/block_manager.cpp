@@ -27,6 +27,14 @@
 //  only under a registered parent (or as a first block), and free_seq puts a
 //  sequence's cached blocks on the LRU list last block first, so a child is
 //  always evicted before its parent and no key can name a reused parent.
+//
+//  Swap ("大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置", section
+//  "生产部署注意事项": when GPU memory runs short, requests' KV cache moves out to
+//  CPU memory and back when GPU memory is free): a host pool of equal blocks
+//  on its own LIFO list.  swap_out moves the blocks a sequence holds alone, in
+//  logical order, and frees their GPU blocks; shared blocks stay resident and
+//  referenced.  swap_in takes fresh GPU blocks for them.  Both are all or
+//  nothing and report the block copies the caller runs.
 
 #include "block_manager.hpp"
 
@@ -171,7 +179,7 @@ pa_status BlockManager::allocate_prefix(int64_t seq, const int32_t* tokens, int 
 
 pa_status BlockManager::fork(int64_t parent, int64_t child) {
     auto it = seqs_.find(parent);
-    if (it == seqs_.end() || seqs_.count(child)) return PA_ERR_INVALID_ARG;
+    if (it == seqs_.end() || seqs_.count(child) || it->second.swapped) return PA_ERR_INVALID_ARG;
     Seq c = it->second;
     for (int32_t b : c.table) ref_[b] += 1;
     seqs_.emplace(child, std::move(c));
@@ -189,7 +197,7 @@ pa_status BlockManager::append_token(int64_t seq, int32_t token, int64_t* slot, 
 pa_status BlockManager::append(int64_t seq, int32_t token, bool known, int64_t* slot, int32_t* cow_src,
                                int32_t* cow_dst) {
     auto it = seqs_.find(seq);
-    if (it == seqs_.end()) return PA_ERR_INVALID_ARG;
+    if (it == seqs_.end() || it->second.swapped) return PA_ERR_INVALID_ARG;
     Seq& s = it->second;
     const int64_t pos = s.ctx;
     int32_t src = -1, dst = -1;
@@ -230,6 +238,22 @@ pa_status BlockManager::free_seq(int64_t seq) {
     auto it = seqs_.find(seq);
     if (it == seqs_.end()) return PA_ERR_INVALID_ARG;
     std::vector<int32_t> cached;
+    const Seq& sq = it->second;
+    if (sq.swapped) {
+        // host blocks go back to their list; shared GPU references are dropped
+        for (size_t j = 0; j < sq.table.size(); ++j) {
+            const int32_t b = sq.table[j];
+            if (sq.on_cpu[j]) {
+                cpu_free_.push_back(b);
+            } else {
+                if (ref_[b] <= 0) return PA_ERR_INVALID_ARG;
+                if (--ref_[b] == 0) free_.push_back(b);
+            }
+        }
+        --num_swapped_;
+        seqs_.erase(it);
+        return PA_OK;
+    }
     for (int32_t b : it->second.table) {
         if (ref_[b] <= 0) return PA_ERR_INVALID_ARG;  // corrupted counts; never expected
         if (--ref_[b] == 0) {
@@ -244,12 +268,90 @@ pa_status BlockManager::free_seq(int64_t seq) {
     return PA_OK;
 }
 
+pa_status BlockManager::set_cpu_blocks(int n) {
+    if (n < 0 || num_swapped_ > 0) return PA_ERR_INVALID_ARG;
+    num_cpu_blocks_ = n;
+    cpu_free_.clear();
+    for (int i = 0; i < n; ++i) cpu_free_.push_back(i);
+    return PA_OK;
+}
+
+bool BlockManager::swapped(int64_t seq) const {
+    const Seq* s = find(seq);
+    return s && s->swapped;
+}
+
+int BlockManager::swap_out_need(int64_t seq) const {
+    const Seq* s = find(seq);
+    if (!s || s->swapped) return -1;
+    int n = 0;
+    for (int32_t b : s->table) n += ref_[b] == 1;
+    return n;
+}
+
+int BlockManager::swap_in_need(int64_t seq) const {
+    const Seq* s = find(seq);
+    if (!s || !s->swapped) return -1;
+    int n = 0;
+    for (char c : s->on_cpu) n += c != 0;
+    return n;
+}
+
+pa_status BlockManager::swap_out(int64_t seq, std::vector<int32_t>& pairs) {
+    if (prefix_cache_) return PA_ERR_UNSUPPORTED;
+    const int need = swap_out_need(seq);
+    if (need < 0) return PA_ERR_INVALID_ARG;
+    if (need > (int)cpu_free_.size()) return PA_ERR_NO_BLOCKS;
+    Seq& s = seqs_[seq];
+    s.swapped = true;
+    s.on_cpu.assign(s.table.size(), 0);
+    pairs.clear();
+    for (size_t j = 0; j < s.table.size(); ++j) {
+        const int32_t g = s.table[j];
+        if (ref_[g] != 1) continue;              // shared: stays resident, still referenced
+        const int32_t c = cpu_free_.back();
+        cpu_free_.pop_back();
+        pairs.push_back(g);
+        pairs.push_back(c);
+        ref_[g] = 0;
+        free_.push_back(g);
+        s.table[j] = c;
+        s.on_cpu[j] = 1;
+    }
+    ++num_swapped_;
+    return PA_OK;
+}
+
+pa_status BlockManager::swap_in(int64_t seq, std::vector<int32_t>& pairs) {
+    const int need = swap_in_need(seq);
+    if (need < 0) return PA_ERR_INVALID_ARG;
+    if (need > (int)free_.size()) return PA_ERR_NO_BLOCKS;
+    Seq& s = seqs_[seq];
+    pairs.clear();
+    for (size_t j = 0; j < s.table.size(); ++j) {
+        if (!s.on_cpu[j]) continue;
+        const int32_t c = s.table[j];
+        const int32_t g = free_.back();
+        free_.pop_back();
+        ref_[g] = 1;
+        pairs.push_back(c);
+        pairs.push_back(g);
+        cpu_free_.push_back(c);
+        s.table[j] = g;
+    }
+    s.on_cpu.clear();
+    s.swapped = false;
+    --num_swapped_;
+    return PA_OK;
+}
+
 void BlockManager::usage(int64_t* held_blocks, int64_t* filled_slots) const {
     // a shared block is counted once, filled up to the furthest of its holders
     std::vector<int32_t> fill(num_blocks_, 0);
     for (const auto& kv : seqs_) {
         const Seq& s = kv.second;
         for (size_t j = 0; j < s.table.size(); ++j) {
+            if (s.swapped && s.on_cpu[j]) continue;              // a host block
             int64_t f = s.ctx - (int64_t)j * block_size_;
             int32_t n = (int32_t)(f < block_size_ ? f : block_size_);
             if (n > fill[s.table[j]]) fill[s.table[j]] = n;
@@ -273,7 +375,7 @@ const BlockManager::Seq* BlockManager::find(int64_t seq) const {
 
 pa_status BlockManager::slots(int64_t seq, int64_t start, int64_t count, int64_t* out) const {
     const Seq* s = find(seq);
-    if (!s || start < 0 || count < 0) return PA_ERR_INVALID_ARG;
+    if (!s || s->swapped || start < 0 || count < 0) return PA_ERR_INVALID_ARG;
     if (start + count > (int64_t)s->table.size() * block_size_) return PA_ERR_INVALID_ARG;
     for (int64_t p = start; p < start + count; ++p)
         out[p - start] = (int64_t)s->table[p / block_size_] * block_size_ + p % block_size_;
@@ -365,7 +467,7 @@ pa_status pa_bm_pack(const pa_bm* bm, const int64_t* seq_ids, int n, int width, 
         return PA_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i) {
         const BlockManager::Seq* s = bm->impl.find(seq_ids[i]);
-        if (!s || (int)s->table.size() > width) return PA_ERR_INVALID_ARG;
+        if (!s || s->swapped || (int)s->table.size() > width) return PA_ERR_INVALID_ARG;
         int32_t* row = tables + (int64_t)i * width;
         int len = (int)s->table.size();
         for (int j = 0; j < width; ++j) row[j] = j < len ? s->table[j] : -1;
@@ -409,6 +511,47 @@ pa_status pa_bm_cache_stats(const pa_bm* bm, int* cached_blocks, int* evictable_
 pa_status pa_bm_usage(const pa_bm* bm, int64_t* held_blocks, int64_t* filled_slots) {
     if (!bm) return PA_ERR_INVALID_ARG;
     bm->impl.usage(held_blocks, filled_slots);
+    return PA_OK;
+}
+
+pa_status pa_bm_set_cpu_blocks(pa_bm* bm, int num_cpu_blocks) {
+    return bm ? bm->impl.set_cpu_blocks(num_cpu_blocks) : PA_ERR_INVALID_ARG;
+}
+
+static pa_status swap_common(pa_bm* bm, int64_t seq_id, int32_t* pairs, int cap, int* n, bool out) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    const int need = out ? bm->impl.swap_out_need(seq_id) : bm->impl.swap_in_need(seq_id);
+    if (need < 0) return PA_ERR_INVALID_ARG;
+    if (n) *n = need;
+    if (need > cap || (need > 0 && !pairs)) return PA_ERR_INVALID_ARG;   // nothing changed
+    std::vector<int32_t> p;
+    pa_status st = out ? bm->impl.swap_out(seq_id, p) : bm->impl.swap_in(seq_id, p);
+    if (st != PA_OK) return st;
+    for (size_t i = 0; i < p.size(); ++i) pairs[i] = p[i];
+    return PA_OK;
+}
+
+pa_status pa_bm_swap_out(pa_bm* bm, int64_t seq_id, int32_t* pairs, int cap, int* n) {
+    return swap_common(bm, seq_id, pairs, cap, n, true);
+}
+
+pa_status pa_bm_swap_in(pa_bm* bm, int64_t seq_id, int32_t* pairs, int cap, int* n) {
+    return swap_common(bm, seq_id, pairs, cap, n, false);
+}
+
+pa_status pa_bm_swapped(const pa_bm* bm, int64_t seq_id, int* swapped) {
+    if (!bm || !swapped || !bm->impl.find(seq_id)) return PA_ERR_INVALID_ARG;
+    *swapped = bm->impl.swapped(seq_id) ? 1 : 0;
+    return PA_OK;
+}
+
+pa_status pa_bm_cpu_free_list(const pa_bm* bm, int32_t* out, int cap, int* n) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    const auto& fl = bm->impl.cpu_free_list();
+    int len = (int)fl.size();
+    if (n) *n = len;
+    if (len > cap || (len > 0 && !out)) return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < len; ++i) out[i] = fl[i];
     return PA_OK;
 }
 

@@ -20,6 +20,8 @@ class BlockManager {
         int64_t ctx = 0;              // tokens held
         std::vector<int32_t> tail;    // token ids of the partly filled last block (prefix cache)
         bool tail_known = true;       // false once a token was appended without its id
+        bool swapped = false;         // swapped out to the host pool
+        std::vector<char> on_cpu;     // while swapped: per logical block, 1 = host block id
     };
 
     BlockManager(int num_blocks, int block_size, const int32_t* initial_free_order);
@@ -41,6 +43,15 @@ class BlockManager {
     int64_t hits() const { return hits_; }
     int64_t lookups() const { return lookups_; }
     const std::list<int32_t>& evictable() const { return lru_; }
+
+    // host swap pool
+    pa_status set_cpu_blocks(int n);
+    pa_status swap_out(int64_t seq, std::vector<int32_t>& pairs);   // (gpu, cpu) pairs
+    pa_status swap_in(int64_t seq, std::vector<int32_t>& pairs);    // (cpu, gpu) pairs
+    int swap_out_need(int64_t seq) const;                           // host blocks swap_out takes, or -1
+    int swap_in_need(int64_t seq) const;                            // GPU blocks swap_in takes, or -1
+    bool swapped(int64_t seq) const;
+    const std::vector<int32_t>& cpu_free_list() const { return cpu_free_; }
 
     // blocks held by live sequences, and their slots holding a token of some holder
     void usage(int64_t* held_blocks, int64_t* filled_slots) const;
@@ -73,6 +84,10 @@ class BlockManager {
     std::vector<std::list<int32_t>::iterator> lru_pos_;
     std::vector<char> in_lru_;
     int64_t hits_ = 0, lookups_ = 0;
+    // host swap pool: LIFO free list of host block ids
+    std::vector<int32_t> cpu_free_;
+    int num_cpu_blocks_ = 0;
+    int num_swapped_ = 0;
 };
 
 }  // namespace pa_host

@@ -13,6 +13,7 @@
 
 #include "device/cache_ops.cuh"
 #include "device/decode.cuh"
+#include "device/verify.cuh"
 #include "pa.h"
 
 namespace {
@@ -259,6 +260,32 @@ pa_status launch_reduce(const pa_dev::DecodeArgs& a, int D, cudaStream_t stream)
     return launch_dependent(pa_dev::reduce_kernel<T, 128>, dim3(grid), dim3(128), 0, stream, a);
 }
 
+template <typename T, int D>
+pa_status launch_verify(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int64_t pair_upper,
+                        cudaStream_t stream) {
+    using C = pa_dev::VerifyCfg<T, D>;
+    auto kern = pa_dev::verify_kernel<T, D>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    static std::atomic<uint64_t> configured{0};
+    static std::atomic<int> occ_of[kMaxDevices];
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) != cudaSuccess)
+            return PA_ERR_CUDA;
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, C::THREADS, C::SMEM) != cudaSuccess || occ <= 0)
+            return PA_ERR_CUDA;
+        if (dev < kMaxDevices) occ_of[dev].store(occ);
+        configured.fetch_or(bit);
+    }
+    const int occ = dev < kMaxDevices ? std::max(1, occ_of[dev].load()) : 1;
+    const int64_t items_upper = pair_upper * a.num_kv_heads * a.n_gchunks;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items_upper, (int64_t)device_sms(dev) * occ));
+    LaunchScope scope(PA_KERNEL_VERIFY, stream);
+    return launch_dependent(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream, a, tk, tv);
+}
+
 int query_chunk(int group, bool tensor) {
     if (tensor) return 8;                  // mma n = 8: one tile holds up to 8 queries
     int g = std::min(group, 8);
@@ -375,6 +402,37 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
     return launch_status();
 }
 
+pa_status pa_swap_blocks(void* dst_k, void* dst_v, int dst_blocks, const void* src_k, const void* src_v,
+                         int src_blocks, const int32_t* pairs, int num_pairs, const pa_cache_desc* cache,
+                         void* stream) {
+    if (!cache || cache->num_kv_heads <= 0 || !valid_dtype(cache->dtype)) return PA_ERR_INVALID_ARG;
+    if (!supported_block_size(cache->block_size) || !supported_head_dim(cache->head_dim)) return PA_ERR_UNSUPPORTED;
+    if (num_pairs < 0 || dst_blocks <= 0 || src_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!dst_k || !dst_v || !src_k || !src_v || !pairs) return PA_ERR_INVALID_ARG;
+    if (!aligned16(dst_k) || !aligned16(dst_v) || !aligned16(src_k) || !aligned16(src_v)) return PA_ERR_INVALID_ARG;
+    // every pointer must be reachable from the device: device memory or pinned host memory
+    const void* ptrs[5] = {dst_k, dst_v, src_k, src_v, pairs};
+    void* dptr[5];
+    for (int i = 0; i < 5; ++i) {
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, ptrs[i]) != cudaSuccess) {
+            cudaGetLastError();
+            return PA_ERR_INVALID_ARG;
+        }
+        if (at.type == cudaMemoryTypeUnregistered || !at.devicePointer) return PA_ERR_INVALID_ARG;
+        dptr[i] = at.devicePointer;      // the address through which kernels reach ptrs[i]
+    }
+    const int64_t block_vecs =
+        (int64_t)cache->block_size * cache->num_kv_heads * cache->head_dim * elem_bytes(cache->dtype) / 16;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    LaunchScope scope(PA_KERNEL_SWAP, s);
+    pa_dev::swap_blocks_kernel<<<dim3((unsigned)num_pairs, 2), 256, 0, s>>>(
+        static_cast<uint4*>(dptr[0]), static_cast<uint4*>(dptr[1]), dst_blocks, static_cast<const uint4*>(dptr[2]),
+        static_cast<const uint4*>(dptr[3]), src_blocks, static_cast<const int32_t*>(dptr[4]), block_vecs);
+    return launch_status();
+}
+
 size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_context_len, int partition_size) {
     const int P = resolve_partition(partition_size);
     if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 || !valid_partition(P)) return 0;
@@ -430,6 +488,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     a.num_blocks = num_blocks;
     a.partition_size = P;
     a.max_partitions = (int)maxP;
+    a.num_queries = 1;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (maxP > 1) {
@@ -473,6 +532,99 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
         case PA_F16: return launch_reduce<__half>(a, head_dim, s);
         default: return launch_reduce<__nv_bfloat16>(a, head_dim, s);
     }
+}
+
+size_t pa_verify_workspace_size(int num_seqs, int num_queries, int num_heads, int head_dim, int max_context_len,
+                                int partition_size) {
+    if (num_queries <= 0) return 0;
+    return pa_decode_workspace_size(num_seqs, num_queries * num_heads, head_dim, max_context_len, partition_size);
+}
+
+pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                    const int32_t* context_lens, float scale, int block_size, int num_kv_heads, int num_seqs,
+                    int num_queries, int num_heads, int head_dim, int max_blocks_per_seq, int max_context_len,
+                    int num_blocks, pa_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+        max_context_len < 0 || !valid_dtype(dtype) || !std::isfinite(scale) || num_queries <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (dtype == PA_F32 || num_queries > 64) return PA_ERR_UNSUPPORTED;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    const int P = resolve_partition(partition_size);
+    if (!valid_partition(P)) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+    if ((int64_t)num_blocks * block_size > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    const int64_t table_cap = (int64_t)max_blocks_per_seq * block_size;
+    const int64_t cap = std::min<int64_t>(max_context_len, table_cap);
+    if (cap > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
+    const int64_t maxP = partitions_for(cap, P);
+    if (maxP > kMaxPartitions) return PA_ERR_UNSUPPORTED;
+    const int group = num_heads / num_kv_heads;
+    const int rows = group * num_queries;
+    const int n_chunks = (rows + 63) / 64;
+    if ((int64_t)num_seqs * maxP * num_kv_heads * n_chunks > INT32_MAX) return PA_ERR_INVALID_ARG;
+    if ((int64_t)num_seqs * num_queries * num_heads > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
+
+    pa_dev::DecodeArgs a{};
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.num_seqs = num_seqs;
+    a.num_heads = num_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.group = group;
+    a.n_gchunks = n_chunks;
+    a.log2_bs = block_size == 8 ? 3 : block_size == 16 ? 4 : 5;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.ctx_cap = (int)cap;
+    a.num_blocks = num_blocks;
+    a.partition_size = P;
+    a.max_partitions = (int)maxP;
+    a.num_queries = num_queries;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (maxP > 1) {
+        // partial rows are [num_seqs][Q][num_heads]: the decode layout with Q x num_heads heads
+        const WsLayout L = ws_layout(num_seqs, (int64_t)num_queries * num_heads, head_dim, maxP);
+        if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return PA_ERR_INVALID_ARG;
+        char* ws = static_cast<char*>(workspace);
+        a.plan = reinterpret_cast<const int2*>(ws + L.plan);
+        a.plan_count = reinterpret_cast<const int*>(ws + L.count);
+        a.part_m = reinterpret_cast<float*>(ws + L.m);
+        a.part_l = reinterpret_cast<float*>(ws + L.l);
+        a.part_o = reinterpret_cast<float*>(ws + L.o);
+        a.merge_count = nullptr;
+        LaunchScope scope(PA_KERNEL_PLAN, s);
+        const int threads = std::min(1024, std::max(32, (num_seqs + 31) / 32 * 32));
+        if (launch_dependent(pa_dev::plan_kernel, dim3(1), dim3(threads), 2 * (maxP + 1) * sizeof(int), s, a,
+                             reinterpret_cast<int2*>(ws + L.plan), reinterpret_cast<int*>(ws + L.count),
+                             reinterpret_cast<int*>(ws + L.counters), 0) != PA_OK)
+            return PA_ERR_CUDA;
+    }
+    CUtensorMap tk, tv;
+    if (!encode_pool_map(&tk, k_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, block_size) ||
+        !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, block_size))
+        return PA_ERR_CUDA;
+    const int64_t pair_upper = (int64_t)num_seqs * maxP;
+    pa_status st;
+    if (dtype == PA_F16)
+        st = head_dim == 64 ? launch_verify<__half, 64>(a, tk, tv, pair_upper, s)
+                            : launch_verify<__half, 128>(a, tk, tv, pair_upper, s);
+    else
+        st = head_dim == 64 ? launch_verify<__nv_bfloat16, 64>(a, tk, tv, pair_upper, s)
+                            : launch_verify<__nv_bfloat16, 128>(a, tk, tv, pair_upper, s);
+    if (st != PA_OK || maxP <= 1) return st;
+    pa_dev::DecodeArgs r = a;               // the reduce sees rows [s][i][h] as num_queries * num_heads heads
+    r.num_heads = num_queries * num_heads;
+    return dtype == PA_F16 ? launch_reduce<__half>(r, head_dim, s) : launch_reduce<__nv_bfloat16>(r, head_dim, s);
 }
 
 pa_status pa_step(const pa_step_host* h, const pa_step_device* d, void* k_cache, void* v_cache,

@@ -3,6 +3,7 @@ include/pa.h declares, and its host block manager and scheduler agree
 bit-exactly with the oracle's Python models (golden traces and random op
 streams).  No CUDA call is made here."""
 
+import ctypes
 import json
 import os
 import re
@@ -256,3 +257,20 @@ def test_full_trace_host_side_lockstep(pa):
         preempted += len(a.preempted)
         mb.check()
     assert preempted > 0
+
+
+def test_verify_workspace_and_argument_rules(pa):
+    """pa_verify's scratch is decode's with Q x heads rows; its argument checks
+    return before any device work (so they run without a GPU)."""
+    lib = pa.lib()
+    assert pa.pa_verify_workspace_size(8, 6, 64, 128, 32768) == pa.pa_decode_workspace_size(8, 6 * 64, 128, 32768)
+    assert pa.pa_verify_workspace_size(8, 6, 64, 128, 512) == 0
+    assert pa.pa_verify_workspace_size(8, 0, 64, 128, 32768) == 0
+    nul = ctypes.c_void_p(0)
+    args = lambda Q, dt, hq=64: (nul, nul, nul, nul, nul, nul, 0.1, 16, 8, 4, Q, hq, 128, 8, 128, 64, dt, 0, nul, 0,
+                                 nul)
+    assert lib.pa_verify(*args(6, 0)) == 2            # fp32: unsupported (tensor cores only)
+    assert lib.pa_verify(*args(65, 2)) == 2           # more than 64 query rows per sequence
+    assert lib.pa_verify(*args(0, 2)) == 1            # no query rows
+    assert lib.pa_verify(*args(6, 2, hq=60)) == 1     # heads not a multiple of kv heads
+    assert lib.pa_verify(*args(6, 2)) == 1            # null pointers
