@@ -507,11 +507,31 @@ pa_status pa_sched_counts_get(const pa_sched* s, pa_sched_counts* c);
 /* The last step's record.  Any pointer may be NULL to skip that array.
  *   finished/admitted/preempted: sequence ids in event order.
  *   ops: num_ops entries in issue order; op_kind[i] = 0 for a cache write
- *        (a = seq, b = position, c = slot) or 1 for a copy-on-write block copy
- *        (a = src block, b = dst block, c = -1).  A copy must be applied after
- *        every earlier write and before every later one.  Ops made dead by a
- *        preemption in the same step are not listed, so no slot appears twice.
+ *        (a = seq, b = position, c = slot), 1 for a copy-on-write block copy
+ *        (a = src block, b = dst block, c = -1), and with preemption by swap
+ *        2 for a swap-out copy (a = GPU block, b = host block) or 3 for a
+ *        swap-in copy (a = host block, b = GPU block).  Ops apply in issue
+ *        order: a copy after every earlier write and before every later one.
+ *        Ops made dead by a preemption in the same step are not listed, so no
+ *        slot appears twice within a run of consecutive writes.
  *   running/context_lens: the batch to decode, in admission order. */
+/* Preemption mode ([P3] "大模型推理显存优化实战：PagedAttention机制原理与vLLM连续
+ * 批处理配置", section "生产部署注意事项"): PA_PREEMPT_RECOMPUTE (default) frees a
+ * victim's blocks and re-writes its history on re-admission; PA_PREEMPT_SWAP
+ * swaps it out to the block manager's host pool when its private blocks fit
+ * (else recomputes) and swaps it back in, before any new admission, once its
+ * host blocks + 1 fit the step's budget.  Swapped sequences keep their
+ * progress and come back in FIFO order. */
+#define PA_PREEMPT_RECOMPUTE 0
+#define PA_PREEMPT_SWAP 1
+pa_status pa_sched_set_preemption(pa_sched* s, int mode);
+
+/* The last step's swap events: ids swapped out and in (in event order), and
+ * the sequences currently waiting swapped out. */
+pa_status pa_sched_swap_counts(const pa_sched* s, int* num_swapped_out, int* num_swapped_in,
+                               int* num_swapped);
+pa_status pa_sched_swap_record(const pa_sched* s, int64_t* swapped_out, int64_t* swapped_in);
+
 pa_status pa_sched_record(const pa_sched* s, int64_t* finished, int64_t* admitted,
                           int64_t* preempted, int32_t* op_kind, int64_t* op_a, int64_t* op_b,
                           int64_t* op_c, int64_t* running, int32_t* context_lens);

@@ -38,6 +38,27 @@ preemption frees blocks, every op of the step that targets a freed block (a
 write into it, a copy into it) is dropped from the record: that work is dead,
 and a freed block can be taken again later in the same step, so keeping it
 would list one slot twice.  Within a step every slot is written at most once.
+
+Preemption by swap (``preempt="swap"``, with a ``SwappingBlockManager``; [P3]
+"大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置", section
+"生产部署注意事项": KV cache moved out to CPU memory when GPU memory runs short
+and back in later), readings adopted:
+
+* A victim whose privately held blocks fit the host pool is swapped out
+  instead of freed: ("so", gpu, cpu) copies join ``ops`` right there, the
+  victim keeps its progress and joins the FIFO swapped queue.  Its writes of
+  this step stay (the copies carry them out).  When the host pool is short,
+  the victim is recomputed as above.
+* Before admission, swapped sequences come back first, in queue order, each
+  needing its host blocks + 1 (its next token) from the step's budget:
+  ("si", cpu, gpu) copies, and it rejoins the running batch.  New requests are
+  admitted only once the swapped queue is empty.
+* A recompute preemption drops the dead ops of the step as above ("so" ops
+  target host blocks and always stay).  A preemption happens only when no
+  GPU block is free, so at that moment every block a swap-out freed earlier
+  in the step has been taken again: only the recomputed victim's own ops
+  become dead.  Ops run in issue order; consecutive writes form one launch,
+  and within one such run every slot is distinct.
 """
 
 from dataclasses import dataclass, field
@@ -76,6 +97,9 @@ class StepRecord:
     writes: list = field(default_factory=list)      # (seq, position, slot)
     cow: list = field(default_factory=list)         # (src, dst)
     ops: list = field(default_factory=list)         # ("w", seq, pos, slot) | ("c", src, dst)
+                                                    # | ("so", gpu, cpu) | ("si", cpu, gpu)
+    swapped_out: list = field(default_factory=list)
+    swapped_in: list = field(default_factory=list)
     running: list = field(default_factory=list)     # seq ids, admission order
     context_lens: list = field(default_factory=list)
 
@@ -87,18 +111,30 @@ class StepRecord:
         self.cow.append((src, dst))
         self.ops.append(("c", src, dst))
 
+    def swap(self, kind, a, b):
+        self.ops.append((kind, a, b))
+
     def drop_dead(self, bm):
-        """Remove ops whose target block is back on the free list."""
+        """Remove ops whose target GPU block is back on the free list."""
         bs = bm.block_size
-        live = lambda op: bm.ref[op[3] // bs if op[0] == "w" else op[2]] > 0
+
+        def live(op):
+            if op[0] == "so":                     # targets a host block
+                return True
+            return bm.ref[op[3] // bs if op[0] == "w" else op[2]] > 0
+
         self.ops = [op for op in self.ops if live(op)]
         self.writes = [(o[1], o[2], o[3]) for o in self.ops if o[0] == "w"]
         self.cow = [(o[1], o[2]) for o in self.ops if o[0] == "c"]
 
 
 class Scheduler:
-    def __init__(self, bm, max_running, prefix_seq=-1):
+    def __init__(self, bm, max_running, prefix_seq=-1, preempt="recompute"):
+        if preempt not in ("recompute", "swap"):
+            raise ValueError(preempt)
         self.bm = bm
+        self.preempt = preempt
+        self.swapped = []          # swapped-out sequences, FIFO
         self.max_running = int(max_running)
         self.prefix_seq = prefix_seq
         self.prefix_len = bm.context_len(prefix_seq) if prefix_seq >= 0 else 0
@@ -147,8 +183,21 @@ class Scheduler:
 
     def _preempt_last(self, rec):
         victim = self.running.pop()
-        self.bm.free(victim.seq_id)
-        rec.drop_dead(self.bm)
+        bm = self.bm
+        if self.preempt == "swap":
+            try:
+                pairs = bm.swap_out(victim.seq_id)
+            except NoBlocks:
+                pairs = None
+            if pairs is not None:
+                for g, c in pairs:
+                    rec.swap("so", g, c)
+                self.swapped.append(victim)
+                rec.swapped_out.append(victim.seq_id)
+                rec.preempted.append(victim.seq_id)
+                return victim
+        bm.free(victim.seq_id)
+        rec.drop_dead(bm)
         self.waiting.insert(0, victim)
         rec.preempted.append(victim.seq_id)
         return victim
@@ -165,9 +214,21 @@ class Scheduler:
             else:
                 keep.append(s)
         self.running = keep
-        # 2. admit (FCFS, stop at the first request that does not fit)
+        # 2. swapped sequences come back first, then admission (FCFS, stop at the
+        # first request that does not fit), only once none is left swapped out
         budget = bm.num_free
-        while self.waiting and budget > 0 and len(self.running) < self.max_running:
+        while self.swapped and len(self.running) < self.max_running:
+            s = self.swapped[0]
+            need = sum(bm.on_cpu[s.seq_id]) + 1
+            if need > budget:
+                break
+            self.swapped.pop(0)
+            budget -= need
+            for c, g in bm.swap_in(s.seq_id):
+                rec.swap("si", c, g)
+            self.running.append(s)
+            rec.swapped_in.append(s.seq_id)
+        while not self.swapped and self.waiting and budget > 0 and len(self.running) < self.max_running:
             s = self.waiting[0]
             need = self._required(s)
             if need > budget:

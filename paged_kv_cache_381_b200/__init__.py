@@ -483,10 +483,12 @@ class BlockManager:
 class Scheduler:
     """Iteration-level batching over a BlockManager (pa_sched_*)."""
 
-    def __init__(self, bm, max_running, prefix_seq=-1):
+    def __init__(self, bm, max_running, prefix_seq=-1, preempt="recompute"):
         self.bm = bm           # keeps the block manager alive
         self._h = ctypes.c_void_p()
         _check(lib().pa_sched_create(bm.handle, max_running, prefix_seq, ctypes.byref(self._h)), "pa_sched_create")
+        _check(lib().pa_sched_set_preemption(self._h, {"recompute": 0, "swap": 1}[preempt]),
+               "pa_sched_set_preemption")
 
     def __del__(self):
         h = getattr(self, "_h", None)
@@ -512,7 +514,14 @@ class Scheduler:
         ctx = np.zeros(c.num_running, np.int32)
         _check(lib().pa_sched_record(self._h, _ptr(fin), _ptr(adm), _ptr(pre), _ptr(kind), _ptr(oa), _ptr(ob),
                                      _ptr(oc), _ptr(run), _ptr(ctx)), "pa_sched_record")
-        ops = [("w", int(a), int(b), int(cc)) if k == 0 else ("c", int(a), int(b))
+        names = {1: "c", 2: "so", 3: "si"}
+        ops = [("w", int(a), int(b), int(cc)) if k == 0 else (names[k], int(a), int(b))
                for k, a, b, cc in zip(kind.tolist(), oa.tolist(), ob.tolist(), oc.tolist())]
+        n_out, n_in, n_q = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        _check(lib().pa_sched_swap_counts(self._h, ctypes.byref(n_out), ctypes.byref(n_in), ctypes.byref(n_q)),
+               "pa_sched_swap_counts")
+        so, si = np.zeros(n_out.value, np.int64), np.zeros(n_in.value, np.int64)
+        _check(lib().pa_sched_swap_record(self._h, _ptr(so), _ptr(si)), "pa_sched_swap_record")
         return {"finished": fin.tolist(), "admitted": adm.tolist(), "preempted": pre.tolist(), "ops": ops,
-                "running": run.tolist(), "context_lens": ctx.tolist(), "num_waiting": c.num_waiting}
+                "running": run.tolist(), "context_lens": ctx.tolist(), "num_waiting": c.num_waiting,
+                "swapped_out": so.tolist(), "swapped_in": si.tolist(), "num_swapped": n_q.value}

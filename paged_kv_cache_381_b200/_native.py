@@ -94,6 +94,9 @@ SIGNATURES = {
     "pa_sched_destroy": (None, [c_void_p]),
     "pa_sched_add_request": (c_int, [c_void_p, c_int64, c_int, c_int, c_int, c_int64, c_int]),
     "pa_sched_step": (c_int, [c_void_p]),
+    "pa_sched_set_preemption": (c_int, [c_void_p, c_int]),
+    "pa_sched_swap_counts": (c_int, [c_void_p, P(c_int), P(c_int), P(c_int)]),
+    "pa_sched_swap_record": (c_int, [c_void_p, c_void_p, c_void_p]),
     "pa_sched_counts_get": (c_int, [c_void_p, P(SchedCounts)]),
     "pa_sched_record": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_void_p, c_void_p, c_void_p]),

@@ -62,6 +62,11 @@ struct VerifyCfg {
     static constexpr int OFF_RED = ((OFF_STATS + (2 * NCW * 16 + 4) * 4) + 127) / 128 * 128;
     static constexpr int RED_STRIDE = D + 8;                // floats per row (spreads banks)
     static constexpr int RED_BYTES = NCW * 16 * RED_STRIDE * 4;
+    // The item's query rows wait in shared memory (not registers) while its
+    // slots stream by, in the region the epilogue later uses for the warps'
+    // partial outputs; rows padded by 16 bytes so ldmatrix rows spread over banks.
+    static constexpr int Q_STRIDE = D * ELT + 16;
+    static_assert(ROWS * Q_STRIDE <= RED_BYTES, "query tile must fit the merge buffer");
     static constexpr size_t SMEM = 1024 + (size_t)OFF_RED + RED_BYTES;
     static_assert(ELT == 2, "tensor path: fp16 / bf16");
     static_assert(ROW_BYTES % 128 == 0 && HALF_BYTES % 1024 == 0, "swizzled boxes need 1024-byte alignment");
@@ -93,6 +98,7 @@ __global__ void __launch_bounds__(VerifyCfg<T, D>::THREADS, 2)
     float* wl = wm + C::NCW * 16;                                    // [NCW][16] row sum
     volatile int* abort_flag = reinterpret_cast<volatile int*>(wl + C::NCW * 16);
     float* red = reinterpret_cast<float*>(smem + C::OFF_RED);        // [NCW][16][RED_STRIDE]
+    unsigned char* qs = smem + C::OFF_RED;                           // [ROWS][Q_STRIDE] bytes, same region
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -236,18 +242,26 @@ __global__ void __launch_bounds__(VerifyCfg<T, D>::THREADS, 2)
         int pos_lo, pos_hi;
         row_of(rt * 16 + gid, orow_lo, pos_lo);
         row_of(rt * 16 + gid + 8, orow_hi, pos_hi);
-        uint32_t qa[KS][4];
-        if (active) {
-            const T* qlo = qg + (orow_lo < 0 ? 0 : orow_lo) * D + 2 * tig;
-            const T* qhi = qg + (orow_hi < 0 ? 0 : orow_hi) * D + 2 * tig;
-#pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-                qa[kk][0] = orow_lo >= 0 ? __ldg(reinterpret_cast<const unsigned int*>(qlo + kk * 16)) : 0u;
-                qa[kk][1] = orow_hi >= 0 ? __ldg(reinterpret_cast<const unsigned int*>(qhi + kk * 16)) : 0u;
-                qa[kk][2] = orow_lo >= 0 ? __ldg(reinterpret_cast<const unsigned int*>(qlo + kk * 16 + 8)) : 0u;
-                qa[kk][3] = orow_hi >= 0 ? __ldg(reinterpret_cast<const unsigned int*>(qhi + kk * 16 + 8)) : 0u;
+        // query rows of the chunk -> shared memory (rows past the chunk as zeros); the
+        // previous item's epilogue ended with a barrier, so the region is free
+        {
+            constexpr int VPR = D * C::ELT / 16;                   // 16-byte vectors per row
+            for (int e = ctid; e < C::ROWS * VPR; e += NCT) {
+                const int lr = e / VPR;
+                const int vcol = e - lr * VPR;
+                int64_t orow;
+                int pos;
+                row_of(lr, orow, pos);
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (orow >= 0) v = __ldg(reinterpret_cast<const uint4*>(qg + orow * D) + vcol);
+                *reinterpret_cast<uint4*>(qs + lr * C::Q_STRIDE + vcol * 16) = v;
             }
+            named_barrier(1, NCT);
         }
+        // ldmatrix address of this lane in the warp's 16-row query tile: matrix lane/8 ->
+        // (+8 rows if odd, +8 columns if >= 2)
+        const uint32_t qaddr = smem_addr(qs) + (rt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * C::Q_STRIDE +
+                               (lane >> 4) * 16;
         float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
         float oacc[DT][4];
 #pragma unroll
@@ -266,22 +280,38 @@ __global__ void __launch_bounds__(VerifyCfg<T, D>::THREADS, 2)
                 const int tb = w.t0 + st * C::STAGE_ROWS;             // position of slot row 0
                 const uint32_t kb = smem_addr(smem + (c % C::NSTAGES) * C::SLOT_BYTES);
                 const uint32_t vb = kb + C::HALF_BYTES;
-                // ---- S = Q K^T over the slot's 32 tokens (4 n-tiles)
-                float sc[4][4];
+                // ---- S = Q K^T over the slot's 32 tokens (4 n-tiles).  Even and odd
+                // k-steps accumulate separately: 8 independent mma chains of depth
+                // KS / 2 instead of 4 of depth KS.  Rows past the partition are
+                // computed too and masked below.
+                float sc[4][4], se[4][4];
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                for (int nt = 0; nt < 4; ++nt) {
+                    sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                    se[nt][0] = se[nt][1] = se[nt][2] = se[nt][3] = 0.f;
+                }
 #pragma unroll
-                for (int np = 0; np < 2; ++np) {
-                    if (np * 16 >= rows) break;
-                    const uint32_t base = kb + row_base(np * 16 + krow);
+                for (int kk = 0; kk < KS; ++kk) {
+                    const int cidx = 2 * kk + kch;
+                    const uint32_t off = (cidx >> 3) * box_bytes + (((cidx & 7) ^ x) << 4);
+                    uint32_t qf[4];
+                    ldsm_x4(qaddr + kk * 32, qf[0], qf[1], qf[2], qf[3]);
 #pragma unroll
-                    for (int kk = 0; kk < KS; ++kk) {
-                        const int cidx = 2 * kk + kch;
+                    for (int np = 0; np < 2; ++np) {
                         uint32_t b0, b1, b2, b3;
-                        ldsm_x4(base + (cidx >> 3) * box_bytes + (((cidx & 7) ^ x) << 4), b0, b1, b2, b3);
-                        M::mma(sc[2 * np], qa[kk], b0, b1);
-                        M::mma(sc[2 * np + 1], qa[kk], b2, b3);
+                        ldsm_x4(kb + row_base(np * 16 + krow) + off, b0, b1, b2, b3);
+                        float (&c0)[4] = (kk & 1) ? se[2 * np] : sc[2 * np];
+                        float (&c1)[4] = (kk & 1) ? se[2 * np + 1] : sc[2 * np + 1];
+                        M::mma(c0, qf, b0, b1);
+                        M::mma(c1, qf, b2, b3);
                     }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    sc[nt][0] += se[nt][0];
+                    sc[nt][1] += se[nt][1];
+                    sc[nt][2] += se[nt][2];
+                    sc[nt][3] += se[nt][3];
                 }
                 // ---- causal mask, slot max, rescale of the running state
                 float mx_lo = -INFINITY, mx_hi = -INFINITY;
@@ -329,8 +359,7 @@ __global__ void __launch_bounds__(VerifyCfg<T, D>::THREADS, 2)
                 }
                 // ---- O += P V (p as a 16-bit value plus its remainder: two mma per tile)
 #pragma unroll
-                for (int kc = 0; kc < 2; ++kc) {
-                    if (kc * 16 >= rows) break;
+                for (int kc = 0; kc < 2; ++kc) {     // a k-chunk past the partition has p = 0 and masked V
                     uint32_t ah[4], al[4];
                     split_pack<M>(sc[2 * kc][0], sc[2 * kc][1], ah[0], al[0]);
                     split_pack<M>(sc[2 * kc][2], sc[2 * kc][3], ah[1], al[1]);

@@ -20,6 +20,19 @@
 // A preemption drops from it every op whose target block the preemption
 // returned to the free list (dead work; the block may be taken again later in
 // the same step), so within a step every slot is written at most once.
+//
+// Preemption by swap ("大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置",
+// section "生产部署注意事项": KV cache moved out to CPU memory when GPU memory
+// runs short, back in later), when selected: a victim whose private blocks fit
+// the host pool is swapped out instead (its "so" copies join the op list; its
+// writes of the step stay, since the copies carry them out) and waits in a
+// FIFO swapped queue; swapped sequences come back before any admission, each
+// needing its host blocks + 1 from the budget ("si" copies), and new requests
+// are admitted only once none is left.  Swap-out ops target host blocks and
+// are never dead; a preemption happens only when no GPU block is free, so the
+// blocks a swap-out freed earlier in the step are all taken again by then and
+// only the recomputed victim's own ops die.  Ops run in issue order;
+// consecutive writes form one launch with distinct slots.
 
 #include <deque>
 #include <new>
@@ -49,6 +62,9 @@ struct pa_sched {
     int64_t prefix_len = 0;
     std::deque<SeqState> waiting;
     std::vector<SeqState> running;
+    int preempt_mode = PA_PREEMPT_RECOMPUTE;
+    std::deque<SeqState> swapped;
+    std::vector<int64_t> swapped_out, swapped_in;
     // record of the last step
     std::vector<int64_t> finished, admitted, preempted;
     std::vector<int32_t> op_kind;
@@ -62,13 +78,19 @@ struct pa_sched {
     void rec_copy(int32_t src, int32_t dst) {
         op_kind.push_back(1); op_a.push_back(src); op_b.push_back(dst); op_c.push_back(-1);
     }
-    // Remove ops (writes into, copies into) whose target block is free again.
+    void rec_swap(int kind, int32_t a, int32_t b) {
+        op_kind.push_back(kind); op_a.push_back(a); op_b.push_back(b); op_c.push_back(-1);
+    }
+    // Remove ops (writes into, copies into, swap-ins into) whose target GPU block
+    // is free again; swap-outs target host blocks and stay.
     void drop_dead_ops() {
         const int bs = bm->block_size();
         size_t w = 0;
         for (size_t i = 0; i < op_kind.size(); ++i) {
-            const int64_t block = op_kind[i] == 0 ? op_c[i] / bs : op_b[i];
-            if (bm->ref((int32_t)block) == 0) continue;
+            if (op_kind[i] != 2) {
+                const int64_t block = op_kind[i] == 0 ? op_c[i] / bs : op_b[i];
+                if (bm->ref((int32_t)block) == 0) continue;
+            }
             op_kind[w] = op_kind[i]; op_a[w] = op_a[i]; op_b[w] = op_b[i]; op_c[w] = op_c[i];
             ++w;
         }
@@ -119,6 +141,7 @@ pa_status pa_sched::admit(SeqState s) {
 
 pa_status pa_sched::step() {
     finished.clear(); admitted.clear(); preempted.clear();
+    swapped_out.clear(); swapped_in.clear();
     op_kind.clear(); op_a.clear(); op_b.clear(); op_c.clear();
     run_ids.clear(); run_ctx.clear();
     pa_status st;
@@ -134,9 +157,22 @@ pa_status pa_sched::step() {
         }
     }
     running.swap(keep);
-    // 2. admit, FCFS against the free-block budget
+    // 2. swapped sequences come back first; then admit, FCFS against the free-block
+    // budget, only once none is left swapped out
     int64_t budget = bm->num_free();
-    while (!waiting.empty() && budget > 0 && (int)running.size() < max_running) {
+    std::vector<int32_t> pairs;
+    while (!swapped.empty() && (int)running.size() < max_running) {
+        const SeqState& head = swapped.front();
+        const int64_t need = bm->swap_in_need(head.id) + 1;
+        if (need > budget) break;
+        if ((st = bm->swap_in(head.id, pairs)) != PA_OK) return st;
+        for (size_t k = 0; k < pairs.size(); k += 2) rec_swap(3, pairs[k], pairs[k + 1]);
+        budget -= need;
+        swapped_in.push_back(head.id);
+        running.push_back(head);
+        swapped.pop_front();
+    }
+    while (swapped.empty() && !waiting.empty() && budget > 0 && (int)running.size() < max_running) {
         const SeqState& head = waiting.front();
         int64_t need = required(head);
         if (need > budget) break;
@@ -156,6 +192,17 @@ pa_status pa_sched::step() {
         if (st == PA_ERR_NO_BLOCKS) {
             SeqState victim = running.back();
             running.pop_back();
+            if (preempt_mode == PA_PREEMPT_SWAP) {
+                const int need = bm->swap_out_need(victim.id);
+                if (need >= 0 && need <= (int)bm->cpu_free_list().size()) {
+                    if ((st = bm->swap_out(victim.id, pairs)) != PA_OK) return st;
+                    for (size_t k = 0; k < pairs.size(); k += 2) rec_swap(2, pairs[k], pairs[k + 1]);
+                    swapped_out.push_back(victim.id);
+                    preempted.push_back(victim.id);
+                    swapped.push_back(victim);
+                    continue;
+                }
+            }
             if ((st = bm->free_seq(victim.id)) != PA_OK) return st;
             drop_dead_ops();
             preempted.push_back(victim.id);
@@ -198,6 +245,28 @@ pa_status pa_sched_create(pa_bm* bm, int max_running, int64_t prefix_seq, pa_sch
 }
 
 void pa_sched_destroy(pa_sched* s) { delete s; }
+
+pa_status pa_sched_set_preemption(pa_sched* s, int mode) {
+    if (!s || (mode != PA_PREEMPT_RECOMPUTE && mode != PA_PREEMPT_SWAP)) return PA_ERR_INVALID_ARG;
+    if (mode == PA_PREEMPT_RECOMPUTE && !s->swapped.empty()) return PA_ERR_INVALID_ARG;
+    s->preempt_mode = mode;
+    return PA_OK;
+}
+
+pa_status pa_sched_swap_counts(const pa_sched* s, int* num_swapped_out, int* num_swapped_in, int* num_swapped) {
+    if (!s) return PA_ERR_INVALID_ARG;
+    if (num_swapped_out) *num_swapped_out = (int)s->swapped_out.size();
+    if (num_swapped_in) *num_swapped_in = (int)s->swapped_in.size();
+    if (num_swapped) *num_swapped = (int)s->swapped.size();
+    return PA_OK;
+}
+
+pa_status pa_sched_swap_record(const pa_sched* s, int64_t* swapped_out, int64_t* swapped_in) {
+    if (!s) return PA_ERR_INVALID_ARG;
+    if (swapped_out) for (size_t i = 0; i < s->swapped_out.size(); ++i) swapped_out[i] = s->swapped_out[i];
+    if (swapped_in) for (size_t i = 0; i < s->swapped_in.size(); ++i) swapped_in[i] = s->swapped_in[i];
+    return PA_OK;
+}
 
 pa_status pa_sched_add_request(pa_sched* s, int64_t seq_id, int prompt_len, int output_len,
                                int shares_prefix, int64_t fork_child, int fork_output_len) {

@@ -92,7 +92,11 @@ def _dry_peak(tc, reqs):
     return peak
 
 
-def test_continuous_batching_trace():
+@pytest.mark.parametrize("preempt", ["recompute", "swap"])
+def test_continuous_batching_trace(preempt):
+    """With preempt="swap", victims move to a pinned host pool (a quarter of the
+    GPU pool) and come back before new admissions; the swap copies run with
+    pa_swap_blocks in issue order among the writes and copy-on-write copies."""
     assert torch.cuda.is_available()
     from paged_kv_cache_381_b200 import build
     build.build()
@@ -102,12 +106,17 @@ def test_continuous_batching_trace():
     streams = Streams(tc, reqs)
     nb = int(math.ceil(tc.pool_frac * _dry_peak(tc, reqs)))
     order = np.random.default_rng(SEED).permutation(nb).astype(np.int32)
+    ncpu = nb // 4 if preempt == "swap" else 0
     bm = pa.BlockManager(nb, tc.block_size, order)
-    model_bm = obm.BlockManager(nb, tc.block_size, order.tolist())
+    bm.set_cpu_blocks(ncpu)
+    if preempt == "swap":
+        model_bm = obm.SwappingBlockManager(nb, tc.block_size, ncpu, order.tolist())
+    else:
+        model_bm = obm.BlockManager(nb, tc.block_size, order.tolist())
     for m in (bm, model_bm):
         m.allocate(wl.PREFIX_SEQ, tc.prefix_len)
-    sch = pa.Scheduler(bm, tc.max_running, wl.PREFIX_SEQ)
-    model = osch.Scheduler(model_bm, tc.max_running, wl.PREFIX_SEQ)
+    sch = pa.Scheduler(bm, tc.max_running, wl.PREFIX_SEQ, preempt=preempt)
+    model = osch.Scheduler(model_bm, tc.max_running, wl.PREFIX_SEQ, preempt=preempt)
     for q in reqs:
         sch.add_request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child, q.fork_output_len)
         model.add_request(osch.Request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child,
@@ -116,6 +125,8 @@ def test_continuous_batching_trace():
     dev = torch.device("cuda")
     kc = torch.zeros((nb, bs, H, D), dtype=torch.float16, device=dev)
     vc = torch.zeros_like(kc)
+    hk = torch.zeros((max(ncpu, 1), bs, H, D), dtype=torch.float16).pin_memory()
+    hv = torch.zeros_like(hk).pin_memory()
     kflat, vflat = kc.view(nb * bs, H, D), vc.view(nb * bs, H, D)
 
     def write(ws):
@@ -131,27 +142,36 @@ def test_continuous_batching_trace():
     write(pre)
 
     r = np.random.default_rng(11)
-    saw = {"preempt": 0, "cow": 0, "blocked": 0, "finish": 0}
+    saw = {"preempt": 0, "cow": 0, "blocked": 0, "finish": 0, "so": 0, "si": 0}
     for step in range(tc.steps):
         rec = sch.step()
         mrec = model.step()
         assert rec["finished"] == mrec.finished and rec["admitted"] == mrec.admitted, step
         assert rec["preempted"] == mrec.preempted and rec["ops"] == [tuple(o) for o in mrec.ops], step
         assert rec["running"] == mrec.running and rec["context_lens"] == mrec.context_lens, step
+        assert rec["swapped_out"] == mrec.swapped_out and rec["swapped_in"] == mrec.swapped_in, step
         saw["preempt"] += len(rec["preempted"])
         saw["finish"] += len(rec["finished"])
         if rec["num_waiting"] > 0 and len(rec["running"]) < tc.max_running:
             saw["blocked"] += 1
-        # apply writes and copies in issue order
+        # apply writes, copies and swap copies in issue order
         run = []
         for op in rec["ops"]:
             if op[0] == "w":
                 run.append(op[1:])
-            else:
-                write(run)
-                run = []
+                continue
+            write(run)
+            run = []
+            pair = torch.tensor([[op[1], op[2]]], dtype=torch.int32, device=dev)
+            if op[0] == "c":
                 saw["cow"] += 1
-                pa.pa_copy_blocks(kc, vc, torch.tensor([[op[1], op[2]]], dtype=torch.int32, device=dev))
+                pa.pa_copy_blocks(kc, vc, pair)
+            elif op[0] == "so":
+                saw["so"] += 1
+                pa.pa_swap_blocks(hk, hv, kc, vc, pair)
+            else:
+                saw["si"] += 1
+                pa.pa_swap_blocks(kc, vc, hk, hv, pair)
         write(run)
         running, ctx = rec["running"], rec["context_lens"]
         if not running:
@@ -195,3 +215,5 @@ def test_continuous_batching_trace():
     assert saw["cow"] >= 1, saw
     assert saw["blocked"] >= 1, saw
     assert saw["finish"] >= 1, saw
+    if preempt == "swap":
+        assert saw["so"] >= 1 and saw["si"] >= 1, saw

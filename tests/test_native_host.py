@@ -171,18 +171,20 @@ def _load_traces():
 @pytest.mark.parametrize("tr", _load_traces(), ids=lambda t: t["name"])
 def test_scheduler_golden_traces(pa, tr):
     bm = pa.BlockManager(tr["num_blocks"], tr["block_size"], tr["initial_free_order"])
+    bm.set_cpu_blocks(tr.get("num_cpu_blocks", 0))
     prefix = -1
     if tr["prefix"]:
         prefix = tr["prefix"]["seq"]
         bm.allocate(prefix, tr["prefix"]["tokens"])
-    sch = pa.Scheduler(bm, tr["max_running"], prefix)
+    sch = pa.Scheduler(bm, tr["max_running"], prefix, preempt=tr.get("preempt", "recompute"))
     for q in tr["requests"]:
         sch.add_request(q["seq"], q["prompt"], q["output"], q.get("shares_prefix", False),
                         q.get("fork_child", -1), q.get("fork_output", 0))
     for i, exp in enumerate(tr["steps"]):
         rec = sch.step()
-        for key in ("finished", "admitted", "preempted", "running", "context_lens"):
-            assert rec[key] == exp[key], (i, key, rec[key])
+        for key in ("finished", "admitted", "preempted", "running", "context_lens", "swapped_out", "swapped_in"):
+            if key in exp:
+                assert rec[key] == exp[key], (i, key, rec[key])
         assert [list(o) for o in rec["ops"]] == exp["ops"], (i, rec["ops"])
 
 
@@ -274,3 +276,35 @@ def test_verify_workspace_and_argument_rules(pa):
     assert lib.pa_verify(*args(0, 2)) == 1            # no query rows
     assert lib.pa_verify(*args(6, 2, hq=60)) == 1     # heads not a multiple of kv heads
     assert lib.pa_verify(*args(6, 2)) == 1            # null pointers
+
+
+@pytest.mark.parametrize("ncpu,nb", [(6, 60), (40, 60), (400, 50)])
+def test_scheduler_swap_matches_model(pa, ncpu, nb):
+    """Preemption by swap: C++ and Python agree every step (ops incl. swap
+    copies, swapped ids, free lists of both pools)."""
+    tc = wl.TraceConfig(block_size=4, max_running=12, num_requests=40, steps=150, prefix_len=10,
+                        prompt_hi=30, output_mean=14.0, fork_every=4)
+    reqs = wl.make_trace_requests(tc, 5)
+    order = np.random.default_rng(9).permutation(nb).tolist()
+    mb = obm.SwappingBlockManager(nb, tc.block_size, ncpu, order)
+    nbm = pa.BlockManager(nb, tc.block_size, order)
+    nbm.set_cpu_blocks(ncpu)
+    for m in (mb, nbm):
+        m.allocate(wl.PREFIX_SEQ, tc.prefix_len)
+    ms = osch.Scheduler(mb, tc.max_running, wl.PREFIX_SEQ, preempt="swap")
+    ns = pa.Scheduler(nbm, tc.max_running, wl.PREFIX_SEQ, preempt="swap")
+    for q in reqs:
+        ms.add_request(osch.Request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child,
+                                    q.fork_output_len))
+        ns.add_request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child, q.fork_output_len)
+    n_so = 0
+    for step in range(tc.steps):
+        a, b = ms.step(), ns.step()
+        assert [tuple(o) for o in a.ops] == b["ops"], step
+        assert (a.finished, a.admitted, a.preempted) == (b["finished"], b["admitted"], b["preempted"]), step
+        assert (a.swapped_out, a.swapped_in) == (b["swapped_out"], b["swapped_in"]), step
+        assert a.running == b["running"] and a.context_lens == b["context_lens"], step
+        assert len(ms.swapped) == b["num_swapped"], step
+        assert mb.free_list == nbm.free_list() and mb.cpu_free == nbm.cpu_free_list(), step
+        n_so += len(a.swapped_out)
+    assert n_so > 0

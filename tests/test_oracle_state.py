@@ -198,12 +198,16 @@ def _load_traces():
 
 
 def _build(tr):
-    bm = obm.BlockManager(tr["num_blocks"], tr["block_size"], tr["initial_free_order"])
+    if tr.get("preempt") == "swap":
+        bm = obm.SwappingBlockManager(tr["num_blocks"], tr["block_size"], tr["num_cpu_blocks"],
+                                      tr["initial_free_order"])
+    else:
+        bm = obm.BlockManager(tr["num_blocks"], tr["block_size"], tr["initial_free_order"])
     prefix = -1
     if tr["prefix"]:
         prefix = tr["prefix"]["seq"]
         bm.allocate(prefix, tr["prefix"]["tokens"])
-    sch = osch.Scheduler(bm, tr["max_running"], prefix)
+    sch = osch.Scheduler(bm, tr["max_running"], prefix, preempt=tr.get("preempt", "recompute"))
     for q in tr["requests"]:
         sch.add_request(osch.Request(q["seq"], q["prompt"], q["output"], q.get("shares_prefix", False),
                                      q.get("fork_child", -1), q.get("fork_output", 0)))
@@ -221,6 +225,8 @@ def test_scheduler_golden_traces(tr):
         assert [list(o) for o in rec.ops] == exp["ops"], (i, rec.ops)
         assert rec.running == exp["running"], (i, rec.running)
         assert rec.context_lens == exp["context_lens"], (i, rec.context_lens)
+        if "swapped_out" in exp:
+            assert (rec.swapped_out, rec.swapped_in) == (exp["swapped_out"], exp["swapped_in"]), i
         bm.check()
 
 
@@ -285,3 +291,76 @@ def test_scheduler_random_trace_invariants():
                 assert shadow.get(sl) == (stream_of(seq, p), p), (seq, p)
     assert first_admit == sorted(first_admit)
     assert saw_preempt and saw_cow
+
+
+def _swap_trace_run(tc, reqs, nb, ncpu, seed, record_cls=None):
+    """Run the scheduler model with preemption by swap; replay its ops on a
+    shadow of GPU and host slots; check every sequence's content each step."""
+    bm = obm.SwappingBlockManager(nb, tc.block_size, ncpu, np.random.default_rng(seed).permutation(nb).tolist())
+    bm.allocate(wl.PREFIX_SEQ, tc.prefix_len)
+    sch = osch.Scheduler(bm, tc.max_running, wl.PREFIX_SEQ, preempt="swap")
+    for q in reqs:
+        sch.add_request(osch.Request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix,
+                                     q.fork_child, q.fork_output_len))
+    bs = tc.block_size
+    gpu, cpu = {}, {}
+    for p, sl in enumerate(bm.slots(wl.PREFIX_SEQ, 0, tc.prefix_len)):
+        gpu[sl] = (wl.PREFIX_SEQ, p)
+    parent_of = {q.fork_child: q.seq_id for q in reqs if q.fork_child >= 0}
+    fork_pos = {q.fork_child: (tc.prefix_len if q.shares_prefix else 0) + q.prompt_len
+                for q in reqs if q.fork_child >= 0}
+    share = {q.seq_id: q.shares_prefix for q in reqs}
+
+    def stream_of(seq, pos):
+        if seq in parent_of and pos < fork_pos[seq]:
+            return stream_of(parent_of[seq], pos)
+        if share.get(seq, False) and pos < tc.prefix_len:
+            return wl.PREFIX_SEQ
+        return seq
+
+    saw = {"so": 0, "si": 0, "recompute": 0}
+    for _ in range(tc.steps):
+        rec = sch.step()
+        run = []
+        for op in rec.ops:
+            if op[0] == "w":
+                run.append(op[3])
+                gpu[op[3]] = (stream_of(op[1], op[2]), op[2])
+                continue
+            assert len(run) == len(set(run)), "a slot written twice in one run of writes"
+            run = []
+            src, dst = (gpu, gpu) if op[0] == "c" else (gpu, cpu) if op[0] == "so" else (cpu, gpu)
+            for o in range(bs):
+                if op[1] * bs + o in src:
+                    dst[op[2] * bs + o] = src[op[1] * bs + o]
+            if op[0] in saw:
+                saw[op[0]] += 1
+        assert len(run) == len(set(run))
+        saw["recompute"] += len(rec.preempted) - len(rec.swapped_out)
+        bm.check()
+        for seq, n in zip(rec.running, rec.context_lens):
+            for p, sl in enumerate(bm.slots(seq, 0, n)):
+                assert gpu.get(sl) == (stream_of(seq, p), p), (seq, p)
+        for s in sch.swapped:             # swapped out: host blocks it moved, GPU blocks it shares
+            t, loc = bm.tables[s.seq_id], bm.on_cpu[s.seq_id]
+            for p in range(bm.ctx[s.seq_id]):
+                store = cpu if loc[p // bs] else gpu
+                assert store.get(t[p // bs] * bs + p % bs) == (stream_of(s.seq_id, p), p), (s.seq_id, p)
+    return saw
+
+
+SWAP_TC = wl.TraceConfig(block_size=4, max_running=12, num_requests=40, steps=150, prefix_len=10,
+                         prompt_hi=30, output_mean=14.0, fork_every=4)
+
+
+@pytest.mark.parametrize("ncpu", [6, 40, 400])
+def test_scheduler_swap_trace_content(ncpu):
+    """Preemption by swap on a scaled-down trace: every running sequence reads
+    its own tokens every step, and so does every swapped-out one where its
+    table says (host or shared GPU blocks); consecutive writes never repeat a
+    slot.  A small host pool also forces recompute fallbacks."""
+    reqs = wl.make_trace_requests(SWAP_TC, 5)
+    saw = _swap_trace_run(SWAP_TC, reqs, 60, ncpu, 9)
+    assert saw["so"] > 0 and saw["si"] > 0, saw
+    if ncpu == 6:
+        assert saw["recompute"] > 0, saw
