@@ -63,6 +63,9 @@ def parse():
                    help="merge split partitions with the reduce kernel or inside the decode kernel")
     p.add_argument("--num-seqs", type=int, default=0,
                    help="keep only the first N sequences (smaller cases for profiling)")
+    p.add_argument("--swap-mb", type=int, default=0,
+                   help="> 0: time pa_swap_blocks moving this many MiB of blocks (K and V) between the "
+                        "device pool and a pinned host pool, against one contiguous copy of the same bytes")
     p.add_argument("--queries", type=int, default=1,
                    help="candidate tokens per sequence: > 1 times the verification pass (pa_verify) "
                         "of speculative decoding instead of decode")
@@ -473,10 +476,70 @@ def run_native(args):
     return 0
 
 
+def run_swap(args):
+    """Host-link throughput of pa_swap_blocks: random (source, destination)
+    block pairs of the 70B-shaped pool (16 tokens x 8 kv heads x 128 x bf16 =
+    32 KiB per block and pool), device -> pinned host and back, against a
+    single contiguous cudaMemcpyAsync of the same byte count (the copy engine
+    over the same link) as the reference."""
+    import torch
+    from paged_kv_cache_381_b200 import build
+    build.build()
+    import paged_kv_cache_381_b200 as pa
+    dev = torch.device("cuda", 0)
+    blk = (16, 8, 128)
+    block_bytes = 2 * 16 * 8 * 128 * 2                      # K and V
+    n = max(1, (args.swap_mb << 20) // block_bytes)
+    nb_dev, nb_host = 2 * n, 2 * n
+    dk = torch.randn((nb_dev,) + blk, device=dev).to(torch.bfloat16)
+    dv = torch.randn((nb_dev,) + blk, device=dev).to(torch.bfloat16)
+    hk = torch.empty((nb_host,) + blk, dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    r = np.random.default_rng(args.seed)
+    out_pairs = torch.from_numpy(np.stack([r.choice(nb_dev, n, replace=False),
+                                           r.choice(nb_host, n, replace=False)], 1).astype(np.int32)).to(dev)
+    in_pairs = torch.from_numpy(np.stack([out_pairs[:, 1].cpu().numpy(),
+                                          r.choice(nb_dev, n, replace=False)], 1).astype(np.int32)).to(dev)
+    flat_d = torch.empty(n * block_bytes, dtype=torch.uint8, device=dev)
+    flat_h = torch.empty(n * block_bytes, dtype=torch.uint8).pin_memory()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for a, b in ev:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return sorted(a.elapsed_time(b) for a, b in ev)[len(ev) // 2]
+
+    steps = max(5, min(args.steps, 50))
+    args.steps = steps
+    t_out = timed(lambda: pa.pa_swap_blocks(hk, hv, dk, dv, out_pairs))
+    t_in = timed(lambda: pa.pa_swap_blocks(dk, dv, hk, hv, in_pairs))
+    t_d2h = timed(lambda: flat_h.copy_(flat_d, non_blocking=True))
+    t_h2d = timed(lambda: flat_d.copy_(flat_h, non_blocking=True))
+    err = pa.pa_get_device_error()
+    gb = n * block_bytes / 1e9
+    res = {"metric": "swap: GB/s of K/V blocks moved over the host link (pa_swap_blocks)", "unit": "GB/s",
+           "value": gb / (t_out * 1e-3), "n_gpus": 1, "steps": steps, "higher_is_better": True,
+           "blocks": int(n), "bytes_per_call": int(n * block_bytes),
+           "swap_out": {"ms": t_out, "gbs": gb / (t_out * 1e-3), "copy_engine_gbs": gb / (t_d2h * 1e-3)},
+           "swap_in": {"ms": t_in, "gbs": gb / (t_in * 1e-3), "copy_engine_gbs": gb / (t_h2d * 1e-3)},
+           "reference": "one contiguous cudaMemcpyAsync of the same bytes (copy engine), median of the steps",
+           "device_error_flags": err, "dtype": "bf16", "data": "synthetic"}
+    print(json.dumps(res))
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.swap_mb > 0:
+        return run_swap(args)
     return run_native(args)
 
 
