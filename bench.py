@@ -401,36 +401,43 @@ def run_native(args):
                 "block_tables": batch.block_tables.cpu().pin_memory(),
                 "context_lens": batch.context_lens.cpu().pin_memory(),
                 "out": torch.empty_like(q, device="cpu").pin_memory()}
-        devb = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
-        devb["workspace"] = batch.workspace
+        # two staging sets: step i+1's inputs and step i-1's output cross the host
+        # link while step i computes (pa_pipeline); the split-K workspace is shared,
+        # since the computes themselves stay in order on one stream
+        sets = []
+        for _ in range(2):
+            d = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+            d["workspace"] = batch.workspace
+            sets.append(d)
         h2d = sum(host[k].numel() * host[k].element_size() for k in host if k != "out")
         d2h = host["out"].numel() * host["out"].element_size()
+        pipe = pa.Pipeline(2)
 
-        def e2e_step():
-            pa.pa_step(host, devb, batch.k_cache, batch.v_cache, cfg.scale, batch.max_context_len, P)
+        def e2e_run(n):
+            pipe.begin(q)
+            for i in range(n):
+                pipe.step(i % 2, host, sets[i % 2], batch.k_cache, batch.v_cache, cfg.scale, batch.max_context_len, P)
+            pipe.end(q)
 
-        for _ in range(3):
-            e2e_step()
-            flush.zero_()
+        e2e_run(3)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        for i in range(args.steps):
-            ev2[i][0].record()
-            e2e_step()
-            ev2[i][1].record()
-            flush.zero_()
+        # inputs (1.1 GB of K/V per step) are larger than L2: no flush inside this run
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        e2e_run(args.steps)
+        e1.record()
         torch.cuda.synchronize()
-        ems = sum(a.elapsed_time(b) for a, b in ev2) / args.steps
+        ems = e0.elapsed_time(e1) / args.steps
         if world > 1:
             t = torch.tensor([ems], dtype=torch.float64, device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ems = float(t[0])
         e2e = {"value": world * step_kv / (ems * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": ems,
-               "tokens_per_s": world * len(lens) / (ems * 1e-3)}
+               "tokens_per_s": world * len(lens) / (ems * 1e-3),
+               "how": "pa_pipeline: each step's H2D and D2H overlap the neighbouring steps' compute"}
 
     peak, peak_kind = measured_peaks()
     if Q > 1:

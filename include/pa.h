@@ -281,6 +281,31 @@ pa_status pa_step(const pa_step_host* host, const pa_step_device* dev, void* k_c
                   void* v_cache, const pa_step_shape* shape, void* stream);
 
 /*
+ * pa_pipeline -- pa_step with its host<->device copies on two copy streams
+ * owned by the pipeline, so that consecutive steps overlap: while step i
+ * computes on `stream`, step i+1's inputs travel host->device and step i-1's
+ * output travels device->host.  The caller provides `depth` staging sets
+ * (pa_step_device, each with its own buffers and workspace) and uses set
+ * i % depth for step i; the pipeline orders, per set, the input copies after
+ * the previous compute that read the set, the compute after those copies and
+ * after the previous output copy that read the set's `out`, and the output
+ * copy after the compute.  Host buffers are read and written asynchronously:
+ * keep them unchanged (inputs) and unread (output) until pa_pipeline_end
+ * returns or its work on `stream` has completed.
+ *   pa_pipeline_begin   the copy streams wait for work enqueued on `stream` so far
+ *   pa_pipeline_step    one layer-step as pa_step (same arguments) on staging set `set`
+ *   pa_pipeline_end     `stream` waits for every copy enqueued so far
+ * Not thread-safe per pipeline.
+ */
+typedef struct pa_pipeline pa_pipeline;
+pa_status pa_pipeline_create(int depth, pa_pipeline** out);
+void pa_pipeline_destroy(pa_pipeline* p);
+pa_status pa_pipeline_begin(pa_pipeline* p, void* stream);
+pa_status pa_pipeline_step(pa_pipeline* p, int set, const pa_step_host* host, const pa_step_device* dev,
+                           void* k_cache, void* v_cache, const pa_step_shape* shape, void* stream);
+pa_status pa_pipeline_end(pa_pipeline* p, void* stream);
+
+/*
  * Arithmetic used by pa_decode's score and output contractions (process-wide):
  *   PA_MATH_AUTO   tensor cores (mma m16n8k16, fp32 accumulate) for fp16 / bf16,
  *                  CUDA-core fp32 FMAs for fp32 -- the default;

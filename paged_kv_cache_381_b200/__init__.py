@@ -226,13 +226,7 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scal
     return out
 
 
-def pa_step(host, dev, k_cache, v_cache, scale, max_context_len, partition_size=0, stream=None):
-    """One layer-step from host buffers (see include/pa.h, pa_step).
-
-    host: dict of pinned CPU tensors q, k, v, slot_mapping, block_tables,
-    context_lens, out (and optionally cow_pairs); dev: dict of CUDA tensors of
-    the same shapes plus ``workspace``.
-    """
+def _step_structs(host, dev, k_cache, scale, max_context_len, partition_size):
     nb, bs, hkv, d = k_cache.shape
     S, Hq, D = host["q"].shape
     T = int(host["slot_mapping"].numel())
@@ -247,9 +241,49 @@ def pa_step(host, dev, k_cache, v_cache, scale, max_context_len, partition_size=
                             ptr(dev["out"]), ptr(ws), 0 if ws is None else int(ws.numel()))
     shape = _native.StepShape(S, Hq, hkv, D, bs, nb, int(host["block_tables"].shape[1]), int(max_context_len), T,
                               ncow, _dtype_code(k_cache), float(scale), int(partition_size))
+    return h, dv, shape
+
+
+def pa_step(host, dev, k_cache, v_cache, scale, max_context_len, partition_size=0, stream=None):
+    """One layer-step from host buffers (see include/pa.h, pa_step).
+
+    host: dict of pinned CPU tensors q, k, v, slot_mapping, block_tables,
+    context_lens, out (and optionally cow_pairs); dev: dict of CUDA tensors of
+    the same shapes plus ``workspace``.
+    """
+    h, dv, shape = _step_structs(host, dev, k_cache, scale, max_context_len, partition_size)
     st = lib().pa_step(ctypes.byref(h), ctypes.byref(dv), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
                        ctypes.byref(shape), _stream(k_cache, stream))
     _check(st, "pa_step")
+
+
+class Pipeline:
+    """pa_step with overlapped host<->device copies (pa_pipeline_*): use
+    staging set i % depth for step i; bracket a run of steps with begin/end."""
+
+    def __init__(self, depth=2):
+        self._h = ctypes.c_void_p()
+        _check(lib().pa_pipeline_create(int(depth), ctypes.byref(self._h)), "pa_pipeline_create")
+        self.depth = int(depth)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            lib().pa_pipeline_destroy(h)
+            self._h = None
+
+    def begin(self, like, stream=None):
+        _check(lib().pa_pipeline_begin(self._h, _stream(like, stream)), "pa_pipeline_begin")
+
+    def step(self, set_index, host, dev, k_cache, v_cache, scale, max_context_len, partition_size=0, stream=None):
+        h, dv, shape = _step_structs(host, dev, k_cache, scale, max_context_len, partition_size)
+        st = lib().pa_pipeline_step(self._h, int(set_index), ctypes.byref(h), ctypes.byref(dv),
+                                    _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), ctypes.byref(shape),
+                                    _stream(k_cache, stream))
+        _check(st, "pa_pipeline_step")
+
+    def end(self, like, stream=None):
+        _check(lib().pa_pipeline_end(self._h, _stream(like, stream)), "pa_pipeline_end")
 
 
 def pa_get_device_error(stream=None):

@@ -55,6 +55,12 @@ SIGNATURES = {
                                   c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p]),
     "pa_copy_blocks": (c_int, [c_void_p, c_void_p, c_void_p, c_int, P(CacheDesc), c_void_p]),
     "pa_step": (c_int, [P(StepHost), P(StepDevice), c_void_p, c_void_p, P(StepShape), c_void_p]),
+    "pa_pipeline_create": (c_int, [c_int, P(c_void_p)]),
+    "pa_pipeline_destroy": (None, [c_void_p]),
+    "pa_pipeline_begin": (c_int, [c_void_p, c_void_p]),
+    "pa_pipeline_step": (c_int, [c_void_p, c_int, P(StepHost), P(StepDevice), c_void_p, c_void_p, P(StepShape),
+                                 c_void_p]),
+    "pa_pipeline_end": (c_int, [c_void_p, c_void_p]),
     "pa_get_device_error": (c_int, [P(c_uint32), c_void_p]),
     "pa_status_string": (ctypes.c_char_p, [c_int]),
     "pa_launch_count": (c_int64, []),

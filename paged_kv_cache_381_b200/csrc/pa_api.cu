@@ -296,6 +296,49 @@ int query_chunk(int group, bool tensor) {
 
 }  // namespace
 
+namespace {
+
+pa_status step_compute(const pa_step_device* d, void* k_cache, void* v_cache, const pa_step_shape* sh, void* stream) {
+    pa_cache_desc cd{sh->num_blocks, sh->block_size, sh->num_kv_heads, sh->head_dim, sh->dtype};
+    pa_status st = PA_OK;
+    if (sh->num_cow > 0 && (st = pa_copy_blocks(k_cache, v_cache, d->cow_pairs, sh->num_cow, &cd, stream)) != PA_OK)
+        return st;
+    if ((st = pa_cache_write(d->k, d->v, k_cache, v_cache, d->slot_mapping, sh->num_tokens, &cd, stream)) != PA_OK)
+        return st;
+    return pa_decode(d->out, d->q, k_cache, v_cache, d->block_tables, d->context_lens, sh->scale, sh->block_size,
+                     sh->num_kv_heads, sh->num_seqs, sh->num_heads, sh->head_dim, sh->max_blocks_per_seq,
+                     sh->max_context_len, sh->num_blocks, sh->dtype, sh->partition_size, d->workspace,
+                     d->workspace_bytes, stream);
+}
+
+bool step_inputs(const pa_step_host* h, const pa_step_device* d, const pa_step_shape* sh, cudaStream_t s) {
+    const size_t e = elem_bytes(sh->dtype);
+    const size_t qbytes = (size_t)sh->num_seqs * sh->num_heads * sh->head_dim * e;
+    const size_t kvbytes = (size_t)sh->num_tokens * sh->num_kv_heads * sh->head_dim * e;
+    auto h2d = [&](void* dst, const void* src, size_t n) -> bool {
+        if (n == 0) return true;
+        if (!dst || !src) return false;
+        return cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    };
+    return h2d(d->q, h->q, qbytes) && h2d(d->k, h->k, kvbytes) && h2d(d->v, h->v, kvbytes) &&
+           h2d(d->slot_mapping, h->slot_mapping, (size_t)sh->num_tokens * sizeof(int64_t)) &&
+           h2d(d->block_tables, h->block_tables, (size_t)sh->num_seqs * sh->max_blocks_per_seq * sizeof(int32_t)) &&
+           h2d(d->context_lens, h->context_lens, (size_t)sh->num_seqs * sizeof(int32_t)) &&
+           h2d(d->cow_pairs, h->cow_pairs, (size_t)sh->num_cow * 2 * sizeof(int32_t));
+}
+
+bool step_output(const pa_step_host* h, const pa_step_device* d, const pa_step_shape* sh, cudaStream_t s) {
+    const size_t qbytes = (size_t)sh->num_seqs * sh->num_heads * sh->head_dim * elem_bytes(sh->dtype);
+    if (qbytes == 0) return true;
+    return h->out && d->out && cudaMemcpyAsync(h->out, d->out, qbytes, cudaMemcpyDeviceToHost, s) == cudaSuccess;
+}
+
+bool step_shape_ok(const pa_step_shape* sh) {
+    return sh->num_seqs >= 0 && sh->num_tokens >= 0 && sh->num_cow >= 0 && valid_dtype(sh->dtype);
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* pa_status_string(pa_status s) {
@@ -629,35 +672,95 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
 
 pa_status pa_step(const pa_step_host* h, const pa_step_device* d, void* k_cache, void* v_cache,
                   const pa_step_shape* sh, void* stream) {
-    if (!h || !d || !sh || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
-    if (sh->num_seqs < 0 || sh->num_tokens < 0 || sh->num_cow < 0 || !valid_dtype(sh->dtype)) return PA_ERR_INVALID_ARG;
+    if (!h || !d || !sh || !k_cache || !v_cache || !step_shape_ok(sh)) return PA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t e = elem_bytes(sh->dtype);
-    const size_t qbytes = (size_t)sh->num_seqs * sh->num_heads * sh->head_dim * e;
-    const size_t kvbytes = (size_t)sh->num_tokens * sh->num_kv_heads * sh->head_dim * e;
-    auto h2d = [&](void* dst, const void* src, size_t n) -> bool {
-        if (n == 0) return true;
-        if (!dst || !src) return false;
-        return cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, s) == cudaSuccess;
-    };
-    if (!h2d(d->q, h->q, qbytes) || !h2d(d->k, h->k, kvbytes) || !h2d(d->v, h->v, kvbytes) ||
-        !h2d(d->slot_mapping, h->slot_mapping, (size_t)sh->num_tokens * sizeof(int64_t)) ||
-        !h2d(d->block_tables, h->block_tables, (size_t)sh->num_seqs * sh->max_blocks_per_seq * sizeof(int32_t)) ||
-        !h2d(d->context_lens, h->context_lens, (size_t)sh->num_seqs * sizeof(int32_t)) ||
-        !h2d(d->cow_pairs, h->cow_pairs, (size_t)sh->num_cow * 2 * sizeof(int32_t)))
+    if (!step_inputs(h, d, sh, s)) return PA_ERR_CUDA;
+    pa_status st = step_compute(d, k_cache, v_cache, sh, stream);
+    if (st != PA_OK) return st;
+    return step_output(h, d, sh, s) ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // extern "C"
+
+struct pa_pipeline {
+    int depth = 0;
+    int device = 0;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    std::vector<cudaEvent_t> staged, computed, drained;   // per staging set
+    cudaEvent_t mark = nullptr;
+    ~pa_pipeline() {
+        for (auto* v : {&staged, &computed, &drained})
+            for (cudaEvent_t e : *v)
+                if (e) cudaEventDestroy(e);
+        if (mark) cudaEventDestroy(mark);
+        if (h2d) cudaStreamDestroy(h2d);
+        if (d2h) cudaStreamDestroy(d2h);
+    }
+};
+
+
+extern "C" {
+
+pa_status pa_pipeline_create(int depth, pa_pipeline** out) {
+    if (!out || depth < 1 || depth > 16) return PA_ERR_INVALID_ARG;
+    *out = nullptr;
+    pa_pipeline* p = new (std::nothrow) pa_pipeline();
+    if (!p) return PA_ERR_INVALID_ARG;
+    p->depth = depth;
+    bool ok = cudaGetDevice(&p->device) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p->d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&p->mark, cudaEventDisableTiming) == cudaSuccess;
+    for (auto* v : {&p->staged, &p->computed, &p->drained}) {
+        v->assign(depth, nullptr);
+        for (int i = 0; i < depth && ok; ++i) ok = cudaEventCreateWithFlags(&(*v)[i], cudaEventDisableTiming) == cudaSuccess;
+    }
+    if (!ok) {
+        delete p;
         return PA_ERR_CUDA;
-    pa_cache_desc cd{sh->num_blocks, sh->block_size, sh->num_kv_heads, sh->head_dim, sh->dtype};
-    pa_status st = PA_OK;
-    if (sh->num_cow > 0 && (st = pa_copy_blocks(k_cache, v_cache, d->cow_pairs, sh->num_cow, &cd, stream)) != PA_OK)
-        return st;
-    if ((st = pa_cache_write(d->k, d->v, k_cache, v_cache, d->slot_mapping, sh->num_tokens, &cd, stream)) != PA_OK)
-        return st;
-    if ((st = pa_decode(d->out, d->q, k_cache, v_cache, d->block_tables, d->context_lens, sh->scale, sh->block_size,
-                        sh->num_kv_heads, sh->num_seqs, sh->num_heads, sh->head_dim, sh->max_blocks_per_seq,
-                        sh->max_context_len, sh->num_blocks, sh->dtype, sh->partition_size, d->workspace,
-                        d->workspace_bytes, stream)) != PA_OK)
-        return st;
-    if (qbytes && (!h->out || !d->out || cudaMemcpyAsync(h->out, d->out, qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess))
+    }
+    *out = p;
+    return PA_OK;
+}
+
+void pa_pipeline_destroy(pa_pipeline* p) { delete p; }
+
+pa_status pa_pipeline_begin(pa_pipeline* p, void* stream) {
+    if (!p) return PA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaEventRecord(p->mark, s) != cudaSuccess || cudaStreamWaitEvent(p->h2d, p->mark, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(p->d2h, p->mark, 0) != cudaSuccess)
+        return PA_ERR_CUDA;
+    return PA_OK;
+}
+
+pa_status pa_pipeline_step(pa_pipeline* p, int set, const pa_step_host* h, const pa_step_device* d, void* k_cache,
+                           void* v_cache, const pa_step_shape* sh, void* stream) {
+    if (!p || set < 0 || set >= p->depth || !h || !d || !sh || !k_cache || !v_cache || !step_shape_ok(sh))
+        return PA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // inputs: after the previous compute that read this set
+    if (cudaStreamWaitEvent(p->h2d, p->computed[set], 0) != cudaSuccess) return PA_ERR_CUDA;
+    if (!step_inputs(h, d, sh, p->h2d) || cudaEventRecord(p->staged[set], p->h2d) != cudaSuccess) return PA_ERR_CUDA;
+    // compute: after the inputs, and after the previous output copy read this set's `out`
+    if (cudaStreamWaitEvent(s, p->staged[set], 0) != cudaSuccess ||
+        cudaStreamWaitEvent(s, p->drained[set], 0) != cudaSuccess)
+        return PA_ERR_CUDA;
+    pa_status st = step_compute(d, k_cache, v_cache, sh, stream);
+    if (st != PA_OK) return st;
+    if (cudaEventRecord(p->computed[set], s) != cudaSuccess) return PA_ERR_CUDA;
+    // output: after the compute
+    if (cudaStreamWaitEvent(p->d2h, p->computed[set], 0) != cudaSuccess || !step_output(h, d, sh, p->d2h) ||
+        cudaEventRecord(p->drained[set], p->d2h) != cudaSuccess)
+        return PA_ERR_CUDA;
+    return PA_OK;
+}
+
+pa_status pa_pipeline_end(pa_pipeline* p, void* stream) {
+    if (!p) return PA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaEventRecord(p->mark, p->h2d) != cudaSuccess || cudaStreamWaitEvent(s, p->mark, 0) != cudaSuccess ||
+        cudaEventRecord(p->mark, p->d2h) != cudaSuccess || cudaStreamWaitEvent(s, p->mark, 0) != cudaSuccess)
         return PA_ERR_CUDA;
     return PA_OK;
 }

@@ -321,6 +321,48 @@ def test_pa_step_from_host_buffers_matches_device_path():
     _no_device_error()
 
 
+def test_pipeline_overlapped_steps_match_device_path():
+    """pa_pipeline over 5 steps with 2 staging sets, a different query per step
+    (own pinned host buffers): every step's host output equals the device
+    path's decode of the same query, bit for bit."""
+    cfg = wl.CONFIGS["70b"]
+    inp = wl.make_decode_inputs(cfg, 22, context_lens=np.array([3000, 17, 600, 1, 4096, 250, 70]))
+    b = DeviceBatch(inp)
+    b.step_write()
+    S, Hq, D = b.q.shape
+    slots = np.array([b.bm.slots(s, int(n) - 1, 1)[0] for s, n in enumerate(b.lens)], dtype=np.int64)
+    k_new = np.stack([inp.k_hist[s][-1] for s in range(S)])
+    v_new = np.stack([inp.v_hist[s][-1] for s in range(S)])
+    pin = lambda t: t.pin_memory()
+    mcl = int(b.lens.max())
+    g = torch.Generator(device="cuda").manual_seed(5)
+    qs = [torch.randn((S, Hq, D), generator=g, device="cuda").to(torch.bfloat16) for _ in range(5)]
+    refs = []
+    for q in qs:
+        out = torch.empty_like(q)
+        pa.pa_decode(out, q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, cfg.scale, max_context_len=mcl)
+        refs.append(to_storage(out, "bf16"))
+    common = {"k": pin(to_device(k_new, "bf16", "cpu")), "v": pin(to_device(v_new, "bf16", "cpu")),
+              "slot_mapping": pin(torch.from_numpy(slots)), "block_tables": pin(b.block_tables.cpu()),
+              "context_lens": pin(b.context_lens.cpu())}
+    hosts = [dict(common, q=pin(q.cpu()), out=pin(torch.full_like(q, float("nan"), device="cpu"))) for q in qs]
+    ws = torch.empty(max(1, pa.pa_decode_workspace_size(S, Hq, D, mcl)), dtype=torch.uint8, device="cuda")
+    sets = []
+    for _ in range(2):
+        d = {k: torch.empty_like(v, device="cuda") for k, v in hosts[0].items()}
+        d["workspace"] = ws
+        sets.append(d)
+    pipe = pa.Pipeline(2)
+    pipe.begin(b.k_cache)
+    for i, h in enumerate(hosts):
+        pipe.step(i % 2, h, sets[i % 2], b.k_cache, b.v_cache, cfg.scale, mcl)
+    pipe.end(b.k_cache)
+    torch.cuda.synchronize()
+    for h, ref in zip(hosts, refs):
+        assert np.array_equal(to_storage(h["out"], "bf16"), ref)
+    _no_device_error()
+
+
 def test_launch_count_and_profile(merge_mode):
     cfg = _grid_cfg("bf16", 128, 16, 8)
     inp = wl.make_decode_inputs(cfg, 14, context_lens=(2000, 30))
