@@ -66,6 +66,8 @@ def parse():
     p.add_argument("--swap-mb", type=int, default=0,
                    help="> 0: time pa_swap_blocks moving this many MiB of blocks (K and V) between the "
                         "device pool and a pinned host pool, against one contiguous copy of the same bytes")
+    p.add_argument("--verify-kernel", default="mma_sync", choices=["mma_sync", "tcgen05"],
+                   help="tensor-core path of the verification pass (with --queries > 1)")
     p.add_argument("--queries", type=int, default=1,
                    help="candidate tokens per sequence: > 1 times the verification pass (pa_verify) "
                         "of speculative decoding instead of decode")
@@ -320,6 +322,7 @@ def run_native(args):
     from paged_kv_cache_381_b200.batch import PagedBatch
     pa.set_decode_math(pa.MATH_AUTO if args.math == "auto" else pa.MATH_SIMT)
     pa.set_split_merge(pa.MERGE_KERNEL if args.merge == "kernel" else pa.MERGE_FUSED)
+    pa.set_verify_kernel(pa.VERIFY_TCGEN05 if args.verify_kernel == "tcgen05" else pa.VERIFY_MMA_SYNC)
 
     cfg = wl.CONFIGS[args.workload]
     seed = args.seed + rank                       # independent replica per rank
@@ -471,6 +474,7 @@ def run_native(args):
         result["metric"] = VERIFY_METRIC
         result["tokens_per_s"] = world * len(lens) * Q / (ms * 1e-3)
         result["config"]["queries_per_seq"] = Q
+        result["config"]["verify_kernel"] = args.verify_kernel
         result["tensor"] = {"flops_per_launch": fl, "achieved_tflops": fl / (dec_ms * 1e-3) / 1e12,
                             "peak_tflops": tpeak, "frac": fl / (dec_ms * 1e-3) / 1e12 / tpeak,
                             "peak_source": tkind, "note": "plain flops; P.V runs as two mma (16-bit value + remainder)"}

@@ -182,6 +182,18 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
                     void* stream);
 
 /*
+ * Tensor-core path of pa_verify (process-wide):
+ *   PA_VERIFY_MMA_SYNC  warp-level mma.m16n8k16 with accumulators in registers
+ *   PA_VERIFY_TCGEN05   tcgen05.mma issued by one thread, accumulators in tensor
+ *                       memory, operands in shared memory
+ * Same results within the stated tolerance; bits differ between the two.
+ */
+#define PA_VERIFY_MMA_SYNC 0
+#define PA_VERIFY_TCGEN05 1
+pa_status pa_set_verify_kernel(int kind);
+int pa_get_verify_kernel(void);
+
+/*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
  * memory.  The pages have no counterpart to this call: it exists for users of
  * this library whose device memory is already spoken for (a serving engine

@@ -322,6 +322,18 @@ def get_split_merge():
     return int(lib().pa_get_split_merge())
 
 
+VERIFY_MMA_SYNC, VERIFY_TCGEN05 = 0, 1
+
+
+def set_verify_kernel(kind):
+    """pa_verify's tensor-core path: VERIFY_MMA_SYNC or VERIFY_TCGEN05."""
+    _check(lib().pa_set_verify_kernel(int(kind)), "pa_set_verify_kernel")
+
+
+def get_verify_kernel():
+    return int(lib().pa_get_verify_kernel())
+
+
 def launch_count():
     return int(lib().pa_launch_count())
 

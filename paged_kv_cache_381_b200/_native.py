@@ -67,6 +67,8 @@ SIGNATURES = {
     "pa_set_decode_math": (c_int, [c_int]),
     "pa_get_decode_math": (c_int, []),
     "pa_set_split_merge": (c_int, [c_int]),
+    "pa_set_verify_kernel": (c_int, [c_int]),
+    "pa_get_verify_kernel": (c_int, []),
     "pa_get_split_merge": (c_int, []),
     "pa_profile_begin": (c_int, []),
     "pa_profile_begin_mask": (c_int, [c_uint32]),

@@ -14,6 +14,7 @@
 #include "device/cache_ops.cuh"
 #include "device/decode.cuh"
 #include "device/verify.cuh"
+#include "device/verify_tc.cuh"
 #include "pa.h"
 
 namespace {
@@ -286,6 +287,35 @@ pa_status launch_verify(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, cons
     return launch_dependent(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream, a, tk, tv);
 }
 
+template <typename T, int D>
+pa_status launch_verify_tc(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                           int64_t pair_upper, cudaStream_t stream) {
+    using C = pa_dev::VerifyTcCfg<T, D>;
+    auto kern = pa_dev::verify_tc_kernel<T, D>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    static std::atomic<uint64_t> configured{0};
+    static std::atomic<int> occ_of[kMaxDevices];
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) != cudaSuccess)
+            return PA_ERR_CUDA;
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, C::THREADS, C::SMEM) != cudaSuccess || occ <= 0)
+            return PA_ERR_CUDA;
+        if (dev < kMaxDevices) occ_of[dev].store(occ);
+        configured.fetch_or(bit);
+    }
+    // two CTAs per SM at most: each holds 256 of the SM's 512 TMEM columns
+    const int occ = std::min(2, dev < kMaxDevices ? std::max(1, occ_of[dev].load()) : 1);
+    const int64_t items_upper = pair_upper * a.num_kv_heads * a.n_gchunks;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items_upper, (int64_t)device_sms(dev) * occ));
+    LaunchScope scope(PA_KERNEL_VERIFY, stream);
+    return launch_dependent(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream, a, tk, tv);
+}
+
+std::atomic<int> g_verify_kernel{PA_VERIFY_MMA_SYNC};
+
 int query_chunk(int group, bool tensor) {
     if (tensor) return 8;                  // mma n = 8: one tile holds up to 8 queries
     int g = std::min(group, 8);
@@ -370,6 +400,14 @@ pa_status pa_set_split_merge(int mode) {
 }
 
 int pa_get_split_merge(void) { return g_split_merge.load(); }
+
+pa_status pa_set_verify_kernel(int kind) {
+    if (kind != PA_VERIFY_MMA_SYNC && kind != PA_VERIFY_TCGEN05) return PA_ERR_INVALID_ARG;
+    g_verify_kernel.store(kind);
+    return PA_OK;
+}
+
+int pa_get_verify_kernel(void) { return g_verify_kernel.load(); }
 
 pa_status pa_profile_begin(void) { return pa_profile_begin_mask(0xffffffffu); }
 
@@ -657,13 +695,23 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
         !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, block_size))
         return PA_ERR_CUDA;
     const int64_t pair_upper = (int64_t)num_seqs * maxP;
+    const bool tc5 = g_verify_kernel.load(std::memory_order_relaxed) == PA_VERIFY_TCGEN05;
     pa_status st;
-    if (dtype == PA_F16)
-        st = head_dim == 64 ? launch_verify<__half, 64>(a, tk, tv, pair_upper, s)
-                            : launch_verify<__half, 128>(a, tk, tv, pair_upper, s);
-    else
-        st = head_dim == 64 ? launch_verify<__nv_bfloat16, 64>(a, tk, tv, pair_upper, s)
-                            : launch_verify<__nv_bfloat16, 128>(a, tk, tv, pair_upper, s);
+    if (dtype == PA_F16) {
+        if (tc5)
+            st = head_dim == 64 ? launch_verify_tc<__half, 64>(a, tk, tv, pair_upper, s)
+                                : launch_verify_tc<__half, 128>(a, tk, tv, pair_upper, s);
+        else
+            st = head_dim == 64 ? launch_verify<__half, 64>(a, tk, tv, pair_upper, s)
+                                : launch_verify<__half, 128>(a, tk, tv, pair_upper, s);
+    } else {
+        if (tc5)
+            st = head_dim == 64 ? launch_verify_tc<__nv_bfloat16, 64>(a, tk, tv, pair_upper, s)
+                                : launch_verify_tc<__nv_bfloat16, 128>(a, tk, tv, pair_upper, s);
+        else
+            st = head_dim == 64 ? launch_verify<__nv_bfloat16, 64>(a, tk, tv, pair_upper, s)
+                                : launch_verify<__nv_bfloat16, 128>(a, tk, tv, pair_upper, s);
+    }
     if (st != PA_OK || maxP <= 1) return st;
     pa_dev::DecodeArgs r = a;               // the reduce sees rows [s][i][h] as num_queries * num_heads heads
     r.num_heads = num_queries * num_heads;

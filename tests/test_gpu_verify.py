@@ -31,6 +31,15 @@ def _gpu():
     yield
 
 
+@pytest.fixture(autouse=True, params=["mma_sync", "tcgen05"])
+def verify_kind(request):
+    """Every case runs on both tensor-core paths of pa_verify."""
+    before = pa.get_verify_kernel()
+    pa.set_verify_kernel(pa.VERIFY_TCGEN05 if request.param == "tcgen05" else pa.VERIFY_MMA_SYNC)
+    yield request.param
+    pa.set_verify_kernel(before)
+
+
 def _cfg(dtype="bf16", Hq=16, Hkv=2, D=128, bs=16, lens=(6, 17, 40, 100)):
     return wl.DecodeConfig("verify", dtype, len(lens), Hq, Hkv, D, bs, "fixed", fixed_lengths=tuple(lens))
 
