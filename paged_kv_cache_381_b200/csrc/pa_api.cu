@@ -298,7 +298,9 @@ pa_status launch_verify_tc(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, c
     static std::atomic<int> occ_of[kMaxDevices];
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) != cudaSuccess)
+        // the whole unified L1 as shared memory, so that two CTAs fit
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) != cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
             return PA_ERR_CUDA;
         int occ = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, C::THREADS, C::SMEM) != cudaSuccess || occ <= 0)
