@@ -63,8 +63,8 @@ struct VerifyTcCfg {
     static constexpr int OFF_Q = NSLOTS * SLOT_BYTES;
     static constexpr int OFF_P = OFF_Q + Q_BYTES;            // tile (buffer b, part h) at (2 b + h) * P_TILE
     static constexpr int OFF_BAR = OFF_P + 4 * P_TILE;
-    // barriers: full[NSLOTS], empty[NSLOTS], s_full[2], q_full, q_empty, p_full, o_full, o_empty, drain
-    static constexpr int NBAR = 2 * NSLOTS + 8;
+    // barriers: full[NSLOTS], empty[NSLOTS], s_full[2], q_full, q_empty, p_full, o_full[2], o_empty, drain
+    static constexpr int NBAR = 2 * NSLOTS + 9;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;      // allocated TMEM address
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
     static constexpr int OFF_TABLE = (OFF_ABORT + 4 + 15) / 16 * 16;
@@ -128,9 +128,9 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     uint64_t* q_full = s_full + 2;               // Q tile written (128 arrivals)
     uint64_t* q_empty = s_full + 3;              // last S of the item done (commit)
     uint64_t* p_full = s_full + 4;               // chunk's S read, O rescaled, p written (128 arrivals)
-    uint64_t* o_full = s_full + 5;               // P.V of a chunk done (commit)
-    uint64_t* o_empty = s_full + 6;              // O read by the epilogue (128 arrivals)
-    uint64_t* drain = s_full + 7;                // every MMA done, before TMEM is freed
+    uint64_t* o_full = s_full + 5;               // [2] P.V of a chunk using P buffer b done (commit)
+    uint64_t* o_empty = s_full + 7;              // O read by the epilogue (128 arrivals)
+    uint64_t* drain = s_full + 8;                // every MMA done, before TMEM is freed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + C::OFF_TABLE);
@@ -149,7 +149,8 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         mbar_init(q_full, 128);
         mbar_init(q_empty, 1);
         mbar_init(p_full, 128);
-        mbar_init(o_full, 1);
+        mbar_init(&o_full[0], 1);
+        mbar_init(&o_full[1], 1);
         mbar_init(o_empty, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 }
                 __syncwarp();
             }
-            if (lane == 0) tc::commit(o_full);
+            if (lane == 0) tc::commit(&o_full[buf]);
             __syncwarp();
             return true;
         };
@@ -351,7 +352,11 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         T* outg = static_cast<T*>(a.out);
         const int Q = a.num_queries;
         const int R = a.group * Q;
-        uint32_t qe_ph = 0, o_ph = 0, gch = 0;
+        uint32_t qe_ph = 0, gch = 0;
+        // P.V of global chunk g (P buffer g & 1) done: its use of o_full[g & 1] is g >> 1
+        auto wait_pv = [&](uint32_t g) -> bool {
+            return mbar_wait(&o_full[g & 1u], (g >> 1) & 1u, abort_flag);
+        };
         bool ok = true;
         for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
             const WorkItem w = decode_item(a, i, false);
@@ -426,9 +431,14 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     cmax = fmaxf(cmax, z);
                 }
                 cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 16));
-                const float m_new = fmaxf(m_run, cmax);
+                // Lazy reference max: p = 2^(z - m_run) stays <= 2^8, so the reference only
+                // moves (and O is rescaled) when a score beats it by more than 8 in base-2
+                // units; a row that has seen nothing yet takes the chunk max (its O is zero).
+                const bool fresh = m_run == -INFINITY;
+                const bool raise = fresh ? cmax != -INFINITY : cmax > m_run + 8.f;
+                const float m_new = raise ? cmax : m_run;
                 const float base = m_new == -INFINITY ? 0.f : m_new;       // a row that saw nothing yet
-                const float corr = exp2f(m_run - base);
+                const float corr = raise && !fresh ? exp2f(m_run - m_new) : 1.f;
                 uint32_t hi[16], lo[16];
                 float lsum = 0.f;
 #pragma unroll
@@ -438,24 +448,25 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     lsum += p0 + p1;
                     split_pack<MO>(p0, p1, hi[k >> 1], lo[k >> 1]);
                 }
-                // the previous chunk's P.V must be done before O is rescaled
-                if (c > 0) {
-                    if (!(ok = mbar_wait(o_full, o_ph, abort_flag))) break;
-                    o_ph ^= 1u;
+                const uint32_t gc = gch + c;
+                // O rescale: only when some row of this warp moved its reference, after the
+                // previous chunk's P.V has landed
+                if (c > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+                    if (!(ok = wait_pv(gc - 1))) break;
                     tc::fence_after_sync();
-                    if (__any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll 1
-                        for (int g = 0; g < D / 64; ++g) {
-                            uint32_t o[32];
-                            tc::ld16x2(tmem + lane_addr + C::O_COL + g * 64, o);
-                            tc::wait_ld();
+                    for (int g = 0; g < D / 64; ++g) {
+                        uint32_t o[32];
+                        tc::ld16x2(tmem + lane_addr + C::O_COL + g * 64, o);
+                        tc::wait_ld();
 #pragma unroll
-                            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * corr);
-                            tc::st16x2(tmem + lane_addr + C::O_COL + g * 64, o);
-                        }
-                        tc::wait_st();
+                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * corr);
+                        tc::st16x2(tmem + lane_addr + C::O_COL + g * 64, o);
                     }
+                    tc::wait_st();
                 }
+                // P buffer gc & 1 was last read by the P.V of chunk gc - 2
+                if (gc >= 2 && !(ok = wait_pv(gc - 2))) break;
                 m_run = m_new;
                 l_run = l_run * corr + lsum;
                 // p of row m, tokens half*32 .. +31 of the chunk: 16-byte chunks 4*half .. +3 of the row
@@ -474,8 +485,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             gch += nc;
             if (!ok) break;
             // ---- epilogue: O after the last chunk, normalised row or partition partials
-            if (!(ok = mbar_wait(o_full, o_ph, abort_flag))) break;
-            o_ph ^= 1u;
+            if (!(ok = wait_pv(gch - 1))) break;
             tc::fence_after_sync();
             const float l_row = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
             const bool single = w.np == 1;

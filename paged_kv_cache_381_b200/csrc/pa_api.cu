@@ -302,9 +302,15 @@ pa_status launch_verify_tc(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, c
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) != cudaSuccess ||
             cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
             return PA_ERR_CUDA;
-        int occ = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, C::THREADS, C::SMEM) != cudaSuccess || occ <= 0)
+        // CTAs per SM from the shared memory (1 KB reserved per CTA) and the registers
+        int smem_sm = 0;
+        cudaFuncAttributes fa;
+        if (cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
             return PA_ERR_CUDA;
+        const int by_smem = smem_sm / (int)(C::SMEM + 1024);
+        const int by_regs = 65536 / std::max(1, fa.numRegs * C::THREADS);
+        const int occ = std::max(1, std::min(by_smem, by_regs));
         if (dev < kMaxDevices) occ_of[dev].store(occ);
         configured.fetch_or(bit);
     }
