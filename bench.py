@@ -66,7 +66,7 @@ def parse():
     p.add_argument("--swap-mb", type=int, default=0,
                    help="> 0: time pa_swap_blocks moving this many MiB of blocks (K and V) between the "
                         "device pool and a pinned host pool, against one contiguous copy of the same bytes")
-    p.add_argument("--verify-kernel", default="mma_sync", choices=["mma_sync", "tcgen05"],
+    p.add_argument("--verify-kernel", default="auto", choices=["auto", "mma_sync", "tcgen05"],
                    help="tensor-core path of the verification pass (with --queries > 1)")
     p.add_argument("--queries", type=int, default=1,
                    help="candidate tokens per sequence: > 1 times the verification pass (pa_verify) "
@@ -322,7 +322,8 @@ def run_native(args):
     from paged_kv_cache_381_b200.batch import PagedBatch
     pa.set_decode_math(pa.MATH_AUTO if args.math == "auto" else pa.MATH_SIMT)
     pa.set_split_merge(pa.MERGE_KERNEL if args.merge == "kernel" else pa.MERGE_FUSED)
-    pa.set_verify_kernel(pa.VERIFY_TCGEN05 if args.verify_kernel == "tcgen05" else pa.VERIFY_MMA_SYNC)
+    pa.set_verify_kernel({"auto": pa.VERIFY_AUTO, "tcgen05": pa.VERIFY_TCGEN05,
+                          "mma_sync": pa.VERIFY_MMA_SYNC}[args.verify_kernel])
 
     cfg = wl.CONFIGS[args.workload]
     seed = args.seed + rank                       # independent replica per rank

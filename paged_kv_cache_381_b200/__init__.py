@@ -322,11 +322,11 @@ def get_split_merge():
     return int(lib().pa_get_split_merge())
 
 
-VERIFY_MMA_SYNC, VERIFY_TCGEN05 = 0, 1
+VERIFY_MMA_SYNC, VERIFY_TCGEN05, VERIFY_AUTO = 0, 1, 2
 
 
 def set_verify_kernel(kind):
-    """pa_verify's tensor-core path: VERIFY_MMA_SYNC or VERIFY_TCGEN05."""
+    """pa_verify's tensor-core path: VERIFY_MMA_SYNC, VERIFY_TCGEN05 or VERIFY_AUTO (default)."""
     _check(lib().pa_set_verify_kernel(int(kind)), "pa_set_verify_kernel")
 
 

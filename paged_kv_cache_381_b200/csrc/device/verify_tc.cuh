@@ -73,39 +73,8 @@ struct VerifyTcCfg {
     static constexpr int THREADS = 6 * 32;
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(SLOT_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0 && P_TILE % 1024 == 0, "1024-byte atoms");
+    static_assert((M * D * 2 / 16) % 128 == 0, "q tile chunks per staging thread");
 };
-
-// Slot stream of an item with `nst` slots of 32 tokens: chunk c holds slots
-// 2c and 2c+1; the stream is K(0), then for every chunk c: K(c+1) (if any),
-// V(c).  Position k of the stream -> (slot, V or K).
-__device__ __forceinline__ void tc_stream_slot(int k, int nst, int& slot, bool& is_v) {
-    const int nc = (nst + 1) / 2;
-    const int first = min(2, nst);
-    slot = 0;
-    is_v = false;
-    if (k < first) {
-        slot = k;
-        return;
-    }
-    int rem = k - first;
-    for (int c = 0; c < nc; ++c) {
-        if (c + 1 < nc) {
-            const int nk = min(2, nst - 2 * (c + 1));
-            if (rem < nk) {
-                slot = 2 * (c + 1) + rem;
-                return;
-            }
-            rem -= nk;
-        }
-        const int nv = min(2, nst - 2 * c);
-        if (rem < nv) {
-            slot = 2 * c + rem;
-            is_v = true;
-            return;
-        }
-        rem -= nv;
-    }
-}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
@@ -178,7 +147,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             prefetch_tmap(&tmap_v);
         }
         const uint64_t policy = l2_policy_evict_first();
-        uint32_t seq = 0;                                   // ring uses so far
+        uint32_t seq = 0;                                   // ring uses so far (K K V K V ... order)
         bool ok = true;
         for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
             const WorkItem w = decode_item(a, i, lane == 0);
@@ -196,28 +165,38 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             }
             __syncwarp();
             const int nst = (w.n + C::SLOT_ROWS - 1) / C::SLOT_ROWS;
-            for (int k = 0; k < 2 * nst; ++k, ++seq) {
-                int st;
-                bool is_v;
-                tc_stream_slot(k, nst, st, is_v);
-                const int slot = seq % C::NSLOTS;
-                if (!mbar_wait(&empty[slot], ((seq / C::NSLOTS) & 1u) ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
+            const int nc = (nst + 1) / 2;
+            // the chunk's K or V slots in one round: both ring slots are waited for,
+            // then one warp instruction issues every box (16 lanes per slot)
+            auto issue = [&](int c, bool is_v) -> bool {
+                const int nb = min(2, nst - 2 * c);
+                for (int j = 0; j < nb; ++j) {
+                    const uint32_t sq = seq + j;
+                    if (!mbar_wait(&empty[sq % C::NSLOTS], ((sq / C::NSLOTS) & 1u) ^ 1u, abort_flag)) return false;
                 }
-                const int rows = min(C::SLOT_ROWS, w.n - st * C::SLOT_ROWS);
-                const int nb = (rows + bs - 1) >> a.log2_bs;       // whole blocks
-                const int nbox = nb * C::NH;
-                if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbox * box_bytes));
+                const int j = lane >> 4;
+                const int e = lane & 15;
+                const int st = 2 * c + j;
+                const int slot = (seq + j) % C::NSLOTS;
+                const int rows = j < nb ? min(C::SLOT_ROWS, w.n - st * C::SLOT_ROWS) : 0;
+                const int nbk = (rows + bs - 1) >> a.log2_bs;      // whole blocks
+                if (j < nb && e == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbk * C::NH * box_bytes));
                 __syncwarp();
-                if (lane < nbox) {
-                    const int half = lane / nb;                     // slice
-                    const int b = lane - half * nb;                 // block within the slot
+                if (e < nbk * C::NH) {
+                    const int half = e / nbk;                       // slice
+                    const int b = e - half * nbk;                   // block within the slot
                     const int phys = tbl[((st * C::SLOT_ROWS) >> a.log2_bs) + b];
                     tma_load_3d(smem + slot * C::SLOT_BYTES + half * C::SLICE_BYTES + b * box_bytes,
                                 is_v ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
                                 half * C::BOX_ELEMS, w.h, phys * bs, &full[slot], policy);
                 }
+                seq += nb;
+                return true;
+            };
+            if (!(ok = issue(0, false))) break;
+            for (int c = 0; c < nc && ok; ++c) {
+                if (c + 1 < nc && !(ok = issue(c + 1, false))) break;
+                ok = issue(c, true);
             }
         }
         if (!ok) {
@@ -392,16 +371,25 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             }
             qe_ph ^= 1u;
             {
+                // all loads of this thread first, then the swizzled stores
                 constexpr int VPR = D * 2 / 16;           // 16-byte chunks per row
-                for (int e = ctid; e < C::M * VPR; e += 128) {
-                    const int lr = e / VPR;
-                    const int cc = e - lr * VPR;
+                constexpr int PER = C::M * VPR / 128;     // chunks per thread
+                uint4 v[PER];
+#pragma unroll
+                for (int u = 0; u < PER; ++u) {
+                    const int e = ctid + u * 128;
                     int64_t orow;
                     int pos;
-                    row_of(lr, orow, pos);
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (orow >= 0) v = __ldg(reinterpret_cast<const uint4*>(qg + orow * D) + cc);
-                    *reinterpret_cast<uint4*>(qs + (cc >> 3) * C::Q_SLICE + lr * 128 + (((cc & 7) ^ (lr & 7)) << 4)) = v;
+                    row_of(e / VPR, orow, pos);
+                    v[u] = orow >= 0 ? __ldg(reinterpret_cast<const uint4*>(qg + orow * D) + (e % VPR))
+                                     : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < PER; ++u) {
+                    const int e = ctid + u * 128;
+                    const int lr = e / VPR;
+                    const int cc = e % VPR;
+                    *reinterpret_cast<uint4*>(qs + (cc >> 3) * C::Q_SLICE + lr * 128 + (((cc & 7) ^ (lr & 7)) << 4)) = v[u];
                 }
                 tc::fence_proxy_async_smem();
                 mbar_arrive(q_full);

@@ -322,7 +322,7 @@ pa_status launch_verify_tc(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, c
     return launch_dependent(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream, a, tk, tv);
 }
 
-std::atomic<int> g_verify_kernel{PA_VERIFY_MMA_SYNC};
+std::atomic<int> g_verify_kernel{PA_VERIFY_AUTO};
 
 int query_chunk(int group, bool tensor) {
     if (tensor) return 8;                  // mma n = 8: one tile holds up to 8 queries
@@ -410,7 +410,7 @@ pa_status pa_set_split_merge(int mode) {
 int pa_get_split_merge(void) { return g_split_merge.load(); }
 
 pa_status pa_set_verify_kernel(int kind) {
-    if (kind != PA_VERIFY_MMA_SYNC && kind != PA_VERIFY_TCGEN05) return PA_ERR_INVALID_ARG;
+    if (kind != PA_VERIFY_MMA_SYNC && kind != PA_VERIFY_TCGEN05 && kind != PA_VERIFY_AUTO) return PA_ERR_INVALID_ARG;
     g_verify_kernel.store(kind);
     return PA_OK;
 }
@@ -703,7 +703,8 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
         !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, block_size))
         return PA_ERR_CUDA;
     const int64_t pair_upper = (int64_t)num_seqs * maxP;
-    const bool tc5 = g_verify_kernel.load(std::memory_order_relaxed) == PA_VERIFY_TCGEN05;
+    const int vk = g_verify_kernel.load(std::memory_order_relaxed);
+    const bool tc5 = vk == PA_VERIFY_TCGEN05 || (vk == PA_VERIFY_AUTO && rows > 16);
     pa_status st;
     if (dtype == PA_F16) {
         if (tc5)

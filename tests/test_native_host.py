@@ -278,6 +278,22 @@ def test_verify_workspace_and_argument_rules(pa):
     assert lib.pa_verify(*args(6, 2)) == 1            # null pointers
 
 
+def test_verify_kernel_selection(pa):
+    """The process-wide tensor-core path of pa_verify: AUTO by default, the
+    three named kinds accepted, anything else rejected with nothing changed."""
+    assert pa.get_verify_kernel() == pa.VERIFY_AUTO
+    try:
+        for k in (pa.VERIFY_MMA_SYNC, pa.VERIFY_TCGEN05, pa.VERIFY_AUTO):
+            pa.set_verify_kernel(k)
+            assert pa.get_verify_kernel() == k
+        pa.set_verify_kernel(pa.VERIFY_TCGEN05)
+        assert pa.lib().pa_set_verify_kernel(3) == 1
+        assert pa.lib().pa_set_verify_kernel(-1) == 1
+        assert pa.get_verify_kernel() == pa.VERIFY_TCGEN05
+    finally:
+        pa.set_verify_kernel(pa.VERIFY_AUTO)
+
+
 @pytest.mark.parametrize("ncpu,nb", [(6, 60), (40, 60), (400, 50)])
 def test_scheduler_swap_matches_model(pa, ncpu, nb):
     """Preemption by swap: C++ and Python agree every step (ops incl. swap
