@@ -43,8 +43,14 @@ WORKLOAD_NAMES = {
 }
 METRIC = "paged decode attention: KV GB/s read (% of B200 HBM peak); decode tokens/s"
 VERIFY_METRIC = "paged verification attention (speculative decoding): KV GB/s read; verified tokens/s"
-KERNEL_SOURCES = ["paged_kv_cache_381_b200/csrc/device/decode.cuh",
-                  "paged_kv_cache_381_b200/csrc/device/common.cuh"]
+_DEV = "paged_kv_cache_381_b200/csrc/device/"
+# the sources each timed kernel is built from: a recorded ncu traffic figure is
+# reported only while their hash is the one it was taken on
+KERNEL_SOURCES = {
+    "decode": [_DEV + "decode.cuh", _DEV + "common.cuh"],
+    "verify": [_DEV + "verify.cuh", _DEV + "decode.cuh", _DEV + "common.cuh"],
+    "verify_tc": [_DEV + "verify_tc.cuh", _DEV + "tcgen05.cuh", _DEV + "decode.cuh", _DEV + "common.cuh"],
+}
 
 
 def parse():
@@ -68,6 +74,11 @@ def parse():
                         "device pool and a pinned host pool, against one contiguous copy of the same bytes")
     p.add_argument("--verify-kernel", default="auto", choices=["auto", "mma_sync", "tcgen05"],
                    help="tensor-core path of the verification pass (with --queries > 1)")
+    p.add_argument("--partition-size", type=int, default=0,
+                   help="split-K partition in tokens (power of two >= the block size); 0: the workload's (512)")
+    p.add_argument("--profile-all", action="store_true",
+                   help="event-time every library launch (kernel_ms per kernel); the events between "
+                        "dependent launches cost the step its launch overlap, so ms_per_step rises")
     p.add_argument("--queries", type=int, default=1,
                    help="candidate tokens per sequence: > 1 times the verification pass (pa_verify) "
                         "of speculative decoding instead of decode")
@@ -83,23 +94,27 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_hash():
+def kernel_hash(kernel="decode"):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"decode_{workload}_traffic.json")
+def traffic_profile_name(kernel, workload, queries):
+    return f"{kernel}_{workload}_traffic.json" if queries == 1 else f"{kernel}_{workload}_q{queries}_traffic.json"
+
+
+def recorded_traffic(kernel, workload, queries=1):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary for this
+    workload, if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", traffic_profile_name(kernel, workload, queries))
     if not os.path.exists(path):
         return None
     with open(path) as f:
         j = json.load(f)
-    if j.get("kernel_source_sha256_16") != kernel_hash():
+    if j.get("kernel_source_sha256_16") != kernel_hash(kernel):
         return None
     return j.get("dram_bytes_per_launch")
 
@@ -341,7 +356,7 @@ def run_native(args):
         q = torch.randn((len(lens), Q, cfg.num_heads, cfg.head_dim), generator=gq, device=dev,
                         dtype=torch.float32).to(d.q.dtype)
     out = torch.empty_like(q)
-    P = cfg.partition_size
+    P = args.partition_size or cfg.partition_size
     batch.ensure_workspace(cfg.num_heads, P)
     step_kv = kv_bytes(cfg, lens)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -349,7 +364,13 @@ def run_native(args):
     torch.cuda.synchronize()
     pa.pa_get_device_error()
 
-    kernel = "verify" if Q > 1 else "decode"
+    kernel = "verify" if Q > 1 else "decode"      # the library's launch-profile id
+    if Q == 1:
+        kname = "decode"
+    elif args.verify_kernel == "tcgen05" or (args.verify_kernel == "auto" and cfg.num_heads // cfg.num_kv_heads * Q > 16):
+        kname = "verify_tc"       # the choice pa_verify makes for VERIFY_AUTO
+    else:
+        kname = "verify"
 
     def step():
         batch.write_new_tokens()
@@ -370,7 +391,7 @@ def run_native(args):
     clocks.start()
     time.sleep(0.3)
     launches0 = pa.launch_count()
-    pa.profile_begin([kernel])            # events around the attention kernel only
+    pa.profile_begin(None if args.profile_all else [kernel])   # default: the attention kernel only
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -446,10 +467,9 @@ def run_native(args):
     peak, peak_kind = measured_peaks()
     if Q > 1:
         dec_bytes = verify_kernel_bytes(cfg, lens, P, Q)
-        traffic = None
     else:
         dec_bytes = decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused")
-        traffic = recorded_traffic(args.workload)
+    traffic = None if args.num_seqs else recorded_traffic(kname, args.workload, Q)
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     value = world * step_kv / (ms * 1e-3) / 1e9
     result = {
@@ -464,7 +484,7 @@ def run_native(args):
         "tokens_per_s": world * len(lens) / (ms * 1e-3),
         "kernel_ms": {k: v[0] / max(1, v[1]) for k, v in prof.items() if v[1]},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": f"{kernel}_kernel", "algorithmic_bytes": dec_bytes,
+                     "traffic": traffic, "kernel": f"{kname}_kernel", "algorithmic_bytes": dec_bytes,
                      "peak_source": peak_kind},
         "gpu_launches": int(launches), "device_error_flags": err, "wall_s": wall,
         "e2e": e2e, "clocks": clk,

@@ -263,13 +263,17 @@ class Pipeline:
 
     def __init__(self, depth=2):
         self._h = ctypes.c_void_p()
+        self._destroy = lib().pa_pipeline_destroy
         _check(lib().pa_pipeline_create(int(depth), ctypes.byref(self._h)), "pa_pipeline_create")
         self.depth = int(depth)
 
     def __del__(self):
+        # the destroy call was bound at construction: module globals may already be
+        # gone when this runs at interpreter exit
         h = getattr(self, "_h", None)
-        if h:
-            lib().pa_pipeline_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h and destroy is not None:
+            destroy(h)
             self._h = None
 
     def begin(self, like, stream=None):
@@ -374,14 +378,18 @@ class BlockManager:
 
     def __init__(self, num_blocks, block_size, initial_free_order=None):
         self._h = ctypes.c_void_p()
+        self._destroy = lib().pa_bm_destroy
         order = None if initial_free_order is None else _i32(initial_free_order)
         _check(lib().pa_bm_create(num_blocks, block_size, _ptr(order), ctypes.byref(self._h)), "pa_bm_create")
         self.num_blocks, self.block_size = num_blocks, block_size
 
     def __del__(self):
+        # the destroy call was bound at construction: module globals may already be
+        # gone when this runs at interpreter exit
         h = getattr(self, "_h", None)
-        if h:
-            lib().pa_bm_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h and destroy is not None:
+            destroy(h)
             self._h = None
 
     @property
@@ -532,14 +540,18 @@ class Scheduler:
     def __init__(self, bm, max_running, prefix_seq=-1, preempt="recompute"):
         self.bm = bm           # keeps the block manager alive
         self._h = ctypes.c_void_p()
+        self._destroy = lib().pa_sched_destroy
         _check(lib().pa_sched_create(bm.handle, max_running, prefix_seq, ctypes.byref(self._h)), "pa_sched_create")
         _check(lib().pa_sched_set_preemption(self._h, {"recompute": 0, "swap": 1}[preempt]),
                "pa_sched_set_preemption")
 
     def __del__(self):
+        # the destroy call was bound at construction: module globals may already be
+        # gone when this runs at interpreter exit
         h = getattr(self, "_h", None)
-        if h:
-            lib().pa_sched_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h and destroy is not None:
+            destroy(h)
             self._h = None
 
     def add_request(self, seq_id, prompt_len, output_len, shares_prefix=False, fork_child=-1, fork_output_len=0):

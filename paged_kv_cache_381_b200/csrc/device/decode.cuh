@@ -230,9 +230,6 @@ __device__ __forceinline__ void merge_partitions(const DecodeArgs& a, int64_t ro
 #ifndef PA_DECODE_MIN_CTAS
 #define PA_DECODE_MIN_CTAS 4
 #endif
-#ifndef PA_DECODE_PRODUCER_BATCH
-#define PA_DECODE_PRODUCER_BATCH 1   // measured: 2 stages per round is not faster here
-#endif
 
 template <typename T, int D, int GC, bool TENSOR>
 struct DecodeCfg {
@@ -248,8 +245,6 @@ struct DecodeCfg {
     static constexpr int STAGE_BYTES = STAGE_ROWS * ROW_BYTES;
     static constexpr int NSTAGES = PA_DECODE_STAGES;
     static constexpr int NCW = 4;                   // consumer warps
-    static constexpr int PB = PA_DECODE_PRODUCER_BATCH;   // stages the producer issues per round
-    static constexpr int LPS = 32 / PB;                    // producer lanes per stage of a round
     static constexpr int THREADS = (NCW + 1) * 32;
     static constexpr int MAX_PARTITION = 1024;
     static constexpr int MAX_TABLE = MAX_PARTITION / 8;
@@ -277,8 +272,6 @@ struct DecodeCfg {
     // use (another warp's) is still in flight, and the parity test would answer
     // "complete" for the wrong phase.
     static_assert(NSTAGES % NCW == 0, "ring depth must be a multiple of the consumer warps");
-    static_assert(PB >= 1 && PB <= NSTAGES && 32 % PB == 0, "producer rounds");
-    static_assert((STAGE_ROWS / 8) * NH <= LPS, "one lane per box of a stage (8-token blocks at most)");
     // + 1024: the dynamic shared-memory base is rounded up to 1024 bytes in the kernel
     static size_t smem_bytes(int partition) {
         const size_t scores = (size_t)partition * LSTRIDE * 4;
@@ -369,32 +362,25 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
             __syncwarp();
             for (int pass = 0; pass < 2 && ok; ++pass) {
                 const void* tmap = pass ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
-                // PB stages per round: their slots are waited for first, then one warp
-                // instruction issues every box of the round (32 / PB lanes per stage)
-                for (int st0 = 0; st0 < nst; st0 += C::PB) {
-                    const int nb = min(C::PB, nst - st0);
-                    for (int j = 0; j < nb && ok; ++j) {
-                        const uint32_t sq = stage + j;
-                        ok = mbar_wait(&empty[sq % C::NSTAGES], ((sq / C::NSTAGES) & 1u) ^ 1u, abort_flag);
+                for (int st = 0; st < nst; ++st, ++stage) {
+                    const int slot = stage % C::NSTAGES;
+                    const uint32_t parity = ((stage / C::NSTAGES) & 1u) ^ 1u;
+                    if (!mbar_wait(&empty[slot], parity, abort_flag)) {
+                        ok = false;
+                        break;
                     }
-                    if (!ok) break;
-                    const int j = lane / C::LPS;                    // stage of this lane within the round
-                    const int e = lane - j * C::LPS;                // box of this lane within its stage
-                    const int st = st0 + j;
-                    const uint32_t sq = stage + j;
-                    const int slot = sq % C::NSTAGES;
-                    const int rows = j < nb ? min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS) : 0;
-                    const int nbox = ((rows + bs - 1) >> a.log2_bs) * C::NH;   // whole blocks are loaded
-                    if (j < nb && e == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbox * box_bytes));
+                    const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
+                    const int nblk_st = (rows + bs - 1) >> a.log2_bs;      // whole blocks are loaded
+                    const int nbox = nblk_st * C::NH;
+                    if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbox * box_bytes));
                     __syncwarp();
-                    if (e < nbox) {
-                        const int b = e / C::NH;
-                        const int half = e - b * C::NH;
+                    if (lane < nbox) {
+                        const int b = lane / C::NH;
+                        const int half = lane - b * C::NH;
                         const int phys = tbl[((st * C::STAGE_ROWS) >> a.log2_bs) + b];
                         tma_load_3d(smem + slot * C::STAGE_BYTES + (b * C::NH + half) * box_bytes, tmap,
                                     half * C::BOX_ELEMS, w.h, phys * bs, &full[slot], policy);
                     }
-                    stage += nb;
                 }
             }
         }

@@ -102,6 +102,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same descriptor for a start address `bytes` further on (a multiple of 16):
+// the address field is the low 14 bits of (address >> 4), and shared-memory
+// addresses stay below 2^18, so the add never carries out of the field.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
+
 // Instruction descriptor, kind::f16 with fp32 accumulation: A/B format (0 fp16,
 // 1 bf16), operand majors (0 K-major, 1 MN-major), N >> 3, M >> 4.
 __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, bool b_mn_major, int m, int n) {

@@ -9,19 +9,25 @@
 // Design (2 CTAs per SM, each holding 256 of the SM's 512 TMEM columns):
 //  * Item = (sequence, 512-token partition, kv head, chunk of <= 64 query
 //    rows).  The rows form one M = 64 tile; the partition is walked in chunks
-//    of 64 tokens = 2 slots of 32.
-//  * Warp 0 streams K and V slots through TMA tiled boxes into one ring (slot
-//    = 32 token rows of one kv head, its 128-byte head_dim slices one after
-//    the other, 128-byte swizzle), K running one chunk ahead of V:
-//    K0 K1 V0 K2 V1 ... .
+//    of 64 tokens.
+//  * Warp 0 streams K and V chunks through TMA tiled boxes into a ring of
+//    three slots (slot = 64 token rows of one kv head; each 128-byte head_dim
+//    slice of the 64 rows is one 128-byte-swizzled array), K running one
+//    chunk ahead of V: K0 K1 V0 K2 V1 ... .  A slot is refilled once the
+//    products that read its previous contents are done: the producer waits
+//    on the same commit barrier the softmax (S done) or the next rescale
+//    (P.V done) waits on, so no separate release barrier is committed.
 //  * Warp 1 issues, from one thread, in the same order:
-//        S(c) [64 x 64]  = Q K^T   2 x KS MMAs M=64 N=32 K=16, into one of two S buffers
-//        O    [64 x D]  += P V     2 x 2 x 2 MMAs M=64 N=D K=16 (P K-major from shared
+//        S(c) [64 x 64]  = Q K^T   KS MMAs M=64 N=64 K=16, into one of two S buffers
+//        O    [64 x D]  += P V     4 x 2 MMAs M=64 N=D K=16 (P K-major from shared
 //                                  memory, V MN-major: the slot as loaded)
 //    so S(c+1) is computed while the softmax of chunk c runs.  TMEM columns:
-//    S buffers [0, 64) and [64, 128), O [128, 128 + D).  A ring slot is
-//    released by a tcgen05.commit once the MMAs reading it are done.  P is
-//    split into a 16-bit value and its remainder (two products), as in decode.
+//    S buffers [0, 64) and [64, 128), O [128, 128 + D).  P is split into a
+//    16-bit value and its remainder (two products), as in decode.  A
+//    tcgen05.mma costs its issuing thread about as much as a commit or a
+//    barrier test, whatever its N, so the chunk is covered by as few
+//    instructions as the shapes allow: one commit per product group, one
+//    barrier wait per chunk of K or V.
 //  * Warps 2-5 (one TMEM lane quarter each; a quarter's first 16 lanes hold 16
 //    rows of an M = 64 accumulator, read as two half-warps of 32 columns)
 //    stage q, take the exact max of the chunk (causal mask), rescale O in TMEM
@@ -38,8 +44,11 @@
 
 namespace pa_dev {
 
-#ifndef PA_VERIFY_TC_SLOTS
-#define PA_VERIFY_TC_SLOTS 6
+#ifndef PA_VERIFY_TC_PSPLIT
+#define PA_VERIFY_TC_PSPLIT 1    // 1: P.V as two products (16-bit p and its remainder); 0: 16-bit p only
+#endif
+#ifndef PA_VERIFY_TC_PBUF
+#define PA_VERIFY_TC_PBUF 2      // P tiles in shared memory: 2 = double-buffered, 1 = single
 #endif
 
 template <typename T, int D>
@@ -47,24 +56,28 @@ struct VerifyTcCfg {
     static constexpr int ELT = 2;
     static constexpr int NH = D * ELT / 128;                 // 128-byte head_dim slices
     static constexpr int BOX_ELEMS = 128 / ELT;
-    static constexpr int SLOT_ROWS = 32;
-    static constexpr int SLICE_BYTES = SLOT_ROWS * 128;      // one slice of a slot
+    static constexpr int CHUNK = 64;                         // tokens per chunk = rows of a ring slot
+    static constexpr int SLICE_BYTES = CHUNK * 128;          // one head_dim slice of a slot
     static constexpr int SLOT_BYTES = NH * SLICE_BYTES;
-    static constexpr int NSLOTS = PA_VERIFY_TC_SLOTS;
-    static constexpr int CHUNK = 64;                         // tokens per softmax chunk
+    // Three slots: K(c+1) and V(c) in use while the next K or V loads.  Deeper
+    // rings would break the refill rule: a slot's previous contents must be the
+    // third-last stream element, whose commit barrier cannot have moved two
+    // phases on by the time the producer tests it.
+    static constexpr int NSLOTS = 3;
     static constexpr int M = 64;                             // query rows per item
     static constexpr int Q_SLICE = M * 128;                  // one 128-byte slice of the Q tile
     static constexpr int Q_BYTES = NH * Q_SLICE;
     static constexpr int P_TILE = M * 128;                   // 64 rows x 64 tokens, one 128-byte atom column
+    static constexpr int PBUF = PA_VERIFY_TC_PBUF;
     static constexpr int TMEM_COLS = 256;
     static constexpr int S_COL = 0;                          // S buffer b: [64 b, 64 b + 64)
     static constexpr int O_COL = 128;
-    // shared memory: ring, Q, P (2 buffers x {value, remainder}), barriers, table
+    // shared memory: ring, Q, P (buffers x {value, remainder}), barriers, table
     static constexpr int OFF_Q = NSLOTS * SLOT_BYTES;
     static constexpr int OFF_P = OFF_Q + Q_BYTES;            // tile (buffer b, part h) at (2 b + h) * P_TILE
-    static constexpr int OFF_BAR = OFF_P + 4 * P_TILE;
-    // barriers: full[NSLOTS], empty[NSLOTS], s_full[2], q_full, q_empty, p_full, o_full[2], o_empty, drain
-    static constexpr int NBAR = 2 * NSLOTS + 9;
+    static constexpr int OFF_BAR = OFF_P + 2 * PBUF * P_TILE;
+    // barriers: full[NSLOTS], s_full[2], q_full, q_empty, p_full, o_full[2], o_empty, drain
+    static constexpr int NBAR = NSLOTS + 9;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;      // allocated TMEM address
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
     static constexpr int OFF_TABLE = (OFF_ABORT + 4 + 15) / 16 * 16;
@@ -74,6 +87,8 @@ struct VerifyTcCfg {
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(SLOT_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0 && P_TILE % 1024 == 0, "1024-byte atoms");
     static_assert((M * D * 2 / 16) % 128 == 0, "q tile chunks per staging thread");
+    static_assert(PBUF == 1 || PBUF == 2, "P buffers");
+    static_assert(CHUNK / 8 * NH <= 32, "one producer lane per box of a slot (8-token blocks at least)");
 };
 
 template <typename T, int D>
@@ -84,16 +99,15 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     using Tr = ElemTraits<T>;
     using MO = MmaOps<T>;
     constexpr bool BF16 = !std::is_same<T, __half>::value;
-    constexpr uint32_t IDESC_S = tc::idesc_f16(BF16, false, C::M, C::SLOT_ROWS);
+    constexpr uint32_t IDESC_S = tc::idesc_f16(BF16, false, C::M, C::CHUNK);
     constexpr uint32_t IDESC_PV = tc::idesc_f16(BF16, true, C::M, D);
     constexpr int KS = D / 16;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* full = bar;
-    uint64_t* empty = bar + C::NSLOTS;
-    uint64_t* s_full = bar + 2 * C::NSLOTS;      // [2] S of a chunk in buffer b done (commit)
+    uint64_t* full = bar;                        // [NSLOTS] a slot's TMA bytes landed
+    uint64_t* s_full = bar + C::NSLOTS;          // [2] S of a chunk in buffer b done (commit)
     uint64_t* q_full = s_full + 2;               // Q tile written (128 arrivals)
     uint64_t* q_empty = s_full + 3;              // last S of the item done (commit)
     uint64_t* p_full = s_full + 4;               // chunk's S read, O rescaled, p written (128 arrivals)
@@ -109,10 +123,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < C::NSLOTS; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-        }
+        for (int i = 0; i < C::NSLOTS; ++i) mbar_init(&full[i], 1);
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
         mbar_init(q_full, 128);
@@ -147,7 +158,10 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             prefetch_tmap(&tmap_v);
         }
         const uint64_t policy = l2_policy_evict_first();
-        uint32_t seq = 0;                                   // ring uses so far (K K V K V ... order)
+        uint32_t seq = 0;                                   // stream elements issued so far
+        uint32_t gch = 0;                                   // chunks of earlier items
+        // the last three stream elements (oldest first): chunk index << 1 | is_v
+        uint32_t h0 = 0, h1 = 0, h2 = 0;
         bool ok = true;
         for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
             const WorkItem w = decode_item(a, i, lane == 0);
@@ -164,33 +178,32 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 tbl[j] = id;
             }
             __syncwarp();
-            const int nst = (w.n + C::SLOT_ROWS - 1) / C::SLOT_ROWS;
-            const int nc = (nst + 1) / 2;
-            // the chunk's K or V slots in one round: both ring slots are waited for,
-            // then one warp instruction issues every box (16 lanes per slot)
+            const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
+            // K or V of chunk c into the next slot, once the products that read the
+            // slot's previous contents (the third-last element) are done
             auto issue = [&](int c, bool is_v) -> bool {
-                const int nb = min(2, nst - 2 * c);
-                for (int j = 0; j < nb; ++j) {
-                    const uint32_t sq = seq + j;
-                    if (!mbar_wait(&empty[sq % C::NSLOTS], ((sq / C::NSLOTS) & 1u) ^ 1u, abort_flag)) return false;
+                if (seq >= (uint32_t)C::NSLOTS) {
+                    const uint32_t g = h0 >> 1;
+                    uint64_t* done = (h0 & 1u) ? &o_full[g & 1u] : &s_full[g & 1u];
+                    if (!mbar_wait(done, (g >> 1) & 1u, abort_flag)) return false;
                 }
-                const int j = lane >> 4;
-                const int e = lane & 15;
-                const int st = 2 * c + j;
-                const int slot = (seq + j) % C::NSLOTS;
-                const int rows = j < nb ? min(C::SLOT_ROWS, w.n - st * C::SLOT_ROWS) : 0;
-                const int nbk = (rows + bs - 1) >> a.log2_bs;      // whole blocks
-                if (j < nb && e == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbk * C::NH * box_bytes));
+                const int slot = seq % C::NSLOTS;
+                const int rows = min(C::CHUNK, w.n - c * C::CHUNK);
+                const int nbk = (rows + bs - 1) >> a.log2_bs;          // whole blocks
+                if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbk * C::NH * box_bytes));
                 __syncwarp();
-                if (e < nbk * C::NH) {
-                    const int half = e / nbk;                       // slice
-                    const int b = e - half * nbk;                   // block within the slot
-                    const int phys = tbl[((st * C::SLOT_ROWS) >> a.log2_bs) + b];
+                if (lane < nbk * C::NH) {
+                    const int half = lane / nbk;                        // slice
+                    const int b = lane - half * nbk;                    // block within the chunk
+                    const int phys = tbl[((c * C::CHUNK) >> a.log2_bs) + b];
                     tma_load_3d(smem + slot * C::SLOT_BYTES + half * C::SLICE_BYTES + b * box_bytes,
                                 is_v ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
                                 half * C::BOX_ELEMS, w.h, phys * bs, &full[slot], policy);
                 }
-                seq += nb;
+                h0 = h1;
+                h1 = h2;
+                h2 = ((gch + (uint32_t)c) << 1) | (is_v ? 1u : 0u);
+                ++seq;
                 return true;
             };
             if (!(ok = issue(0, false))) break;
@@ -198,6 +211,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 if (c + 1 < nc && !(ok = issue(c + 1, false))) break;
                 ok = issue(c, true);
             }
+            gch += nc;
         }
         if (!ok) {
             if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
@@ -216,66 +230,63 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         // ------------------------------------------------------------ MMA issue
         uint32_t seq = 0, q_ph = 0, p_ph = 0, oe_ph = 0, gch = 0;
         bool ok = true;
-        const uint32_t qb = smem_addr(qs), pb = smem_addr(ps);
-        // S(c) = Q K^T for the chunk's slots, into S buffer `buf`
-        auto issue_s = [&](int c, int nst, uint32_t buf) -> bool {
-            const int nsl = min(2, nst - 2 * c);
-            for (int j = 0; j < nsl; ++j, ++seq) {
-                const int slot = seq % C::NSLOTS;
-                if (!mbar_wait(&full[slot], (seq / C::NSLOTS) & 1u, abort_flag)) return false;
-                tc::fence_after_sync();
-                if (lane == 0) {
-                    const uint32_t kb = smem_addr(smem + slot * C::SLOT_BYTES);
+        // operand descriptors built once; every MMA adds a byte offset to one of them
+        const uint64_t qdesc = tc::sw128_desc(smem_addr(qs), 16, 1024);                 // Q, K-major
+        const uint64_t pdesc = tc::sw128_desc(smem_addr(ps), 16, 1024);                 // P, K-major
+        const uint64_t kdesc = tc::sw128_desc(smem_addr(smem), 16, 1024);               // slot 0 as K, K-major
+        const uint64_t vdesc = tc::sw128_desc(smem_addr(smem), C::SLICE_BYTES, 1024);   // slot 0 as V, MN-major
+        // S(c) = Q K^T over the chunk's 64 tokens, into S buffer `buf` (token columns
+        // past the partition read stale rows; the softmax masks them)
+        auto issue_s = [&](uint32_t buf) -> bool {
+            const int slot = seq % C::NSLOTS;
+            if (!mbar_wait(&full[slot], (seq / C::NSLOTS) & 1u, abort_flag)) return false;
+            tc::fence_after_sync();
+            if (lane == 0) {
+                const uint64_t kd = tc::desc_add(kdesc, slot * C::SLOT_BYTES);
+                const uint32_t d = tmem + C::S_COL + buf * 64;
 #pragma unroll
-                    for (int kk = 0; kk < KS; ++kk) {
-                        const uint32_t koff = (kk >> 2) * C::SLICE_BYTES + (kk & 3) * 32;
-                        const uint32_t qoff = (kk >> 2) * C::Q_SLICE + (kk & 3) * 32;
-                        tc::mma_ss(tmem + C::S_COL + buf * 64 + j * C::SLOT_ROWS, tc::sw128_desc(qb + qoff, 16, 1024),
-                                   tc::sw128_desc(kb + koff, 16, 1024), IDESC_S, kk > 0);
-                    }
-                    tc::commit(&empty[slot]);                 // the K slot is free once these are done
+                for (int kk = 0; kk < KS; ++kk) {
+                    const uint32_t koff = (kk >> 2) * C::SLICE_BYTES + (kk & 3) * 32;
+                    const uint32_t qoff = (kk >> 2) * C::Q_SLICE + (kk & 3) * 32;
+                    tc::mma_ss(d, tc::desc_add(qdesc, qoff), tc::desc_add(kd, koff), IDESC_S, kk > 0);
                 }
-                __syncwarp();
+                tc::commit(&s_full[buf]);           // also frees the slot for the producer
             }
-            if (lane == 0) tc::commit(&s_full[buf]);
             __syncwarp();
+            ++seq;
             return true;
         };
-        // O += P V for the chunk's slots, p from P buffer `buf`
-        auto issue_pv = [&](int c, int nst, int n, uint32_t buf, bool first) -> bool {
-            const int nsl = min(2, nst - 2 * c);
-            for (int j = 0; j < nsl; ++j, ++seq) {
-                const int slot = seq % C::NSLOTS;
-                if (!mbar_wait(&full[slot], (seq / C::NSLOTS) & 1u, abort_flag)) return false;
-                const int rows = min(C::SLOT_ROWS, n - (2 * c + j) * C::SLOT_ROWS);
-                if (rows < C::SLOT_ROWS) {
-                    // rows past the partition (stale or unwritten pool rows, maybe NaN):
-                    // zero them so p = 0 meets finite values
-                    uint4* vrow = reinterpret_cast<uint4*>(smem + slot * C::SLOT_BYTES);
-                    for (int e = lane; e < C::NH * C::SLOT_ROWS * 8; e += 32)
-                        if (((e >> 3) % C::SLOT_ROWS) >= rows) vrow[e] = make_uint4(0u, 0u, 0u, 0u);
-                    tc::fence_proxy_async_smem();
-                }
-                __syncwarp();
-                tc::fence_after_sync();
-                if (lane == 0) {
-                    const uint32_t vb = smem_addr(smem + slot * C::SLOT_BYTES);
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {                      // 16 tokens per MMA
-                        const uint32_t poff = (j * C::SLOT_ROWS + ks * 16) * 2;   // within the 128-byte atom row
-                        const uint64_t bdesc = tc::sw128_desc(vb + ks * 16 * 128, C::SLICE_BYTES, 1024);
-                        const bool acc = !(first && j == 0 && ks == 0);
-                        tc::mma_ss(tmem + C::O_COL, tc::sw128_desc(pb + (2 * buf) * C::P_TILE + poff, 16, 1024),
-                                   bdesc, IDESC_PV, acc);
-                        tc::mma_ss(tmem + C::O_COL, tc::sw128_desc(pb + (2 * buf + 1) * C::P_TILE + poff, 16, 1024),
-                                   bdesc, IDESC_PV, true);
-                    }
-                    tc::commit(&empty[slot]);
-                }
-                __syncwarp();
+        // O += P V over the chunk's tokens, p from P buffer `buf` (buffer 0 when single)
+        auto issue_pv = [&](int c, int n, uint32_t buf, bool first) -> bool {
+            const uint32_t pbuf = C::PBUF == 2 ? buf : 0u;
+            const int slot = seq % C::NSLOTS;
+            if (!mbar_wait(&full[slot], (seq / C::NSLOTS) & 1u, abort_flag)) return false;
+            const int rows = min(C::CHUNK, n - c * C::CHUNK);
+            if (rows < C::CHUNK) {
+                // rows past the partition (stale or unwritten rows, maybe NaN): zero them
+                // so that p = 0 meets finite values
+                uint4* vrow = reinterpret_cast<uint4*>(smem + slot * C::SLOT_BYTES);
+                for (int e = lane; e < C::NH * C::CHUNK * 8; e += 32)
+                    if (((e >> 3) % C::CHUNK) >= rows) vrow[e] = make_uint4(0u, 0u, 0u, 0u);
+                tc::fence_proxy_async_smem();
             }
-            if (lane == 0) tc::commit(&o_full[buf]);
             __syncwarp();
+            tc::fence_after_sync();
+            if (lane == 0) {
+                const uint64_t vd = tc::desc_add(vdesc, slot * C::SLOT_BYTES);
+                const uint64_t pd = tc::desc_add(pdesc, 2 * pbuf * C::P_TILE);
+#pragma unroll
+                for (int ks = 0; ks < C::CHUNK / 16; ++ks) {             // 16 tokens per MMA
+                    const uint64_t bd = tc::desc_add(vd, ks * 16 * 128);
+                    tc::mma_ss(tmem + C::O_COL, tc::desc_add(pd, ks * 32), bd, IDESC_PV, ks > 0 || !first);
+#if PA_VERIFY_TC_PSPLIT
+                    tc::mma_ss(tmem + C::O_COL, tc::desc_add(pd, C::P_TILE + ks * 32), bd, IDESC_PV, true);
+#endif
+                }
+                tc::commit(&o_full[buf]);           // also frees the slot for the producer
+            }
+            __syncwarp();
+            ++seq;
             return true;
         };
         for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
@@ -287,14 +298,13 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             }
             q_ph ^= 1u;
             tc::fence_after_sync();
-            const int nst = (w.n + C::SLOT_ROWS - 1) / C::SLOT_ROWS;
-            const int nc = (nst + 1) / 2;
-            if (!(ok = issue_s(0, nst, gch & 1u))) break;
+            const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
+            if (!(ok = issue_s(gch & 1u))) break;
             if (nc == 1 && lane == 0) tc::commit(q_empty);        // last S of the item: Q may be replaced
             __syncwarp();
             for (int c = 0; c < nc && ok; ++c) {
                 if (c + 1 < nc) {
-                    if (!(ok = issue_s(c + 1, nst, (gch + c + 1) & 1u))) break;
+                    if (!(ok = issue_s((gch + c + 1) & 1u))) break;
                     if (c + 2 == nc && lane == 0) tc::commit(q_empty);
                     __syncwarp();
                 }
@@ -306,7 +316,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     oe_ph ^= 1u;
                 }
                 tc::fence_after_sync();
-                if (!(ok = issue_pv(c, nst, w.n, (gch + c) & 1u, c == 0))) break;
+                if (!(ok = issue_pv(c, w.n, (gch + c) & 1u, c == 0))) break;
             }
             gch += nc;
         }
@@ -398,8 +408,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             int pos;
             row_of(m, orow, pos);
             float m_run = -INFINITY, l_run = 0.f;        // l: this thread's half of the row
-            const int nst = (w.n + C::SLOT_ROWS - 1) / C::SLOT_ROWS;
-            const int nc = (nst + 1) / 2;
+            const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
             for (int c = 0; c < nc && ok; ++c) {
                 const uint32_t buf = (gch + c) & 1u;
                 if (!(ok = mbar_wait(&s_full[buf], ((gch + c) >> 1) & 1u, abort_flag))) break;
@@ -433,8 +442,14 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 for (int k = 0; k < 32; k += 2) {
                     const float p0 = exp2f(__uint_as_float(r[k]) - base);
                     const float p1 = exp2f(__uint_as_float(r[k + 1]) - base);
+#if PA_VERIFY_TC_PSPLIT
                     lsum += p0 + p1;
                     split_pack<MO>(p0, p1, hi[k >> 1], lo[k >> 1]);
+#else
+                    hi[k >> 1] = MO::pack(p0, p1);            // the sum takes p as the product sees it
+                    const float2 h = MO::unpack(hi[k >> 1]);
+                    lsum += h.x + h.y;
+#endif
                 }
                 const uint32_t gc = gch + c;
                 // O rescale: only when some row of this warp moved its reference, after the
@@ -453,18 +468,20 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     }
                     tc::wait_st();
                 }
-                // P buffer gc & 1 was last read by the P.V of chunk gc - 2
-                if (gc >= 2 && !(ok = wait_pv(gc - 2))) break;
+                // the P buffer this chunk writes was last read by the P.V of chunk gc - PBUF
+                if (gc >= (uint32_t)C::PBUF && !(ok = wait_pv(gc - C::PBUF))) break;
                 m_run = m_new;
                 l_run = l_run * corr + lsum;
                 // p of row m, tokens half*32 .. +31 of the chunk: 16-byte chunks 4*half .. +3 of the row
-                unsigned char* pt = ps + (2 * buf) * C::P_TILE + m * 128;
+                unsigned char* pt = ps + (C::PBUF == 2 ? 2 * buf : 0u) * C::P_TILE + m * 128;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const int off = (((half * 4 + q4) ^ (m & 7)) << 4);
                     *reinterpret_cast<uint4*>(pt + off) = make_uint4(hi[4 * q4], hi[4 * q4 + 1], hi[4 * q4 + 2], hi[4 * q4 + 3]);
+#if PA_VERIFY_TC_PSPLIT
                     *reinterpret_cast<uint4*>(pt + C::P_TILE + off) =
                         make_uint4(lo[4 * q4], lo[4 * q4 + 1], lo[4 * q4 + 2], lo[4 * q4 + 3]);
+#endif
                 }
                 tc::fence_proxy_async_smem();
                 tc::fence_before_sync();
