@@ -367,7 +367,7 @@ def run_native(args):
     kernel = "verify" if Q > 1 else "decode"      # the library's launch-profile id
     if Q == 1:
         kname = "decode"
-    elif args.verify_kernel == "tcgen05" or (args.verify_kernel == "auto" and cfg.num_heads // cfg.num_kv_heads * Q > 16):
+    elif args.verify_kernel in ("tcgen05", "auto"):
         kname = "verify_tc"       # the choice pa_verify makes for VERIFY_AUTO
     else:
         kname = "verify"

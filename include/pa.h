@@ -184,15 +184,15 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
 /*
  * Tensor-core path of pa_verify (process-wide):
  *   PA_VERIFY_MMA_SYNC  warp-level mma.m16n8k16 with accumulators in registers
- *   PA_VERIFY_TCGEN05   tcgen05.mma issued by one thread, accumulators in tensor
- *                       memory, operands in shared memory (M = 64 query rows per
- *                       item: it pays when num_heads / num_kv_heads x Q is large)
- *   PA_VERIFY_AUTO      the first for at most 16 rows per kv head, else the second
+ *   PA_VERIFY_TCGEN05   tcgen05.mma issued by one thread, accumulators and p in
+ *                       tensor memory, K/V and q in shared memory (M = 64 query
+ *                       rows per item); the faster kernel at every measured shape
+ *   PA_VERIFY_AUTO      the kernel measured fastest: PA_VERIFY_TCGEN05
  * Same results within the stated tolerance; bits differ between the two.
  */
 #define PA_VERIFY_MMA_SYNC 0
 #define PA_VERIFY_TCGEN05 1
-#define PA_VERIFY_AUTO 2    /* default: tcgen05 when a kv head carries more than 16 query rows */
+#define PA_VERIFY_AUTO 2    /* default: the tcgen05 kernel */
 pa_status pa_set_verify_kernel(int kind);
 int pa_get_verify_kernel(void);
 

@@ -11,28 +11,28 @@
 //    rows).  The rows form one M = 64 tile; the partition is walked in chunks
 //    of 64 tokens.
 //  * Warp 0 streams K and V chunks through TMA tiled boxes into a ring of
-//    three slots (slot = 64 token rows of one kv head; each 128-byte head_dim
+//    five slots (slot = 64 token rows of one kv head; each 128-byte head_dim
 //    slice of the 64 rows is one 128-byte-swizzled array), K running one
 //    chunk ahead of V: K0 K1 V0 K2 V1 ... .  A slot is refilled once the
 //    products that read its previous contents are done: the producer waits
-//    on the same commit barrier the softmax (S done) or the next rescale
-//    (P.V done) waits on, so no separate release barrier is committed.
+//    on the commit barrier the softmax (S done) or the epilogue (P.V done)
+//    waits on, so no separate release barrier is committed.
 //  * Warp 1 issues, from one thread, in the same order:
 //        S(c) [64 x 64]  = Q K^T   KS MMAs M=64 N=64 K=16, into one of two S buffers
-//        O    [64 x D]  += P V     4 x 2 MMAs M=64 N=D K=16 (P K-major from shared
-//                                  memory, V MN-major: the slot as loaded)
+//        O    [64 x D]  += P V     4 (x 2) MMAs M=64 N=D K=16, P read from tensor
+//                                  memory, V MN-major from the slot as loaded
 //    so S(c+1) is computed while the softmax of chunk c runs.  TMEM columns:
-//    S buffers [0, 64) and [64, 128), O [128, 128 + D).  P is split into a
-//    16-bit value and its remainder (two products), as in decode.  A
-//    tcgen05.mma costs its issuing thread about as much as a commit or a
-//    barrier test, whatever its N, so the chunk is covered by as few
-//    instructions as the shapes allow: one commit per product group, one
-//    barrier wait per chunk of K or V.
+//    S buffers [0, 64) and [64, 128), O [128, 128 + D).  A tcgen05.mma costs
+//    its issuing thread about as much as a commit or a barrier test, whatever
+//    its N, so a chunk is covered by as few instructions as the shapes allow.
 //  * Warps 2-5 (one TMEM lane quarter each; a quarter's first 16 lanes hold 16
 //    rows of an M = 64 accumulator, read as two half-warps of 32 columns)
 //    stage q, take the exact max of the chunk (causal mask), rescale O in TMEM
-//    when the running max grows, write p to shared memory, and finally read O,
-//    normalise and store (or store the partition's partials).
+//    when the running max grows by more than 8 (base 2), write p over the
+//    chunk's S columns, and finally read O, normalise and store (or store the
+//    partition's partials).  For bf16, p is split into a 16-bit value and its
+//    remainder (two products, as in decode); an fp16 p keeps 11 significant
+//    bits and goes in one product.
 //  * All waits are bounded; TMEM is freed after a final commit has drained
 //    the MMAs.
 #pragma once
@@ -45,10 +45,21 @@
 namespace pa_dev {
 
 #ifndef PA_VERIFY_TC_PSPLIT
-#define PA_VERIFY_TC_PSPLIT 1    // 1: P.V as two products (16-bit p and its remainder); 0: 16-bit p only
+// 1: P.V as two products (16-bit p and its remainder); 0: the 16-bit p only;
+// 2: split for bf16 only (an fp16 p already carries 11 significant bits)
+#define PA_VERIFY_TC_PSPLIT 2
+#endif
+#ifndef PA_VERIFY_TC_SLOTS
+#define PA_VERIFY_TC_SLOTS 5
+#endif
+#ifndef PA_VERIFY_TC_PTMEM
+#define PA_VERIFY_TC_PTMEM 1     // 1: p written to tensor memory over its S buffer, P.V reads A from there
+#endif
+#ifndef PA_VERIFY_TC_PWAR
+#define PA_VERIFY_TC_PWAR 1      // with p in tensor memory: S of chunk g waits for P.V of chunk g - 2
 #endif
 #ifndef PA_VERIFY_TC_PBUF
-#define PA_VERIFY_TC_PBUF 2      // P tiles in shared memory: 2 = double-buffered, 1 = single
+#define PA_VERIFY_TC_PBUF 1      // P tiles in shared memory: 2 = double-buffered, 1 = single
 #endif
 
 template <typename T, int D>
@@ -59,16 +70,21 @@ struct VerifyTcCfg {
     static constexpr int CHUNK = 64;                         // tokens per chunk = rows of a ring slot
     static constexpr int SLICE_BYTES = CHUNK * 128;          // one head_dim slice of a slot
     static constexpr int SLOT_BYTES = NH * SLICE_BYTES;
-    // Three slots: K(c+1) and V(c) in use while the next K or V loads.  Deeper
-    // rings would break the refill rule: a slot's previous contents must be the
-    // third-last stream element, whose commit barrier cannot have moved two
-    // phases on by the time the producer tests it.
-    static constexpr int NSLOTS = 3;
+    // K(c+1) and V(c) are in use while the rest of the ring loads.  The commit
+    // barriers of S and P.V come in four copies (chunk g uses copy g % 4), so a
+    // refill that waits on the element NSLOTS back in the stream can never see
+    // its barrier four phases on: the same copy's next use is at least seven
+    // elements later.
+    static constexpr int NSLOTS = PA_VERIFY_TC_SLOTS;
+    static constexpr int NPH = 4;                            // copies of the S / P.V commit barriers
     static constexpr int M = 64;                             // query rows per item
     static constexpr int Q_SLICE = M * 128;                  // one 128-byte slice of the Q tile
     static constexpr int Q_BYTES = NH * Q_SLICE;
     static constexpr int P_TILE = M * 128;                   // 64 rows x 64 tokens, one 128-byte atom column
-    static constexpr int PBUF = PA_VERIFY_TC_PBUF;
+    static constexpr bool PTMEM = PA_VERIFY_TC_PTMEM != 0;
+    static constexpr int PBUF = PTMEM ? 0 : PA_VERIFY_TC_PBUF;  // P tiles in shared memory
+    static constexpr bool PSPLIT =
+        PA_VERIFY_TC_PSPLIT == 2 ? !std::is_same<T, __half>::value : PA_VERIFY_TC_PSPLIT != 0;
     static constexpr int TMEM_COLS = 256;
     static constexpr int S_COL = 0;                          // S buffer b: [64 b, 64 b + 64)
     static constexpr int O_COL = 128;
@@ -76,8 +92,8 @@ struct VerifyTcCfg {
     static constexpr int OFF_Q = NSLOTS * SLOT_BYTES;
     static constexpr int OFF_P = OFF_Q + Q_BYTES;            // tile (buffer b, part h) at (2 b + h) * P_TILE
     static constexpr int OFF_BAR = OFF_P + 2 * PBUF * P_TILE;
-    // barriers: full[NSLOTS], s_full[2], q_full, q_empty, p_full, o_full[2], o_empty, drain
-    static constexpr int NBAR = NSLOTS + 9;
+    // barriers: full[NSLOTS], s_full[NPH], q_full, q_empty, p_full, o_full[NPH], o_empty, drain
+    static constexpr int NBAR = NSLOTS + 2 * NPH + 5;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;      // allocated TMEM address
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
     static constexpr int OFF_TABLE = (OFF_ABORT + 4 + 15) / 16 * 16;
@@ -87,7 +103,8 @@ struct VerifyTcCfg {
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(SLOT_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0 && P_TILE % 1024 == 0, "1024-byte atoms");
     static_assert((M * D * 2 / 16) % 128 == 0, "q tile chunks per staging thread");
-    static_assert(PBUF == 1 || PBUF == 2, "P buffers");
+    static_assert(PTMEM || PBUF == 1 || PBUF == 2, "P buffers");
+    static_assert(NSLOTS >= 3 && NSLOTS <= 7, "ring refill rule");
     static_assert(CHUNK / 8 * NH <= 32, "one producer lane per box of a slot (8-token blocks at least)");
 };
 
@@ -107,13 +124,13 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* full = bar;                        // [NSLOTS] a slot's TMA bytes landed
-    uint64_t* s_full = bar + C::NSLOTS;          // [2] S of a chunk in buffer b done (commit)
-    uint64_t* q_full = s_full + 2;               // Q tile written (128 arrivals)
-    uint64_t* q_empty = s_full + 3;              // last S of the item done (commit)
-    uint64_t* p_full = s_full + 4;               // chunk's S read, O rescaled, p written (128 arrivals)
-    uint64_t* o_full = s_full + 5;               // [2] P.V of a chunk using P buffer b done (commit)
-    uint64_t* o_empty = s_full + 7;              // O read by the epilogue (128 arrivals)
-    uint64_t* drain = s_full + 8;                // every MMA done, before TMEM is freed
+    uint64_t* s_full = bar + C::NSLOTS;          // [NPH] S of chunk g done (commit), copy g % NPH
+    uint64_t* q_full = s_full + C::NPH;          // Q tile written (128 arrivals)
+    uint64_t* q_empty = q_full + 1;              // last S of the item done (commit)
+    uint64_t* p_full = q_full + 2;               // chunk's S read, O rescaled, p written (128 arrivals)
+    uint64_t* o_full = q_full + 3;               // [NPH] P.V of chunk g done (commit), copy g % NPH
+    uint64_t* o_empty = o_full + C::NPH;         // O read by the epilogue (128 arrivals)
+    uint64_t* drain = o_empty + 1;               // every MMA done, before TMEM is freed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + C::OFF_TABLE);
@@ -124,13 +141,13 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NSLOTS; ++i) mbar_init(&full[i], 1);
-        mbar_init(&s_full[0], 1);
-        mbar_init(&s_full[1], 1);
+        for (int i = 0; i < C::NPH; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&o_full[i], 1);
+        }
         mbar_init(q_full, 128);
         mbar_init(q_empty, 1);
         mbar_init(p_full, 128);
-        mbar_init(&o_full[0], 1);
-        mbar_init(&o_full[1], 1);
         mbar_init(o_empty, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -160,8 +177,10 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         const uint64_t policy = l2_policy_evict_first();
         uint32_t seq = 0;                                   // stream elements issued so far
         uint32_t gch = 0;                                   // chunks of earlier items
-        // the last three stream elements (oldest first): chunk index << 1 | is_v
-        uint32_t h0 = 0, h1 = 0, h2 = 0;
+        // the last NSLOTS stream elements (oldest first): chunk index << 1 | is_v
+        uint32_t hist[C::NSLOTS];
+#pragma unroll
+        for (int k = 0; k < C::NSLOTS; ++k) hist[k] = 0;
         bool ok = true;
         for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
             const WorkItem w = decode_item(a, i, lane == 0);
@@ -180,12 +199,12 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             __syncwarp();
             const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
             // K or V of chunk c into the next slot, once the products that read the
-            // slot's previous contents (the third-last element) are done
+            // slot's previous contents (the element NSLOTS back) are done
             auto issue = [&](int c, bool is_v) -> bool {
                 if (seq >= (uint32_t)C::NSLOTS) {
-                    const uint32_t g = h0 >> 1;
-                    uint64_t* done = (h0 & 1u) ? &o_full[g & 1u] : &s_full[g & 1u];
-                    if (!mbar_wait(done, (g >> 1) & 1u, abort_flag)) return false;
+                    const uint32_t g = hist[0] >> 1;
+                    uint64_t* done = (hist[0] & 1u) ? &o_full[g % C::NPH] : &s_full[g % C::NPH];
+                    if (!mbar_wait(done, (g / C::NPH) & 1u, abort_flag)) return false;
                 }
                 const int slot = seq % C::NSLOTS;
                 const int rows = min(C::CHUNK, w.n - c * C::CHUNK);
@@ -200,9 +219,9 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                                 is_v ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
                                 half * C::BOX_ELEMS, w.h, phys * bs, &full[slot], policy);
                 }
-                h0 = h1;
-                h1 = h2;
-                h2 = ((gch + (uint32_t)c) << 1) | (is_v ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k + 1 < C::NSLOTS; ++k) hist[k] = hist[k + 1];
+                hist[C::NSLOTS - 1] = ((gch + (uint32_t)c) << 1) | (is_v ? 1u : 0u);
                 ++seq;
                 return true;
             };
@@ -235,11 +254,18 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         const uint64_t pdesc = tc::sw128_desc(smem_addr(ps), 16, 1024);                 // P, K-major
         const uint64_t kdesc = tc::sw128_desc(smem_addr(smem), 16, 1024);               // slot 0 as K, K-major
         const uint64_t vdesc = tc::sw128_desc(smem_addr(smem), C::SLICE_BYTES, 1024);   // slot 0 as V, MN-major
-        // S(c) = Q K^T over the chunk's 64 tokens, into S buffer `buf` (token columns
-        // past the partition read stale rows; the softmax masks them)
-        auto issue_s = [&](uint32_t buf) -> bool {
+        // S of global chunk g = Q K^T over its 64 tokens, into S buffer g & 1 (token
+        // columns past the partition read stale rows; the softmax masks them)
+        auto issue_s = [&](uint32_t g) -> bool {
+            const uint32_t buf = g & 1u;
             const int slot = seq % C::NSLOTS;
             if (!mbar_wait(&full[slot], (seq / C::NSLOTS) & 1u, abort_flag)) return false;
+            if constexpr (C::PTMEM && PA_VERIFY_TC_PWAR) {
+                // the buffer holds p of chunk g - 2, read by the P.V issued just before: a
+                // later product may not overwrite an operand the tensor core is still
+                // reading, so that P.V completes first
+                if (g >= 2 && !mbar_wait(&o_full[(g - 2) % C::NPH], ((g - 2) / C::NPH) & 1u, abort_flag)) return false;
+            }
             tc::fence_after_sync();
             if (lane == 0) {
                 const uint64_t kd = tc::desc_add(kdesc, slot * C::SLOT_BYTES);
@@ -250,15 +276,16 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     const uint32_t qoff = (kk >> 2) * C::Q_SLICE + (kk & 3) * 32;
                     tc::mma_ss(d, tc::desc_add(qdesc, qoff), tc::desc_add(kd, koff), IDESC_S, kk > 0);
                 }
-                tc::commit(&s_full[buf]);           // also frees the slot for the producer
+                tc::commit(&s_full[g % C::NPH]);    // also frees the slot for the producer
             }
             __syncwarp();
             ++seq;
             return true;
         };
-        // O += P V over the chunk's tokens, p from P buffer `buf` (buffer 0 when single)
-        auto issue_pv = [&](int c, int n, uint32_t buf, bool first) -> bool {
-            const uint32_t pbuf = C::PBUF == 2 ? buf : 0u;
+        // O += P V over the tokens of chunk c (global chunk g), p from P buffer g & 1
+        // (buffer 0 when single)
+        auto issue_pv = [&](int c, int n, uint32_t g, bool first) -> bool {
+            const uint32_t pbuf = C::PBUF == 2 ? (g & 1u) : 0u;
             const int slot = seq % C::NSLOTS;
             if (!mbar_wait(&full[slot], (seq / C::NSLOTS) & 1u, abort_flag)) return false;
             const int rows = min(C::CHUNK, n - c * C::CHUNK);
@@ -275,15 +302,21 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             if (lane == 0) {
                 const uint64_t vd = tc::desc_add(vdesc, slot * C::SLOT_BYTES);
                 const uint64_t pd = tc::desc_add(pdesc, 2 * pbuf * C::P_TILE);
+                // p in tensor memory: value in S buffer columns [0, 32), remainder in [32, 64)
+                const uint32_t pt = tmem + C::S_COL + (g & 1u) * 64;
 #pragma unroll
                 for (int ks = 0; ks < C::CHUNK / 16; ++ks) {             // 16 tokens per MMA
                     const uint64_t bd = tc::desc_add(vd, ks * 16 * 128);
-                    tc::mma_ss(tmem + C::O_COL, tc::desc_add(pd, ks * 32), bd, IDESC_PV, ks > 0 || !first);
-#if PA_VERIFY_TC_PSPLIT
-                    tc::mma_ss(tmem + C::O_COL, tc::desc_add(pd, C::P_TILE + ks * 32), bd, IDESC_PV, true);
-#endif
+                    if constexpr (C::PTMEM) {
+                        tc::mma_ts(tmem + C::O_COL, pt + ks * 8, bd, IDESC_PV, ks > 0 || !first);
+                        if constexpr (C::PSPLIT) tc::mma_ts(tmem + C::O_COL, pt + 32 + ks * 8, bd, IDESC_PV, true);
+                    } else {
+                        tc::mma_ss(tmem + C::O_COL, tc::desc_add(pd, ks * 32), bd, IDESC_PV, ks > 0 || !first);
+                        if constexpr (C::PSPLIT)
+                            tc::mma_ss(tmem + C::O_COL, tc::desc_add(pd, C::P_TILE + ks * 32), bd, IDESC_PV, true);
+                    }
                 }
-                tc::commit(&o_full[buf]);           // also frees the slot for the producer
+                tc::commit(&o_full[g % C::NPH]);    // also frees the slot for the producer
             }
             __syncwarp();
             ++seq;
@@ -299,12 +332,12 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             q_ph ^= 1u;
             tc::fence_after_sync();
             const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
-            if (!(ok = issue_s(gch & 1u))) break;
+            if (!(ok = issue_s(gch))) break;
             if (nc == 1 && lane == 0) tc::commit(q_empty);        // last S of the item: Q may be replaced
             __syncwarp();
             for (int c = 0; c < nc && ok; ++c) {
                 if (c + 1 < nc) {
-                    if (!(ok = issue_s((gch + c + 1) & 1u))) break;
+                    if (!(ok = issue_s(gch + c + 1))) break;
                     if (c + 2 == nc && lane == 0) tc::commit(q_empty);
                     __syncwarp();
                 }
@@ -316,7 +349,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     oe_ph ^= 1u;
                 }
                 tc::fence_after_sync();
-                if (!(ok = issue_pv(c, w.n, (gch + c) & 1u, c == 0))) break;
+                if (!(ok = issue_pv(c, w.n, gch + c, c == 0))) break;
             }
             gch += nc;
         }
@@ -342,76 +375,77 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         const int Q = a.num_queries;
         const int R = a.group * Q;
         uint32_t qe_ph = 0, gch = 0;
-        // P.V of global chunk g (P buffer g & 1) done: its use of o_full[g & 1] is g >> 1
+        // P.V of global chunk g done: barrier copy g % NPH, its (g / NPH)-th phase
         auto wait_pv = [&](uint32_t g) -> bool {
-            return mbar_wait(&o_full[g & 1u], (g >> 1) & 1u, abort_flag);
+            return mbar_wait(&o_full[g % C::NPH], (g / C::NPH) & 1u, abort_flag);
+        };
+        // output row and query position of local row lr of item w (orow < 0: no row)
+        auto row_in = [&](const WorkItem& w, int ctx, int lr, int64_t& orow, int& pos) {
+            const int r0 = w.gc * C::M;
+            if (lr >= min(C::M, R - r0)) {
+                orow = -1;
+                pos = -1;
+                return;
+            }
+            const int r = r0 + lr;
+            const int qi = r / a.group;
+            const int g = r - qi * a.group;
+            orow = ((int64_t)w.s * Q + qi) * a.num_heads + (int64_t)w.h * a.group + g;
+            pos = ctx - Q + qi;
+        };
+        // item w's query rows as the A tile (rows past the chunk are zero), once the
+        // previous item's last S product no longer reads the tile
+        auto stage_q = [&](const WorkItem& w, int ctx) -> bool {
+            if (!mbar_wait(q_empty, qe_ph ^ 1u, abort_flag)) return false;
+            qe_ph ^= 1u;
+            // all loads of this thread first, then the swizzled stores
+            constexpr int VPR = D * 2 / 16;               // 16-byte chunks per row
+            constexpr int PER = C::M * VPR / 128;         // chunks per thread
+            uint4 v[PER];
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int e = ctid + u * 128;
+                int64_t orow;
+                int pos;
+                row_in(w, ctx, e / VPR, orow, pos);
+                v[u] = orow >= 0 ? __ldg(reinterpret_cast<const uint4*>(qg + orow * D) + (e % VPR))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int e = ctid + u * 128;
+                const int lr = e / VPR;
+                const int cc = e % VPR;
+                *reinterpret_cast<uint4*>(qs + (cc >> 3) * C::Q_SLICE + lr * 128 + (((cc & 7) ^ (lr & 7)) << 4)) = v[u];
+            }
+            tc::fence_proxy_async_smem();
+            mbar_arrive(q_full);
+            return true;
         };
         bool ok = true;
+        int staged = -1;                                 // item whose Q tile is already written
         for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
             const WorkItem w = decode_item(a, i, false);
             const int ctx = clamp_context(a, w.s, false);
-            const int r0 = w.gc * C::M;
-            const int nr = min(C::M, R - r0);
-            auto row_of = [&](int lr, int64_t& orow, int& pos) {
-                if (lr >= nr) {
-                    orow = -1;
-                    pos = -1;
-                    return;
-                }
-                const int r = r0 + lr;
-                const int qi = r / a.group;
-                const int g = r - qi * a.group;
-                orow = ((int64_t)w.s * Q + qi) * a.num_heads + (int64_t)w.h * a.group + g;
-                pos = ctx - Q + qi;
-            };
             if (w.n == 0) {                              // empty context: zero rows
+                const int nr = min(C::M, R - w.gc * C::M);
                 for (int e = ctid; e < nr * D; e += 128) {
                     int64_t orow;
                     int pos;
-                    row_of(e / D, orow, pos);
+                    row_in(w, ctx, e / D, orow, pos);
                     outg[orow * D + (e % D)] = Tr::from_float(0.f);
                 }
                 continue;
             }
-            // ---- this item's query rows as the A tile (rows past the chunk are zero), once
-            // the previous item's last S product no longer reads the tile
-            if (!mbar_wait(q_empty, qe_ph ^ 1u, abort_flag)) {
-                ok = false;
-                break;
-            }
-            qe_ph ^= 1u;
-            {
-                // all loads of this thread first, then the swizzled stores
-                constexpr int VPR = D * 2 / 16;           // 16-byte chunks per row
-                constexpr int PER = C::M * VPR / 128;     // chunks per thread
-                uint4 v[PER];
-#pragma unroll
-                for (int u = 0; u < PER; ++u) {
-                    const int e = ctid + u * 128;
-                    int64_t orow;
-                    int pos;
-                    row_of(e / VPR, orow, pos);
-                    v[u] = orow >= 0 ? __ldg(reinterpret_cast<const uint4*>(qg + orow * D) + (e % VPR))
-                                     : make_uint4(0u, 0u, 0u, 0u);
-                }
-#pragma unroll
-                for (int u = 0; u < PER; ++u) {
-                    const int e = ctid + u * 128;
-                    const int lr = e / VPR;
-                    const int cc = e % VPR;
-                    *reinterpret_cast<uint4*>(qs + (cc >> 3) * C::Q_SLICE + lr * 128 + (((cc & 7) ^ (lr & 7)) << 4)) = v[u];
-                }
-                tc::fence_proxy_async_smem();
-                mbar_arrive(q_full);
-            }
+            if (staged != i && !(ok = stage_q(w, ctx))) break;
             int64_t orow;
             int pos;
-            row_of(m, orow, pos);
+            row_in(w, ctx, m, orow, pos);
             float m_run = -INFINITY, l_run = 0.f;        // l: this thread's half of the row
             const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
             for (int c = 0; c < nc && ok; ++c) {
                 const uint32_t buf = (gch + c) & 1u;
-                if (!(ok = mbar_wait(&s_full[buf], ((gch + c) >> 1) & 1u, abort_flag))) break;
+                if (!(ok = mbar_wait(&s_full[(gch + c) % C::NPH], ((gch + c) / C::NPH) & 1u, abort_flag))) break;
                 tc::fence_after_sync();
                 uint32_t r[32];
                 tc::ld16x2(tmem + lane_addr + C::S_COL + buf * 64, r);
@@ -442,14 +476,14 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 for (int k = 0; k < 32; k += 2) {
                     const float p0 = exp2f(__uint_as_float(r[k]) - base);
                     const float p1 = exp2f(__uint_as_float(r[k + 1]) - base);
-#if PA_VERIFY_TC_PSPLIT
-                    lsum += p0 + p1;
-                    split_pack<MO>(p0, p1, hi[k >> 1], lo[k >> 1]);
-#else
-                    hi[k >> 1] = MO::pack(p0, p1);            // the sum takes p as the product sees it
-                    const float2 h = MO::unpack(hi[k >> 1]);
-                    lsum += h.x + h.y;
-#endif
+                    if constexpr (C::PSPLIT) {
+                        lsum += p0 + p1;
+                        split_pack<MO>(p0, p1, hi[k >> 1], lo[k >> 1]);
+                    } else {
+                        hi[k >> 1] = MO::pack(p0, p1);            // the sum takes p as the product sees it
+                        const float2 h = MO::unpack(hi[k >> 1]);
+                        lsum += h.x + h.y;
+                    }
                 }
                 const uint32_t gc = gch + c;
                 // O rescale: only when some row of this warp moved its reference, after the
@@ -468,27 +502,56 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     }
                     tc::wait_st();
                 }
-                // the P buffer this chunk writes was last read by the P.V of chunk gc - PBUF
-                if (gc >= (uint32_t)C::PBUF && !(ok = wait_pv(gc - C::PBUF))) break;
                 m_run = m_new;
                 l_run = l_run * corr + lsum;
-                // p of row m, tokens half*32 .. +31 of the chunk: 16-byte chunks 4*half .. +3 of the row
-                unsigned char* pt = ps + (C::PBUF == 2 ? 2 * buf : 0u) * C::P_TILE + m * 128;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int off = (((half * 4 + q4) ^ (m & 7)) << 4);
-                    *reinterpret_cast<uint4*>(pt + off) = make_uint4(hi[4 * q4], hi[4 * q4 + 1], hi[4 * q4 + 2], hi[4 * q4 + 3]);
-#if PA_VERIFY_TC_PSPLIT
-                    *reinterpret_cast<uint4*>(pt + C::P_TILE + off) =
-                        make_uint4(lo[4 * q4], lo[4 * q4 + 1], lo[4 * q4 + 2], lo[4 * q4 + 3]);
-#endif
+                if constexpr (C::PTMEM || C::PBUF == 2) {
+                    // p_full counts one arrival per thread and phase: a warp that is a chunk
+                    // ahead of the others must not arrive before the previous chunk's phase
+                    // completes, or its arrival would count toward that phase.  (With a
+                    // single P buffer the wait for the previous P.V below implies this.)
+                    if (gc >= 1 && !(ok = mbar_wait(p_full, (gc - 1) & 1u, abort_flag))) break;
                 }
-                tc::fence_proxy_async_smem();
+                if constexpr (C::PTMEM) {
+                    // p over this chunk's S columns (already read): tokens half*32 .. +31 of row m
+                    // are value columns half*16 .. +15 and remainder columns 32 + half*16 .. +15.
+                    // The buffer's previous p was read by P.V of chunk gc - 2, which the tensor
+                    // core finished before it wrote S of this chunk there.
+                    tc::st16x2_x16(tmem + lane_addr + C::S_COL + buf * 64, hi);
+                    if constexpr (C::PSPLIT) tc::st16x2_x16(tmem + lane_addr + C::S_COL + buf * 64 + 32, lo);
+                    tc::wait_st();
+                } else {
+                    // the P buffer this chunk writes was last read by the P.V of chunk gc - PBUF
+                    if (gc >= (uint32_t)C::PBUF && !(ok = wait_pv(gc - C::PBUF))) break;
+                    // p of row m, tokens half*32 .. +31 of the chunk: 16-byte chunks 4*half .. +3 of the row
+                    unsigned char* pt = ps + (C::PBUF == 2 ? 2 * buf : 0u) * C::P_TILE + m * 128;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int off = (((half * 4 + q4) ^ (m & 7)) << 4);
+                        *reinterpret_cast<uint4*>(pt + off) =
+                            make_uint4(hi[4 * q4], hi[4 * q4 + 1], hi[4 * q4 + 2], hi[4 * q4 + 3]);
+                        if constexpr (C::PSPLIT)
+                            *reinterpret_cast<uint4*>(pt + C::P_TILE + off) =
+                                make_uint4(lo[4 * q4], lo[4 * q4 + 1], lo[4 * q4 + 2], lo[4 * q4 + 3]);
+                    }
+                    tc::fence_proxy_async_smem();
+                }
                 tc::fence_before_sync();
                 mbar_arrive(p_full);
             }
             gch += nc;
             if (!ok) break;
+            // ---- the next item's Q tile now, so that its first S products run while
+            // this item's epilogue does
+            {
+                const int inext = i + gridDim.x;
+                if (inext < total) {
+                    const WorkItem wn = decode_item(a, inext, false);
+                    if (wn.n > 0) {
+                        if (!(ok = stage_q(wn, clamp_context(a, wn.s, false)))) break;
+                        staged = inext;
+                    }
+                }
+            }
             // ---- epilogue: O after the last chunk, normalised row or partition partials
             if (!(ok = wait_pv(gch - 1))) break;
             tc::fence_after_sync();

@@ -704,7 +704,7 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
         return PA_ERR_CUDA;
     const int64_t pair_upper = (int64_t)num_seqs * maxP;
     const int vk = g_verify_kernel.load(std::memory_order_relaxed);
-    const bool tc5 = vk == PA_VERIFY_TCGEN05 || (vk == PA_VERIFY_AUTO && rows > 16);
+    const bool tc5 = vk != PA_VERIFY_MMA_SYNC;
     pa_status st;
     if (dtype == PA_F16) {
         if (tc5)
