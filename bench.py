@@ -466,6 +466,7 @@ def run_native(args):
 
     peak, peak_kind = measured_peaks()
     if Q > 1:
+        P = pa.pa_verify_partition_size(len(lens), Q, cfg.num_heads, cfg.num_kv_heads, P)   # what pa_verify used
         dec_bytes = verify_kernel_bytes(cfg, lens, P, Q)
     else:
         dec_bytes = decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused")

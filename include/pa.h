@@ -153,6 +153,15 @@ size_t pa_verify_workspace_size(int num_seqs, int num_queries, int num_heads, in
                                 int max_context_len, int partition_size);
 
 /*
+ * The partition pa_verify uses for these shapes: partition_size itself when
+ * non-zero, else 1024 tokens when a kv head carries R = num_heads /
+ * num_kv_heads x num_queries >= 32 query rows and num_seqs x num_kv_heads x
+ * ceil(R / 64) >= 592, else 512.  No device work; never fails (argument checks
+ * are pa_verify's).
+ */
+int pa_verify_partition_size(int num_seqs, int num_queries, int num_heads, int num_kv_heads, int partition_size);
+
+/*
  * pa_verify -- multi-query paged attention: the target model's verification
  * pass of speculative decoding ([P1] "大模型推理引擎高频优化：连续批处理、
  * PagedAttention 与 KV Cache 实战拆解", section 5: a draft model proposes a
@@ -171,7 +180,8 @@ size_t pa_verify_workspace_size(int num_seqs, int num_queries, int num_heads, in
  * row.  fp16 and bf16 only (tensor cores; fp32 returns PA_ERR_UNSUPPORTED);
  * 1 <= Q <= 64.  Long contexts are split and merged as in pa_decode; the
  * workspace (>= pa_verify_workspace_size bytes, 256-byte aligned) holds the
- * partials.
+ * partials.  partition_size 0 lets pa_verify_partition_size choose (512 or
+ * 1024 tokens); pa_verify_workspace_size(..., 0) covers either.
  */
 pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, const int32_t* context_lens, float scale,

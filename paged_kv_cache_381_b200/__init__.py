@@ -165,6 +165,11 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block
     return out
 
 
+def pa_verify_partition_size(num_seqs, num_queries, num_heads, num_kv_heads, partition_size=0):
+    """The partition (tokens) pa_verify uses for these shapes."""
+    return int(lib().pa_verify_partition_size(num_seqs, num_queries, num_heads, num_kv_heads, partition_size))
+
+
 def pa_verify_workspace_size(num_seqs, num_queries, num_heads, head_dim, max_context_len, partition_size=0):
     return int(lib().pa_verify_workspace_size(num_seqs, num_queries, num_heads, head_dim, max_context_len,
                                               partition_size))

@@ -41,6 +41,8 @@
 //    runs through its remaining work without touching the stages.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace pa_dev {
@@ -837,81 +839,91 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, int2* pl
         if (tid == 0) carry += warp_tot[nw - 1];
         __syncthreads();
     }
+    // level 1 lists every split sequence once, as (s, 1): the reduce walks it
+    if (tid == 0) {
+        count[1] = L > 1 ? cur[1] : 0;           // its first plan slot
+        count[2] = L > 1 ? cur[0] - cur[1] : 0;  // its size: sequences with more than one partition
+    }
+    __syncthreads();
     for (int s = tid; s < a.num_seqs; s += blockDim.x) {
         const int np = partitions_of(a, clamp_context(a, s, false));
         for (int p = 0; p < np; ++p) plan[atomicAdd(&cur[p], 1)] = make_int2(s, p);
     }
     __syncthreads();
-    if (tid == 0) *count = carry;
+    if (tid == 0) count[0] = carry;
 }
 
 // Log-sum-exp merge of a sequence's partitions (base-2 units): with
 // M = max_i m_i, w_i = 2^(m_i - M):  out = sum_i w_i o_i / sum_i w_i l_i.
-// One warp per (sequence, query head) -- for the verification pass, per
-// (sequence, query row, head) with num_heads = rows x heads; sequences with one
-// partition were finished by the attention kernel.
+// One warp per (split sequence, query head) -- for the verification pass, per
+// (sequence, query row, head) with num_heads = rows x heads.  The split
+// sequences come from the plan (its level 1: one (s, 1) entry per sequence with
+// more than one partition), walked by a persistent grid; sequences with one
+// partition were finished by the attention kernel.  A row's m, l and its first
+// RB partials are all requested before the max and sum are formed.
+constexpr int kReduceWarps = 8;                   // warps per reduce CTA
 template <typename T, int D>
-__global__ void __launch_bounds__(128) reduce_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const DecodeArgs a) {
     using Tr = ElemTraits<T>;
-    grid_dependency_wait();                       // the decode kernel's partials must be complete
+    constexpr int PER = D / 32;                   // floats of a partial row per lane
+    constexpr int RB = 8;                         // partials in flight per lane
+    using Vec = typename std::conditional<PER == 4, float4, float2>::type;
+    grid_dependency_wait();                       // the plan and the partials must be complete
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * 4 + warp;
-    if (row >= (int64_t)a.num_seqs * a.num_heads) return;
-    const int s = (int)(row / a.num_heads);
-    const int np = partitions_of(a, clamp_context(a, s, false));
-    if (np <= 1) return;
-    const float* pm = a.part_m + row * a.max_partitions;
-    const float* pl = a.part_l + row * a.max_partitions;
-    float M = -INFINITY;
-    for (int i = lane; i < np; i += 32) M = fmaxf(M, pm[i]);
-    M = warp_max(M);
-    float L = 0.f;
-    for (int i = lane; i < np; i += 32) L += exp2f(pm[i] - M) * pl[i];
-    L = warp_sum(L);
-    constexpr int PER = D / 32;
-    float o[PER];
+    const int split_base = a.plan_count[1];
+    const int64_t units = (int64_t)a.plan_count[2] * a.num_heads;
+    for (int64_t u = (int64_t)blockIdx.x * kReduceWarps + warp; u < units; u += (int64_t)gridDim.x * kReduceWarps) {
+        const int k = (int)(u / a.num_heads);
+        const int h = (int)(u - (int64_t)k * a.num_heads);
+        const int s = a.plan[split_base + k].x;
+        const int np = partitions_of(a, clamp_context(a, s, false));
+        const int64_t row = (int64_t)s * a.num_heads + h;
+        const float* pm = a.part_m + row * a.max_partitions;
+        const float* pl = a.part_l + row * a.max_partitions;
+        const float* po = a.part_o + row * a.max_partitions * D + lane * PER;
+        Vec x[RB];
+        float mb[RB];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) o[j] = 0.f;
-    const float* po = a.part_o + row * a.max_partitions * D + lane * PER;
-    // partitions in order; each lane computes one weight per 32 partitions and
-    // the loads of 8 partitions are issued before their FMAs
-    for (int b = 0; b < np; b += 32) {
-        const float wl = b + lane < np ? exp2f(pm[b + lane] - M) : 0.f;
-        const int cnt = min(32, np - b);
-        int i = 0;
-        for (; i + 8 <= cnt; i += 8) {
-            float x[8][PER];
+        for (int j = 0; j < RB; ++j)
+            if (j < np) {
+                x[j] = *reinterpret_cast<const Vec*>(po + (int64_t)j * D);
+                mb[j] = pm[j];
+            }
+        float M = -INFINITY;
+        for (int i = lane; i < np; i += 32) M = fmaxf(M, pm[i]);
+        M = warp_max(M);
+        float L = 0.f;
+        for (int i = lane; i < np; i += 32) L += exp2f(pm[i] - M) * pl[i];
+        L = warp_sum(L);
+        float o[PER];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float* src = po + (int64_t)(b + i + j) * D;
-                if constexpr (PER == 4) {
-                    const float4 v = *reinterpret_cast<const float4*>(src);
-                    x[j][0] = v.x; x[j][1] = v.y; x[j][2] = v.z; x[j][3] = v.w;
-                } else {
-                    const float2 v = *reinterpret_cast<const float2*>(src);
-                    x[j][0] = v.x; x[j][1] = v.y;
+        for (int j = 0; j < PER; ++j) o[j] = 0.f;
+        // partitions in order
+        for (int b = 0; b < np; b += RB) {
+            if (b > 0) {
+#pragma unroll
+                for (int j = 0; j < RB; ++j)
+                    if (b + j < np) {
+                        x[j] = *reinterpret_cast<const Vec*>(po + (int64_t)(b + j) * D);
+                        mb[j] = pm[b + j];
+                    }
+            }
+#pragma unroll
+            for (int j = 0; j < RB; ++j)
+                if (b + j < np) {
+                    const float wgt = exp2f(mb[j] - M);
+                    const float* xv = reinterpret_cast<const float*>(&x[j]);
+#pragma unroll
+                    for (int q = 0; q < PER; ++q) o[q] = fmaf(wgt, xv[q], o[q]);
                 }
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float wgt = __shfl_sync(0xffffffffu, wl, i + j);
-#pragma unroll
-                for (int k = 0; k < PER; ++k) o[k] = fmaf(wgt, x[j][k], o[k]);
-            }
         }
-        for (; i < cnt; ++i) {
-            const float wgt = __shfl_sync(0xffffffffu, wl, i);
-            const float* src = po + (int64_t)(b + i) * D;
+        T* out = static_cast<T*>(a.out) + row * D + lane * PER;
+        // L == 0 only for a verification row that sees no token (context shorter
+        // than the query rows): a zero row, as for an empty context
 #pragma unroll
-            for (int k = 0; k < PER; ++k) o[k] = fmaf(wgt, src[k], o[k]);
-        }
+        for (int j = 0; j < PER; ++j) out[j] = Tr::from_float(L > 0.f ? o[j] / L : 0.f);
     }
-    T* out = static_cast<T*>(a.out) + row * D + lane * PER;
-    // L == 0 only for a verification row that sees no token (context shorter
-    // than the query rows): a zero row, as for an empty context
-#pragma unroll
-    for (int j = 0; j < PER; ++j) out[j] = Tr::from_float(L > 0.f ? o[j] / L : 0.f);
 }
 
 }  // namespace pa_dev

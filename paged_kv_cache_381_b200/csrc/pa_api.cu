@@ -254,11 +254,16 @@ pa_status dispatch_head_dim(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, 
 
 template <typename T>
 pa_status launch_reduce(const pa_dev::DecodeArgs& a, int D, cudaStream_t stream) {
+    // persistent: the number of split rows is known only on the device (plan)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
     const int64_t rows = (int64_t)a.num_seqs * a.num_heads;
-    const unsigned grid = (unsigned)((rows + 3) / 4);
+    const int64_t blocks_needed = (rows + pa_dev::kReduceWarps - 1) / pa_dev::kReduceWarps;
+    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)device_sms(dev) * 4));
+    const dim3 block(pa_dev::kReduceWarps * 32);
     LaunchScope scope(PA_KERNEL_REDUCE, stream);
-    if (D == 64) return launch_dependent(pa_dev::reduce_kernel<T, 64>, dim3(grid), dim3(128), 0, stream, a);
-    return launch_dependent(pa_dev::reduce_kernel<T, 128>, dim3(grid), dim3(128), 0, stream, a);
+    if (D == 64) return launch_dependent(pa_dev::reduce_kernel<T, 64>, dim3(grid), block, 0, stream, a);
+    return launch_dependent(pa_dev::reduce_kernel<T, 128>, dim3(grid), block, 0, stream, a);
 }
 
 template <typename T, int D>
@@ -623,6 +628,20 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     }
 }
 
+int pa_verify_partition_size(int num_seqs, int num_queries, int num_heads, int num_kv_heads, int partition_size) {
+    if (partition_size != 0) return partition_size;
+    if (num_seqs <= 0 || num_queries <= 0 || num_kv_heads <= 0 || num_heads <= 0) return kDefaultPartition;
+    const int64_t rows = (int64_t)num_heads / num_kv_heads * num_queries;
+    const int64_t items = (int64_t)num_seqs * num_kv_heads * ((rows + 63) / 64);
+    // A split partition writes rows x (head_dim + 2) fp32 partials per kv head, which
+    // the reduce reads back: at 32 rows or more that is over a tenth of the K/V bytes
+    // of a 512-token partition.  There, and with enough (sequence, kv head) items to
+    // fill the GPU without splitting, 1024-token partitions halve the partials and the
+    // per-item start-up of the kernel (their workspace need is below the 512-token one
+    // that pa_verify_workspace_size reports for partition_size 0).
+    return rows >= 32 && items >= 4 * 148 ? 1024 : kDefaultPartition;
+}
+
 size_t pa_verify_workspace_size(int num_seqs, int num_queries, int num_heads, int head_dim, int max_context_len,
                                 int partition_size) {
     if (num_queries <= 0) return 0;
@@ -640,7 +659,10 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
     if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     if (dtype == PA_F32 || num_queries > 64) return PA_ERR_UNSUPPORTED;
     if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
-    const int P = resolve_partition(partition_size);
+    const int group = num_heads / num_kv_heads;
+    const int rows = group * num_queries;
+    const int n_chunks = (rows + 63) / 64;
+    const int P = pa_verify_partition_size(num_seqs, num_queries, num_heads, num_kv_heads, partition_size);
     if (!valid_partition(P)) return PA_ERR_INVALID_ARG;
     if (num_seqs == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
@@ -651,9 +673,6 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
     if (cap > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
     const int64_t maxP = partitions_for(cap, P);
     if (maxP > kMaxPartitions) return PA_ERR_UNSUPPORTED;
-    const int group = num_heads / num_kv_heads;
-    const int rows = group * num_queries;
-    const int n_chunks = (rows + 63) / 64;
     if ((int64_t)num_seqs * maxP * num_kv_heads * n_chunks > INT32_MAX) return PA_ERR_INVALID_ARG;
     if ((int64_t)num_seqs * num_queries * num_heads > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
 

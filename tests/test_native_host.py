@@ -278,6 +278,22 @@ def test_verify_workspace_and_argument_rules(pa):
     assert lib.pa_verify(*args(6, 2)) == 1            # null pointers
 
 
+def test_verify_partition_choice(pa):
+    """partition_size 0: 1024 tokens once a kv head carries >= 32 query rows
+    and (sequence, kv head, 64-row chunk) items reach 592, else 512; an
+    explicit size is kept; the 0-partition workspace covers the 1024 choice."""
+    assert pa.pa_verify_partition_size(256, 6, 64, 8) == 1024       # 48 rows, 2048 items
+    assert pa.pa_verify_partition_size(64, 6, 32, 32) == 512        # 6 rows
+    assert pa.pa_verify_partition_size(8, 6, 64, 8) == 512          # 64 items
+    assert pa.pa_verify_partition_size(74, 4, 64, 8) == 1024        # 32 rows, 592 items
+    assert pa.pa_verify_partition_size(73, 4, 64, 8) == 512         # 584 items
+    assert pa.pa_verify_partition_size(256, 3, 64, 8) == 512        # 24 rows
+    assert pa.pa_verify_partition_size(8, 16, 64, 8) == 512         # 128 rows per kv head: 2 chunks, 128 items
+    assert pa.pa_verify_partition_size(256, 6, 64, 8, 256) == 256
+    for S, Q, Hq, D, ctx in ((256, 6, 64, 128, 8192), (64, 6, 32, 128, 2048), (8, 4, 64, 64, 32768)):
+        assert pa.pa_verify_workspace_size(S, Q, Hq, D, ctx, 0) >= pa.pa_verify_workspace_size(S, Q, Hq, D, ctx, 1024)
+
+
 def test_verify_kernel_selection(pa):
     """The process-wide tensor-core path of pa_verify: AUTO by default, the
     three named kinds accepted, anything else rejected with nothing changed."""
