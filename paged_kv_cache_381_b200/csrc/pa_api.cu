@@ -13,6 +13,7 @@
 
 #include "device/cache_ops.cuh"
 #include "device/decode.cuh"
+#include "device/split_merge.cuh"
 #include "device/verify.cuh"
 #include "device/verify_tc.cuh"
 #include "pa.h"
