@@ -62,6 +62,14 @@ namespace pa_dev {
 #define PA_VERIFY_TC_PBUF 1      // P tiles in shared memory: 2 = double-buffered, 1 = single
 #endif
 
+// 2^x by the PTX ex2.approx instruction (relative error about 2^-22; -inf -> +0;
+// results below the normal range flush to zero)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <typename T, int D>
 struct VerifyTcCfg {
     static constexpr int ELT = 2;
@@ -453,14 +461,27 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 // exact max of the chunk's visible scores (base-2 units); this thread holds
                 // tokens c*64 + half*32 + k of row m
                 const int t0 = c * C::CHUNK + half * 32;
+                // With a positive scale the max commutes with scaling: scores stay raw (masked
+                // ones -inf), the max is scaled once and p = 2^(fma(s, scale, -base)).  A
+                // thread whose 32 tokens are all visible (most chunks) skips the mask.
+                const float sl2 = a.scale_log2;
+                const bool raw = sl2 > 0.f;
+                const bool all_visible = t0 + 31 < w.n && w.t0 + t0 + 31 <= pos;
                 float cmax = -INFINITY;
+                if (raw && all_visible) {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int t = t0 + k;
-                    const float z = (t < w.n && w.t0 + t <= pos) ? __uint_as_float(r[k]) * a.scale_log2 : -INFINITY;
-                    r[k] = __float_as_uint(z);
-                    cmax = fmaxf(cmax, z);
+                    for (int k = 0; k < 32; ++k) cmax = fmaxf(cmax, __uint_as_float(r[k]));
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int t = t0 + k;
+                        const float x = __uint_as_float(r[k]);
+                        const float z = (t < w.n && w.t0 + t <= pos) ? (raw ? x : x * sl2) : -INFINITY;
+                        r[k] = __float_as_uint(z);
+                        cmax = fmaxf(cmax, z);
+                    }
                 }
+                if (raw) cmax *= sl2;                    // -inf stays -inf
                 cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 16));
                 // Lazy reference max: p = 2^(z - m_run) stays <= 2^8, so the reference only
                 // moves (and O is rescaled) when a score beats it by more than 8 in base-2
@@ -472,10 +493,11 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 const float corr = raise && !fresh ? exp2f(m_run - m_new) : 1.f;
                 uint32_t hi[16], lo[16];
                 float lsum = 0.f;
+                const float sc = raw ? sl2 : 1.f;       // scores are raw, or already scaled
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
-                    const float p0 = exp2f(__uint_as_float(r[k]) - base);
-                    const float p1 = exp2f(__uint_as_float(r[k + 1]) - base);
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(r[k]), sc, -base));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(r[k + 1]), sc, -base));
                     if constexpr (C::PSPLIT) {
                         lsum += p0 + p1;
                         split_pack<MO>(p0, p1, hi[k >> 1], lo[k >> 1]);
