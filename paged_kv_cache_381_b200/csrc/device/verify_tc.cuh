@@ -58,6 +58,9 @@ namespace pa_dev {
 #ifndef PA_VERIFY_TC_PWAR
 #define PA_VERIFY_TC_PWAR 1      // with p in tensor memory: S of chunk g waits for P.V of chunk g - 2
 #endif
+#ifndef PA_VERIFY_TC_TWO_ISSUERS
+#define PA_VERIFY_TC_TWO_ISSUERS 1   // 1: S and P.V products issued by two warps; 0: one thread issues both
+#endif
 #ifndef PA_VERIFY_TC_PBUF
 #define PA_VERIFY_TC_PBUF 1      // P tiles in shared memory: 2 = double-buffered, 1 = single
 #endif
@@ -107,7 +110,13 @@ struct VerifyTcCfg {
     static constexpr int OFF_TABLE = (OFF_ABORT + 4 + 15) / 16 * 16;
     static constexpr int MAX_TABLE = 1024 / 8;
     static constexpr size_t SMEM = 1024 + (size_t)OFF_TABLE + MAX_TABLE * 4;
-    static constexpr int THREADS = 6 * 32;
+    // A tcgen05.mma costs its issuing thread about 57 cycles whatever its N; two
+    // issuing warps (S in warp 1, P.V in warp 6) double the rate the chunks need.
+    // The S warp's wait for P.V of chunk g - 2 orders the two streams where they
+    // share tensor memory, so this needs p in tensor memory with that wait.
+    static constexpr bool TWO_ISSUERS = PA_VERIFY_TC_TWO_ISSUERS != 0 && PTMEM && PA_VERIFY_TC_PWAR != 0;
+    static constexpr int PV_WARP = TWO_ISSUERS ? 6 : 1;
+    static constexpr int THREADS = (TWO_ISSUERS ? 7 : 6) * 32;
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(SLOT_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0 && P_TILE % 1024 == 0, "1024-byte atoms");
     static_assert((M * D * 2 / 16) % 128 == 0, "q tile chunks per staging thread");
@@ -138,7 +147,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     uint64_t* p_full = q_full + 2;               // chunk's S read, O rescaled, p written (128 arrivals)
     uint64_t* o_full = q_full + 3;               // [NPH] P.V of chunk g done (commit), copy g % NPH
     uint64_t* o_empty = o_full + C::NPH;         // O read by the epilogue (128 arrivals)
-    uint64_t* drain = o_empty + 1;               // every MMA done, before TMEM is freed
+    uint64_t* drain = o_empty + 1;               // every MMA done, before TMEM is freed (one commit per issuer)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + C::OFF_TABLE);
@@ -157,7 +166,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         mbar_init(q_empty, 1);
         mbar_init(p_full, 128);
         mbar_init(o_empty, 128);
-        mbar_init(drain, 1);
+        mbar_init(drain, C::TWO_ISSUERS ? 2 : 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -253,8 +262,10 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             }
         }
     }
-    if (warp == 1) {
+    if (warp == 1 || warp == C::PV_WARP) {
         // ------------------------------------------------------------ MMA issue
+        const bool do_s = warp == 1;                     // issues S products (and commits q_empty)
+        const bool do_pv = warp == C::PV_WARP;           // issues P.V products
         uint32_t seq = 0, q_ph = 0, p_ph = 0, oe_ph = 0, gch = 0;
         bool ok = true;
         // operand descriptors built once; every MMA adds a byte offset to one of them
@@ -262,16 +273,17 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         const uint64_t pdesc = tc::sw128_desc(smem_addr(ps), 16, 1024);                 // P, K-major
         const uint64_t kdesc = tc::sw128_desc(smem_addr(smem), 16, 1024);               // slot 0 as K, K-major
         const uint64_t vdesc = tc::sw128_desc(smem_addr(smem), C::SLICE_BYTES, 1024);   // slot 0 as V, MN-major
-        // S of global chunk g = Q K^T over its 64 tokens, into S buffer g & 1 (token
-        // columns past the partition read stale rows; the softmax masks them)
-        auto issue_s = [&](uint32_t g) -> bool {
+        // S of global chunk g = Q K^T over its 64 tokens (stream element pos), into S
+        // buffer g & 1 (token columns past the partition read stale rows; the softmax
+        // masks them)
+        auto issue_s = [&](uint32_t pos, uint32_t g) -> bool {
             const uint32_t buf = g & 1u;
-            const int slot = seq % C::NSLOTS;
-            if (!mbar_wait(&full[slot], (seq / C::NSLOTS) & 1u, abort_flag)) return false;
+            const int slot = pos % C::NSLOTS;
+            if (!mbar_wait(&full[slot], (pos / C::NSLOTS) & 1u, abort_flag)) return false;
             if constexpr (C::PTMEM && PA_VERIFY_TC_PWAR) {
-                // the buffer holds p of chunk g - 2, read by the P.V issued just before: a
-                // later product may not overwrite an operand the tensor core is still
-                // reading, so that P.V completes first
+                // the buffer holds p of chunk g - 2, read by P.V of that chunk: a later
+                // product may not overwrite an operand the tensor core may still read
+                // (nor, with two issuers, one not yet read), so that P.V completes first
                 if (g >= 2 && !mbar_wait(&o_full[(g - 2) % C::NPH], ((g - 2) / C::NPH) & 1u, abort_flag)) return false;
             }
             tc::fence_after_sync();
@@ -287,15 +299,14 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 tc::commit(&s_full[g % C::NPH]);    // also frees the slot for the producer
             }
             __syncwarp();
-            ++seq;
             return true;
         };
-        // O += P V over the tokens of chunk c (global chunk g), p from P buffer g & 1
-        // (buffer 0 when single)
-        auto issue_pv = [&](int c, int n, uint32_t g, bool first) -> bool {
+        // O += P V over the tokens of chunk c (global chunk g, stream element pos), p from
+        // P buffer g & 1 (buffer 0 when single)
+        auto issue_pv = [&](uint32_t pos, int c, int n, uint32_t g, bool first) -> bool {
             const uint32_t pbuf = C::PBUF == 2 ? (g & 1u) : 0u;
-            const int slot = seq % C::NSLOTS;
-            if (!mbar_wait(&full[slot], (seq / C::NSLOTS) & 1u, abort_flag)) return false;
+            const int slot = pos % C::NSLOTS;
+            if (!mbar_wait(&full[slot], (pos / C::NSLOTS) & 1u, abort_flag)) return false;
             const int rows = min(C::CHUNK, n - c * C::CHUNK);
             if (rows < C::CHUNK) {
                 // rows past the partition (stale or unwritten rows, maybe NaN): zero them
@@ -327,51 +338,75 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 tc::commit(&o_full[g % C::NPH]);    // also frees the slot for the producer
             }
             __syncwarp();
-            ++seq;
             return true;
+        };
+        // P.V of chunk c, once its p is written (and, for the item's first chunk, the
+        // previous item's O has been read out)
+        auto pv_chunk = [&](uint32_t pos, int c, int n, uint32_t g) -> bool {
+            if (!mbar_wait(p_full, p_ph, abort_flag)) return false;
+            p_ph ^= 1u;
+            if (c == 0) {
+                if (!mbar_wait(o_empty, oe_ph ^ 1u, abort_flag)) return false;
+                oe_ph ^= 1u;
+            }
+            tc::fence_after_sync();
+            return issue_pv(pos, c, n, g, c == 0);
         };
         for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
             const WorkItem w = decode_item(a, i, false);
             if (w.n == 0) continue;
-            if (!mbar_wait(q_full, q_ph, abort_flag)) {
-                ok = false;
-                break;
-            }
-            q_ph ^= 1u;
-            tc::fence_after_sync();
             const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
-            if (!(ok = issue_s(gch))) break;
-            if (nc == 1 && lane == 0) tc::commit(q_empty);        // last S of the item: Q may be replaced
-            __syncwarp();
-            for (int c = 0; c < nc && ok; ++c) {
-                if (c + 1 < nc) {
-                    if (!(ok = issue_s(gch + c + 1))) break;
-                    if (c + 2 == nc && lane == 0) tc::commit(q_empty);
-                    __syncwarp();
+            // stream positions of the item's elements: K0, then K(c+1), V(c) per chunk
+            auto kpos = [&](int c) -> uint32_t { return seq + (c == 0 ? 0u : (uint32_t)(2 * c - 1)); };
+            auto vpos = [&](int c) -> uint32_t {
+                return seq + (c + 1 < nc ? (uint32_t)(2 * c + 2) : (uint32_t)(2 * nc - 1));
+            };
+            if (do_s) {
+                if (!mbar_wait(q_full, q_ph, abort_flag)) {
+                    ok = false;
+                    break;
                 }
-                if (!(ok = mbar_wait(p_full, p_ph, abort_flag))) break;
-                p_ph ^= 1u;
-                if (c == 0) {
-                    // the previous item's O has been read out before this item's first P.V
-                    if (!(ok = mbar_wait(o_empty, oe_ph ^ 1u, abort_flag))) break;
-                    oe_ph ^= 1u;
-                }
+                q_ph ^= 1u;
                 tc::fence_after_sync();
-                if (!(ok = issue_pv(c, w.n, gch + c, c == 0))) break;
             }
+            if constexpr (C::TWO_ISSUERS) {
+                if (do_s) {
+                    for (int c = 0; c < nc && ok; ++c) {
+                        ok = issue_s(kpos(c), gch + c);
+                        if (ok && c + 1 == nc && lane == 0) tc::commit(q_empty);   // Q may be replaced
+                        __syncwarp();
+                    }
+                } else {
+                    for (int c = 0; c < nc && ok; ++c) ok = pv_chunk(vpos(c), c, w.n, gch + c);
+                }
+            } else {
+                // one thread: S(c+1) is issued before P.V(c), so it runs during softmax(c)
+                if (!(ok = issue_s(kpos(0), gch))) break;
+                if (nc == 1 && lane == 0) tc::commit(q_empty);        // last S of the item: Q may be replaced
+                __syncwarp();
+                for (int c = 0; c < nc && ok; ++c) {
+                    if (c + 1 < nc) {
+                        if (!(ok = issue_s(kpos(c + 1), gch + c + 1))) break;
+                        if (c + 2 == nc && lane == 0) tc::commit(q_empty);
+                        __syncwarp();
+                    }
+                    ok = pv_chunk(vpos(c), c, w.n, gch + c);
+                }
+            }
+            seq += 2 * nc;
             gch += nc;
         }
         if (!ok) {
             if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
             *abort_flag = 1;
         }
-        // drain: every MMA issued above has completed before TMEM is released
+        // drain: every MMA this warp issued has completed before TMEM is released
         if (lane == 0) tc::commit(drain);
         __syncwarp();
         const volatile int never = 0;
         mbar_wait(drain, 0, &never);
     }
-    if (warp >= 2) {
+    if (warp >= 2 && warp < 6) {
         // ------------------------------------------------- softmax and epilogue
         const int ctid = threadIdx.x - 64;               // 0..127
         const int quarter = warp & 3;                    // TMEM lanes 32*quarter .. +15 hold rows 16*quarter ..
