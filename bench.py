@@ -95,10 +95,15 @@ def measured_peaks():
 
 
 def kernel_hash(kernel="decode"):
+    """Hash of the kernel's sources without // comments and blank lines, so that a
+    comment edit does not void a recorded traffic figure."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -7,9 +7,9 @@
 // items, partitions, partials and the reduce are shared with decode.
 //
 // Design (2 CTAs per SM, each holding 256 of the SM's 512 TMEM columns):
-//  * Item = (sequence, 512-token partition, kv head, chunk of <= 64 query
-//    rows).  The rows form one M = 64 tile; the partition is walked in chunks
-//    of 64 tokens.
+//  * Item = (sequence, partition of 512 or 1024 tokens, kv head, chunk of <= 64
+//    query rows).  The rows form one M = 64 tile; the partition is walked in
+//    chunks of 64 tokens.
 //  * Warp 0 streams K and V chunks through TMA tiled boxes into a ring of
 //    five slots (slot = 64 token rows of one kv head; each 128-byte head_dim
 //    slice of the 64 rows is one 128-byte-swizzled array), K running one
@@ -17,17 +17,21 @@
 //    products that read its previous contents are done: the producer waits
 //    on the commit barrier the softmax (S done) or the epilogue (P.V done)
 //    waits on, so no separate release barrier is committed.
-//  * Warp 1 issues, from one thread, in the same order:
+//  * One elected thread of warp 1 issues the S products, one of warp 6 the P.V
+//    products:
 //        S(c) [64 x 64]  = Q K^T   KS MMAs M=64 N=64 K=16, into one of two S buffers
 //        O    [64 x D]  += P V     4 (x 2) MMAs M=64 N=D K=16, P read from tensor
 //                                  memory, V MN-major from the slot as loaded
-//    so S(c+1) is computed while the softmax of chunk c runs.  TMEM columns:
-//    S buffers [0, 64) and [64, 128), O [128, 128 + D).  A tcgen05.mma costs
-//    its issuing thread about as much as a commit or a barrier test, whatever
-//    its N, so a chunk is covered by as few instructions as the shapes allow.
+//    S(c+1) is computed while the softmax of chunk c runs; S(c) waits for P.V
+//    of chunk c - 2, the last reader of its buffer.  TMEM columns: S buffers
+//    [0, 64) and [64, 128), O [128, 128 + D).  A tcgen05.mma costs its issuing
+//    thread about as much as a commit or a barrier test, whatever its N, so a
+//    chunk is covered by as few instructions as the shapes allow, over two
+//    issuers.
 //  * Warps 2-5 (one TMEM lane quarter each; a quarter's first 16 lanes hold 16
 //    rows of an M = 64 accumulator, read as two half-warps of 32 columns)
-//    stage q, take the exact max of the chunk (causal mask), rescale O in TMEM
+//    stage q, take the exact max of the chunk (causal mask, only where a
+//    thread's tokens need it; max over raw scores, scaled once), rescale O in TMEM
 //    when the running max grows by more than 8 (base 2), write p over the
 //    chunk's S columns, and finally read O, normalise and store (or store the
 //    partition's partials).  For bf16, p is split into a 16-bit value and its
