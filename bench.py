@@ -319,6 +319,24 @@ def run_reference(args):
 # native arm
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(values, device):
+    """Each value's maximum over the ranks of the default process group (the
+    values themselves without one): a multi-GPU time is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_gbs(world, bytes_per_rank, ms):
+    """Whole-job throughput: every rank moved bytes_per_rank in the slowest
+    rank's ms (replicas: weak scaling)."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -417,10 +435,7 @@ def run_native(args):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     ms = sum(step_ms) / len(step_ms)
     dec_ms = prof[kernel][0] / max(1, prof[kernel][1])
-    if world > 1:
-        t = torch.tensor([ms, dec_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, dec_ms = float(t[0]), float(t[1])
+    ms, dec_ms = max_over_ranks([ms, dec_ms], dev)
 
     # ---- e2e: the same step from pinned host buffers through pa_step
     e2e = None
@@ -460,11 +475,8 @@ def run_native(args):
         e1.record()
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / args.steps
-        if world > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t[0])
-        e2e = {"value": world * step_kv / (ems * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+        (ems,) = max_over_ranks([ems], dev)
+        e2e = {"value": whole_job_gbs(world, step_kv, ems), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": ems,
                "tokens_per_s": world * len(lens) / (ems * 1e-3),
                "how": "pa_pipeline: each step's H2D and D2H overlap the neighbouring steps' compute"}
@@ -477,7 +489,7 @@ def run_native(args):
         dec_bytes = decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused")
     traffic = None if args.num_seqs else recorded_traffic(kname, args.workload, Q)
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
-    value = world * step_kv / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_kv, ms)
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
