@@ -302,30 +302,38 @@ pa_status launch_verify_tc(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, c
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
     static std::atomic<uint64_t> configured{0};
     static std::atomic<int> occ_of[kMaxDevices];
+    static std::atomic<int> smem_of[kMaxDevices];
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
-        // the whole unified L1 as shared memory, so that two CTAs fit
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) != cudaSuccess ||
-            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
-            return PA_ERR_CUDA;
-        // CTAs per SM from the shared memory (1 KB reserved per CTA) and the registers
         int smem_sm = 0;
         cudaFuncAttributes fa;
         if (cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
             cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
             return PA_ERR_CUDA;
-        const int by_smem = smem_sm / (int)(C::SMEM + 1024);
+        // Each CTA holds 256 of the SM's 512 TMEM columns: a third CTA on an SM would
+        // only wait in tcgen05.alloc.  The shared memory asked for is raised until a
+        // third no longer fits (1 KB reserved per CTA); the kernel uses C::SMEM of it.
+        const int smem = std::max((int)C::SMEM, smem_sm / 3 - 1024 + 16);
+        // the whole unified L1 as shared memory, so that two CTAs fit
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+            return PA_ERR_CUDA;
+        // CTAs per SM from the shared memory and the registers
+        const int by_smem = smem_sm / (smem + 1024);
         const int by_regs = 65536 / std::max(1, fa.numRegs * C::THREADS);
         const int occ = std::max(1, std::min(by_smem, by_regs));
-        if (dev < kMaxDevices) occ_of[dev].store(occ);
+        if (dev < kMaxDevices) {
+            occ_of[dev].store(occ);
+            smem_of[dev].store(smem);
+        }
         configured.fetch_or(bit);
     }
-    // two CTAs per SM at most: each holds 256 of the SM's 512 TMEM columns
     const int occ = std::min(2, dev < kMaxDevices ? std::max(1, occ_of[dev].load()) : 1);
+    const size_t smem = dev < kMaxDevices && smem_of[dev].load() > 0 ? (size_t)smem_of[dev].load() : C::SMEM;
     const int64_t items_upper = pair_upper * a.num_kv_heads * a.n_gchunks;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items_upper, (int64_t)device_sms(dev) * occ));
     LaunchScope scope(PA_KERNEL_VERIFY, stream);
-    return launch_dependent(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, stream, a, tk, tv);
+    return launch_dependent(kern, dim3((unsigned)grid), dim3(C::THREADS), smem, stream, a, tk, tv);
 }
 
 std::atomic<int> g_verify_kernel{PA_VERIFY_AUTO};
