@@ -233,7 +233,8 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbk * C::NH * box_bytes));
                 __syncwarp();
                 if (lane < nbk * C::NH) {
-                    const int half = lane / nbk;                        // slice
+                    static_assert(C::NH <= 2, "one or two slices");
+                    const int half = C::NH == 2 && lane >= nbk ? 1 : 0;  // slice
                     const int b = lane - half * nbk;                    // block within the chunk
                     const int phys = tbl[((c * C::CHUNK) >> a.log2_bs) + b];
                     tma_load_3d(smem + slot * C::SLOT_BYTES + half * C::SLICE_BYTES + b * box_bytes,
