@@ -495,18 +495,25 @@ pa_status pa_bm_set_cpu_blocks(pa_bm* bm, int num_cpu_blocks);
 
 /* Swap a resident sequence out: every block it holds ALONE (count 1) moves to
  * a host block, in logical order, and the GPU block goes back to the free
- * list; shared blocks stay resident and referenced.  pairs receives
- * *n (gpu, cpu) pairs ([n][2], cap pairs of room) for pa_swap_blocks, which
- * must run before the freed GPU blocks are written again.  All or nothing:
- * PA_ERR_NO_BLOCKS when the host pool is short, PA_ERR_INVALID_ARG when cap
- * is short (nothing changes; *n tells the need); PA_ERR_UNSUPPORTED with the
- * prefix cache on.  A swapped-out sequence cannot append, fork, pack or give
- * slots until it is swapped in; pa_bm_free releases it. */
+ * list; shared blocks stay resident and referenced.  With the prefix cache
+ * on, such a block that the cache names keeps its name and waits on the
+ * evictable list instead (last block first), its K/V reusable on the GPU
+ * until evicted.  pairs receives *n (gpu, cpu) pairs ([n][2], cap pairs of
+ * room) for pa_swap_blocks, which must run before the released GPU blocks are
+ * written again.  All or nothing: PA_ERR_NO_BLOCKS when the host pool is
+ * short, PA_ERR_INVALID_ARG when cap is short (nothing changes; *n tells the
+ * need).  A swapped-out sequence cannot append, fork, pack or give slots
+ * until it is swapped in; pa_bm_free releases it. */
 pa_status pa_bm_swap_out(pa_bm* bm, int64_t seq_id, int32_t* pairs, int cap, int* n);
 
-/* Swap a sequence back in: a fresh GPU block (taken from the free list) for
- * each of its host blocks, in logical order; pairs receives the (cpu, gpu)
- * copies.  All or nothing, as for pa_bm_swap_out. */
+/* Swap a sequence back in, in logical order: a block it left named in the
+ * prefix cache is taken back with no copy while the cache still names it by
+ * the same key (another holder may share it meanwhile); every other host
+ * block gets a fresh GPU block (free list first, else an evicted one) and a
+ * (cpu, gpu) copy in pairs.  Needs as many free blocks (free list + evictable)
+ * as the sequence has host blocks; all or nothing, as for pa_bm_swap_out.  On
+ * success *n is the number of copies (at most the host blocks; the cap check
+ * uses the host block count). */
 pa_status pa_bm_swap_in(pa_bm* bm, int64_t seq_id, int32_t* pairs, int cap, int* n);
 
 /* *swapped = 1 while the sequence is swapped out; the host free list from

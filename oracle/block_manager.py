@@ -485,3 +485,143 @@ class SwappingBlockManager(BlockManager):
         cf = set(self.cpu_free)
         assert len(cf) == len(self.cpu_free) and cf.isdisjoint(cpu_held)
         assert cf | set(cpu_held) == set(range(self.num_cpu_blocks)), "host block lost"
+
+
+class PrefixSwappingBlockManager(PrefixCachingBlockManager):
+    """Prefix cache and host swap pool together (oracle; test infrastructure only).
+
+    The two sections of [P3] "大模型推理显存优化实战：PagedAttention机制原理与vLLM
+    连续批处理配置" ("Prefix Caching前缀复用优化", "生产部署注意事项") at once.
+    Everything of PrefixCachingBlockManager holds; swap follows
+    SwappingBlockManager with these readings where the two meet:
+
+    * ``swap_out`` copies every block the sequence holds alone to a host
+      block, in logical order.  Such a block that the cache names keeps its
+      name and joins the evictable list (last block first, as ``free`` does),
+      so its K/V stays reusable on the GPU until it is evicted; the others go
+      to the free list.  The sequence remembers each named block and its name.
+    * ``swap_in`` needs as many free GPU blocks (free list + evictable) as the
+      sequence has host blocks, all or nothing.  In logical order, a
+      remembered block that the cache still names by the same name is taken
+      back (off the evictable list if it is there; another holder may have
+      referenced it meanwhile) with no copy; any other host block gets a
+      fresh block (which may evict) and a (cpu, gpu) copy.  Host blocks go
+      back to their list.  Blocks filled in this way are not named again.
+    * ``free`` of a swapped-out sequence returns its host blocks and drops its
+      GPU references; named blocks reaching zero join the evictable list last
+      block first.
+    """
+
+    def __init__(self, num_blocks, block_size, num_cpu_blocks, initial_free_order=None):
+        super().__init__(num_blocks, block_size, initial_free_order)
+        self.num_cpu_blocks = int(num_cpu_blocks)
+        self.cpu_free = list(range(self.num_cpu_blocks))
+        self.on_cpu = {}         # seq id -> per logical block, True = host block
+        self.left = {}           # seq id -> per logical block, (GPU block, name) left in the cache, or None
+
+    def swapped(self, seq):
+        return seq in self.on_cpu
+
+    def swap_out(self, seq):
+        if seq not in self.tables or seq in self.on_cpu:
+            raise InvalidArg(f"sequence {seq} is not resident")
+        table = self.tables[seq]
+        alone = [j for j, b in enumerate(table) if self.ref[b] == 1]
+        if len(alone) > len(self.cpu_free):
+            raise NoBlocks(f"need {len(alone)} host blocks, {len(self.cpu_free)} free")
+        loc, left, named, pairs = [False] * len(table), [None] * len(table), [], []
+        for j in alone:
+            g = table[j]
+            c = self.cpu_free.pop()
+            pairs.append((g, c))
+            self.ref[g] = 0
+            if g in self.name:
+                named.append(g)
+                left[j] = (g, self.name[g])
+            else:
+                self.free_list.append(g)
+            table[j] = c
+            loc[j] = True
+        self.evictable.extend(reversed(named))
+        self.on_cpu[seq], self.left[seq] = loc, left
+        return pairs
+
+    def swap_in(self, seq):
+        if seq not in self.on_cpu:
+            raise InvalidArg(f"sequence {seq} is not swapped out")
+        table, loc, left = self.tables[seq], self.on_cpu[seq], self.left[seq]
+        need = sum(loc)
+        if need > self.num_free:
+            raise NoBlocks(f"need {need} blocks, {self.num_free} free")
+        pairs = []
+        for j, here in enumerate(loc):
+            if not here:
+                continue
+            c = table[j]
+            kept = left[j]
+            if kept is not None and self.cache.get(kept[1]) == kept[0]:
+                g = kept[0]                     # still cached under the same name: no copy
+                if g in self.evictable:
+                    self.evictable.remove(g)
+                self.ref[g] += 1
+            else:
+                g = self._take()
+                self.ref[g] = 1
+                pairs.append((c, g))
+            self.cpu_free.append(c)
+            table[j] = g
+        del self.on_cpu[seq], self.left[seq]
+        return pairs
+
+    def fork(self, parent, child):
+        if parent in self.on_cpu:
+            raise InvalidArg(f"sequence {parent} is swapped out")
+        super().fork(parent, child)
+
+    def _append(self, seq, token):
+        if seq in self.on_cpu:
+            raise InvalidArg(f"sequence {seq} is swapped out")
+        return super()._append(seq, token)
+
+    def free(self, seq):
+        if seq not in self.on_cpu:
+            return super().free(seq)
+        named = []
+        for b, here in zip(self.tables[seq], self.on_cpu[seq]):
+            if here:
+                self.cpu_free.append(b)
+                continue
+            if self.ref[b] <= 0:
+                raise AssertionError("reference count underflow")
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                if b in self.name:
+                    named.append(b)
+                else:
+                    self.free_list.append(b)
+        self.evictable.extend(reversed(named))
+        del self.tables[seq], self.ctx[seq], self.tokens[seq], self.on_cpu[seq], self.left[seq]
+
+    def check(self):
+        held, cpu_held = {}, []
+        for seq, table in self.tables.items():
+            assert len(table) == ceil_div(self.ctx[seq], self.block_size), seq
+            loc = self.on_cpu.get(seq, [False] * len(table))
+            for b, here in zip(table, loc):
+                if here:
+                    cpu_held.append(b)
+                else:
+                    held[b] = held.get(b, 0) + 1
+        for b in range(self.num_blocks):
+            assert self.ref[b] == held.get(b, 0), (b, self.ref[b], held.get(b, 0))
+        free, ev = set(self.free_list), set(self.evictable)
+        assert len(free) == len(self.free_list) and len(ev) == len(self.evictable), "duplicate"
+        assert not (free & ev) and not (free & held.keys()) and not (ev & held.keys()), "block in two places"
+        assert free | ev | set(held) == set(range(self.num_blocks)), "block lost"
+        assert ev <= set(self.name), "evictable block without a name"
+        assert not (free & set(self.name)), "named block on the free list"
+        assert {self.cache[k]: k for k in self.cache} == self.name, "cache and names disagree"
+        assert len(set(cpu_held)) == len(cpu_held), "host block held twice"
+        cf = set(self.cpu_free)
+        assert len(cf) == len(self.cpu_free) and cf.isdisjoint(cpu_held)
+        assert cf | set(cpu_held) == set(range(self.num_cpu_blocks)), "host block lost"

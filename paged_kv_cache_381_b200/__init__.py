@@ -482,7 +482,7 @@ class BlockManager:
             _check(st, what)
         out = np.zeros((n.value, 2), dtype=np.int32)
         _check(fn(self._h, seq, _ptr(out), n.value, ctypes.byref(n)), what)
-        return out
+        return out[:n.value]                # a swap-in may copy fewer blocks than it takes back
 
     def swap_out(self, seq):
         """(gpu, cpu) block pairs [n, 2] to copy device -> host."""

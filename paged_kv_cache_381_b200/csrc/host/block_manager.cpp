@@ -95,6 +95,13 @@ void BlockManager::release_block(int32_t b) {
     }
 }
 
+void BlockManager::unlink_lru(int32_t b) {
+    if (in_lru_[b]) {
+        lru_.erase(lru_pos_[b]);
+        in_lru_[b] = 0;
+    }
+}
+
 std::string BlockManager::make_key(int32_t parent, const int32_t* tokens) const {
     std::string k(sizeof(int32_t) * (1 + block_size_), '\0');
     std::memcpy(&k[0], &parent, sizeof(int32_t));
@@ -240,16 +247,23 @@ pa_status BlockManager::free_seq(int64_t seq) {
     std::vector<int32_t> cached;
     const Seq& sq = it->second;
     if (sq.swapped) {
-        // host blocks go back to their list; shared GPU references are dropped
+        // host blocks go back to their list; shared GPU references are dropped (named
+        // blocks reaching zero wait on the LRU list, last block first)
         for (size_t j = 0; j < sq.table.size(); ++j) {
             const int32_t b = sq.table[j];
             if (sq.on_cpu[j]) {
                 cpu_free_.push_back(b);
             } else {
                 if (ref_[b] <= 0) return PA_ERR_INVALID_ARG;
-                if (--ref_[b] == 0) free_.push_back(b);
+                if (--ref_[b] == 0) {
+                    if (key_of_.count(b))
+                        cached.push_back(b);
+                    else
+                        free_.push_back(b);
+                }
             }
         }
+        for (auto r = cached.rbegin(); r != cached.rend(); ++r) release_block(*r);
         --num_swapped_;
         seqs_.erase(it);
         return PA_OK;
@@ -298,14 +312,16 @@ int BlockManager::swap_in_need(int64_t seq) const {
 }
 
 pa_status BlockManager::swap_out(int64_t seq, std::vector<int32_t>& pairs) {
-    if (prefix_cache_) return PA_ERR_UNSUPPORTED;
     const int need = swap_out_need(seq);
     if (need < 0) return PA_ERR_INVALID_ARG;
     if (need > (int)cpu_free_.size()) return PA_ERR_NO_BLOCKS;
     Seq& s = seqs_[seq];
     s.swapped = true;
     s.on_cpu.assign(s.table.size(), 0);
+    s.left_block.assign(s.table.size(), -1);
+    s.left_key.assign(s.table.size(), std::string());
     pairs.clear();
+    std::vector<int32_t> named;
     for (size_t j = 0; j < s.table.size(); ++j) {
         const int32_t g = s.table[j];
         if (ref_[g] != 1) continue;              // shared: stays resident, still referenced
@@ -314,10 +330,18 @@ pa_status BlockManager::swap_out(int64_t seq, std::vector<int32_t>& pairs) {
         pairs.push_back(g);
         pairs.push_back(c);
         ref_[g] = 0;
-        free_.push_back(g);
+        auto k = key_of_.find(g);
+        if (k != key_of_.end()) {                // stays named and reusable until evicted
+            named.push_back(g);
+            s.left_block[j] = g;
+            s.left_key[j] = k->second;
+        } else {
+            free_.push_back(g);
+        }
         s.table[j] = c;
         s.on_cpu[j] = 1;
     }
+    for (auto r = named.rbegin(); r != named.rend(); ++r) release_block(*r);   // last block first
     ++num_swapped_;
     return PA_OK;
 }
@@ -325,21 +349,33 @@ pa_status BlockManager::swap_out(int64_t seq, std::vector<int32_t>& pairs) {
 pa_status BlockManager::swap_in(int64_t seq, std::vector<int32_t>& pairs) {
     const int need = swap_in_need(seq);
     if (need < 0) return PA_ERR_INVALID_ARG;
-    if (need > (int)free_.size()) return PA_ERR_NO_BLOCKS;
+    if (need > num_free()) return PA_ERR_NO_BLOCKS;
     Seq& s = seqs_[seq];
     pairs.clear();
     for (size_t j = 0; j < s.table.size(); ++j) {
         if (!s.on_cpu[j]) continue;
         const int32_t c = s.table[j];
-        const int32_t g = free_.back();
-        free_.pop_back();
-        ref_[g] = 1;
-        pairs.push_back(c);
-        pairs.push_back(g);
+        int32_t g = s.left_block.empty() ? -1 : s.left_block[j];
+        if (g >= 0) {
+            // taken back with no copy while the cache still names it by the same key
+            auto b = block_of_.find(s.left_key[j]);
+            if (b == block_of_.end() || b->second != g) g = -1;
+        }
+        if (g >= 0) {
+            unlink_lru(g);
+            ++ref_[g];
+        } else {
+            g = take_block();                     // may evict
+            ref_[g] = 1;
+            pairs.push_back(c);
+            pairs.push_back(g);
+        }
         cpu_free_.push_back(c);
         s.table[j] = g;
     }
     s.on_cpu.clear();
+    s.left_block.clear();
+    s.left_key.clear();
     s.swapped = false;
     --num_swapped_;
     return PA_OK;
@@ -528,6 +564,8 @@ static pa_status swap_common(pa_bm* bm, int64_t seq_id, int32_t* pairs, int cap,
     pa_status st = out ? bm->impl.swap_out(seq_id, p) : bm->impl.swap_in(seq_id, p);
     if (st != PA_OK) return st;
     for (size_t i = 0; i < p.size(); ++i) pairs[i] = p[i];
+    // the copies made: a swap-in takes blocks still cached back without one
+    if (n) *n = (int)(p.size() / 2);
     return PA_OK;
 }
 

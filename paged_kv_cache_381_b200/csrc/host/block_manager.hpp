@@ -22,6 +22,10 @@ class BlockManager {
         bool tail_known = true;       // false once a token was appended without its id
         bool swapped = false;         // swapped out to the host pool
         std::vector<char> on_cpu;     // while swapped: per logical block, 1 = host block id
+        // while swapped, prefix cache on: per logical block, the GPU block left named in
+        // the cache (-1: none) and its key, to take it back without a copy
+        std::vector<int32_t> left_block;
+        std::vector<std::string> left_key;
     };
 
     BlockManager(int num_blocks, int block_size, const int32_t* initial_free_order);
@@ -70,6 +74,7 @@ class BlockManager {
     std::string make_key(int32_t parent, const int32_t* tokens) const;
     void register_block(int32_t block, int32_t parent, const int32_t* tokens);
     void release_block(int32_t block);                      // ref reached zero
+    void unlink_lru(int32_t block);                         // a cached block is referenced again
 
     int num_blocks_;
     int block_size_;
