@@ -39,3 +39,34 @@ def test_kernel_hash_ignores_comments(tmp_path, monkeypatch):
     assert bench.kernel_hash("probe") == h0
     src.write_text("int f() { return 2; }\n")
     assert bench.kernel_hash("probe") != h0
+
+
+def _cfg():
+    from paged_kv_cache_381_b200 import workloads as wl
+    return wl.DecodeConfig("bytes", "bf16", 3, 4, 2, 64, 16, "fixed", fixed_lengths=(10, 20, 40))
+
+
+def test_algorithmic_bytes_hand_example():
+    """Contexts 10, 20, 40 with 16-token partitions and blocks; 4 query / 2 kv
+    heads, head_dim 64, bf16.  By hand: K/V 70 tokens x 2 x 2 heads x 64 x 2 B
+    = 35840; q 3 x 4 x 64 x 2 = 1536; the one single-partition sequence's rows
+    4 x 64 x 2 = 512; partials of 2 + 3 partitions x 4 heads x (64 + 2) x 4 B
+    = 5280; table entries (1 + 2 + 3) blocks x 2 kv heads x 4 B = 48."""
+    import numpy as np
+    cfg, lens = _cfg(), np.array([10, 20, 40])
+    assert bench.kv_bytes(cfg, lens) == 35840
+    assert bench.decode_kernel_bytes(cfg, lens, 16) == 35840 + 1536 + 512 + 5280 + 48
+    # merged in the kernel: every final row written, partials written and read back
+    assert bench.decode_kernel_bytes(cfg, lens, 16, fused=True) == 35840 + 1536 + 1536 + 2 * 5280 + 48
+    # one partition for everything: no partials
+    assert bench.decode_kernel_bytes(cfg, lens, 64) == 35840 + 1536 + 1536 + 48
+
+
+def test_verify_bytes_and_flops_hand_example():
+    """Two query rows per sequence: q and rows double, partials double; flops
+    4 x D x Hq x (visible positions) with 9 + 10, 19 + 20, 39 + 40 visible."""
+    import numpy as np
+    cfg, lens = _cfg(), np.array([10, 20, 40])
+    assert bench.verify_kernel_bytes(cfg, lens, 16, 2) == 35840 + 3072 + 1024 + 10560 + 48
+    assert bench.verify_flops(cfg, lens, 2) == 4 * 64 * 4 * (19 + 39 + 79)
+    assert bench.verify_kernel_bytes(cfg, lens, 16, 1) == bench.decode_kernel_bytes(cfg, lens, 16)
