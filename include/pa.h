@@ -531,6 +531,13 @@ pa_status pa_bm_cache_stats(const pa_bm* bm, int* cached_blocks, int* evictable_
  * too small, which returns PA_ERR_INVALID_ARG). */
 pa_status pa_bm_evictable(const pa_bm* bm, int32_t* out, int cap, int* n);
 
+/* Drop the cache key of `block`, which must be cached with count zero (on the
+ * evictable list), and put it on the free list.  For K/V that must not be
+ * found again: the writes that filled the block were abandoned (a scheduler
+ * preempted their sequence within the same step).  PA_ERR_INVALID_ARG when the
+ * block is out of range, referenced or not cached; nothing changes then. */
+pa_status pa_bm_forget(pa_bm* bm, int32_t block);
+
 /* ------------------------------------------------------------------------ */
 /* Host scheduler: iteration-level (continuous) batching                     */
 /* ------------------------------------------------------------------------ */
@@ -592,6 +599,43 @@ pa_status pa_sched_swap_record(const pa_sched* s, int64_t* swapped_out, int64_t*
 pa_status pa_sched_record(const pa_sched* s, int64_t* finished, int64_t* admitted,
                           int64_t* preempted, int32_t* op_kind, int64_t* op_a, int64_t* op_b,
                           int64_t* op_c, int64_t* running, int32_t* context_lens);
+
+/* ---- admission through the prefix cache ([P3] "Prefix Caching前缀复用优化") ----
+ *
+ * Token id of position `position` of sequence `seq_id`, the token whose K/V a
+ * decode step writes there (in a server: the token sampled at the previous
+ * step).  Called from pa_sched_step on the calling thread; must be pure for a
+ * given (seq_id, position), since a retried reservation asks again. */
+typedef int32_t (*pa_token_fn)(void* ctx, int64_t seq_id, int64_t position);
+
+/* Switch the scheduler to admission through the prefix cache.  Needs
+ * pa_bm_enable_prefix_cache on its block manager, token_fn non-NULL, and no
+ * request queued yet; prefix_tokens[0..n) are the ids of the prefix holder's
+ * tokens (n = its length when the scheduler was made with prefix_seq >= 0,
+ * else 0; the holder should have been made by pa_bm_allocate_prefix so that
+ * its full blocks are cached).  Then:
+ *   - requests come in through pa_sched_add_request_tokens (pa_sched_add_request
+ *     returns PA_ERR_INVALID_ARG); a prefix-sharing request's token history is
+ *     prefix_tokens followed by its own;
+ *   - admission calls pa_bm_allocate_prefix with the whole history (prompt,
+ *     plus the tokens generated so far when a recomputed sequence comes back)
+ *     and lists cache writes only for positions past the cached blocks; the
+ *     budget charge is the same as without the cache;
+ *   - each decode reservation is pa_bm_append_token with token_fn's id;
+ *   - a recompute preemption first frees the victim, then forgets
+ *     (pa_bm_forget) every block that an op of this step targets and that is
+ *     left cached with count zero, in op order, then drops the dead ops: K/V
+ *     whose writes are dropped must not be found by a later lookup.  Cached
+ *     blocks written in earlier steps keep their keys.
+ * Default off: the scheduler behaves exactly as described above. */
+pa_status pa_sched_enable_prefix_cache(pa_sched* s, const int32_t* prefix_tokens, int n,
+                                       pa_token_fn token_fn, void* ctx);
+
+/* pa_sched_add_request with the request's own prompt token ids tokens[0..prompt_len)
+ * (copied); only with admission through the prefix cache. */
+pa_status pa_sched_add_request_tokens(pa_sched* s, int64_t seq_id, const int32_t* tokens, int prompt_len,
+                                      int output_len, int shares_prefix, int64_t fork_child,
+                                      int fork_output_len);
 
 #ifdef __cplusplus
 }

@@ -301,6 +301,15 @@ class PrefixCachingBlockManager(BlockManager):
         t = self.tokens[parent]
         self.tokens[child] = None if t is None else list(t)
 
+    def forget(self, b):
+        """Drop the name of an unreferenced cached block and free it (its K/V is
+        not to be trusted, e.g. writes into it were abandoned)."""
+        if self.ref[b] != 0 or b not in self.name:
+            raise InvalidArg(f"block {b} is not an unreferenced cached block")
+        self.evictable.remove(b)
+        del self.cache[self.name.pop(b)]
+        self.free_list.append(b)
+
     def _append(self, seq, token):
         if seq not in self.tables:
             raise InvalidArg(f"unknown sequence {seq}")

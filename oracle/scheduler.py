@@ -59,6 +59,28 @@ and back in later), readings adopted:
   in the step has been taken again: only the recomputed victim's own ops
   become dead.  Ops run in issue order; consecutive writes form one launch,
   and within one such run every slot is distinct.
+
+Admission through the prefix cache (``prefix_cache=True``, with a
+prefix-caching manager; [P3] "大模型推理显存优化实战：PagedAttention机制原理与vLLM连续批处理配置",
+section "Prefix Caching前缀复用优化": a request whose prompt begins with cached
+KV references those blocks and skips their prefill), readings adopted:
+
+* Requests carry their prompt token ids; a prefix-sharing request's tokens
+  are the system prefix's ids (given to the scheduler) followed by its own.
+  The token a sequence generates at position p comes from ``token_fn(seq,
+  p)``, an input (it stands in for the sampled token; the tests pass the
+  counter-based generator of the input module, which the C++ scheduler
+  implements from the same published definition).
+* Admission calls ``allocate_prefix`` with the sequence's whole token history
+  (prompt, and on re-admission the tokens generated so far) and records cache
+  writes only past the cached part.  The budget charge is unchanged (it does
+  not count on hits).  Decode appends go through ``append_token``.
+* A recompute preemption frees the victim as usual; then every block that an
+  op of this step targets and that is now unreferenced but still named is
+  forgotten (name dropped, back to the free list) before the dead ops are
+  dropped: a block whose writes are abandoned must not be found by a later
+  lookup.  A named block written in earlier steps keeps its name and waits
+  on the evictable list, so a re-admission finds it again.
 """
 
 from dataclasses import dataclass, field
@@ -74,6 +96,7 @@ class Request:
     shares_prefix: bool = False
     fork_child: int = -1       # id of a parallel-sampling child, -1 for none
     fork_output_len: int = 0
+    tokens: list = None        # own prompt token ids (prefix-cache admission)
 
 
 @dataclass
@@ -87,6 +110,7 @@ class _Seq:
     fork_output_len: int = 0
     forked: bool = False
     is_child: bool = False
+    tokens: list = None        # whole token history (prefix-cache admission)
 
 
 @dataclass
@@ -129,9 +153,15 @@ class StepRecord:
 
 
 class Scheduler:
-    def __init__(self, bm, max_running, prefix_seq=-1, preempt="recompute"):
+    def __init__(self, bm, max_running, prefix_seq=-1, preempt="recompute", prefix_cache=False,
+                 prefix_tokens=None, token_fn=None):
         if preempt not in ("recompute", "swap"):
             raise ValueError(preempt)
+        self.prefix_cache = bool(prefix_cache)
+        self.prefix_tokens = [int(t) for t in (prefix_tokens or [])]
+        self.token_fn = token_fn
+        if self.prefix_cache and token_fn is None:
+            raise ValueError("prefix-cache admission needs the generated tokens")
         self.bm = bm
         self.preempt = preempt
         self.swapped = []          # swapped-out sequences, FIFO
@@ -145,9 +175,14 @@ class Scheduler:
         if req.shares_prefix and self.prefix_seq < 0:
             raise ValueError("prefix-sharing request without a prefix holder")
         base = self.prefix_len if req.shares_prefix else 0
-        self.waiting.append(_Seq(req.seq_id, req.output_len, req.shares_prefix,
-                                 base + req.prompt_len, 0, req.fork_child,
-                                 req.fork_output_len))
+        s = _Seq(req.seq_id, req.output_len, req.shares_prefix, base + req.prompt_len, 0, req.fork_child,
+                 req.fork_output_len)
+        if self.prefix_cache:
+            own = [int(t) for t in req.tokens]
+            if len(own) != req.prompt_len:
+                raise ValueError("prompt tokens and prompt length disagree")
+            s.tokens = (list(self.prefix_tokens) if req.shares_prefix else []) + own
+        self.waiting.append(s)
 
     def _unshared(self, s):
         return s.history - (self.prefix_len if s.shares_prefix else 0)
@@ -160,7 +195,11 @@ class Scheduler:
 
     def _admit(self, s, rec):
         bm = self.bm
-        if s.shares_prefix:
+        if self.prefix_cache:
+            cached = bm.allocate_prefix(s.seq_id, s.tokens[:s.history])
+            for pos, slot in enumerate(bm.slots(s.seq_id, cached, s.history - cached), start=cached):
+                rec.write(s.seq_id, pos, slot)
+        elif s.shares_prefix:
             bm.fork(self.prefix_seq, s.seq_id)
             for pos in range(self.prefix_len, s.history):
                 slot, src, dst = bm.append_slot(s.seq_id)
@@ -178,6 +217,8 @@ class Scheduler:
             bm.fork(s.seq_id, s.fork_child)
             child = _Seq(s.fork_child, s.fork_output_len, s.shares_prefix,
                          s.history, 0, is_child=True)
+            if self.prefix_cache:
+                child.tokens = list(s.tokens[:s.history])
             self.running.append(child)
             rec.admitted.append(child.seq_id)
 
@@ -197,6 +238,20 @@ class Scheduler:
                 rec.preempted.append(victim.seq_id)
                 return victim
         bm.free(victim.seq_id)
+        if self.prefix_cache:
+            # blocks this step targets that are now unreferenced but still named:
+            # their writes are about to be dropped, so their names must go too
+            bs = bm.block_size
+            seen = set()
+            for op in rec.ops:
+                if op[0] == "so":
+                    continue
+                b = op[3] // bs if op[0] == "w" else op[2]
+                if b in seen:
+                    continue
+                seen.add(b)
+                if bm.ref[b] == 0 and b in bm.name:
+                    bm.forget(b)
         rec.drop_dead(bm)
         self.waiting.insert(0, victim)
         rec.preempted.append(victim.seq_id)
@@ -244,7 +299,11 @@ class Scheduler:
         while i < len(self.running):
             s = self.running[i]
             try:
-                slot, src, dst = bm.append_slot(s.seq_id)
+                if self.prefix_cache:
+                    tok = int(self.token_fn(s.seq_id, s.history))
+                    slot, src, dst = bm.append_token(s.seq_id, tok)
+                else:
+                    slot, src, dst = bm.append_slot(s.seq_id)
             except NoBlocks:
                 victim = self._preempt_last(rec)
                 if victim is s:
@@ -253,6 +312,9 @@ class Scheduler:
             if src >= 0:
                 rec.copy(src, dst)
             rec.write(s.seq_id, s.history, slot)
+            if self.prefix_cache:
+                del s.tokens[s.history:]
+                s.tokens.append(tok)
             s.history += 1
             s.generated += 1
             i += 1

@@ -531,6 +531,10 @@ class BlockManager:
                "pa_bm_cache_stats")
         return c.value, e.value, h.value, l.value
 
+    def forget(self, block):
+        """Drop the cache key of an unreferenced cached block and free it."""
+        _check(lib().pa_bm_forget(self._h, int(block)), "pa_bm_forget")
+
     def evictable(self):
         """Evictable cached blocks, next victim first."""
         out = np.zeros(self.num_blocks, dtype=np.int32)
@@ -542,13 +546,28 @@ class BlockManager:
 class Scheduler:
     """Iteration-level batching over a BlockManager (pa_sched_*)."""
 
-    def __init__(self, bm, max_running, prefix_seq=-1, preempt="recompute"):
+    def __init__(self, bm, max_running, prefix_seq=-1, preempt="recompute", prefix_cache=False,
+                 prefix_tokens=None, token_fn=None):
+        """``prefix_cache=True`` admits through the block manager's prefix cache
+        (pa_sched_enable_prefix_cache): ``prefix_tokens`` are the prefix
+        holder's token ids, ``token_fn(seq_id, position)`` gives the token id a
+        decode step writes at that position, and requests need their ``tokens``."""
         self.bm = bm           # keeps the block manager alive
         self._h = ctypes.c_void_p()
         self._destroy = lib().pa_sched_destroy
+        self._token_cb = None
         _check(lib().pa_sched_create(bm.handle, max_running, prefix_seq, ctypes.byref(self._h)), "pa_sched_create")
         _check(lib().pa_sched_set_preemption(self._h, {"recompute": 0, "swap": 1}[preempt]),
                "pa_sched_set_preemption")
+        if prefix_cache:
+            if token_fn is None:
+                raise ValueError("admission through the prefix cache needs token_fn")
+            fn = token_fn
+            # kept on self: the library calls it back from every step
+            self._token_cb = _native.TokenFn(lambda _ctx, seq, pos: int(fn(seq, pos)))
+            toks = np.ascontiguousarray(prefix_tokens if prefix_tokens is not None else [], dtype=np.int32)
+            _check(lib().pa_sched_enable_prefix_cache(self._h, _ptr(toks), toks.size, self._token_cb, None),
+                   "pa_sched_enable_prefix_cache")
 
     def __del__(self):
         # the destroy call was bound at construction: module globals may already be
@@ -559,9 +578,18 @@ class Scheduler:
             destroy(h)
             self._h = None
 
-    def add_request(self, seq_id, prompt_len, output_len, shares_prefix=False, fork_child=-1, fork_output_len=0):
-        _check(lib().pa_sched_add_request(self._h, seq_id, prompt_len, output_len, int(bool(shares_prefix)),
-                                          fork_child, fork_output_len), "pa_sched_add_request")
+    def add_request(self, seq_id, prompt_len, output_len, shares_prefix=False, fork_child=-1, fork_output_len=0,
+                    tokens=None):
+        if tokens is None:
+            _check(lib().pa_sched_add_request(self._h, seq_id, prompt_len, output_len, int(bool(shares_prefix)),
+                                              fork_child, fork_output_len), "pa_sched_add_request")
+            return
+        toks = np.ascontiguousarray(tokens, dtype=np.int32)
+        if toks.size != prompt_len:
+            raise ValueError("prompt tokens and prompt length disagree")
+        _check(lib().pa_sched_add_request_tokens(self._h, seq_id, _ptr(toks), prompt_len, output_len,
+                                                 int(bool(shares_prefix)), fork_child, fork_output_len),
+               "pa_sched_add_request_tokens")
 
     def step(self):
         """Run one iteration; returns the step record as a dict of lists."""

@@ -11,6 +11,9 @@ c_int, c_int32, c_int64, c_size_t, c_float, c_double, c_void_p, c_uint32 = (
     ctypes.c_double, ctypes.c_void_p, ctypes.c_uint32)
 P = ctypes.POINTER
 
+# pa_token_fn: token id of (seq_id, position), called back from pa_sched_step
+TokenFn = ctypes.CFUNCTYPE(c_int32, c_void_p, c_int64, c_int64)
+
 
 class CacheDesc(ctypes.Structure):
     _fields_ = [("num_blocks", c_int), ("block_size", c_int), ("num_kv_heads", c_int),
@@ -109,6 +112,9 @@ SIGNATURES = {
     "pa_sched_counts_get": (c_int, [c_void_p, P(SchedCounts)]),
     "pa_sched_record": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_void_p, c_void_p, c_void_p]),
+    "pa_bm_forget": (c_int, [c_void_p, c_int32]),
+    "pa_sched_enable_prefix_cache": (c_int, [c_void_p, c_void_p, c_int, TokenFn, c_void_p]),
+    "pa_sched_add_request_tokens": (c_int, [c_void_p, c_int64, c_void_p, c_int, c_int, c_int, c_int64, c_int]),
 }
 
 _lib = None

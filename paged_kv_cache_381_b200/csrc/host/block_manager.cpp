@@ -102,6 +102,19 @@ void BlockManager::unlink_lru(int32_t b) {
     }
 }
 
+// A cached block with count zero whose K/V is not to be trusted (the writes
+// that filled it were abandoned): its key goes, and the block returns to the
+// free list instead of waiting on the LRU list.
+pa_status BlockManager::forget(int32_t b) {
+    if (b < 0 || b >= num_blocks_ || ref_[b] != 0 || !key_of_.count(b)) return PA_ERR_INVALID_ARG;
+    unlink_lru(b);
+    auto it = key_of_.find(b);
+    block_of_.erase(it->second);
+    key_of_.erase(it);
+    free_.push_back(b);
+    return PA_OK;
+}
+
 std::string BlockManager::make_key(int32_t parent, const int32_t* tokens) const {
     std::string k(sizeof(int32_t) * (1 + block_size_), '\0');
     std::memcpy(&k[0], &parent, sizeof(int32_t));
@@ -591,6 +604,10 @@ pa_status pa_bm_cpu_free_list(const pa_bm* bm, int32_t* out, int cap, int* n) {
     if (len > cap || (len > 0 && !out)) return PA_ERR_INVALID_ARG;
     for (int i = 0; i < len; ++i) out[i] = fl[i];
     return PA_OK;
+}
+
+pa_status pa_bm_forget(pa_bm* bm, int32_t block) {
+    return bm ? bm->impl.forget(block) : PA_ERR_INVALID_ARG;
 }
 
 pa_status pa_bm_evictable(const pa_bm* bm, int32_t* out, int cap, int* n) {

@@ -47,6 +47,8 @@ class BlockManager {
     int64_t hits() const { return hits_; }
     int64_t lookups() const { return lookups_; }
     const std::list<int32_t>& evictable() const { return lru_; }
+    bool named(int32_t b) const { return key_of_.count(b) != 0; }
+    pa_status forget(int32_t b);      // drop an unreferenced cached block's name, free it
 
     // host swap pool
     pa_status set_cpu_blocks(int n);

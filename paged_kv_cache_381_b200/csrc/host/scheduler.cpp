@@ -33,6 +33,17 @@
 // blocks a swap-out freed earlier in the step are all taken again by then and
 // only the recomputed victim's own ops die.  Ops run in issue order;
 // consecutive writes form one launch with distinct slots.
+//
+// Admission through the prefix cache ("大模型推理显存优化实战：PagedAttention机制原理与
+// vLLM连续批处理配置", section "Prefix Caching前缀复用优化": a request whose prompt
+// starts with cached KV references those blocks and skips their prefill), when
+// enabled: each sequence carries its token history; admission allocates through
+// the cache with the whole history and lists writes only past the cached
+// blocks; decode reservations record their token ids (from a caller-given
+// function) so that filled blocks get cached.  A recompute preemption forgets
+// every block that this step's ops target and that the preemption left cached
+// with no holder, before dropping the dead ops, so no later lookup finds K/V
+// whose writes were abandoned.
 
 #include <deque>
 #include <new>
@@ -51,6 +62,7 @@ struct SeqState {
     int64_t fork_child = -1;
     int64_t fork_output_len = 0;
     bool forked = false;
+    std::vector<int32_t> tokens;   // token history (admission through the prefix cache)
 };
 
 }  // namespace
@@ -71,6 +83,11 @@ struct pa_sched {
     std::vector<int64_t> op_a, op_b, op_c;
     std::vector<int64_t> run_ids;
     std::vector<int32_t> run_ctx;
+    // admission through the prefix cache
+    bool prefix_cache = false;
+    std::vector<int32_t> prefix_tokens;
+    pa_token_fn token_fn = nullptr;
+    void* token_ctx = nullptr;
 
     void rec_write(int64_t seq, int64_t pos, int64_t slot) {
         op_kind.push_back(0); op_a.push_back(seq); op_b.push_back(pos); op_c.push_back(slot);
@@ -96,6 +113,21 @@ struct pa_sched {
         }
         op_kind.resize(w); op_a.resize(w); op_b.resize(w); op_c.resize(w);
     }
+    // Recompute preemption with the prefix cache: blocks targeted by this step's
+    // ops, left cached with count zero by the victim's release, lose their keys.
+    pa_status forget_abandoned() {
+        const int bs = bm->block_size();
+        std::vector<char> seen(bm->num_blocks(), 0);
+        pa_status st;
+        for (size_t i = 0; i < op_kind.size(); ++i) {
+            if (op_kind[i] == 2) continue;
+            const int32_t b = (int32_t)(op_kind[i] == 0 ? op_c[i] / bs : op_b[i]);
+            if (seen[b]) continue;
+            seen[b] = 1;
+            if (bm->ref(b) == 0 && bm->named(b) && (st = bm->forget(b)) != PA_OK) return st;
+        }
+        return PA_OK;
+    }
     int64_t own_tokens(const SeqState& s) const { return s.history - (s.shares_prefix ? prefix_len : 0); }
     int64_t required(const SeqState& s) const {
         int64_t need = pa_host::ceil_div(own_tokens(s), bm->block_size()) + 1;
@@ -108,7 +140,14 @@ struct pa_sched {
 
 pa_status pa_sched::admit(SeqState s) {
     pa_status st;
-    if (s.shares_prefix) {
+    if (prefix_cache) {
+        int cached = 0;
+        if ((st = bm->allocate_prefix(s.id, s.tokens.data(), (int)s.history, &cached)) != PA_OK) return st;
+        const int64_t count = s.history - cached;
+        std::vector<int64_t> slots(count);
+        if (count > 0 && (st = bm->slots(s.id, cached, count, slots.data())) != PA_OK) return st;
+        for (int64_t k = 0; k < count; ++k) rec_write(s.id, cached + k, slots[k]);
+    } else if (s.shares_prefix) {
         if ((st = bm->fork(prefix_seq, s.id)) != PA_OK) return st;
         for (int64_t pos = prefix_len; pos < s.history; ++pos) {
             int64_t slot; int32_t src, dst;
@@ -133,6 +172,7 @@ pa_status pa_sched::admit(SeqState s) {
         c.output_len = s.fork_output_len;
         c.shares_prefix = s.shares_prefix;
         c.history = s.history;
+        if (prefix_cache) c.tokens.assign(s.tokens.begin(), s.tokens.begin() + s.history);
         running.push_back(c);
         admitted.push_back(c.id);
     }
@@ -188,7 +228,13 @@ pa_status pa_sched::step() {
     while (i < running.size()) {
         SeqState& s = running[i];
         int64_t slot; int32_t src, dst;
-        st = bm->append_slot(s.id, &slot, &src, &dst);
+        int32_t tok = 0;
+        if (prefix_cache) {
+            tok = token_fn(token_ctx, s.id, s.history);
+            st = bm->append_token(s.id, tok, &slot, &src, &dst);
+        } else {
+            st = bm->append_slot(s.id, &slot, &src, &dst);
+        }
         if (st == PA_ERR_NO_BLOCKS) {
             SeqState victim = running.back();
             running.pop_back();
@@ -204,6 +250,7 @@ pa_status pa_sched::step() {
                 }
             }
             if ((st = bm->free_seq(victim.id)) != PA_OK) return st;
+            if (prefix_cache && (st = forget_abandoned()) != PA_OK) return st;
             drop_dead_ops();
             preempted.push_back(victim.id);
             waiting.push_front(victim);
@@ -212,6 +259,10 @@ pa_status pa_sched::step() {
         if (st != PA_OK) return st;
         if (src >= 0) rec_copy(src, dst);
         rec_write(s.id, s.history, slot);
+        if (prefix_cache) {
+            s.tokens.resize(s.history);
+            s.tokens.push_back(tok);
+        }
         s.history += 1;
         s.generated += 1;
         ++i;
@@ -268,8 +319,8 @@ pa_status pa_sched_swap_record(const pa_sched* s, int64_t* swapped_out, int64_t*
     return PA_OK;
 }
 
-pa_status pa_sched_add_request(pa_sched* s, int64_t seq_id, int prompt_len, int output_len,
-                               int shares_prefix, int64_t fork_child, int fork_output_len) {
+static pa_status queue_request(pa_sched* s, int64_t seq_id, const int32_t* tokens, int prompt_len,
+                               int output_len, int shares_prefix, int64_t fork_child, int fork_output_len) {
     if (!s || prompt_len < 0 || output_len < 0 || fork_output_len < 0) return PA_ERR_INVALID_ARG;
     if (shares_prefix && s->prefix_seq < 0) return PA_ERR_INVALID_ARG;
     SeqState q;
@@ -279,7 +330,36 @@ pa_status pa_sched_add_request(pa_sched* s, int64_t seq_id, int prompt_len, int 
     q.history = (q.shares_prefix ? s->prefix_len : 0) + prompt_len;
     q.fork_child = fork_child;
     q.fork_output_len = fork_output_len;
-    s->waiting.push_back(q);
+    if (s->prefix_cache) {
+        if (q.shares_prefix) q.tokens = s->prefix_tokens;
+        if (prompt_len > 0) q.tokens.insert(q.tokens.end(), tokens, tokens + prompt_len);
+    }
+    s->waiting.push_back(std::move(q));
+    return PA_OK;
+}
+
+pa_status pa_sched_add_request(pa_sched* s, int64_t seq_id, int prompt_len, int output_len,
+                               int shares_prefix, int64_t fork_child, int fork_output_len) {
+    if (s && s->prefix_cache) return PA_ERR_INVALID_ARG;     // needs the prompt's token ids
+    return queue_request(s, seq_id, nullptr, prompt_len, output_len, shares_prefix, fork_child, fork_output_len);
+}
+
+pa_status pa_sched_add_request_tokens(pa_sched* s, int64_t seq_id, const int32_t* tokens, int prompt_len,
+                                      int output_len, int shares_prefix, int64_t fork_child,
+                                      int fork_output_len) {
+    if (!s || !s->prefix_cache || (prompt_len > 0 && !tokens)) return PA_ERR_INVALID_ARG;
+    return queue_request(s, seq_id, tokens, prompt_len, output_len, shares_prefix, fork_child, fork_output_len);
+}
+
+pa_status pa_sched_enable_prefix_cache(pa_sched* s, const int32_t* prefix_tokens, int n, pa_token_fn token_fn,
+                                       void* ctx) {
+    if (!s || !token_fn || !s->bm->prefix_cache() || n < 0 || (n > 0 && !prefix_tokens)) return PA_ERR_INVALID_ARG;
+    if (n != (s->prefix_seq >= 0 ? s->prefix_len : 0)) return PA_ERR_INVALID_ARG;
+    if (!s->waiting.empty() || !s->running.empty() || !s->swapped.empty()) return PA_ERR_INVALID_ARG;
+    s->prefix_cache = true;
+    s->prefix_tokens.assign(prefix_tokens, prefix_tokens + n);
+    s->token_fn = token_fn;
+    s->token_ctx = ctx;
     return PA_OK;
 }
 

@@ -318,6 +318,18 @@ def _splitmix64(x):
     return z ^ (z >> np.uint64(31))
 
 
+def generated_token(seq, pos, vocab):
+    """Token id a synthetic decode produced for position ``pos`` of sequence
+    ``seq``: SplitMix64 of (seq x 0x100000001B3 + pos) mod 2^64, modulo vocab.
+    Stands in for the sampled token when a scheduler names blocks by their
+    token ids."""
+    m = 0xFFFFFFFFFFFFFFFF
+    z = ((int(seq) * 0x100000001B3 + int(pos)) + 0x9E3779B97F4A7C15) & m
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & m
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & m
+    return (z ^ (z >> 31)) % int(vocab)
+
+
 _ROW_TABLES = {}
 
 
