@@ -322,3 +322,37 @@ def test_prefix_mode_argument_rules(pa):
     plain_s = pa.Scheduler(plain, 4)
     with pytest.raises(pa.PagedAttentionError):        # tokens without the prefix-cache mode
         plain_s.add_request(1, 2, 2, tokens=[1, 2])
+
+
+def test_no_holder_replayed_prompts(pa):
+    """Admission through the cache with no prefix holder: repeated prompts alone
+    make the hits; C++ and model agree and the content check holds."""
+    bs, nb = 2, 40
+    r = np.random.default_rng(11)
+    base = [int(x) for x in r.integers(0, VOCAB, 12)]
+    order = r.permutation(nb).tolist()
+    mbm = obm.PrefixCachingBlockManager(nb, bs, order)
+    nbm = pa.BlockManager(nb, bs, order)
+    nbm.enable_prefix_cache()
+    ms = osch.Scheduler(mbm, 6, prefix_cache=True, token_fn=token_fn)
+    ns = pa.Scheduler(nbm, 6, prefix_cache=True, prefix_tokens=[], token_fn=token_fn)
+    reqs, prompts = [], []
+    for i in range(24):
+        n = int(r.integers(3, 16))
+        p = (base + [int(x) for x in r.integers(0, VOCAB, n)])[:n] if i % 2 else \
+            [int(x) for x in r.integers(0, VOCAB, n)]
+        q = wl.TraceRequest(seq_id=i, prompt_len=n, output_len=int(r.integers(1, 9)), shares_prefix=False,
+                            fork_child=-1, fork_output_len=0)
+        reqs.append(q)
+        prompts.append(p)
+        ms.add_request(osch.Request(i, n, q.output_len, tokens=p))
+        ns.add_request(i, n, q.output_len, tokens=p)
+    content = _Content(bs, [], reqs, prompts)
+    for step in range(60):
+        a, b = ms.step(), ns.step()
+        assert [tuple(o) for o in a.ops] == b["ops"], step
+        assert a.running == b["running"] and a.context_lens == b["context_lens"], step
+        assert mbm.free_list == nbm.free_list() and mbm.evictable == nbm.evictable(), step
+        content.apply(b["ops"])
+        content.check(lambda s: nbm.block_table(s), b["running"], b["context_lens"])
+    assert mbm.hits > 0 and not ms.running and not ms.waiting
