@@ -559,7 +559,12 @@ pa_status pa_sched_add_request(pa_sched* s, int64_t seq_id, int prompt_len, int 
 /* Run one iteration ([P1] 2.2): finish, admit (FCFS, stop at the first request
  * that does not fit the free-block budget), then reserve every running
  * sequence's next slot, preempting the most recently admitted sequence when
- * the pool is exhausted.  The step's record is kept until the next call. */
+ * the pool is exhausted.  The step's record is kept until the next call.
+ * The budget charge covers every block an admission takes, so the block
+ * manager's own calls do not fail inside a step; if one does (the block
+ * manager was changed behind the scheduler's back), its status is returned and
+ * the scheduler and block manager are left part-way through the step: destroy
+ * both. */
 pa_status pa_sched_step(pa_sched* s);
 
 /* Sizes of the last step's record. */
