@@ -617,8 +617,10 @@ typedef int32_t (*pa_token_fn)(void* ctx, int64_t seq_id, int64_t position);
  * pa_bm_enable_prefix_cache on its block manager, token_fn non-NULL, and no
  * request queued yet; prefix_tokens[0..n) are the ids of the prefix holder's
  * tokens (n = its length when the scheduler was made with prefix_seq >= 0,
- * else 0; the holder should have been made by pa_bm_allocate_prefix so that
- * its full blocks are cached).  Then:
+ * else 0).  Each full block of the holder must be the block the cache names
+ * for these ids (make the holder with pa_bm_allocate_prefix): then every
+ * admission takes at most the blocks the budget charges it.  Otherwise, or
+ * when the holder is swapped out, PA_ERR_INVALID_ARG.  Then:
  *   - requests come in through pa_sched_add_request_tokens (pa_sched_add_request
  *     returns PA_ERR_INVALID_ARG); a prefix-sharing request's token history is
  *     prefix_tokens followed by its own;

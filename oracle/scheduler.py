@@ -71,6 +71,9 @@ KV references those blocks and skips their prefill), readings adopted:
   p)``, an input (it stands in for the sampled token; the tests pass the
   counter-based generator of the input module, which the C++ scheduler
   implements from the same published definition).
+* The prefix holder's full blocks must be the cached blocks of the prefix
+  ids (checked at construction).  Then a prefix-sharing admission finds all
+  of them, and no admission takes more blocks than the budget charges it.
 * Admission calls ``allocate_prefix`` with the sequence's whole token history
   (prompt, and on re-admission the tokens generated so far) and records cache
   writes only past the cached part.  The budget charge is unchanged (it does
@@ -162,6 +165,16 @@ class Scheduler:
         self.token_fn = token_fn
         if self.prefix_cache and token_fn is None:
             raise ValueError("prefix-cache admission needs the generated tokens")
+        if self.prefix_cache and prefix_seq >= 0:
+            # every full block of the holder must be the cached block of these
+            # ids, so a sharer finds them all and stays within its charge
+            bs, table = bm.block_size, bm.tables.get(prefix_seq)
+            ok = table is not None and bm.ctx[prefix_seq] == len(self.prefix_tokens)
+            ok = ok and not (hasattr(bm, "swapped") and bm.swapped(prefix_seq))
+            for j in range(len(self.prefix_tokens) // bs if ok else 0):
+                ok = ok and bm.cache.get(tuple(self.prefix_tokens[:(j + 1) * bs])) == table[j]
+            if not ok:
+                raise ValueError("the prefix holder's blocks are not cached under these token ids")
         self.bm = bm
         self.preempt = preempt
         self.swapped = []          # swapped-out sequences, FIFO

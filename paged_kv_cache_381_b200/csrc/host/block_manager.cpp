@@ -115,6 +115,19 @@ pa_status BlockManager::forget(int32_t b) {
     return PA_OK;
 }
 
+bool BlockManager::cached_as(int64_t seq, const int32_t* tokens, int n) const {
+    auto it = seqs_.find(seq);
+    if (it == seqs_.end() || it->second.swapped || it->second.ctx != n || (n > 0 && !tokens)) return false;
+    const std::vector<int32_t>& t = it->second.table;
+    int32_t parent = -1;
+    for (int j = 0; j < n / block_size_; ++j) {
+        auto b = block_of_.find(make_key(parent, tokens + (int64_t)j * block_size_));
+        if (b == block_of_.end() || b->second != t[j]) return false;
+        parent = t[j];
+    }
+    return true;
+}
+
 std::string BlockManager::make_key(int32_t parent, const int32_t* tokens) const {
     std::string k(sizeof(int32_t) * (1 + block_size_), '\0');
     std::memcpy(&k[0], &parent, sizeof(int32_t));

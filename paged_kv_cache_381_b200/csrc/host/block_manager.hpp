@@ -49,6 +49,9 @@ class BlockManager {
     const std::list<int32_t>& evictable() const { return lru_; }
     bool named(int32_t b) const { return key_of_.count(b) != 0; }
     pa_status forget(int32_t b);      // drop an unreferenced cached block's name, free it
+    // true when seq holds exactly n tokens and each of its full blocks is the
+    // block the cache names for those token ids
+    bool cached_as(int64_t seq, const int32_t* tokens, int n) const;
 
     // host swap pool
     pa_status set_cpu_blocks(int n);

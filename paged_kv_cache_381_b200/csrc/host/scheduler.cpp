@@ -355,6 +355,10 @@ pa_status pa_sched_enable_prefix_cache(pa_sched* s, const int32_t* prefix_tokens
                                        void* ctx) {
     if (!s || !token_fn || !s->bm->prefix_cache() || n < 0 || (n > 0 && !prefix_tokens)) return PA_ERR_INVALID_ARG;
     if (n != (s->prefix_seq >= 0 ? s->prefix_len : 0)) return PA_ERR_INVALID_ARG;
+    // the holder's full blocks must be the cached blocks of these ids: then a
+    // prefix-sharing admission finds them all and never takes more blocks than
+    // the budget charges it
+    if (s->prefix_seq >= 0 && !s->bm->cached_as(s->prefix_seq, prefix_tokens, n)) return PA_ERR_INVALID_ARG;
     if (!s->waiting.empty() || !s->running.empty() || !s->swapped.empty()) return PA_ERR_INVALID_ARG;
     s->prefix_cache = true;
     s->prefix_tokens.assign(prefix_tokens, prefix_tokens + n);

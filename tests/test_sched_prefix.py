@@ -356,3 +356,36 @@ def test_no_holder_replayed_prompts(pa):
         content.apply(b["ops"])
         content.check(lambda s: nbm.block_table(s), b["running"], b["context_lens"])
     assert mbm.hits > 0 and not ms.running and not ms.waiting
+
+
+def test_holder_must_be_cached_under_the_prefix_ids(pa):
+    """A holder made without the cache, or prefix ids other than the holder's,
+    are refused by both schedulers: a sharer would then take more blocks than
+    its budget charge."""
+    bs, nb = 4, 32
+    ids = [0, 1, 2, 3, 1, 1, 2, 0, 3, 3]
+    wrong = ids[:5] + [2] + ids[6:]                 # differs in the second block
+    for make_model in (True, False):
+        def manager(cached):
+            if make_model:
+                m = obm.PrefixCachingBlockManager(nb, bs)
+            else:
+                m = pa.BlockManager(nb, bs)
+                m.enable_prefix_cache()
+            if cached:
+                m.allocate_prefix(wl.PREFIX_SEQ, ids)
+            else:
+                m.allocate(wl.PREFIX_SEQ, len(ids))
+            return m
+
+        def sched(m, toks):
+            if make_model:
+                return osch.Scheduler(m, 4, wl.PREFIX_SEQ, prefix_cache=True, prefix_tokens=toks, token_fn=token_fn)
+            return pa.Scheduler(m, 4, wl.PREFIX_SEQ, prefix_cache=True, prefix_tokens=toks, token_fn=token_fn)
+
+        err = ValueError if make_model else pa.PagedAttentionError
+        with pytest.raises(err):
+            sched(manager(False), ids)
+        with pytest.raises(err):
+            sched(manager(True), wrong)
+        sched(manager(True), ids)
