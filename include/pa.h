@@ -361,6 +361,12 @@ int pa_get_split_merge(void);
  * PA_ERR_DEVICE when any bit was set, PA_OK otherwise. */
 pa_status pa_get_device_error(uint32_t* flags, void* stream);
 
+/* Diagnostic of the kernels' bounded waits: launches one CTA on `stream` that
+ * waits on a shared-memory barrier nothing arrives at.  The wait gives up after
+ * its limit (2 s of %globaltimer), the CTA sets PA_DEVERR_TIMEOUT and exits;
+ * read it with pa_get_device_error.  Returns PA_ERR_CUDA if the launch fails. */
+pa_status pa_check_wait_expiry(void* stream);
+
 const char* pa_status_string(pa_status status);
 
 /* ------------------------------------------------------------------------ */

@@ -309,6 +309,14 @@ def pa_get_device_error(stream=None):
 MATH_AUTO, MATH_SIMT, MATH_TENSOR = 0, 1, 2
 
 
+def pa_check_wait_expiry(stream=None):
+    """Launch the bounded-wait diagnostic (one CTA whose wait must expire after
+    about 2 s and set DEVERR_TIMEOUT); read the flag with pa_get_device_error."""
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    _check(lib().pa_check_wait_expiry(ctypes.c_void_p(s.cuda_stream)), "pa_check_wait_expiry")
+
+
 def set_decode_math(mode):
     """Choose tensor-core (default for fp16/bf16) or CUDA-core decode arithmetic."""
     _check(lib().pa_set_decode_math(int(mode)), "pa_set_decode_math")

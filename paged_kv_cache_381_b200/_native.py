@@ -66,6 +66,7 @@ SIGNATURES = {
                                  c_void_p]),
     "pa_pipeline_end": (c_int, [c_void_p, c_void_p]),
     "pa_get_device_error": (c_int, [P(c_uint32), c_void_p]),
+    "pa_check_wait_expiry": (c_int, [c_void_p]),
     "pa_status_string": (ctypes.c_char_p, [c_int]),
     "pa_launch_count": (c_int64, []),
     "pa_set_decode_math": (c_int, [c_int]),

@@ -18,6 +18,25 @@
 #include "device/verify_tc.cuh"
 #include "pa.h"
 
+namespace pa_dev {
+
+// The bounded wait's expiry path on its own: one thread waits on a barrier
+// that nothing arrives at.  The wait must give up after kWaitLimitNs and the
+// CTA must flag PA_DEVERR_TIMEOUT and exit, leaving the context usable.
+__global__ void wait_expiry_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag)) flag_error(PA_DEVERR_TIMEOUT);
+}
+
+}  // namespace pa_dev
+
 namespace {
 
 constexpr int kDefaultPartition = 512;
@@ -848,6 +867,12 @@ pa_status pa_pipeline_end(pa_pipeline* p, void* stream) {
         cudaEventRecord(p->mark, p->d2h) != cudaSuccess || cudaStreamWaitEvent(s, p->mark, 0) != cudaSuccess)
         return PA_ERR_CUDA;
     return PA_OK;
+}
+
+pa_status pa_check_wait_expiry(void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    pa_dev::wait_expiry_kernel<<<1, 32, 0, s>>>();
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_get_device_error(uint32_t* flags, void* stream) {
