@@ -47,6 +47,7 @@
 
 #include <deque>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "block_manager.hpp"
@@ -164,17 +165,19 @@ pa_status pa_sched::admit(SeqState s) {
     admitted.push_back(s.id);
     const bool spawn = s.fork_child >= 0 && !s.forked;
     if (spawn) s.forked = true;
-    running.push_back(s);
+    SeqState c;
     if (spawn) {
         if ((st = bm->fork(s.id, s.fork_child)) != PA_OK) return st;
-        SeqState c;
         c.id = s.fork_child;
         c.output_len = s.fork_output_len;
         c.shares_prefix = s.shares_prefix;
         c.history = s.history;
         if (prefix_cache) c.tokens.assign(s.tokens.begin(), s.tokens.begin() + s.history);
-        running.push_back(c);
+    }
+    running.push_back(std::move(s));
+    if (spawn) {
         admitted.push_back(c.id);
+        running.push_back(std::move(c));
     }
     return PA_OK;
 }
@@ -188,12 +191,12 @@ pa_status pa_sched::step() {
     // 1. finish
     std::vector<SeqState> keep;
     keep.reserve(running.size());
-    for (const SeqState& s : running) {
+    for (SeqState& s : running) {
         if (s.generated >= s.output_len) {
             if ((st = bm->free_seq(s.id)) != PA_OK) return st;
             finished.push_back(s.id);
         } else {
-            keep.push_back(s);
+            keep.push_back(std::move(s));
         }
     }
     running.swap(keep);
@@ -209,7 +212,7 @@ pa_status pa_sched::step() {
         for (size_t k = 0; k < pairs.size(); k += 2) rec_swap(3, pairs[k], pairs[k + 1]);
         budget -= need;
         swapped_in.push_back(head.id);
-        running.push_back(head);
+        running.push_back(std::move(swapped.front()));
         swapped.pop_front();
     }
     while (swapped.empty() && !waiting.empty() && budget > 0 && (int)running.size() < max_running) {
@@ -218,10 +221,10 @@ pa_status pa_sched::step() {
         if (need > budget) break;
         int extra = (head.fork_child >= 0 && !head.forked) ? 1 : 0;
         if ((int)running.size() + 1 + extra > max_running) break;
-        SeqState s = head;
+        SeqState s = std::move(waiting.front());
         waiting.pop_front();
         budget -= need;
-        if ((st = admit(s)) != PA_OK) return st;
+        if ((st = admit(std::move(s))) != PA_OK) return st;
     }
     // 3. reserve every running sequence's next slot, preempting when exhausted
     size_t i = 0;
@@ -236,7 +239,7 @@ pa_status pa_sched::step() {
             st = bm->append_slot(s.id, &slot, &src, &dst);
         }
         if (st == PA_ERR_NO_BLOCKS) {
-            SeqState victim = running.back();
+            SeqState victim = std::move(running.back());
             running.pop_back();
             if (preempt_mode == PA_PREEMPT_SWAP) {
                 const int need = bm->swap_out_need(victim.id);
@@ -245,7 +248,7 @@ pa_status pa_sched::step() {
                     for (size_t k = 0; k < pairs.size(); k += 2) rec_swap(2, pairs[k], pairs[k + 1]);
                     swapped_out.push_back(victim.id);
                     preempted.push_back(victim.id);
-                    swapped.push_back(victim);
+                    swapped.push_back(std::move(victim));
                     continue;
                 }
             }
@@ -253,7 +256,7 @@ pa_status pa_sched::step() {
             if (prefix_cache && (st = forget_abandoned()) != PA_OK) return st;
             drop_dead_ops();
             preempted.push_back(victim.id);
-            waiting.push_front(victim);
+            waiting.push_front(std::move(victim));
             continue;   // retry the same index (or stop if the victim was this one)
         }
         if (st != PA_OK) return st;
