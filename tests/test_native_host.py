@@ -340,3 +340,34 @@ def test_scheduler_swap_matches_model(pa, ncpu, nb):
         assert mb.free_list == nbm.free_list() and mb.cpu_free == nbm.cpu_free_list(), step
         n_so += len(a.swapped_out)
     assert n_so > 0
+
+
+def test_decode_and_cache_write_argument_rules(pa):
+    """pa_decode and pa_cache_write return their argument errors synchronously,
+    before any device work, so these run without a GPU (status codes: 0 ok,
+    1 invalid argument, 2 unsupported)."""
+    lib = pa.lib()
+    nul = ctypes.c_void_p(0)
+
+    def dec(S=4, Hq=64, Hkv=8, D=128, bs=16, dt=2, P=0, scale=0.1):
+        return lib.pa_decode(nul, nul, nul, nul, nul, nul, scale, bs, Hkv, S, Hq, D, 8, 128, 64, dt, P, nul, 0, nul)
+
+    assert dec(S=0) == 0                               # nothing to do
+    assert dec() == 1                                  # null pointers
+    assert dec(Hq=60) == 1                             # heads not a multiple of kv heads
+    assert dec(D=96) == 2                              # head_dim outside {64, 128}
+    assert dec(bs=12) == 2                             # block size outside {8, 16, 32}
+    assert dec(P=100) == 1                             # partition not a multiple of 32
+    assert dec(dt=7) == 1                              # unknown dtype
+    assert dec(scale=float("nan")) == 1
+
+    def cw(T=4, nb=64, bs=16, Hkv=8, D=128, dt=2):
+        desc = pa._native.CacheDesc(nb, bs, Hkv, D, dt)
+        return lib.pa_cache_write(nul, nul, nul, nul, nul, T, ctypes.byref(desc), nul)
+
+    assert cw(T=0) == 0
+    assert cw() == 1                                   # null pointers
+    assert cw(T=-1) == 1
+    assert cw(bs=12) == 2 and cw(D=96) == 2
+    assert cw(nb=0) == 1 and cw(dt=9) == 1
+    assert lib.pa_cache_write(nul, nul, nul, nul, nul, 4, None, nul) == 1
