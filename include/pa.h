@@ -270,7 +270,12 @@ pa_status pa_swap_blocks(void* dst_k, void* dst_v, int dst_blocks, const void* s
  * num_cow > 0), pa_cache_write and pa_decode, and copies `out` back
  * device->host.  The caller provides the device staging buffers (no
  * allocation here).  Returns once the work is enqueued; the host output is
- * valid after the stream synchronizes.
+ * valid after the stream synchronizes.  NULL structs or pools, negative
+ * counts and an unknown dtype return PA_ERR_INVALID_ARG before any copy; the
+ * remaining checks of pa_copy_blocks / pa_cache_write / pa_decode run after
+ * the input copies are enqueued and return their status before their own
+ * launch; a failed copy returns PA_ERR_CUDA.  Host buffers should be pinned
+ * for the copies to be asynchronous.
  */
 typedef struct {
     /* host inputs */
@@ -367,6 +372,8 @@ pa_status pa_get_device_error(uint32_t* flags, void* stream);
  * read it with pa_get_device_error.  Returns PA_ERR_CUDA if the launch fails. */
 pa_status pa_check_wait_expiry(void* stream);
 
+/* A static English description of a status code (never NULL; "unknown status"
+ * for values outside the enum). */
 const char* pa_status_string(pa_status status);
 
 /* ------------------------------------------------------------------------ */
