@@ -599,8 +599,13 @@ class Scheduler:
                                                  int(bool(shares_prefix)), fork_child, fork_output_len),
                "pa_sched_add_request_tokens")
 
-    def step(self):
-        """Run one iteration; returns the step record as a dict of lists."""
+    def step(self, raw=False):
+        """Run one iteration; returns the step record as a dict of lists.
+
+        ``raw=True`` leaves the ops as four numpy arrays (``op_kind``: 0 write,
+        1 copy-on-write, 2 swap-out, 3 swap-in; ``op_a``, ``op_b``, ``op_c`` as in
+        pa_sched_record) instead of a list of tuples, for callers that hand them
+        to the device without looking at each one."""
         _check(lib().pa_sched_step(self._h), "pa_sched_step")
         c = _native.SchedCounts()
         _check(lib().pa_sched_counts_get(self._h, ctypes.byref(c)), "pa_sched_counts_get")
@@ -613,14 +618,20 @@ class Scheduler:
         ctx = np.zeros(c.num_running, np.int32)
         _check(lib().pa_sched_record(self._h, _ptr(fin), _ptr(adm), _ptr(pre), _ptr(kind), _ptr(oa), _ptr(ob),
                                      _ptr(oc), _ptr(run), _ptr(ctx)), "pa_sched_record")
-        names = {1: "c", 2: "so", 3: "si"}
-        ops = [("w", int(a), int(b), int(cc)) if k == 0 else (names[k], int(a), int(b))
-               for k, a, b, cc in zip(kind.tolist(), oa.tolist(), ob.tolist(), oc.tolist())]
+        if raw:
+            ops = None
+        else:
+            names = {1: "c", 2: "so", 3: "si"}
+            ops = [("w", a, b, cc) if k == 0 else (names[k], a, b)
+                   for k, a, b, cc in zip(kind.tolist(), oa.tolist(), ob.tolist(), oc.tolist())]
         n_out, n_in, n_q = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
         _check(lib().pa_sched_swap_counts(self._h, ctypes.byref(n_out), ctypes.byref(n_in), ctypes.byref(n_q)),
                "pa_sched_swap_counts")
         so, si = np.zeros(n_out.value, np.int64), np.zeros(n_in.value, np.int64)
         _check(lib().pa_sched_swap_record(self._h, _ptr(so), _ptr(si)), "pa_sched_swap_record")
-        return {"finished": fin.tolist(), "admitted": adm.tolist(), "preempted": pre.tolist(), "ops": ops,
-                "running": run.tolist(), "context_lens": ctx.tolist(), "num_waiting": c.num_waiting,
-                "swapped_out": so.tolist(), "swapped_in": si.tolist(), "num_swapped": n_q.value}
+        rec = {"finished": fin.tolist(), "admitted": adm.tolist(), "preempted": pre.tolist(), "ops": ops,
+               "running": run.tolist(), "context_lens": ctx.tolist(), "num_waiting": c.num_waiting,
+               "swapped_out": so.tolist(), "swapped_in": si.tolist(), "num_swapped": n_q.value}
+        if raw:
+            rec.update(op_kind=kind, op_a=oa, op_b=ob, op_c=oc)
+        return rec

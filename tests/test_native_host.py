@@ -371,3 +371,30 @@ def test_decode_and_cache_write_argument_rules(pa):
     assert cw(bs=12) == 2 and cw(D=96) == 2
     assert cw(nb=0) == 1 and cw(dt=9) == 1
     assert lib.pa_cache_write(nul, nul, nul, nul, nul, 4, None, nul) == 1
+
+
+def test_scheduler_raw_record_matches_tuples(pa):
+    """step(raw=True) gives the same ops as arrays."""
+    tc = wl.TraceConfig(block_size=4, max_running=12, num_requests=40, steps=80, prefix_len=10,
+                        prompt_hi=30, output_mean=10.0, fork_every=4)
+    reqs = wl.make_trace_requests(tc, 2)
+    order = np.random.default_rng(2).permutation(70).tolist()
+    pair = []
+    for _ in range(2):
+        bm = pa.BlockManager(70, tc.block_size, order)
+        bm.allocate(wl.PREFIX_SEQ, tc.prefix_len)
+        s = pa.Scheduler(bm, tc.max_running, wl.PREFIX_SEQ)
+        for q in reqs:
+            s.add_request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child, q.fork_output_len)
+        pair.append(s)
+    names = {"w": 0, "c": 1, "so": 2, "si": 3}
+    n_ops = 0
+    for step in range(tc.steps):
+        a, b = pair[0].step(), pair[1].step(raw=True)
+        assert b["ops"] is None and a["running"] == b["running"], step
+        assert [names[o[0]] for o in a["ops"]] == b["op_kind"].tolist(), step
+        assert [o[1] for o in a["ops"]] == b["op_a"].tolist(), step
+        assert [o[2] for o in a["ops"]] == b["op_b"].tolist(), step
+        assert [o[3] if o[0] == "w" else -1 for o in a["ops"]] == b["op_c"].tolist(), step
+        n_ops += len(a["ops"])
+    assert n_ops > 0
