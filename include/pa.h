@@ -147,6 +147,29 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     void* stream);
 
 /*
+ * pa_write_decode -- one decode step of a continuous batch in one call: the
+ * new tokens' K/V appended to their slots, then decode attention over the
+ * block tables ([P1] 3.2-3.3 for the append, [P3] "PagedAttention分页注意力机制原理"
+ * for the attention).  Same arguments, layouts, results and errors as
+ *   pa_cache_write(k, v, k_cache, v_cache, slot_mapping, num_tokens, &desc, stream);
+ *   pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, ...);
+ * with desc = {num_blocks, block_size, num_kv_heads, head_dim, dtype}: the
+ * decode sees every row the write appends.  Every argument of both is checked
+ * before anything is launched.  Fewer launches than the two calls: when the
+ * batch is split into partitions, one kernel does the write and orders the
+ * partitions, so the attention kernel follows it directly.  num_tokens == 0
+ * is pa_decode alone.
+ */
+pa_status pa_write_decode(const void* k, const void* v, const int64_t* slot_mapping, int num_tokens,
+                          void* out, const void* q, void* k_cache, void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens, float scale,
+                          int block_size, int num_kv_heads,
+                          int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                          int max_context_len, int num_blocks, pa_dtype dtype,
+                          int partition_size, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
  * Scratch bytes pa_verify needs (zero when every context fits one partition).
  */
 size_t pa_verify_workspace_size(int num_seqs, int num_queries, int num_heads, int head_dim,
@@ -216,10 +239,13 @@ int pa_get_verify_kernel(void);
  * split-K scratch is a fixed device array of PA_NOALLOC_SCRATCH_BYTES inside
  * the library instead of a caller-supplied workspace.
  *   - Every GPU on which the library is loaded holds that array until exit.
- *   - A batch needing more scratch than that (pa_decode_workspace_size) is
- *     rejected with PA_ERR_UNSUPPORTED before any launch.
+ *   - A batch needing more scratch than that (pa_decode_workspace_size, with
+ *     max_context_len capped at max_blocks_per_seq x block_size as pa_decode
+ *     caps it) is rejected with PA_ERR_UNSUPPORTED before any launch.
  *   - The first call on a device looks up the array's device address for that
- *     device; make that first call before any stream capture.
+ *     device and keeps it for the device's current context; make that first
+ *     call before any stream capture.  A call made in another context of the
+ *     device (after cudaDeviceReset, for one) looks the address up again.
  *   - All calls share the array and it keeps the last call's contents (no part
  *     of it needs to start at zero); calls that overlap on the GPU race on it.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
@@ -388,7 +414,8 @@ typedef enum {
     PA_KERNEL_COPY_BLOCKS = 4,
     PA_KERNEL_VERIFY = 5,        /* multi-query (verification) kernel */
     PA_KERNEL_SWAP = 6,          /* block moves between device and host pools */
-    PA_KERNEL_COUNT = 7
+    PA_KERNEL_WRITE_PLAN = 7,    /* pa_write_decode: cache write and plan in one kernel */
+    PA_KERNEL_COUNT = 8
 } pa_kernel_id;
 
 /* Number of kernels this library has launched in the process so far. */

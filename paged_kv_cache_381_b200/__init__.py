@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3:
                 4: "PA_ERR_CUDA", 5: "PA_ERR_DEVICE"}
 PA_ERR_NO_BLOCKS = 3
 DEVERR_SLOT, DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
-KERNELS = ("cache_write", "decode", "reduce", "plan", "copy_blocks", "verify", "swap")
+KERNELS = ("cache_write", "decode", "reduce", "plan", "copy_blocks", "verify", "swap", "write_plan")
 DEFAULT_PARTITION = 512
 
 
@@ -147,7 +147,8 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block
     maxb = block_tables.shape[1] if block_tables.dim() == 2 else 1
     if max_context_len is None:
         max_context_len = maxb * block_size
-    need = pa_decode_workspace_size(S, Hq, D, max_context_len, partition_size)
+    # the library bounds contexts by the table's capacity as well
+    need = pa_decode_workspace_size(S, Hq, D, min(int(max_context_len), maxb * int(block_size)), partition_size)
     ws_ptr, ws_bytes = ctypes.c_void_p(0), 0
     if need:
         if workspace is None:
@@ -162,6 +163,42 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block
                          int(block_size), int(num_kv_heads), S, Hq, D, maxb, int(max_context_len), nb,
                          _dtype_code(q), int(partition_size), ws_ptr, ws_bytes, _stream(q, stream))
     _check(st, "pa_decode")
+    return out
+
+
+def pa_write_decode(k, v, slot_mapping, out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                    block_size=None, num_kv_heads=None, max_context_len=None, partition_size=0, workspace=None,
+                    stream=None):
+    """pa_cache_write of the new rows k, v [T, Hkv, D] through int64 slots, then
+    pa_decode, in one call (fewer launches).  Arguments as for those two."""
+    import torch
+    nb, bs, hkv, d = k_cache.shape
+    block_size = bs if block_size is None else block_size
+    num_kv_heads = hkv if num_kv_heads is None else num_kv_heads
+    S, Hq, D = q.shape
+    maxb = block_tables.shape[1] if block_tables.dim() == 2 else 1
+    if max_context_len is None:
+        max_context_len = maxb * block_size
+    # the library bounds contexts by the table's capacity as well
+    need = pa_decode_workspace_size(S, Hq, D, min(int(max_context_len), maxb * int(block_size)), partition_size)
+    ws_ptr, ws_bytes = ctypes.c_void_p(0), 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        if workspace.numel() < need:
+            raise ValueError(f"workspace needs {need} bytes")
+        ws_ptr, ws_bytes = ctypes.c_void_p(workspace.data_ptr()), int(workspace.numel())
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    T = int(slot_mapping.numel())
+    st = lib().pa_write_decode(_dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping"), T, _dev(out, "out"),
+                               _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                               _dev(block_tables, "block_tables"), _dev(context_lens, "context_lens"), float(scale),
+                               int(block_size), int(num_kv_heads), S, Hq, D, maxb, int(max_context_len), nb,
+                               _dtype_code(q), int(partition_size), ws_ptr, ws_bytes, _stream(q, stream))
+    _check(st, "pa_write_decode")
     return out
 
 

@@ -50,6 +50,9 @@ SIGNATURES = {
     "pa_decode_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "pa_decode": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int, c_int,
                           c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "pa_write_decode": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                c_void_p, c_void_p, c_float, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "pa_verify_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
     "pa_verify_partition_size": (c_int, [c_int, c_int, c_int, c_int, c_int]),
     "pa_verify": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int, c_int,

@@ -18,7 +18,7 @@ import numpy as np
 import torch
 
 from . import (BlockManager, pa_cache_write, pa_decode, pa_decode_workspace_size, pa_verify,
-               pa_verify_workspace_size)
+               pa_verify_workspace_size, pa_write_decode)
 
 
 class PagedBatch:
@@ -97,6 +97,14 @@ class PagedBatch:
         return pa_decode(out, q, self.k_cache, self.v_cache, self.block_tables, self.context_lens, scale,
                          self.block_size, self.num_kv_heads, max_context_len=self.max_context_len,
                          partition_size=partition_size, workspace=ws, stream=stream)
+
+    def step(self, out, q, scale, partition_size=0, stream=None):
+        """write_new_tokens then decode, in one library call (pa_write_decode)."""
+        ws = self.ensure_workspace(q.shape[1], partition_size)
+        return pa_write_decode(self.k_new, self.v_new, self.slot_mapping, out, q, self.k_cache, self.v_cache,
+                               self.block_tables, self.context_lens, scale, self.block_size, self.num_kv_heads,
+                               max_context_len=self.max_context_len, partition_size=partition_size, workspace=ws,
+                               stream=stream)
 
     def verify(self, out, q, scale, partition_size=0, stream=None):
         """q, out: [S, Q, Hq, D] with Q = new_tokens."""

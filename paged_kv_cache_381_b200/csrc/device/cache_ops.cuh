@@ -16,18 +16,16 @@
 
 namespace pa_dev {
 
-// One thread per 16-byte vector of a token row (K and V), grid-stride; many
-// independent loads in flight keep this short kernel from being latency-bound.
-// row_vecs = 16-byte vectors per token row.
-__global__ void __launch_bounds__(256) cache_write_kernel(const uint4* __restrict__ k,
-                                                          const uint4* __restrict__ v,
-                                                          uint4* __restrict__ k_cache,
-                                                          uint4* __restrict__ v_cache,
-                                                          const int64_t* __restrict__ slot_mapping,
-                                                          int num_tokens, int row_vecs, int64_t num_slots) {
+// One thread per 16-byte vector of a token row (K and V), strided over the
+// threads given (`first` = this thread's first vector, `stride` = all the
+// threads' count); many independent loads in flight keep this short work from
+// being latency-bound.  row_vecs = 16-byte vectors per token row.
+__device__ __forceinline__ void write_rows(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                           uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                                           const int64_t* __restrict__ slot_mapping, int num_tokens, int row_vecs,
+                                           int64_t num_slots, int64_t first, int64_t stride) {
     const int64_t total = (int64_t)num_tokens * row_vecs;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
+    for (int64_t i = first; i < total; i += stride) {
         const int64_t t = i / row_vecs;
         const int64_t j = i - t * row_vecs;
         const int64_t slot = __ldg(slot_mapping + t);
@@ -41,6 +39,24 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const uint4* __restric
         k_cache[slot * row_vecs + j] = a;
         v_cache[slot * row_vecs + j] = b;
     }
+}
+
+// The arguments of one cache write (pa_cache_write; also the first part of
+// pa_write_decode's first kernel).
+struct WriteArgs {
+    const uint4* k;
+    const uint4* v;
+    uint4* k_cache;
+    uint4* v_cache;
+    const int64_t* slot_mapping;
+    int num_tokens;
+    int row_vecs;
+    int64_t num_slots;
+};
+
+__global__ void __launch_bounds__(256) cache_write_kernel(const WriteArgs w) {
+    write_rows(w.k, w.v, w.k_cache, w.v_cache, w.slot_mapping, w.num_tokens, w.row_vecs, w.num_slots,
+               (int64_t)blockIdx.x * blockDim.x + threadIdx.x, (int64_t)gridDim.x * blockDim.x);
 }
 
 // grid (num_pairs, 2): blockIdx.y selects the K or V pool.

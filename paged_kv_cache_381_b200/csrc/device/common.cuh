@@ -14,7 +14,15 @@
 namespace pa_dev {
 
 // Error word of the library (one per device context); bits are PA_DEVERR_*.
-// Defined here: the library is one CUDA translation unit.
+// It is defined in this header, so exactly one translation unit of the
+// library may include it -- pa_api.cu, which also holds pa_get_device_error.
+// A second unit including it would get its own copy of the word (the library
+// is built without relocatable device code), and flags raised there would
+// never be read; the check below turns that into a compile error.
+// (pa_noalloc.cu, the library's other CUDA unit, launches nothing itself.)
+#ifndef PA_ERROR_WORD_UNIT
+#error "common.cuh defines the device error word: include it only from pa_api.cu"
+#endif
 __device__ unsigned int g_error = 0;
 
 __device__ __forceinline__ void flag_error(unsigned int bit) { atomicOr(&g_error, bit); }

@@ -13,28 +13,35 @@
 //  * Work item = (sequence, context partition, kv head, query-head chunk).  A
 //    CTA handles all query heads of a kv-head group that share the K/V rows it
 //    streams, so each K/V byte leaves HBM once.  Contexts longer than the
-//    partition size are split; items are ordered longest-first by a small
-//    planning kernel and a persistent grid (a multiple of the SM count) walks
-//    them with a fixed stride.
-//  * One producer warp resolves block ids through the block table (staged in
-//    shared memory) and issues tiled TMA loads into a ring of shared-memory
-//    stages of 32 token rows, each stage completed on an mbarrier with
-//    transaction counts.  The pool is seen by the TMA unit as a 3-D tensor
-//    [num_blocks * block_size rows][num_kv_heads][head_dim]; one box is the
-//    block_size rows of one kv head and one 128-byte slice of head_dim, so a
-//    16-token block of a 128-wide bf16 head arrives in two 2 KiB loads (per-row
-//    256-byte bulk copies were measured to cap a producer warp near 7 GB/s).
-//    Boxes land with the 128-byte swizzle (16-byte chunk index XOR row % 8),
-//    which keeps 8-row ldmatrix and 16-byte vector reads free of bank
-//    conflicts; consumers apply the same XOR when they address a row.
-//  * Four consumer warps: phase 1 computes the scaled scores of every token of
-//    the partition into shared memory (16-byte vector reads, fp32 FMAs, a
-//    transposing butterfly that reduces G partial dot products over the lanes
-//    of a row with G-1 shuffles); phase 2 takes the exact max and the
-//    exponentials (fp32, base 2 with log2(e) folded into the scale) and their
-//    sum; phase 3 accumulates p * V in fp32 registers; an epilogue merges the
-//    warps in a fixed order and either writes the normalised row (one
-//    partition) or the partition's unnormalised output, max and sum.
+//    partition size are split.  A planning kernel sorts the items by length,
+//    longest first, and a persistent grid (a multiple of the SM count) deals
+//    them out in snake order (walk_first / walk_next), which evens out the
+//    CTAs' totals.
+//  * One producer warp looks items up one ahead of their use, publishes each
+//    item's descriptor and q rows (one bulk copy) to the consumers through a
+//    double-buffered shared-memory slot, resolves block ids through the block
+//    table and issues tiled TMA loads into a ring of shared-memory stages of 32
+//    token rows, each stage completed on an mbarrier with transaction counts.
+//    The pool is seen by the TMA unit as a 3-D tensor [num_blocks * block_size
+//    rows][num_kv_heads][head_dim]; one box is the block_size rows of one kv
+//    head and one 128-byte slice of head_dim, so a 16-token block of a
+//    128-wide bf16 head arrives in two 2 KiB loads (per-row 256-byte bulk
+//    copies were measured to cap a producer warp near 7 GB/s).  Boxes land
+//    with the 128-byte swizzle (16-byte chunk index XOR row % 8), which keeps
+//    8-row ldmatrix and 16-byte vector reads free of bank conflicts; consumers
+//    apply the same XOR when they address a row.
+//  * Four consumer warps.  Tensor path (fp16 / bf16): phase 1 splits the K
+//    stages over the warps and writes the scaled scores of every token of the
+//    partition to shared memory with a running max; phase 2 gives each warp a
+//    quarter of head_dim over every V stage, so each warp finishes its own
+//    output columns (and the whole softmax denominator) without a cross-warp
+//    reduction.  CUDA-core path (fp32, or on request): phase 1 as above with
+//    16-byte vector reads, fp32 FMAs and a transposing butterfly that reduces
+//    G partial dot products over the lanes of a row; phase 2 takes the exact
+//    max, exponentials and their sum; phase 3 accumulates p * V per warp over
+//    its stages, and an epilogue merges the warps in a fixed order.  Either
+//    path writes the normalised row (one partition) or the partition's
+//    unnormalised output, max and sum.
 //  * Every reduction order depends only on logical token positions, so the
 //    result is bitwise independent of the physical placement of blocks.
 //  * All waits are bounded: on expiry the CTA records PA_DEVERR_TIMEOUT and
@@ -65,7 +72,8 @@ struct DecodeArgs {
     int partition_size;        // tokens per partition (multiple of 32)
     int max_partitions;        // 1: single pass, no plan / partials
     const int2* plan;          // split mode: (seq, partition), longest first
-    const int* plan_count;
+    const int* plan_count;     // [0]: pairs in the plan, [1]: split sequences
+    const int* split_seqs;     // split mode: the sequences with more than one partition
     float* part_m;             // [num_seqs * num_heads, max_partitions] (log2 units)
     float* part_l;             // [num_seqs * num_heads, max_partitions]
     float* part_o;             // [num_seqs * num_heads, max_partitions, head_dim]
@@ -91,6 +99,12 @@ __device__ __forceinline__ int partitions_of(const DecodeArgs& a, int ctx) {
     return ctx == 0 ? 1 : (ctx + a.partition_size - 1) / a.partition_size;
 }
 
+// (sequence, partition) of a pair index: the plan's entry in split mode, the
+// sequence itself in single-pass mode.
+__device__ __forceinline__ int2 pair_at(const DecodeArgs& a, int pair) {
+    return a.max_partitions == 1 ? make_int2(pair, 0) : a.plan[pair];
+}
+
 __device__ __forceinline__ WorkItem decode_item(const DecodeArgs& a, int i, bool report) {
     const int per = a.num_kv_heads * a.n_gchunks;
     const int pair = i / per;
@@ -98,19 +112,30 @@ __device__ __forceinline__ WorkItem decode_item(const DecodeArgs& a, int i, bool
     WorkItem w;
     w.h = rem / a.n_gchunks;
     w.gc = rem - w.h * a.n_gchunks;
-    if (a.max_partitions == 1) {
-        w.s = pair;
-        w.p = 0;
-    } else {
-        const int2 e = a.plan[pair];
-        w.s = e.x;
-        w.p = e.y;
-    }
+    const int2 e = pair_at(a, pair);
+    w.s = e.x;
+    w.p = e.y;
     const int ctx = clamp_context(a, w.s, report);
     w.np = partitions_of(a, ctx);
     w.t0 = w.p * a.partition_size;
     w.n = min(max(ctx - w.t0, 0), a.partition_size);
     return w;
+}
+
+// The items a CTA of the persistent grid takes.  Round r covers items
+// [r * G, (r + 1) * G) with G = gridDim.x; CTA c takes item r * G + c in even
+// rounds and r * G + G - 1 - c in odd rounds (snake order).  With the plan
+// sorted longest first, the CTA that took a round's longest item takes the
+// next round's shortest, and the per-CTA sums of item lengths stay close to
+// their mean.  The sequence of items is increasing, so a walk ends at the
+// first index past the total.
+__device__ __forceinline__ int walk_first() { return (int)blockIdx.x; }
+
+__device__ __forceinline__ int walk_next(int i) {
+    const int64_t G = gridDim.x;
+    const int64_t r = i / G + 1;
+    const int64_t n = r * G + ((r & 1) ? G - 1 - (int64_t)blockIdx.x : (int64_t)blockIdx.x);
+    return n > 0x7fffffff ? 0x7fffffff : (int)n;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -248,29 +273,42 @@ struct DecodeCfg {
     static constexpr int THREADS = (NCW + 1) * 32;
     static constexpr int MAX_PARTITION = 1024;
     static constexpr int MAX_TABLE = MAX_PARTITION / 8;
+    static constexpr int TPL = MAX_TABLE / 32;      // block-table entries per producer lane
+    // Tensor path: every consumer warp reads every stage (phase 1 work goes to
+    // one warp per stage, phase 2 work to all four), and a stage is free once
+    // all four have released it.  CUDA-core path: each stage belongs to one warp.
+    static constexpr int EMPTY_ARRIVALS = TENSOR ? NCW : 1;
     // scores row stride (floats): the tensor path reads 8-query rows as pairs;
     // the SIMT path pads to GC + 1 so per-query column walks avoid bank conflicts
     static constexpr int LSTRIDE = TENSOR ? GC : (GC == 1 ? 1 : GC + 1);
+    static constexpr int Q_BYTES = GC * ROW_BYTES;  // one item's q rows
     static constexpr int OFF_FULL = NSTAGES * STAGE_BYTES;   // ring at a 1024-byte aligned base
     static constexpr int OFF_EMPTY = OFF_FULL + NSTAGES * 8;
-    static constexpr int OFF_TABLE = OFF_EMPTY + NSTAGES * 8;
-    static constexpr int OFF_STATS = OFF_TABLE + MAX_TABLE * 4;     // wmax, wsum [NCW][GC], m, l [GC], abort
+    static constexpr int OFF_IFULL = OFF_EMPTY + NSTAGES * 8;    // item slot filled (descriptor + q)
+    static constexpr int OFF_IEMPTY = OFF_IFULL + 2 * 8;         // item slot read by every consumer warp
+    static constexpr int OFF_INFO = OFF_IEMPTY + 2 * 8;          // two WorkItem descriptors, 8 ints each
+    static constexpr int OFF_TABLE = OFF_INFO + 2 * 32;
+    static constexpr int OFF_QBUF = (OFF_TABLE + MAX_TABLE * 4 + 127) / 128 * 128;   // two q tiles
+    static constexpr int OFF_STATS = OFF_QBUF + 2 * Q_BYTES;    // wmax, wsum [NCW][GC], m, l [GC], flags
     static constexpr int STATS_FLOATS = 2 * NCW * GC + 2 * GC + 4;
-    // The scores (phases 1-3) and the warps' output partials (epilogue) share
-    // one region: a barrier separates the last score read from the first
-    // partial write.
+    // The scores (phases 1-3) and, on the CUDA-core path, the warps' output
+    // partials (epilogue) share one region: a barrier separates the last score
+    // read from the first partial write.
     static constexpr int OFF_LOGITS = ((OFF_STATS + STATS_FLOATS * 4) + 127) / 128 * 128;
     static constexpr int OFF_RED = OFF_LOGITS;
-    static constexpr int RED_BYTES = NCW * GC * D * 4;
-    static_assert(TENSOR ? (GC == 8 && ELT == 2) : (GC <= LPT), "unsupported query chunk");
+    static constexpr int RED_BYTES = TENSOR ? 0 : NCW * GC * D * 4;
+    static_assert(TENSOR ? (GC == 8 && ELT == 2 && (D / 16) % NCW == 0) : (GC <= LPT), "unsupported query chunk");
     static_assert(LPT >= 1 && LPT <= 32 && (32 % LPT) == 0, "row must span a divisor of the warp");
     static_assert(ROW_BYTES % 128 == 0 && STAGE_BYTES % 1024 == 0, "swizzled boxes need 1024-byte alignment");
-    // Consumer warp w takes the stages st = w, w + NCW, ... of a phase, and a
-    // ring slot is reused every NSTAGES stages.  Only when NSTAGES is a multiple
-    // of NCW does one warp own every use of a slot within a phase; otherwise a
-    // warp could test a slot's full barrier for its next use while the previous
-    // use (another warp's) is still in flight, and the parity test would answer
-    // "complete" for the wrong phase.
+    static_assert(Q_BYTES % 16 == 0 && OFF_QBUF % 16 == 0, "bulk copies need 16-byte sizes and addresses");
+    // CUDA-core path: consumer warp w takes the stages st = w, w + NCW, ... of
+    // a phase, and a ring slot is reused every NSTAGES stages.  Only when
+    // NSTAGES is a multiple of NCW does one warp own every use of a slot within
+    // a phase; otherwise a warp could test a slot's full barrier for its next
+    // use while the previous use (another warp's) is still in flight, and the
+    // parity test would answer "complete" for the wrong phase.  (On the tensor
+    // path every warp waits on every stage in order, which is safe at any
+    // depth; the same rule is kept for both.)
     static_assert(NSTAGES % NCW == 0, "ring depth must be a multiple of the consumer warps");
     // + 1024: the dynamic shared-memory base is rounded up to 1024 bytes in the kernel
     static size_t smem_bytes(int partition) {
@@ -299,7 +337,11 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_FULL);
     uint64_t* empty = reinterpret_cast<uint64_t*>(smem + C::OFF_EMPTY);
+    uint64_t* item_full = reinterpret_cast<uint64_t*>(smem + C::OFF_IFULL);
+    uint64_t* item_empty = reinterpret_cast<uint64_t*>(smem + C::OFF_IEMPTY);
+    int* info = reinterpret_cast<int*>(smem + C::OFF_INFO);           // [2][8]
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + C::OFF_TABLE);
+    unsigned char* qbuf = smem + C::OFF_QBUF;                          // [2][GC][D] elements
     float* wmax = reinterpret_cast<float*>(smem + C::OFF_STATS);   // [NCW][GC]
     float* wsum = wmax + C::NCW * GC;                                // [NCW][GC]
     float* stat_m = wsum + C::NCW * GC;                              // [GC]
@@ -314,7 +356,11 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NSTAGES; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
+            mbar_init(&empty[i], C::EMPTY_ARRIVALS);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&item_full[i], 1);
+            mbar_init(&item_empty[i], C::NCW);
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -324,7 +370,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
     // launched as a programmatic dependent of the plan kernel (or of whatever
     // precedes it): nothing written by earlier kernels is read before this
     grid_dependency_wait();
-    const int pairs = a.max_partitions == 1 ? a.num_seqs : *a.plan_count;
+    const int pairs = a.max_partitions == 1 ? a.num_seqs : a.plan_count[0];
     const int total = pairs * a.num_kv_heads * a.n_gchunks;
     const int bs = 1 << a.log2_bs;
     const int box_bytes = bs * 128;
@@ -343,57 +389,126 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
             prefetch_tmap(&tmap_v);
         }
         const uint64_t policy = l2_policy_evict_first();
-        uint32_t stage = 0;
-        bool ok = true;
-        for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-            const WorkItem w = decode_item(a, i, lane == 0);
-            if (w.n == 0) continue;
-            const int nst = (w.n + C::STAGE_ROWS - 1) / C::STAGE_ROWS;
+        const T* qg = static_cast<const T*>(a.q);
+        // Block ids of an item, requested into registers (lane j holds entries
+        // j, j + 32, ...) one item before they are needed; rows of the table
+        // past the item's blocks are not read.
+        auto request_ids = [&](const WorkItem& w, int32_t (&ids)[C::TPL]) {
             const int nblk = (w.n + bs - 1) >> a.log2_bs;
             const int32_t* trow = a.block_tables + (int64_t)w.s * a.max_blocks_per_seq + (w.t0 >> a.log2_bs);
-            for (int j = lane; j < nblk; j += 32) {
-                int32_t id = trow[j];
-                if (id < 0 || id >= a.num_blocks) {
-                    flag_error(PA_DEVERR_BLOCK_ID);
-                    id = 0;
-                }
-                tbl[j] = id;
+#pragma unroll
+            for (int k = 0; k < C::TPL; ++k) {
+                const int j = lane + 32 * k;
+                ids[k] = j < nblk ? trow[j] : 0;
             }
-            __syncwarp();
-            for (int pass = 0; pass < 2 && ok; ++pass) {
-                const void* tmap = pass ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
-                for (int st = 0; st < nst; ++st, ++stage) {
-                    const int slot = stage % C::NSTAGES;
-                    const uint32_t parity = ((stage / C::NSTAGES) & 1u) ^ 1u;
-                    if (!mbar_wait(&empty[slot], parity, abort_flag)) {
-                        ok = false;
-                        break;
+        };
+        uint32_t stage = 0;
+        uint32_t k = 0;                                   // items published
+        bool ok = true;
+        int i = walk_first();
+        WorkItem w{};
+        int32_t ids[C::TPL];
+        if (i < total) {
+            w = decode_item(a, i, lane == 0);
+            request_ids(w, ids);
+        }
+        for (; i < total && ok; ++k) {
+            // publish the item: descriptor, then its q rows by one bulk copy
+            const int b = k & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&item_empty[b], ((k >> 1) & 1u) ^ 1u, abort_flag))) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                int* dst = info + b * 8;
+                dst[0] = w.s;
+                dst[1] = w.p;
+                dst[2] = w.h;
+                dst[3] = w.gc;
+                dst[4] = w.t0;
+                dst[5] = w.n;
+                dst[6] = w.np;
+                if (w.n > 0) {
+                    const int gq = min(GC, a.group - w.gc * GC);
+                    const int64_t row0 = (int64_t)w.s * a.num_heads + w.h * a.group + w.gc * GC;
+                    mbar_arrive_expect_tx(&item_full[b], (uint32_t)(gq * C::ROW_BYTES));
+                    bulk_copy_g2s(qbuf + b * C::Q_BYTES, qg + row0 * D, (uint32_t)(gq * C::ROW_BYTES),
+                                  &item_full[b]);
+                } else {
+                    mbar_arrive(&item_full[b]);
+                }
+            }
+            // look the next item up while this item's stages wait for ring slots
+            const int inext = walk_next(i);
+            WorkItem wn{};
+            int32_t idn[C::TPL];
+            if (inext < total) {
+                wn = decode_item(a, inext, lane == 0);
+                request_ids(wn, idn);
+            }
+            if (w.n > 0) {
+                const int nst = (w.n + C::STAGE_ROWS - 1) / C::STAGE_ROWS;
+                const int nblk = (w.n + bs - 1) >> a.log2_bs;
+                __syncwarp();                 // the previous item's table reads are done
+#pragma unroll
+                for (int kk = 0; kk < C::TPL; ++kk) {
+                    const int j = lane + 32 * kk;
+                    if (j < nblk) {
+                        int32_t id = ids[kk];
+                        if (id < 0 || id >= a.num_blocks) {
+                            flag_error(PA_DEVERR_BLOCK_ID);
+                            id = 0;
+                        }
+                        tbl[j] = id;
                     }
-                    const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
-                    const int nblk_st = (rows + bs - 1) >> a.log2_bs;      // whole blocks are loaded
-                    const int nbox = nblk_st * C::NH;
-                    if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbox * box_bytes));
-                    __syncwarp();
-                    if (lane < nbox) {
-                        const int b = lane / C::NH;
-                        const int half = lane - b * C::NH;
-                        const int phys = tbl[((st * C::STAGE_ROWS) >> a.log2_bs) + b];
-                        tma_load_3d(smem + slot * C::STAGE_BYTES + (b * C::NH + half) * box_bytes, tmap,
-                                    half * C::BOX_ELEMS, w.h, phys * bs, &full[slot], policy);
+                }
+                __syncwarp();
+                for (int pass = 0; pass < 2 && ok; ++pass) {
+                    const void* tmap = pass ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
+                    for (int st = 0; st < nst; ++st, ++stage) {
+                        const int slot = stage % C::NSTAGES;
+                        const uint32_t parity = ((stage / C::NSTAGES) & 1u) ^ 1u;
+                        if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], parity, abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
+                        const int nblk_st = (rows + bs - 1) >> a.log2_bs;      // whole blocks are loaded
+                        const int nbox = nblk_st * C::NH;
+                        if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbox * box_bytes));
+                        __syncwarp();
+                        if (lane < nbox) {
+                            const int bb = lane / C::NH;
+                            const int half = lane - bb * C::NH;
+                            const int phys = tbl[((st * C::STAGE_ROWS) >> a.log2_bs) + bb];
+                            tma_load_3d(smem + slot * C::STAGE_BYTES + (bb * C::NH + half) * box_bytes, tmap,
+                                        half * C::BOX_ELEMS, w.h, phys * bs, &full[slot], policy);
+                        }
                     }
                 }
             }
+            i = inext;
+            w = wn;
+#pragma unroll
+            for (int kk = 0; kk < C::TPL; ++kk) ids[kk] = idn[kk];
         }
         if (!ok) {
             if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
             *abort_flag = 1;
-            // let copies already issued land before the CTA can retire
+            // let copies already issued land before the CTA can retire: every
+            // stage issued, and the q copy of every item published
+            const volatile int never = 0;
             const uint32_t issued = stage;
             for (int slot = lane; slot < C::NSTAGES; slot += 32) {
                 if ((uint32_t)slot < issued) {
                     const uint32_t last = issued - 1 - ((issued - 1 - slot) % C::NSTAGES);
-                    const volatile int never = 0;
                     mbar_wait(&full[slot], (last / C::NSTAGES) & 1u, &never);
+                }
+            }
+            for (int b = lane; b < 2; b += 32) {
+                if ((uint32_t)b < k) {
+                    const uint32_t last = k - 1 - ((k - 1 - b) & 1u);
+                    mbar_wait(&item_full[b], (last >> 1) & 1u, &never);
                 }
             }
         }
@@ -403,14 +518,16 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
     // -------------------------------------------------------------- consumers
     constexpr int NCT = C::NCW * 32;
     const int ctid = threadIdx.x;
-    const T* qg = static_cast<const T*>(a.q);
     T* outg = static_cast<T*>(a.out);
     uint32_t stage = 0;
 
-    // Wait for a stage this warp owns; false once the CTA has given up.
+    // Wait for a stage; false once the CTA has given up.  The answer is the
+    // same for every lane of the warp (the lanes poll on their own, and the
+    // warp-wide matrix instructions that follow need all of them).
     auto acquire = [&](uint32_t c) -> bool {
         const int slot = c % C::NSTAGES;
-        if (*abort_flag || !mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag)) {
+        const bool got = !*abort_flag && mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
             *abort_flag = 1;
             return false;
         }
@@ -421,12 +538,35 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
         if (lane == 0) mbar_arrive(&empty[c % C::NSTAGES]);
     };
 
-    for (int i = blockIdx.x; i < total; i += gridDim.x) {
-        const WorkItem w = decode_item(a, i, false);
+    uint32_t k = 0;                                       // items taken
+    for (int i = walk_first(); i < total; i = walk_next(i), ++k) {
+        const int b = k & 1;
+        // the item as the producer published it; after a give-up, looked up here
+        // (every warp then still takes the same items through the same barriers)
+        WorkItem w;
+        bool have_q = false;
+        const bool got = !*abort_flag && mbar_wait(&item_full[b], (k >> 1) & 1u, abort_flag);
+        if (__all_sync(0xffffffffu, got)) {
+            const int* src = info + b * 8;
+            w.s = src[0];
+            w.p = src[1];
+            w.h = src[2];
+            w.gc = src[3];
+            w.t0 = src[4];
+            w.n = src[5];
+            w.np = src[6];
+            have_q = true;
+        } else {
+            *abort_flag = 1;
+            w = decode_item(a, i, false);
+        }
         const int gq = min(GC, a.group - w.gc * GC);
         const int hq0 = w.h * a.group + w.gc * GC;
         const int64_t row0 = (int64_t)w.s * a.num_heads + hq0;
+        const unsigned char* qs = qbuf + b * C::Q_BYTES;
         if (w.n == 0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&item_empty[b]);
             for (int e = ctid; e < gq * D; e += NCT) outg[row0 * D + e] = Tr::from_float(0.f);
             continue;
         }
@@ -435,56 +575,62 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
         if constexpr (TENSOR) {
             using M = MmaOps<T>;
             constexpr int KS = D / 16;                 // k-steps over head_dim
+            constexpr int DMW = KS / C::NCW;           // 16-wide head_dim tiles per warp in phase 2
             const int gid = lane >> 2;
             const int tig = lane & 3;
-            // ---- phase 1: S^T tiles, scaled to base-2 units, with a running max
+            // ---- q as B fragments, from the item's tile (rows past the chunk are zero)
             uint32_t qb[KS][2];
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
-                if (gid < gq) {
-                    const T* qrow = qg + (row0 + gid) * D + kk * 16 + tig * 2;
-                    qb[kk][0] = __ldg(reinterpret_cast<const unsigned int*>(qrow));
-                    qb[kk][1] = __ldg(reinterpret_cast<const unsigned int*>(qrow + 8));
+                if (have_q && gid < gq) {
+                    const unsigned char* qrow = qs + gid * C::ROW_BYTES + (kk * 16 + tig * 2) * C::ELT;
+                    qb[kk][0] = *reinterpret_cast<const uint32_t*>(qrow);
+                    qb[kk][1] = *reinterpret_cast<const uint32_t*>(qrow + 8 * C::ELT);
                 } else {
                     qb[kk][0] = qb[kk][1] = 0u;
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&item_empty[b]);
+            // ---- phase 1: S^T tiles of the warp's stages, scaled to base-2 units, with a running max
             float mlo = -INFINITY, mhi = -INFINITY;      // queries 2*tig, 2*tig+1
-            for (int st = warp; st < nst; st += C::NCW) {
+            for (int st = 0; st < nst; ++st) {
                 const uint32_t c = stage + st;
                 if (!acquire(c)) continue;
-                const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
-                const uint32_t sb = smem_addr(smem + (c % C::NSTAGES) * C::STAGE_BYTES);
-                // ldmatrix row address of this lane: matrix lane/8 -> (+8 rows if odd, +8 cols if >= 2);
-                // row % 8 == lane % 8, the swizzle key
-                const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int hi = lane >> 4;
-                const int x = lane & 7;
+                if ((st & (C::NCW - 1)) == warp) {
+                    const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
+                    const uint32_t sb = smem_addr(smem + (c % C::NSTAGES) * C::STAGE_BYTES);
+                    // ldmatrix row address of this lane: matrix lane/8 -> (+8 rows if odd, +8 cols if >= 2);
+                    // row % 8 == lane % 8, the swizzle key
+                    const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int hi = lane >> 4;
+                    const int x = lane & 7;
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                    if (mt * 16 >= rows) break;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    const uint32_t base = sb + row_base(mt * 16 + lrow);
+                    for (int mt = 0; mt < 2; ++mt) {
+                        if (mt * 16 >= rows) break;
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                        const uint32_t base = sb + row_base(mt * 16 + lrow);
 #pragma unroll
-                    for (int kk = 0; kk < KS; ++kk) {
-                        uint32_t af[4];
-                        const int cc = ((kk * 2) & 7) + hi;         // 16-byte chunk within the slice
-                        ldsm_x4(base + (kk >> 2) * box_bytes + ((cc ^ x) << 4), af[0], af[1], af[2], af[3]);
-                        M::mma(acc, af, qb[kk][0], qb[kk][1]);
-                    }
-                    const int t_lo = mt * 16 + gid;            // stage-relative token of acc[0..1]
-                    float* lrow_lo = logits + (st * C::STAGE_ROWS + t_lo) * GC + tig * 2;
-                    if (t_lo < rows) {
-                        const float z0 = acc[0] * a.scale_log2, z1 = acc[1] * a.scale_log2;
-                        *reinterpret_cast<float2*>(lrow_lo) = make_float2(z0, z1);
-                        mlo = fmaxf(mlo, z0);
-                        mhi = fmaxf(mhi, z1);
-                    }
-                    if (t_lo + 8 < rows) {
-                        const float z2 = acc[2] * a.scale_log2, z3 = acc[3] * a.scale_log2;
-                        *reinterpret_cast<float2*>(lrow_lo + 8 * GC) = make_float2(z2, z3);
-                        mlo = fmaxf(mlo, z2);
-                        mhi = fmaxf(mhi, z3);
+                        for (int kk = 0; kk < KS; ++kk) {
+                            uint32_t af[4];
+                            const int cc = ((kk * 2) & 7) + hi;         // 16-byte chunk within the slice
+                            ldsm_x4(base + (kk >> 2) * box_bytes + ((cc ^ x) << 4), af[0], af[1], af[2], af[3]);
+                            M::mma(acc, af, qb[kk][0], qb[kk][1]);
+                        }
+                        const int t_lo = mt * 16 + gid;            // stage-relative token of acc[0..1]
+                        float* lrow_lo = logits + (st * C::STAGE_ROWS + t_lo) * GC + tig * 2;
+                        if (t_lo < rows) {
+                            const float z0 = acc[0] * a.scale_log2, z1 = acc[1] * a.scale_log2;
+                            *reinterpret_cast<float2*>(lrow_lo) = make_float2(z0, z1);
+                            mlo = fmaxf(mlo, z0);
+                            mhi = fmaxf(mhi, z1);
+                        }
+                        if (t_lo + 8 < rows) {
+                            const float z2 = acc[2] * a.scale_log2, z3 = acc[3] * a.scale_log2;
+                            *reinterpret_cast<float2*>(lrow_lo + 8 * GC) = make_float2(z2, z3);
+                            mlo = fmaxf(mlo, z2);
+                            mhi = fmaxf(mhi, z3);
+                        }
                     }
                 }
                 release(c);
@@ -501,19 +647,20 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
             }
             named_barrier(1, NCT);
 
-            // ---- phase 3: p = 2^(z - max) built straight into B fragments; O^T += V^T P^T
+            // ---- phase 2: p = 2^(z - max) built straight into B fragments for every
+            // token; O^T += V^T P^T over this warp's head_dim tiles
             float mg = wmax[gid];
 #pragma unroll
             for (int ww = 1; ww < C::NCW; ++ww) mg = fmaxf(mg, wmax[ww * GC + gid]);
-            float oacc[KS][4];
+            float oacc[DMW][4];
 #pragma unroll
-            for (int dm = 0; dm < KS; ++dm) oacc[dm][0] = oacc[dm][1] = oacc[dm][2] = oacc[dm][3] = 0.f;
+            for (int j = 0; j < DMW; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
             float lsum = 0.f;
             // ldmatrix.trans row address: matrix lane/8 -> (+8 tokens if >= 2, +8 head-dim cols if odd)
             const int vrow = (lane & 7) + (lane >> 4) * 8;
             const int vhi = (lane >> 3) & 1;
             const int vx = lane & 7;
-            for (int st = warp; st < nst; st += C::NCW) {
+            for (int st = 0; st < nst; ++st) {
                 const uint32_t c = stage + st;
                 if (!acquire(c)) continue;
                 const int rows = min(C::STAGE_ROWS, w.n - st * C::STAGE_ROWS);
@@ -537,7 +684,8 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
                     const int vlo = rows - k0;              // valid tokens from k0 on (for masking)
                     const uint32_t base = sb + row_base(mt * 16 + vrow);
 #pragma unroll
-                    for (int dm = 0; dm < KS; ++dm) {
+                    for (int j = 0; j < DMW; ++j) {
+                        const int dm = warp * DMW + j;
                         uint32_t af[4];
                         const int cc = ((dm * 2) & 7) + vhi;
                         ldsm_x4_trans(base + (dm >> 2) * box_bytes + ((cc ^ vx) << 4), af[0], af[1], af[2], af[3]);
@@ -547,40 +695,66 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
                             af[2] = keep_pair(af[2], vlo - 8);
                             af[3] = keep_pair(af[3], vlo - 8);
                         }
-                        M::mma(oacc[dm], af, b0, b1);
-                        M::mma(oacc[dm], af, b0l, b1l);
+                        M::mma(oacc[j], af, b0, b1);
+                        M::mma(oacc[j], af, b0l, b1l);
                     }
                 }
                 release(c);
             }
             stage += nst;
-            // sum of p for query gid over the lanes holding it (tig = 0..3)
+            // sum of p for query gid over the lanes holding it (tig = 0..3): every
+            // warp formed the same sums in the same order
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-            if (tig == 0) wsum[warp * GC + gid] = lsum;
-            named_barrier(1, NCT);            // every warp is done with the scores: reuse them as `red`
-            // O^T fragment: (d = 16*dm + gid [+8], query 2*tig [+1])
-            float* rw = red + warp * GC * D;
+
+            // ---- epilogue: this warp's columns; O^T fragment (d = 16*dm + gid [+8], query 2*tig [+1])
+            const int qa = tig * 2, qc = tig * 2 + 1;
+            const float la = __shfl_sync(0xffffffffu, lsum, qa * 4);     // lane with gid == query
+            const float lc = __shfl_sync(0xffffffffu, lsum, qc * 4);
+            const float ma = __shfl_sync(0xffffffffu, mg, qa * 4);
+            const float mc = __shfl_sync(0xffffffffu, mg, qc * 4);
+            const bool single = (w.np == 1);
+            if (single) {
 #pragma unroll
-            for (int dm = 0; dm < KS; ++dm) {
-                const int d0 = dm * 16 + gid;
-                rw[(tig * 2) * D + d0] = oacc[dm][0];
-                rw[(tig * 2 + 1) * D + d0] = oacc[dm][1];
-                rw[(tig * 2) * D + d0 + 8] = oacc[dm][2];
-                rw[(tig * 2 + 1) * D + d0 + 8] = oacc[dm][3];
-            }
-            named_barrier(1, NCT);
-            if (ctid < GC) {
-                float m = wmax[ctid], l = 0.f;
-#pragma unroll
-                for (int ww = 0; ww < C::NCW; ++ww) {
-                    m = fmaxf(m, wmax[ww * GC + ctid]);
-                    l += wsum[ww * GC + ctid];
+                for (int j = 0; j < DMW; ++j) {
+                    const int d0 = (warp * DMW + j) * 16 + gid;
+                    if (qa < gq) {
+                        T* dst = outg + (row0 + qa) * D + d0;
+                        dst[0] = Tr::from_float(oacc[j][0] / la);
+                        dst[8] = Tr::from_float(oacc[j][2] / la);
+                    }
+                    if (qc < gq) {
+                        T* dst = outg + (row0 + qc) * D + d0;
+                        dst[0] = Tr::from_float(oacc[j][1] / lc);
+                        dst[8] = Tr::from_float(oacc[j][3] / lc);
+                    }
                 }
-                stat_m[ctid] = m;
-                stat_l[ctid] = l;
+            } else {
+                const int64_t pa_ = (row0 + qa) * a.max_partitions + w.p;
+                const int64_t pc_ = (row0 + qc) * a.max_partitions + w.p;
+#pragma unroll
+                for (int j = 0; j < DMW; ++j) {
+                    const int d0 = (warp * DMW + j) * 16 + gid;
+                    if (qa < gq) {
+                        a.part_o[pa_ * D + d0] = oacc[j][0];
+                        a.part_o[pa_ * D + d0 + 8] = oacc[j][2];
+                    }
+                    if (qc < gq) {
+                        a.part_o[pc_ * D + d0] = oacc[j][1];
+                        a.part_o[pc_ * D + d0 + 8] = oacc[j][3];
+                    }
+                }
+                if (warp == 0 && gid == 0) {
+                    if (qa < gq) {
+                        a.part_m[pa_] = ma;
+                        a.part_l[pa_] = la;
+                    }
+                    if (qc < gq) {
+                        a.part_m[pc_] = mc;
+                        a.part_l[pc_] = lc;
+                    }
+                }
             }
-            named_barrier(1, NCT);
         } else {
             constexpr int LS = C::LSTRIDE;
             const int row_in = lane / C::LPT;                 // row within a warp instruction
@@ -592,14 +766,16 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
                 float qf[GC][C::VEC];
 #pragma unroll
                 for (int g = 0; g < GC; ++g) {
-                    if (g < gq) {
-                        const uint4 u = __ldg(reinterpret_cast<const uint4*>(qg + (row0 + g) * D + chunk * C::VEC));
+                    if (have_q && g < gq) {
+                        const uint4 u = *reinterpret_cast<const uint4*>(qs + g * C::ROW_BYTES + chunk * 16);
                         Tr::unpack(u, qf[g]);
                     } else {
 #pragma unroll
                         for (int v = 0; v < C::VEC; ++v) qf[g][v] = 0.f;
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&item_empty[b]);
                 for (int st = warp; st < nst; st += C::NCW) {
                     const uint32_t c = stage + st;
                     if (!acquire(c)) continue;
@@ -698,35 +874,36 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
                 }
             }
             named_barrier(1, NCT);
-        }
 
-        // ---- epilogue: warps merged in a fixed order; final row or partition partials
-        const bool single = (w.np == 1);
-        volatile int* last_flag = abort_flag + 1;
-        for (int e = ctid; e < gq * D; e += NCT) {
-            const int g = e / D;
-            const int d = e - g * D;
-            float o = 0.f;
+            // ---- epilogue: warps merged in a fixed order; final row or partition partials
+            const bool single = (w.np == 1);
+            for (int e = ctid; e < gq * D; e += NCT) {
+                const int g = e / D;
+                const int d = e - g * D;
+                float o = 0.f;
 #pragma unroll
-            for (int ww = 0; ww < C::NCW; ++ww) o += red[(ww * GC + g) * D + d];
-            const int64_t row = row0 + g;
-            if (single) {
-                outg[row * D + d] = Tr::from_float(o / stat_l[g]);
-            } else {
-                const int64_t pidx = row * a.max_partitions + w.p;
-                a.part_o[pidx * D + d] = o;
-                if (d == 0) {
-                    a.part_m[pidx] = stat_m[g];
-                    a.part_l[pidx] = stat_l[g];
+                for (int ww = 0; ww < C::NCW; ++ww) o += red[(ww * GC + g) * D + d];
+                const int64_t row = row0 + g;
+                if (single) {
+                    outg[row * D + d] = Tr::from_float(o / stat_l[g]);
+                } else {
+                    const int64_t pidx = row * a.max_partitions + w.p;
+                    a.part_o[pidx * D + d] = o;
+                    if (d == 0) {
+                        a.part_m[pidx] = stat_m[g];
+                        a.part_l[pidx] = stat_l[g];
+                    }
                 }
             }
         }
-        if (!single && a.merge_count != nullptr) {
+
+        if (w.np != 1 && a.merge_count != nullptr) {
             // The CTA that finishes the last partition of this (sequence, kv head,
             // chunk) merges all of them: partials are published with a fence
             // before the counter increment; the last arriver fences and reads
             // them from L2.  Nothing waits; the merge order is fixed (partition 0
             // first), so the bits do not depend on which CTA ends up merging.
+            volatile int* last_flag = abort_flag + 1;
             __threadfence();
             named_barrier(1, NCT);
             if (ctid == 0) {
@@ -740,6 +917,8 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
                 merge_partitions<T, D>(a, row0, gq, w.np, stat_m, stat_l, warp, lane, ctid, C::NCW);
             }
         }
+        // every warp is done with this item's scores (and statistics) before the
+        // next item's phase 1 writes them
         named_barrier(1, NCT);
     }
     // this CTA's work is done: a dependent kernel (the reduce) may start launching;

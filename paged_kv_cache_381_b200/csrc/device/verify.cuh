@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(VerifyCfg<T, D>::THREADS, 2)
         const uint64_t policy = l2_policy_evict_first();
         uint32_t stage = 0;
         bool ok = true;
-        for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        for (int i = walk_first(); i < total && ok; i = walk_next(i)) {
             const WorkItem w = decode_item(a, i, lane == 0);
             if (w.n == 0) continue;
             const int nst = (w.n + C::STAGE_ROWS - 1) / C::STAGE_ROWS;
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(VerifyCfg<T, D>::THREADS, 2)
         if (lane == 0) mbar_arrive(&empty[c % C::NSTAGES]);
     };
 
-    for (int i = blockIdx.x; i < total; i += gridDim.x) {
+    for (int i = walk_first(); i < total; i = walk_next(i)) {
         const WorkItem w = decode_item(a, i, false);
         const int ctx = clamp_context(a, w.s, false);
         const int r0 = w.gc * C::ROWS;

@@ -197,62 +197,103 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         }
         const uint64_t policy = l2_policy_evict_first();
         uint32_t seq = 0;                                   // stream elements issued so far
+        uint32_t slot = 0;                                  // ring slot of the next element (seq % NSLOTS)
         uint32_t gch = 0;                                   // chunks of earlier items
-        // the last NSLOTS stream elements (oldest first): chunk index << 1 | is_v
-        uint32_t hist[C::NSLOTS];
-#pragma unroll
-        for (int k = 0; k < C::NSLOTS; ++k) hist[k] = 0;
+        // lane k < NSLOTS holds the tag (chunk index << 1 | is_v) of the element
+        // last loaded into slot k: the one NSLOTS back in the stream
+        uint32_t tag = 0;
         bool ok = true;
-        for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-            const WorkItem w = decode_item(a, i, lane == 0);
-            if (w.n == 0) continue;
-            const int nblk = (w.n + bs - 1) >> a.log2_bs;
-            const int32_t* trow = a.block_tables + (int64_t)w.s * a.max_blocks_per_seq + (w.t0 >> a.log2_bs);
-            __syncwarp();
-            for (int j = lane; j < nblk; j += 32) {
-                int32_t id = trow[j];
-                if (id < 0 || id >= a.num_blocks) {
-                    flag_error(PA_DEVERR_BLOCK_ID);
-                    id = 0;
-                }
-                tbl[j] = id;
-            }
-            __syncwarp();
-            const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
-            // K or V of chunk c into the next slot, once the products that read the
-            // slot's previous contents (the element NSLOTS back) are done
-            auto issue = [&](int c, bool is_v) -> bool {
-                if (seq >= (uint32_t)C::NSLOTS) {
-                    const uint32_t g = hist[0] >> 1;
-                    uint64_t* done = (hist[0] & 1u) ? &o_full[g % C::NPH] : &s_full[g % C::NPH];
-                    if (!mbar_wait(done, (g / C::NPH) & 1u, abort_flag)) return false;
-                }
-                const int slot = seq % C::NSLOTS;
-                const int rows = min(C::CHUNK, w.n - c * C::CHUNK);
-                const int nbk = (rows + bs - 1) >> a.log2_bs;          // whole blocks
-                if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbk * C::NH * box_bytes));
-                __syncwarp();
-                if (lane < nbk * C::NH) {
-                    static_assert(C::NH <= 2, "one or two slices");
-                    const int half = C::NH == 2 && lane >= nbk ? 1 : 0;  // slice
-                    const int b = lane - half * nbk;                    // block within the chunk
-                    const int phys = tbl[((c * C::CHUNK) >> a.log2_bs) + b];
-                    tma_load_3d(smem + slot * C::SLOT_BYTES + half * C::SLICE_BYTES + b * box_bytes,
-                                is_v ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
-                                half * C::BOX_ELEMS, w.h, phys * bs, &full[slot], policy);
-                }
+        // Block ids of an item, requested into registers (lane j holds entries
+        // j, j + 32, ...) one item before they are needed.
+        constexpr int TPL = C::MAX_TABLE / 32;
+        auto request_ids = [&](const WorkItem& x, int32_t (&ids)[TPL]) {
+            const int nblk = (x.n + bs - 1) >> a.log2_bs;
+            const int32_t* trow = a.block_tables + (int64_t)x.s * a.max_blocks_per_seq + (x.t0 >> a.log2_bs);
 #pragma unroll
-                for (int k = 0; k + 1 < C::NSLOTS; ++k) hist[k] = hist[k + 1];
-                hist[C::NSLOTS - 1] = ((gch + (uint32_t)c) << 1) | (is_v ? 1u : 0u);
-                ++seq;
-                return true;
-            };
-            if (!(ok = issue(0, false))) break;
-            for (int c = 0; c < nc && ok; ++c) {
-                if (c + 1 < nc && !(ok = issue(c + 1, false))) break;
-                ok = issue(c, true);
+            for (int k = 0; k < TPL; ++k) {
+                const int j = lane + 32 * k;
+                ids[k] = j < nblk ? trow[j] : 0;
             }
-            gch += nc;
+        };
+        int i = walk_first();
+        WorkItem w{};
+        int32_t ids[TPL];
+        if (i < total) {
+            w = decode_item(a, i, lane == 0);
+            request_ids(w, ids);
+        }
+        while (i < total && ok) {
+            // the next item is looked up (its ids requested) once this item's first
+            // element is issued, while the rest wait for ring slots
+            const int inext = walk_next(i);
+            WorkItem wn{};
+            int32_t idn[TPL];
+            bool looked = false;
+            auto look_ahead = [&]() {
+                if (looked) return;
+                looked = true;
+                if (inext < total) {
+                    wn = decode_item(a, inext, lane == 0);
+                    request_ids(wn, idn);
+                }
+            };
+            if (w.n > 0) {
+                const int nblk = (w.n + bs - 1) >> a.log2_bs;
+                __syncwarp();               // the previous item's table reads are done
+#pragma unroll
+                for (int kk = 0; kk < TPL; ++kk) {
+                    const int j = lane + 32 * kk;
+                    if (j < nblk) {
+                        int32_t id = ids[kk];
+                        if (id < 0 || id >= a.num_blocks) {
+                            flag_error(PA_DEVERR_BLOCK_ID);
+                            id = 0;
+                        }
+                        tbl[j] = id;
+                    }
+                }
+                __syncwarp();
+                const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
+                // K or V of chunk c into the next slot, once the products that read the
+                // slot's previous contents (the element NSLOTS back) are done
+                auto issue = [&](int c, bool is_v) -> bool {
+                    if (seq >= (uint32_t)C::NSLOTS) {
+                        const uint32_t prev = __shfl_sync(0xffffffffu, tag, (int)slot);
+                        const uint32_t g = prev >> 1;
+                        uint64_t* done = (prev & 1u) ? &o_full[g % C::NPH] : &s_full[g % C::NPH];
+                        if (!__all_sync(0xffffffffu, mbar_wait(done, (g / C::NPH) & 1u, abort_flag))) return false;
+                    }
+                    const int rows = min(C::CHUNK, w.n - c * C::CHUNK);
+                    const int nbk = (rows + bs - 1) >> a.log2_bs;          // whole blocks
+                    if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)(nbk * C::NH * box_bytes));
+                    __syncwarp();
+                    if (lane < nbk * C::NH) {
+                        static_assert(C::NH <= 2, "one or two slices");
+                        const int half = C::NH == 2 && lane >= nbk ? 1 : 0;  // slice
+                        const int b = lane - half * nbk;                    // block within the chunk
+                        const int phys = tbl[((c * C::CHUNK) >> a.log2_bs) + b];
+                        tma_load_3d(smem + slot * C::SLOT_BYTES + half * C::SLICE_BYTES + b * box_bytes,
+                                    is_v ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
+                                    half * C::BOX_ELEMS, w.h, phys * bs, &full[slot], policy);
+                    }
+                    if (lane == (int)slot) tag = ((gch + (uint32_t)c) << 1) | (is_v ? 1u : 0u);
+                    slot = slot + 1 == (uint32_t)C::NSLOTS ? 0u : slot + 1;
+                    ++seq;
+                    return true;
+                };
+                ok = issue(0, false);
+                look_ahead();
+                for (int c = 0; c < nc && ok; ++c) {
+                    if (c + 1 < nc && !(ok = issue(c + 1, false))) break;
+                    ok = issue(c, true);
+                }
+                gch += nc;
+            }
+            look_ahead();
+            i = inext;
+            w = wn;
+#pragma unroll
+            for (int kk = 0; kk < TPL; ++kk) ids[kk] = idn[kk];
         }
         if (!ok) {
             if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
@@ -357,7 +398,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             tc::fence_after_sync();
             return issue_pv(pos, c, n, g, c == 0);
         };
-        for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        for (int i = walk_first(); i < total && ok; i = walk_next(i)) {
             const WorkItem w = decode_item(a, i, false);
             if (w.n == 0) continue;
             const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
@@ -472,8 +513,9 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         };
         bool ok = true;
         int staged = -1;                                 // item whose Q tile is already written
-        for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-            const WorkItem w = decode_item(a, i, false);
+        WorkItem staged_w{};                             // ... and its descriptor
+        for (int i = walk_first(); i < total && ok; i = walk_next(i)) {
+            const WorkItem w = staged == i ? staged_w : decode_item(a, i, false);
             const int ctx = clamp_context(a, w.s, false);
             if (w.n == 0) {                              // empty context: zero rows
                 const int nr = min(C::M, R - w.gc * C::M);
@@ -605,12 +647,13 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             // ---- the next item's Q tile now, so that its first S products run while
             // this item's epilogue does
             {
-                const int inext = i + gridDim.x;
+                const int inext = walk_next(i);
                 if (inext < total) {
                     const WorkItem wn = decode_item(a, inext, false);
                     if (wn.n > 0) {
                         if (!(ok = stage_q(wn, clamp_context(a, wn.s, false)))) break;
                         staged = inext;
+                        staged_w = wn;
                     }
                 }
             }

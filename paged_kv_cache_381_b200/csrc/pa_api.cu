@@ -11,6 +11,8 @@
 #include <utility>
 #include <vector>
 
+// this unit holds the device error word (device/common.cuh) and reads it
+#define PA_ERROR_WORD_UNIT 1
 #include "device/cache_ops.cuh"
 #include "device/decode.cuh"
 #include "device/split_merge.cuh"
@@ -141,9 +143,37 @@ pa_status check_cache_desc(const pa_cache_desc* c) {
     return PA_OK;
 }
 
+// ------------------------------------------------------------ cache write
+// Checks of pa_cache_write (all before any launch); fills the kernel arguments.
+pa_status write_args(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                     int num_tokens, const pa_cache_desc* cache, pa_dev::WriteArgs* w) {
+    pa_status st = check_cache_desc(cache);
+    if (st != PA_OK) return st;
+    if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+    const int64_t row_bytes = (int64_t)cache->num_kv_heads * cache->head_dim * elem_bytes(cache->dtype);
+    w->k = static_cast<const uint4*>(k);
+    w->v = static_cast<const uint4*>(v);
+    w->k_cache = static_cast<uint4*>(k_cache);
+    w->v_cache = static_cast<uint4*>(v_cache);
+    w->slot_mapping = slot_mapping;
+    w->num_tokens = num_tokens;
+    w->row_vecs = (int)(row_bytes / 16);
+    w->num_slots = (int64_t)cache->num_blocks * cache->block_size;
+    return PA_OK;
+}
+
+// CTAs of 256 threads for a cache write: one thread per 16-byte vector, at most 65,535 CTAs
+unsigned write_grid(const pa_dev::WriteArgs& w) {
+    const int64_t threads = (int64_t)w.num_tokens * w.row_vecs;
+    return (unsigned)std::max<int64_t>(1, std::min<int64_t>((threads + 255) / 256, 65535));
+}
+
 // ------------------------------------------------------------ workspace
 struct WsLayout {
-    size_t plan, count, counters, m, l, o, total;
+    size_t plan, count, split, counters, m, l, o, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -153,8 +183,10 @@ WsLayout ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t maxP) {
     size_t off = 0;
     w.plan = off;
     off = align256(off + (size_t)(S * maxP) * sizeof(int2));
-    w.count = off;
-    off = align256(off + sizeof(int));
+    w.count = off;                                      // pairs in the plan, split sequences
+    off = align256(off + 2 * sizeof(int));
+    w.split = off;                                      // the split sequences
+    off = align256(off + (size_t)S * sizeof(int));
     w.counters = off;                                   // fused-merge counters, <= S * Hq of them
     off = align256(off + (size_t)(S * Hq) * sizeof(int));
     w.m = off;
@@ -176,7 +208,7 @@ int64_t partitions_for(int64_t ctx, int64_t P) { return ctx <= P ? 1 : (ctx + P 
 // ------------------------------------------------------------ decode launch
 std::atomic<int> g_decode_math{PA_MATH_AUTO};
 std::atomic<int> g_split_merge{PA_MERGE_KERNEL};
-constexpr int kMaxPartitions = 4096;    // plan kernel: 2 * kMaxPartitions ints of shared memory
+constexpr int kMaxPartitions = 4096;    // partitions per sequence
 
 // ---------------------------------------------------------------- TMA maps
 // cuTensorMapEncodeTiled is reached through the runtime's driver entry point,
@@ -272,18 +304,32 @@ pa_status dispatch_head_dim(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, 
                    : dispatch_group<T, 128>(a, tk, tv, gc, tensor, pair_upper, st);
 }
 
-template <typename T>
-pa_status launch_reduce(const pa_dev::DecodeArgs& a, int D, cudaStream_t stream) {
-    // persistent: the number of split rows is known only on the device (plan)
+template <typename T, int D>
+pa_status launch_reduce_d(const pa_dev::DecodeArgs& a, cudaStream_t stream) {
+    // persistent, one CTA per resident slot: the number of split rows is known
+    // only on the device (plan)
+    auto kern = pa_dev::reduce_kernel<T, D>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    static std::atomic<int> occ_of[kMaxDevices];
+    const int threads = pa_dev::kReduceWarps * 32;
+    int occ = dev < kMaxDevices ? occ_of[dev].load() : 0;
+    if (occ <= 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, 0) != cudaSuccess || occ <= 0)
+            return PA_ERR_CUDA;
+        if (dev < kMaxDevices) occ_of[dev].store(occ);
+    }
     const int64_t rows = (int64_t)a.num_seqs * a.num_heads;
     const int64_t blocks_needed = (rows + pa_dev::kReduceWarps - 1) / pa_dev::kReduceWarps;
-    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)device_sms(dev) * 4));
-    const dim3 block(pa_dev::kReduceWarps * 32);
+    const unsigned grid =
+        (unsigned)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)device_sms(dev) * occ));
     LaunchScope scope(PA_KERNEL_REDUCE, stream);
-    if (D == 64) return launch_dependent(pa_dev::reduce_kernel<T, 64>, dim3(grid), block, 0, stream, a);
-    return launch_dependent(pa_dev::reduce_kernel<T, 128>, dim3(grid), block, 0, stream, a);
+    return launch_dependent(kern, dim3(grid), dim3(threads), 0, stream, a);
+}
+
+template <typename T>
+pa_status launch_reduce(const pa_dev::DecodeArgs& a, int D, cudaStream_t stream) {
+    return D == 64 ? launch_reduce_d<T, 64>(a, stream) : launch_reduce_d<T, 128>(a, stream);
 }
 
 template <typename T, int D>
@@ -369,17 +415,129 @@ int query_chunk(int group, bool tensor) {
 
 namespace {
 
+// pa_decode, optionally preceded by a cache write (`wr`, pa_write_decode): all
+// checks first, then the launches -- the write and the plan in one kernel when
+// the batch is split, the write kernel alone when it is not.
+pa_status decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, float scale, int block_size, int num_kv_heads, int num_seqs,
+                      int num_heads, int head_dim, int max_blocks_per_seq, int max_context_len, int num_blocks,
+                      pa_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes, void* stream,
+                      const pa_dev::WriteArgs* wr) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+        max_context_len < 0 || !valid_dtype(dtype) || !std::isfinite(scale))
+        return PA_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    const int P = resolve_partition(partition_size);
+    if (!valid_partition(P)) return PA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto write_alone = [&]() -> pa_status {
+        LaunchScope scope(PA_KERNEL_CACHE_WRITE, s);
+        pa_dev::cache_write_kernel<<<write_grid(*wr), 256, 0, s>>>(*wr);
+        return launch_status();
+    };
+    if (num_seqs == 0) return wr ? write_alone() : PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+
+    if ((int64_t)num_blocks * block_size > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    const int64_t table_cap = (int64_t)max_blocks_per_seq * block_size;
+    const int64_t cap = std::min<int64_t>(max_context_len, table_cap);
+    if (cap > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
+    const int64_t maxP = partitions_for(cap, P);
+    if (maxP > kMaxPartitions) return PA_ERR_UNSUPPORTED;
+    const int group = num_heads / num_kv_heads;
+    const int math = g_decode_math.load(std::memory_order_relaxed);
+    const bool tensor = dtype != PA_F32 && math != PA_MATH_SIMT;
+    const int gc = query_chunk(group, tensor);
+    const int n_gchunks = (group + gc - 1) / gc;
+    if ((int64_t)num_seqs * maxP * num_kv_heads * n_gchunks > INT32_MAX) return PA_ERR_INVALID_ARG;
+
+    pa_dev::DecodeArgs a{};
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.num_seqs = num_seqs;
+    a.num_heads = num_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.group = group;
+    a.n_gchunks = n_gchunks;
+    a.log2_bs = block_size == 8 ? 3 : block_size == 16 ? 4 : 5;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.ctx_cap = (int)cap;
+    a.num_blocks = num_blocks;
+    a.partition_size = P;
+    a.max_partitions = (int)maxP;
+    a.num_queries = 1;
+
+    const int box_rows = block_size;          // one TMA box = one block of one kv head, one 128-byte slice
+    CUtensorMap tk, tv;
+    if (!encode_pool_map(&tk, k_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, box_rows) ||
+        !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, box_rows))
+        return PA_ERR_CUDA;
+    if (maxP > 1) {
+        const WsLayout L = ws_layout(num_seqs, num_heads, head_dim, maxP);
+        if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return PA_ERR_INVALID_ARG;
+        char* ws = static_cast<char*>(workspace);
+        a.plan = reinterpret_cast<const int2*>(ws + L.plan);
+        a.plan_count = reinterpret_cast<const int*>(ws + L.count);
+        a.split_seqs = reinterpret_cast<const int*>(ws + L.split);
+        a.part_m = reinterpret_cast<float*>(ws + L.m);
+        a.part_l = reinterpret_cast<float*>(ws + L.l);
+        a.part_o = reinterpret_cast<float*>(ws + L.o);
+        const bool fused = g_split_merge.load(std::memory_order_relaxed) == PA_MERGE_FUSED;
+        int* counters = reinterpret_cast<int*>(ws + L.counters);
+        a.merge_count = fused ? counters : nullptr;
+        const int num_counters = fused ? num_seqs * num_kv_heads * n_gchunks : 0;
+        int2* plan = reinterpret_cast<int2*>(ws + L.plan);
+        int* count = reinterpret_cast<int*>(ws + L.count);
+        int* split = reinterpret_cast<int*>(ws + L.split);
+        if (wr) {
+            LaunchScope scope(PA_KERNEL_WRITE_PLAN, s);
+            const unsigned wb = write_grid(*wr);
+            pa_dev::write_plan_kernel<<<wb + 1, 256, 0, s>>>(*wr, (int)wb, a, plan, count, split, counters,
+                                                             num_counters);
+            if (launch_status() != PA_OK) return PA_ERR_CUDA;
+        } else {
+            LaunchScope scope(PA_KERNEL_PLAN, s);
+            const int threads = std::min(1024, std::max(32, (num_seqs + 31) / 32 * 32));
+            if (launch_dependent(pa_dev::plan_kernel, dim3(1), dim3(threads), 0, s, a, plan, count, split, counters,
+                                 num_counters) != PA_OK)
+                return PA_ERR_CUDA;
+        }
+    } else if (wr && write_alone() != PA_OK) {
+        return PA_ERR_CUDA;
+    }
+    const int64_t pair_upper = (int64_t)num_seqs * maxP;
+    pa_status st;
+    switch (dtype) {
+        case PA_F32: st = dispatch_head_dim<float>(a, tk, tv, head_dim, gc, false, pair_upper, s); break;
+        case PA_F16: st = dispatch_head_dim<__half>(a, tk, tv, head_dim, gc, tensor, pair_upper, s); break;
+        default: st = dispatch_head_dim<__nv_bfloat16>(a, tk, tv, head_dim, gc, tensor, pair_upper, s); break;
+    }
+    if (st != PA_OK || maxP <= 1 || a.merge_count != nullptr) return st;
+    switch (dtype) {
+        case PA_F32: return launch_reduce<float>(a, head_dim, s);
+        case PA_F16: return launch_reduce<__half>(a, head_dim, s);
+        default: return launch_reduce<__nv_bfloat16>(a, head_dim, s);
+    }
+}
+
+
 pa_status step_compute(const pa_step_device* d, void* k_cache, void* v_cache, const pa_step_shape* sh, void* stream) {
     pa_cache_desc cd{sh->num_blocks, sh->block_size, sh->num_kv_heads, sh->head_dim, sh->dtype};
     pa_status st = PA_OK;
     if (sh->num_cow > 0 && (st = pa_copy_blocks(k_cache, v_cache, d->cow_pairs, sh->num_cow, &cd, stream)) != PA_OK)
         return st;
-    if ((st = pa_cache_write(d->k, d->v, k_cache, v_cache, d->slot_mapping, sh->num_tokens, &cd, stream)) != PA_OK)
-        return st;
-    return pa_decode(d->out, d->q, k_cache, v_cache, d->block_tables, d->context_lens, sh->scale, sh->block_size,
-                     sh->num_kv_heads, sh->num_seqs, sh->num_heads, sh->head_dim, sh->max_blocks_per_seq,
-                     sh->max_context_len, sh->num_blocks, sh->dtype, sh->partition_size, d->workspace,
-                     d->workspace_bytes, stream);
+    return pa_write_decode(d->k, d->v, d->slot_mapping, sh->num_tokens, d->out, d->q, k_cache, v_cache,
+                           d->block_tables, d->context_lens, sh->scale, sh->block_size, sh->num_kv_heads,
+                           sh->num_seqs, sh->num_heads, sh->head_dim, sh->max_blocks_per_seq, sh->max_context_len,
+                           sh->num_blocks, sh->dtype, sh->partition_size, d->workspace, d->workspace_bytes, stream);
 }
 
 bool step_inputs(const pa_step_host* h, const pa_step_device* d, const pa_step_shape* sh, cudaStream_t s) {
@@ -489,22 +647,12 @@ pa_status pa_profile_end(double* total_ms, int64_t* launches) {
 
 pa_status pa_cache_write(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
                          int num_tokens, const pa_cache_desc* cache, void* stream) {
-    pa_status st = check_cache_desc(cache);
-    if (st != PA_OK) return st;
-    if (num_tokens < 0) return PA_ERR_INVALID_ARG;
-    if (num_tokens == 0) return PA_OK;
-    if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
-    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
-    const int64_t row_bytes = (int64_t)cache->num_kv_heads * cache->head_dim * elem_bytes(cache->dtype);
-    const int row_vecs = (int)(row_bytes / 16);
-    const int64_t num_slots = (int64_t)cache->num_blocks * cache->block_size;
-    const int64_t threads = (int64_t)num_tokens * row_vecs;
-    const unsigned grid = (unsigned)std::min<int64_t>((threads + 255) / 256, 65535);
+    pa_dev::WriteArgs w{};
+    const pa_status st = write_args(k, v, k_cache, v_cache, slot_mapping, num_tokens, cache, &w);
+    if (st != PA_OK || num_tokens == 0) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     LaunchScope scope(PA_KERNEL_CACHE_WRITE, s);
-    pa_dev::cache_write_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
-                                                     static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
-                                                     slot_mapping, num_tokens, row_vecs, num_slots);
+    pa_dev::cache_write_kernel<<<write_grid(w), 256, 0, s>>>(w);
     return launch_status();
 }
 
@@ -567,93 +715,23 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     const int32_t* context_lens, float scale, int block_size, int num_kv_heads, int num_seqs,
                     int num_heads, int head_dim, int max_blocks_per_seq, int max_context_len, int num_blocks,
                     pa_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes, void* stream) {
-    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
-        max_context_len < 0 || !valid_dtype(dtype) || !std::isfinite(scale))
-        return PA_ERR_INVALID_ARG;
-    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
-    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
-    const int P = resolve_partition(partition_size);
-    if (!valid_partition(P)) return PA_ERR_INVALID_ARG;
-    if (num_seqs == 0) return PA_OK;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size, num_kv_heads, num_seqs,
+                       num_heads, head_dim, max_blocks_per_seq, max_context_len, num_blocks, dtype, partition_size,
+                       workspace, workspace_bytes, stream, nullptr);
+}
 
-    if ((int64_t)num_blocks * block_size > INT32_MAX) return PA_ERR_UNSUPPORTED;
-    const int64_t table_cap = (int64_t)max_blocks_per_seq * block_size;
-    const int64_t cap = std::min<int64_t>(max_context_len, table_cap);
-    if (cap > INT32_MAX / 2) return PA_ERR_INVALID_ARG;
-    const int64_t maxP = partitions_for(cap, P);
-    if (maxP > kMaxPartitions) return PA_ERR_UNSUPPORTED;
-    const int group = num_heads / num_kv_heads;
-    const int math = g_decode_math.load(std::memory_order_relaxed);
-    const bool tensor = dtype != PA_F32 && math != PA_MATH_SIMT;
-    const int gc = query_chunk(group, tensor);
-    const int n_gchunks = (group + gc - 1) / gc;
-    if ((int64_t)num_seqs * maxP * num_kv_heads * n_gchunks > INT32_MAX) return PA_ERR_INVALID_ARG;
-
-    pa_dev::DecodeArgs a{};
-    a.out = out;
-    a.q = q;
-    a.k_cache = k_cache;
-    a.v_cache = v_cache;
-    a.block_tables = block_tables;
-    a.context_lens = context_lens;
-    a.scale_log2 = scale * 1.4426950408889634f;
-    a.num_seqs = num_seqs;
-    a.num_heads = num_heads;
-    a.num_kv_heads = num_kv_heads;
-    a.group = group;
-    a.n_gchunks = n_gchunks;
-    a.log2_bs = block_size == 8 ? 3 : block_size == 16 ? 4 : 5;
-    a.max_blocks_per_seq = max_blocks_per_seq;
-    a.ctx_cap = (int)cap;
-    a.num_blocks = num_blocks;
-    a.partition_size = P;
-    a.max_partitions = (int)maxP;
-    a.num_queries = 1;
-
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (maxP > 1) {
-        const WsLayout L = ws_layout(num_seqs, num_heads, head_dim, maxP);
-        if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-            return PA_ERR_INVALID_ARG;
-        char* ws = static_cast<char*>(workspace);
-        a.plan = reinterpret_cast<const int2*>(ws + L.plan);
-        a.plan_count = reinterpret_cast<const int*>(ws + L.count);
-        a.part_m = reinterpret_cast<float*>(ws + L.m);
-        a.part_l = reinterpret_cast<float*>(ws + L.l);
-        a.part_o = reinterpret_cast<float*>(ws + L.o);
-        const bool fused = g_split_merge.load(std::memory_order_relaxed) == PA_MERGE_FUSED;
-        int* counters = reinterpret_cast<int*>(ws + L.counters);
-        a.merge_count = fused ? counters : nullptr;
-        {
-            LaunchScope scope(PA_KERNEL_PLAN, s);
-            const int threads = std::min(1024, std::max(32, (num_seqs + 31) / 32 * 32));
-            const int num_counters = fused ? num_seqs * num_kv_heads * n_gchunks : 0;
-            if (launch_dependent(pa_dev::plan_kernel, dim3(1), dim3(threads), 2 * (maxP + 1) * sizeof(int), s, a,
-                                 reinterpret_cast<int2*>(ws + L.plan), reinterpret_cast<int*>(ws + L.count),
-                                 counters, num_counters) != PA_OK)
-                return PA_ERR_CUDA;
-        }
-    }
-    const int box_rows = block_size;          // one TMA box = one block of one kv head, one 128-byte slice
-    CUtensorMap tk, tv;
-    if (!encode_pool_map(&tk, k_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, box_rows) ||
-        !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, box_rows))
-        return PA_ERR_CUDA;
-    const int64_t pair_upper = (int64_t)num_seqs * maxP;
-    pa_status st;
-    switch (dtype) {
-        case PA_F32: st = dispatch_head_dim<float>(a, tk, tv, head_dim, gc, false, pair_upper, s); break;
-        case PA_F16: st = dispatch_head_dim<__half>(a, tk, tv, head_dim, gc, tensor, pair_upper, s); break;
-        default: st = dispatch_head_dim<__nv_bfloat16>(a, tk, tv, head_dim, gc, tensor, pair_upper, s); break;
-    }
-    if (st != PA_OK || maxP <= 1 || a.merge_count != nullptr) return st;
-    switch (dtype) {
-        case PA_F32: return launch_reduce<float>(a, head_dim, s);
-        case PA_F16: return launch_reduce<__half>(a, head_dim, s);
-        default: return launch_reduce<__nv_bfloat16>(a, head_dim, s);
-    }
+pa_status pa_write_decode(const void* k, const void* v, const int64_t* slot_mapping, int num_tokens, void* out,
+                          const void* q, void* k_cache, void* v_cache, const int32_t* block_tables,
+                          const int32_t* context_lens, float scale, int block_size, int num_kv_heads, int num_seqs,
+                          int num_heads, int head_dim, int max_blocks_per_seq, int max_context_len, int num_blocks,
+                          pa_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes, void* stream) {
+    const pa_cache_desc cd{num_blocks, block_size, num_kv_heads, head_dim, dtype};
+    pa_dev::WriteArgs w{};
+    const pa_status st = write_args(k, v, k_cache, v_cache, slot_mapping, num_tokens, &cd, &w);
+    if (st != PA_OK) return st;
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size, num_kv_heads, num_seqs,
+                       num_heads, head_dim, max_blocks_per_seq, max_context_len, num_blocks, dtype, partition_size,
+                       workspace, workspace_bytes, stream, num_tokens > 0 ? &w : nullptr);
 }
 
 int pa_verify_partition_size(int num_seqs, int num_queries, int num_heads, int num_kv_heads, int partition_size) {
@@ -734,15 +812,17 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
         char* ws = static_cast<char*>(workspace);
         a.plan = reinterpret_cast<const int2*>(ws + L.plan);
         a.plan_count = reinterpret_cast<const int*>(ws + L.count);
+        a.split_seqs = reinterpret_cast<const int*>(ws + L.split);
         a.part_m = reinterpret_cast<float*>(ws + L.m);
         a.part_l = reinterpret_cast<float*>(ws + L.l);
         a.part_o = reinterpret_cast<float*>(ws + L.o);
         a.merge_count = nullptr;
         LaunchScope scope(PA_KERNEL_PLAN, s);
         const int threads = std::min(1024, std::max(32, (num_seqs + 31) / 32 * 32));
-        if (launch_dependent(pa_dev::plan_kernel, dim3(1), dim3(threads), 2 * (maxP + 1) * sizeof(int), s, a,
+        if (launch_dependent(pa_dev::plan_kernel, dim3(1), dim3(threads), 0, s, a,
                              reinterpret_cast<int2*>(ws + L.plan), reinterpret_cast<int*>(ws + L.count),
-                             reinterpret_cast<int*>(ws + L.counters), 0) != PA_OK)
+                             reinterpret_cast<int*>(ws + L.split), reinterpret_cast<int*>(ws + L.counters),
+                             0) != PA_OK)
             return PA_ERR_CUDA;
     }
     CUtensorMap tk, tv;
