@@ -70,3 +70,24 @@ def test_verify_bytes_and_flops_hand_example():
     assert bench.verify_kernel_bytes(cfg, lens, 16, 2) == 35840 + 3072 + 1024 + 10560 + 48
     assert bench.verify_flops(cfg, lens, 2) == 4 * 64 * 4 * (19 + 39 + 79)
     assert bench.verify_kernel_bytes(cfg, lens, 16, 1) == bench.decode_kernel_bytes(cfg, lens, 16)
+
+
+def test_reference_arm_reports_the_native_config(tmp_path):
+    """The reference arm prints the native arm's config object (same keys and
+    values for the same workload), so the two lines describe one workload."""
+    import json
+    import subprocess
+    import sys
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          "tiny", "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr
+    line = json.loads(res.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    cfg = bench.wl.CONFIGS["tiny"]
+    lens = bench.wl.context_lengths(cfg, bench.wl.rng(0))
+
+    class A:
+        workload, math, merge, partition_size = "tiny", "auto", "kernel", 0
+    assert line["config"] == bench.workload_config(A, cfg, lens, cfg.partition_size, 1)
+    assert line["config"]["kv_bytes_per_step"] == bench.kv_bytes(cfg, lens)
+    assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}

@@ -4,7 +4,7 @@ Tolerances (stated by the task's contract for this path): fp16 / bf16 outputs
 within 2e-3 absolute + 1e-2 relative of the unrounded fp64 oracle; fp32 within
 1e-5 absolute + 1e-5 relative.  Cache writes, block copies and bookkeeping are
 bit-exact.  Full-size workloads (the bench's launch configuration) are checked
-on sampled (sequence, head) rows computed one by one by the oracle.
+on every (sequence, head) row, element by element.
 """
 
 import numpy as np
@@ -16,6 +16,7 @@ from paged_kv_cache_381_b200 import workloads as wl
 from paged_kv_cache_381_b200.batch import PagedBatch
 from tests.gpu_harness import (DeviceBatch, assert_cache_exact, assert_close, free_order_for, oracle_outputs,
                                to_device, to_storage, TORCH_DTYPE)
+from tests.full_size import assert_every_row, oracle_all_rows
 from oracle import attention as oa
 from oracle.numerics import widen
 
@@ -132,6 +133,53 @@ def test_split_vs_single_pass(math_path, merge_mode):
     assert_close(single, ref, "bf16", "single")
     assert_close(split, ref, "bf16", "split")
     assert_close(split, widen(single, "bf16"), "bf16", "split vs single")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("P", [64, 0])
+def test_write_decode_equals_write_then_decode(dtype, P, math_path, merge_mode):
+    """pa_write_decode (the write and the plan in one kernel when the batch is
+    split) gives the bits of pa_cache_write followed by pa_decode: the same
+    pools and the same outputs, and those match the oracle."""
+    if dtype == "f32" and math_path != "auto":
+        pytest.skip("fp32 always uses the CUDA-core path")
+    cfg = _grid_cfg(dtype, 128, 16, 4)
+    lens = (0, 1, 33, 300, 700, 1100) if P else (0, 1, 33, 300, 511, 17)
+    inp = wl.make_decode_inputs(cfg, 60 + P, context_lens=lens)
+    a = DeviceBatch(inp)
+    a.step_write()
+    out_a = a.decode(partition_size=P)
+    b = DeviceBatch(inp)
+    # the same rows and slots as DeviceBatch.step_write, through the fused call
+    S = len(b.lens)
+    hkv, d = cfg.num_kv_heads, cfg.head_dim
+    sd = inp.k_hist[0].dtype
+    slots = np.full(S, -1, dtype=np.int64)
+    k = np.zeros((S, hkv, d), dtype=sd)
+    v = np.zeros((S, hkv, d), dtype=sd)
+    for s_ in range(S):
+        n = int(b.lens[s_])
+        if n > 0:
+            slots[s_] = b.bm.slots(s_, n - 1, 1)[0]
+            k[s_] = inp.k_hist[s_][n - 1]
+            v[s_] = inp.v_hist[s_][n - 1]
+    out_b = torch.empty_like(b.q)
+    n0 = pa.launch_count()
+    pa.pa_write_decode(to_device(k, dtype), to_device(v, dtype), torch.from_numpy(slots).cuda(), out_b, b.q,
+                       b.k_cache, b.v_cache, b.block_tables, b.context_lens, cfg.scale,
+                       max_context_len=int(b.lens.max()), partition_size=P)
+    torch.cuda.synchronize()
+    launches = pa.launch_count() - n0
+    _no_device_error()
+    split = max(lens) > (P or 512)
+    fused = merge_mode == "fused"
+    # split: write+plan, decode (+ reduce); one partition: write, decode
+    assert launches == ((2 if fused else 3) if split else 2)
+    assert np.array_equal(to_storage(out_a, dtype), to_storage(out_b, dtype))
+    assert np.array_equal(to_storage(a.k_cache, dtype), to_storage(b.k_cache, dtype))
+    assert np.array_equal(to_storage(a.v_cache, dtype), to_storage(b.v_cache, dtype))
+    assert_close(to_storage(out_b, dtype), oracle_outputs(inp), dtype, f"write_decode {dtype} P{P}")
+    assert_cache_exact(b)
 
 
 def test_cache_write_bit_exact_all_dtypes():
@@ -380,19 +428,12 @@ def test_launch_count_and_profile(merge_mode):
     assert prof["reduce"][1] == (0 if fused else 1)
 
 
-# -- full-size workloads, sampled rows, in the bench's launch configuration -------
-
-def _sample_rows(lens, Hq, k, seed):
-    r = np.random.default_rng(seed)
-    S = len(lens)
-    rows = {(int(np.argmax(lens)), 0), (int(np.argmax(lens)), Hq - 1), (int(np.argmin(lens)), Hq // 2)}
-    while len(rows) < k:
-        rows.add((int(r.integers(S)), int(r.integers(Hq))))
-    return sorted(rows)
-
+# -- full-size workloads, every row, in the bench's launch configuration ----------
 
 @pytest.mark.parametrize("name", ["7b", "70b", "long"])
-def test_full_size_sampled(name, math_path, merge_mode):
+def test_full_size_every_row(name, math_path, merge_mode):
+    """Every (sequence, head) row of the full-size batch against the fp64
+    oracle, element by element."""
     cfg = wl.CONFIGS[name]
     d = wl.draw_device(cfg, 0)
     batch = PagedBatch(d.k_hist, d.v_hist, d.offsets, d.context_lens, d.num_blocks, cfg.block_size,
@@ -402,16 +443,5 @@ def test_full_size_sampled(name, math_path, merge_mode):
     batch.decode(out, d.q, cfg.scale, partition_size=cfg.partition_size)
     torch.cuda.synchronize()
     _no_device_error()
-    rows = _sample_rows(d.context_lens, cfg.num_heads, 40, 1)
-    G = cfg.num_heads // cfg.num_kv_heads
-    got = to_storage(out, cfg.dtype)
-    ref = []
-    for s, h in rows:
-        a, e = int(d.offsets[s]), int(d.offsets[s + 1])
-        g = h // G
-        K = widen(to_storage(d.k_hist[a:e, g], cfg.dtype), cfg.dtype)
-        V = widen(to_storage(d.v_hist[a:e, g], cfg.dtype), cfg.dtype)
-        ref.append(oa.attend(widen(to_storage(d.q[s, h], cfg.dtype), cfg.dtype), K, V, cfg.scale))
-    assert_close(np.stack([got[s, h] for s, h in rows]), np.stack(ref), cfg.dtype, name)
-    # properties that hold for every row: finite, and bounded by the value range
-    assert torch.isfinite(out.float()).all()
+    ref = oracle_all_rows(d.q, d, cfg)
+    assert_every_row(out, ref, cfg.dtype, f"{name} ({math_path}, {merge_mode})")

@@ -11,9 +11,11 @@ preempted (both asserted).
 Every step: the native scheduler and the oracle's Python model agree on the
 step record bit for bit; its writes and copies are applied on the device in
 issue order (pa_cache_write / pa_copy_blocks); the decode runs over the
-running batch.  Checked: every row written this step, bit-exact; the full
-cache contents of sampled sequences, bit-exact; their decode outputs against
-the fp64 oracle; and every 50 steps the outputs of the whole batch.
+running batch.  Checked: every row written this step, bit-exact; the decode
+output of every running sequence at every step against the fp64 oracle
+(computed on spawned worker processes that draw each history from the
+generators); the full cache contents of sampled sequences, bit-exact, and
+every 50 steps those of the whole batch.
 """
 
 import math
@@ -24,11 +26,10 @@ import torch
 
 import paged_kv_cache_381_b200 as pa
 from paged_kv_cache_381_b200 import workloads as wl
-from oracle import attention as oa
 from oracle import block_manager as obm
 from oracle import scheduler as osch
-from oracle.numerics import widen
 from tests.gpu_harness import assert_close, to_device, to_storage
+from tests.trace_oracle import TraceOracle
 
 pytestmark = pytest.mark.gpu
 
@@ -140,9 +141,21 @@ def test_continuous_batching_trace(preempt):
     # the shared prefix is written once
     pre = [(wl.PREFIX_SEQ, p, int(s)) for p, s in enumerate(bm.slots(wl.PREFIX_SEQ, 0, tc.prefix_len))]
     write(pre)
+    oracle = TraceOracle(SEED, tc, (tc.prefix_len, wl.PREFIX_SEQ, dict(streams.share), dict(streams.parent),
+                                    dict(streams.fork_pos)))
+    try:
+        _trace_steps(tc, sch, model, bm, streams, kc, vc, hk, hv, kflat, vflat, write, oracle, preempt)
+    finally:
+        oracle.close()
+
+
+def _trace_steps(tc, sch, model, bm, streams, kc, vc, hk, hv, kflat, vflat, write, oracle, preempt):
+    H, D, bs = tc.num_kv_heads, tc.head_dim, tc.block_size
+    dev = torch.device("cuda")
 
     r = np.random.default_rng(11)
     saw = {"preempt": 0, "cow": 0, "blocked": 0, "finish": 0, "so": 0, "si": 0}
+    checked = {"rows": 0, "steps": 0}
     for step in range(tc.steps):
         rec = sch.step()
         mrec = model.step()
@@ -184,6 +197,8 @@ def test_continuous_batching_trace(preempt):
         out = torch.empty_like(qd)
         pa.pa_decode(out, qd, kc, vc, torch.from_numpy(tables).to(dev), torch.from_numpy(lens).to(dev), tc.scale,
                      bs, H, max_context_len=int(lens.max()))
+        # every running sequence, every step: the oracle works while the GPU does
+        oracle.submit([(s, c, q[i]) for i, (s, c) in enumerate(zip(running, ctx))])
         torch.cuda.synchronize()
         # rows written this step, still owned by their writer: bit-exact
         live = {s: set() for s in running}
@@ -195,21 +210,22 @@ def test_continuous_batching_trace(preempt):
             owned = np.array([bm.slots(w[0], w[1], 1)[0] == w[2] for w in checks])
             assert np.array_equal(gotk[owned], _rows_for_writes(checks, streams, tc, 0)[owned]), step
             assert np.array_equal(gotv[owned], _rows_for_writes(checks, streams, tc, 1)[owned]), step
-        # sampled sequences (plus every one that copied a block): whole cache + outputs
+        got = to_storage(out, "f16")
+        refs = oracle.results()
+        assert_close(got, np.stack(refs), "f16", f"step {step}, all {len(running)} running sequences")
+        # sampled sequences: their whole cache, bit-exact (every 50 steps: every sequence)
         sample = set(r.choice(len(running), size=min(4, len(running)), replace=False).tolist())
         if step % 50 == 49:
             sample = set(range(len(running)))
-        got = to_storage(out, "f16")
         for i in sorted(sample):
             s, n = running[i], ctx[i]
             sl = torch.from_numpy(bm.slots(s, 0, n)).to(dev)
             K = streams.rows(s, range(n), tc, 0)
             V = streams.rows(s, range(n), tc, 1)
-            if i < 8 or step % 50 == 49:
-                assert np.array_equal(to_storage(kflat.index_select(0, sl), "f16"), K), (step, s)
-                assert np.array_equal(to_storage(vflat.index_select(0, sl), "f16"), V), (step, s)
-            ref = oa.decode_history(widen(q[i], "f16"), widen(K, "f16"), widen(V, "f16"), tc.scale)
-            assert_close(got[i], ref, "f16", f"step {step} seq {s}")
+            assert np.array_equal(to_storage(kflat.index_select(0, sl), "f16"), K), (step, s)
+            assert np.array_equal(to_storage(vflat.index_select(0, sl), "f16"), V), (step, s)
+        checked["rows"] += len(running)
+        checked["steps"] += 1
         assert pa.pa_get_device_error() == 0
     assert saw["preempt"] >= 1, saw
     assert saw["cow"] >= 1, saw
@@ -217,3 +233,5 @@ def test_continuous_batching_trace(preempt):
     assert saw["finish"] >= 1, saw
     if preempt == "swap":
         assert saw["so"] >= 1 and saw["si"] >= 1, saw
+    # every step decoded a running batch, and every row of it was checked
+    assert checked["steps"] == tc.steps and checked["rows"] >= 100 * tc.steps, checked

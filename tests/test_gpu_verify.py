@@ -4,7 +4,7 @@ against the fp64 oracle (oracle.attention.paged_verify).
 Tolerance as for decode: 2e-3 absolute + 1e-2 relative for fp16 / bf16.  The
 cache is filled through the product path (host block manager slots +
 pa_cache_write); the Q candidate tokens are the last Q rows of each history.
-Full-size shapes are checked on sampled (sequence, query, head) rows.
+Full-size shapes are checked on every (sequence, query, head) row.
 """
 
 import numpy as np
@@ -15,6 +15,7 @@ import paged_kv_cache_381_b200 as pa
 from paged_kv_cache_381_b200 import workloads as wl
 from paged_kv_cache_381_b200.batch import PagedBatch
 from tests.gpu_harness import DeviceBatch, assert_close, to_device, to_storage
+from tests.full_size import assert_every_row, oracle_all_rows
 from oracle import attention as oa
 from oracle import cache as oc
 from oracle.numerics import widen
@@ -140,9 +141,10 @@ def test_physical_placement_is_bitwise_invariant():
 
 
 @pytest.mark.parametrize("name", ["70b", "7b"])
-def test_full_size_sampled(name):
+def test_full_size_every_row(name):
     """The decode workload's batch verifying 6 candidate tokens per sequence
-    (the bench's verification configuration), checked on sampled rows."""
+    (the bench's verification configuration): every (sequence, query, head)
+    row against the fp64 oracle."""
     cfg = wl.CONFIGS[name]
     Q = 6
     d = wl.draw_device(cfg, 0)
@@ -157,19 +159,5 @@ def test_full_size_sampled(name):
                  max_context_len=batch.max_context_len)
     torch.cuda.synchronize()
     assert pa.pa_get_device_error() == 0
-    r = np.random.default_rng(11)
-    lens = d.context_lens
-    picks = [(int(s), int(i), int(h)) for s, i, h in zip(r.integers(0, S, 24), r.integers(0, Q, 24),
-                                                          r.integers(0, Hq, 24))]
-    picks += [(int(np.argmax(lens)), Q - 1, 0), (int(np.argmin(lens)), 0, Hq - 1)]
-    G = Hq // cfg.num_kv_heads
-    qs = to_storage(q, cfg.dtype)
-    got = to_storage(out, cfg.dtype)
-    for s, i, h in picks:
-        a = int(d.offsets[s])
-        p = int(lens[s]) - Q + i
-        K = widen(to_storage(d.k_hist[a:a + p + 1, h // G], cfg.dtype), cfg.dtype)
-        V = widen(to_storage(d.v_hist[a:a + p + 1, h // G], cfg.dtype), cfg.dtype)
-        ref = oa.attend(widen(qs[s, i, h], cfg.dtype), K, V, cfg.scale)
-        assert_close(got[s, i, h], ref, cfg.dtype, f"{name} row {(s, i, h)}")
-    assert torch.isfinite(out.float()).all()
+    ref = oracle_all_rows(q, d, cfg, verify=True)
+    assert_every_row(out, ref, cfg.dtype, f"{name} verify")

@@ -373,6 +373,45 @@ def test_decode_and_cache_write_argument_rules(pa):
     assert lib.pa_cache_write(nul, nul, nul, nul, nul, 4, None, nul) == 1
 
 
+def test_write_decode_argument_rules(pa):
+    """pa_write_decode checks every argument of the cache write and of the
+    decode before anything is launched (so these run without a GPU)."""
+    lib = pa.lib()
+    nul = ctypes.c_void_p(0)
+    before = pa.launch_count()
+
+    def wd(T=4, S=4, Hq=64, Hkv=8, D=128, bs=16, dt=2, P=0, scale=0.1, nb=64):
+        return lib.pa_write_decode(nul, nul, nul, T, nul, nul, nul, nul, nul, nul, scale, bs, Hkv, S, Hq, D, 8, 128,
+                                   nb, dt, P, nul, 0, nul)
+
+    assert wd() == 1                                   # null write pointers
+    assert wd(T=-1) == 1
+    assert wd(T=0) == 1                                # no write: the decode's own checks (null pointers)
+    assert wd(T=0, S=0) == 0                           # nothing at all to do
+    assert wd(bs=12) == 2 and wd(D=96) == 2            # unsupported shapes (write checks first)
+    assert wd(T=0, Hq=60) == 1                         # decode checks: heads not a multiple of kv heads
+    assert wd(T=0, P=100) == 1 and wd(T=0, scale=float("nan")) == 1
+    assert wd(dt=7) == 1
+    assert pa.launch_count() == before
+
+
+def test_noalloc_scratch_need_uses_the_table_capacity(pa):
+    """pa_decode_noalloc sizes its scratch need as pa_decode does, from
+    max_context_len capped by the block table's capacity: a generous bound over
+    a small table is not refused, a batch that really needs more than the
+    built-in array is (both decided before any device call)."""
+    lib = pa.lib()
+    nul = ctypes.c_void_p(0)
+
+    def na(mcl, maxb, S=8, Hq=64, D=128, P=0):
+        return lib.pa_decode_noalloc(nul, nul, nul, nul, nul, nul, 0.1, 16, 8, S, Hq, D, maxb, mcl, 64, 2, P, nul)
+
+    assert pa.pa_decode_workspace_size(8, 64, 128, 10 ** 6) > 32 * 1024 * 1024
+    assert na(10 ** 6, 8) == 1          # table holds 128 tokens: one partition, no scratch; then null pointers
+    assert pa.pa_decode_workspace_size(32, 64, 128, 2048 * 16) > 32 * 1024 * 1024
+    assert na(10 ** 6, 2048, S=32) == 2  # 32768 tokens of table, 32 sequences: the scratch exceeds the array
+
+
 def test_scheduler_raw_record_matches_tuples(pa):
     """step(raw=True) gives the same ops as arrays."""
     tc = wl.TraceConfig(block_size=4, max_running=12, num_requests=40, steps=80, prefix_len=10,

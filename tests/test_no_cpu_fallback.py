@@ -36,6 +36,8 @@ def test_device_calls_refuse_host_tensors(pa):
     with pytest.raises(ValueError, match="CUDA tensor"):
         pa.pa_verify(out.view(S, 1, Hq, D), q.view(S, 1, Hq, D), kc, vc, tables, lens, 0.125)
     with pytest.raises(ValueError, match="CUDA tensor"):
+        pa.pa_write_decode(k, k, slots, out, q, kc, vc, tables, lens, 0.125)
+    with pytest.raises(ValueError, match="CUDA tensor"):
         pa.pa_copy_blocks(kc, vc, torch.zeros(1, 2, dtype=torch.int32))
     assert pa.launch_count() == before
 

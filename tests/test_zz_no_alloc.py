@@ -92,3 +92,29 @@ def test_noalloc_single_pass_and_rejection():
     assert big > 32 * 1024 * 1024
     assert _call_noalloc(b, out, 30000, partition_size=32) == PA_ERR_UNSUPPORTED
     assert pa.pa_get_device_error() == 0
+
+
+def test_noalloc_bound_above_table_capacity():
+    """A declared max_context_len far above what the block tables can hold is
+    capped at the table capacity, as pa_decode caps it, so the scratch need
+    fits the built-in array and the call matches pa_decode."""
+    assert torch.cuda.is_available(), "this test needs a CUDA device"
+    cfg = wl.DecodeConfig("noalloc2", "bf16", 4, 64, 8, 128, 16, "fixed")
+    lens = (3000, 17, 1200, 4096)
+    inp = wl.make_decode_inputs(cfg, 19, context_lens=lens)
+    b = DeviceBatch(inp)
+    b.step_write()
+    bound = 10 ** 6
+    assert pa.pa_decode_workspace_size(len(lens), cfg.num_heads, cfg.head_dim, bound) > 32 * 1024 * 1024
+    ref = torch.empty_like(b.q)
+    pa.pa_decode(ref, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, cfg.scale, b.bs,
+                 cfg.num_kv_heads, max_context_len=bound,
+                 workspace=torch.empty(pa.pa_decode_workspace_size(len(lens), cfg.num_heads, cfg.head_dim,
+                                                                   b.block_tables.shape[1] * b.bs),
+                                       dtype=torch.uint8, device="cuda"))
+    out = torch.full_like(b.q, float("nan"))
+    assert _call_noalloc(b, out, bound) == 0
+    torch.cuda.synchronize()
+    assert np.array_equal(to_storage(out, "bf16"), to_storage(ref, "bf16"))
+    assert_close(to_storage(out, "bf16"), oracle_outputs(inp), "bf16", "bound above table capacity")
+    assert pa.pa_get_device_error() == 0
