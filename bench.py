@@ -5,13 +5,19 @@ sequence + decode attention over the block tables) on B200.
     python bench.py --impl reference ...      # the CPU oracle, same workload
 
 Prints one JSON line.  ``value`` is KV bytes read per second over the whole
-step (cache write + plan + decode + reduce), inputs resident in HBM, L2
-flushed between steps (the flush is outside the per-step events).  ``e2e`` is
-the same metric through ``pa_step`` with pinned host buffers, host<->device
-copies inside the timed region.  ``roofline`` is the decode kernel's achieved
-bandwidth (algorithmic bytes / its average event-timed duration) against the
-measured HBM copy bandwidth.  N > 1 runs independent replicas (one per GPU,
-no data-path collective; weak scaling).
+step (cache write + plan in one kernel, decode, reduce: pa_write_decode),
+inputs resident in HBM, L2 flushed between steps (the flush is outside the
+per-step events).  ``e2e`` is the same metric through ``pa_step`` with pinned
+host buffers, host<->device copies inside each step's events, measured like
+``value``; ``e2e.pipelined`` is the overlapped serving loop (pa_pipeline)
+beside the device-only step over the same continuous loop.  ``roofline`` is
+the decode kernel's achieved bandwidth (algorithmic bytes / its average
+event-timed duration) against the measured HBM copy bandwidth.  On the
+default run the other configurations follow as sub-objects: ``workloads``
+(7B-shaped and long split-K decode), ``trace`` (per-step time of the
+continuous-batching trace) and ``verify_q6`` (the verification pass of six
+candidate tokens).  N > 1 runs independent replicas (one per GPU, no
+data-path collective; weak scaling).
 """
 
 import argparse
@@ -64,6 +70,8 @@ def parse():
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="time the 70b workload only (no 7b / long / trace / verification sub-objects)")
     p.add_argument("--math", default="auto", choices=["auto", "simt"],
                    help="decode arithmetic: tensor cores for fp16/bf16 (auto), CUDA cores (simt)")
     p.add_argument("--merge", default="kernel", choices=["kernel", "fused"],
@@ -84,15 +92,6 @@ def parse():
                    help="candidate tokens per sequence: > 1 times the verification pass (pa_verify) "
                         "of speculative decoding instead of decode")
     return p.parse_args()
-
-
-def measured_peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
-        with open(path) as f:
-            j = json.load(f)
-        return float(j["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
 
 
 def kernel_hash(kernel="decode"):
@@ -329,10 +328,21 @@ def cpu_baseline_all_cores(cfg_name, seed, lens, unit_scale, single, min_seconds
                       f"{rounds} rounds, float64 numpy, 1 BLAS thread each, slowest process {t:.1f} s"}
 
 
+def workload_config(args, cfg, lens, P, world):
+    """The ``config`` object of the JSON line: the same keys and values for the
+    native arm and the reference arm of one workload."""
+    return {"workload": WORKLOAD_NAMES[args.workload], "num_seqs": len(lens),
+            "context_tokens": int(np.sum(lens)), "kv_bytes_per_step": kv_bytes(cfg, lens),
+            "partition_size": P or 512, "decode_math": args.math, "split_merge": args.merge,
+            "l2": "flushed between steps (256 MiB write, outside step events)",
+            "parallelism": "replicas" if world > 1 else "single"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     cfg = wl.CONFIGS[args.workload]
     lens = wl.context_lengths(cfg, wl.rng(args.seed))
     seqs = list(range(0, len(lens), 4)) or [0]
@@ -344,14 +354,15 @@ def run_reference(args):
         times = [_time_oracle(cfg, items) for _ in range(args.steps)]
     secs = sum(times) / len(times)
     value = sample_bytes / secs / 1e9
+    full_ms = kv_bytes(cfg, lens) / (value * 1e9) * 1e3          # the whole batch at the sample's rate
     sample = (f"{len(seqs)} of {len(lens)} sequences (every 4th) per step, all {cfg.num_heads} query heads, "
-              f"float64 numpy, 1 BLAS thread")
+              f"float64 numpy, 1 BLAS thread, {secs * 1e3:.1f} ms per sample step")
+    P = args.partition_size or cfg.partition_size
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAMES[args.workload], "num_seqs": len(lens),
-                       "kv_bytes_per_step": sample_bytes, "parallelism": "replicas"},
-            "tokens_per_s": len(seqs) / secs,
+            "config": workload_config(args, cfg, lens, P, world),
+            "tokens_per_s": len(lens) / (full_ms * 1e-3),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -380,6 +391,172 @@ def whole_job_gbs(world, bytes_per_rank, ms):
     return world * bytes_per_rank / (ms * 1e-3) / 1e9
 
 
+def hbm_peak(dev):
+    """HBM copy bandwidth to divide by: MEASURED_PEAKS.json when present, else
+    measured here the same way (a device-to-device copy of 2 GiB, best of 10
+    event-timed copies, read + written bytes)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json)"
+    import torch
+    n = 2 << 30
+    a = torch.empty(n, dtype=torch.uint8, device=dev)
+    b = torch.empty_like(a)
+    a.fill_(1)
+    best = float("inf")
+    for i in range(13):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        b.copy_(a)
+        e1.record()
+        e1.synchronize()
+        if i >= 3:
+            best = min(best, e0.elapsed_time(e1))
+    del a, b
+    return 2 * n / (best * 1e-3) / 1e9, "measured in this run (2 GiB device copy, best of 10)"
+
+
+def decode_case(pa, cfg, seed, dev, P, num_seqs=0, queries=1):
+    """A full-size batch resident in HBM: pools filled, new rows held back."""
+    import torch
+    from paged_kv_cache_381_b200.batch import PagedBatch
+    lens_override = wl.context_lengths(cfg, wl.rng(seed))[:num_seqs] if num_seqs else None
+    d = wl.draw_device(cfg, seed, device=dev, context_lens=lens_override)
+    batch = PagedBatch(d.k_hist, d.v_hist, d.offsets, d.context_lens, d.num_blocks, cfg.block_size, d.free_order,
+                       new_tokens=queries)
+    q = d.q
+    if queries > 1:
+        gq = torch.Generator(device=dev).manual_seed(seed * 7919 + queries)
+        q = torch.randn((len(d.context_lens), queries, cfg.num_heads, cfg.head_dim), generator=gq, device=dev,
+                        dtype=torch.float32).to(d.q.dtype)
+    del d.k_hist, d.v_hist
+    return batch, q, np.asarray(d.context_lens)
+
+
+def time_steps(pa, step, steps, warmup, flush, kernel, profile_all=False, world=1):
+    """Warm up, then time `steps` calls of step() each between two CUDA events
+    on the current stream, L2 flushed between them outside the events; the
+    library's own events time `kernel` (or every kernel) inside."""
+    import torch
+    import torch.distributed as dist
+    for _ in range(max(warmup, 3)):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    launches0 = pa.launch_count()
+    pa.profile_begin(None if profile_all else [kernel])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall0 = time.perf_counter()
+    for i in range(steps):
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+        flush.zero_()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    prof = pa.profile_end()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    return {"step_ms": step_ms, "prof": prof, "launches": pa.launch_count() - launches0, "wall": wall}
+
+
+def roofline(bytes_per_launch, ms, peak, peak_kind, kernel, traffic):
+    achieved = bytes_per_launch / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": traffic, "kernel": kernel, "algorithmic_bytes": int(bytes_per_launch), "peak_source": peak_kind,
+            "spec_peak": SPEC_HBM_GBS, "spec_frac": achieved / SPEC_HBM_GBS}
+
+
+def sub_decode(pa, name, seed, dev, flush, peak, peak_kind, steps=100, warmup=5):
+    """One more decode workload at full size: its step and decode-kernel roofline."""
+    import torch
+    cfg = wl.CONFIGS[name]
+    P = cfg.partition_size
+    batch, q, lens = decode_case(pa, cfg, seed, dev, P)
+    out = torch.empty_like(q)
+    batch.ensure_workspace(cfg.num_heads, P)
+    r = time_steps(pa, lambda: batch.step(out, q, cfg.scale, partition_size=P), steps, warmup, flush, "decode")
+    ms = statistics.mean(r["step_ms"])
+    dec_ms = r["prof"]["decode"][0] / max(1, r["prof"]["decode"][1])
+    step_kv = kv_bytes(cfg, lens)
+    res = {"workload": WORKLOAD_NAMES[name], "dtype": cfg.dtype, "steps": steps, "ms_per_step": ms,
+           "ms_per_step_median": statistics.median(r["step_ms"]), "value": step_kv / (ms * 1e-3) / 1e9,
+           "unit": "GB/s", "pct_of_hbm_peak": step_kv / (ms * 1e-3) / 1e9 / peak, "kv_bytes_per_step": step_kv,
+           "tokens_per_s": len(lens) / (ms * 1e-3), "kernel_ms": {"decode": dec_ms},
+           "roofline": roofline(decode_kernel_bytes(cfg, lens, P), dec_ms, peak, peak_kind, "decode_kernel",
+                                recorded_traffic("decode", name))}
+    del batch, q, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def sub_verify(pa, name, seed, dev, flush, peak, peak_kind, Q=6, steps=100, warmup=5, verify_kernel="auto"):
+    """The verification pass of speculative decoding (Q candidate tokens per
+    sequence) on a decode workload: step, kernel roofline and tensor work."""
+    import torch
+    cfg = wl.CONFIGS[name]
+    batch, q, lens = decode_case(pa, cfg, seed, dev, 0, queries=Q)
+    out = torch.empty_like(q)
+    P = pa.pa_verify_partition_size(len(lens), Q, cfg.num_heads, cfg.num_kv_heads, 0)
+    batch.ensure_workspace(cfg.num_heads, 0)
+
+    def step():
+        batch.write_new_tokens()
+        batch.verify(out, q, cfg.scale)
+    r = time_steps(pa, step, steps, warmup, flush, "verify")
+    ms = statistics.mean(r["step_ms"])
+    k_ms = r["prof"]["verify"][0] / max(1, r["prof"]["verify"][1])
+    kname = "verify_tc" if verify_kernel in ("auto", "tcgen05") else "verify"
+    step_kv = kv_bytes(cfg, lens)
+    tpeak, tkind = measured_tensor_peak()
+    fl = verify_flops(cfg, lens, Q)
+    res = {"workload": WORKLOAD_NAMES[name], "queries_per_seq": Q, "verify_kernel": verify_kernel,
+           "partition_size": P, "steps": steps, "ms_per_step": ms, "ms_per_step_median": statistics.median(r["step_ms"]),
+           "value": step_kv / (ms * 1e-3) / 1e9, "unit": "GB/s", "tokens_per_s": len(lens) * Q / (ms * 1e-3),
+           "kernel_ms": {"verify": k_ms},
+           "roofline": roofline(verify_kernel_bytes(cfg, lens, P, Q), k_ms, peak, peak_kind, f"{kname}_kernel",
+                                recorded_traffic(kname, name, Q)),
+           "tensor": {"flops_per_launch": fl, "achieved_tflops": fl / (k_ms * 1e-3) / 1e12, "peak_tflops": tpeak,
+                      "frac": fl / (k_ms * 1e-3) / 1e12 / tpeak, "peak_source": tkind,
+                      "note": "plain flops; P.V runs as two products (16-bit value + remainder) for bf16"}}
+    del batch, q, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def sub_trace(dev, peak):
+    """Per-step time of the continuous-batching trace (the serving loop): device
+    work of each step and the host scheduler's time, separately."""
+    import torch
+    from paged_kv_cache_381_b200 import trace
+    r = trace.run(wl.TRACE, seed=5, device=dev)
+    d = np.asarray(r["device_ms"])
+    h = np.asarray(r["host_ms"])
+    tc = wl.TRACE
+    res = {"workload": (f"continuous-batching trace: fp16, block 8, {tc.num_heads} q / {tc.num_kv_heads} kv heads, "
+                        f"head_dim {tc.head_dim}, <= {tc.max_running} running, {tc.steps} steps, "
+                        f"{tc.prefix_len}-token shared prefix for half the requests, prompts U[1, 512], "
+                        "outputs geometric (mean 256), pool 75% of the unbounded peak"),
+           "steps_timed": int(r["steps"]), "device_ms_median": float(np.median(d)), "device_ms_p90": float(np.percentile(d, 90)),
+           "device_ms_mean": float(d.mean()), "host_sched_ms_median": float(np.median(h)),
+           "host_sched_ms_p90": float(np.percentile(h, 90)),
+           "kv_gbs": float(np.sum(r["kv_bytes"]) / (d.sum() * 1e-3) / 1e9),
+           "pct_of_hbm_peak": float(np.sum(r["kv_bytes"]) / (d.sum() * 1e-3) / 1e9 / peak),
+           "preemptions": int(r["preempted"]), "admissions": int(r["admitted"]), "num_blocks": int(r["num_blocks"]),
+           "how": ("device: each step's metadata H2D (pinned), copy-on-write copies, prompt writes and "
+                   "pa_write_decode between two events, L2 flushed between steps; host: pa_sched_step + "
+                   "table packing through the Python binding")}
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -400,33 +577,21 @@ def run_native(args):
     if world > 1:
         dist.barrier()
     import paged_kv_cache_381_b200 as pa
-    from paged_kv_cache_381_b200.batch import PagedBatch
     pa.set_decode_math(pa.MATH_AUTO if args.math == "auto" else pa.MATH_SIMT)
     pa.set_split_merge(pa.MERGE_KERNEL if args.merge == "kernel" else pa.MERGE_FUSED)
     pa.set_verify_kernel({"auto": pa.VERIFY_AUTO, "tcgen05": pa.VERIFY_TCGEN05,
                           "mma_sync": pa.VERIFY_MMA_SYNC}[args.verify_kernel])
+    peak, peak_kind = hbm_peak(dev)
 
     cfg = wl.CONFIGS[args.workload]
     seed = args.seed + rank                       # independent replica per rank
-    lens_override = None
-    if args.num_seqs:
-        lens_override = wl.context_lengths(cfg, wl.rng(seed))[:args.num_seqs]
-    d = wl.draw_device(cfg, seed, device=dev, context_lens=lens_override)
     Q = args.queries
-    batch = PagedBatch(d.k_hist, d.v_hist, d.offsets, d.context_lens, d.num_blocks, cfg.block_size, d.free_order,
-                       new_tokens=Q)
-    lens = d.context_lens
-    q = d.q
-    if Q > 1:
-        gq = torch.Generator(device=dev).manual_seed(seed * 7919 + Q)
-        q = torch.randn((len(lens), Q, cfg.num_heads, cfg.head_dim), generator=gq, device=dev,
-                        dtype=torch.float32).to(d.q.dtype)
-    out = torch.empty_like(q)
     P = args.partition_size or cfg.partition_size
+    batch, q, lens = decode_case(pa, cfg, seed, dev, P, num_seqs=args.num_seqs, queries=Q)
+    out = torch.empty_like(q)
     batch.ensure_workspace(cfg.num_heads, P)
     step_kv = kv_bytes(cfg, lens)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    del d.k_hist, d.v_hist
     torch.cuda.synchronize()
     pa.pa_get_device_error()
 
@@ -439,49 +604,25 @@ def run_native(args):
         kname = "verify"
 
     def step():
-        batch.write_new_tokens()
         if Q > 1:
+            batch.write_new_tokens()
             batch.verify(out, q, cfg.scale, partition_size=P)
         else:
-            batch.decode(out, q, cfg.scale, partition_size=P)
+            batch.step(out, q, cfg.scale, partition_size=P)      # pa_write_decode
 
-    for _ in range(max(args.warmup, 3)):
-        step()
-        flush.zero_()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.3)
-    launches0 = pa.launch_count()
-    pa.profile_begin(None if args.profile_all else [kernel])   # default: the attention kernel only
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    wall0 = time.perf_counter()
-    for i in range(args.steps):
-        ev[i][0].record()
-        step()
-        ev[i][1].record()
-        flush.zero_()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    wall = time.perf_counter() - wall0
-    prof = pa.profile_end()
-    launches = pa.launch_count() - launches0
+    r = time_steps(pa, step, args.steps, args.warmup, flush, kernel, args.profile_all, world)
     clk = clocks.stop()
     err = pa.pa_get_device_error()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    ms = sum(step_ms) / len(step_ms)
-    ms_median = statistics.median(step_ms)
+    prof = r["prof"]
+    ms = sum(r["step_ms"]) / len(r["step_ms"])
+    ms_median = statistics.median(r["step_ms"])
     dec_ms = prof[kernel][0] / max(1, prof[kernel][1])
     ms, dec_ms = max_over_ranks([ms, dec_ms], dev)
 
-    # ---- e2e: the same step from pinned host buffers through pa_step
+    # ---- e2e: the same step through the library's host-buffer calls
     e2e = None
     if not args.no_e2e and Q == 1:
         S, Hq, D = q.shape
@@ -490,67 +631,74 @@ def run_native(args):
                 "block_tables": batch.block_tables.cpu().pin_memory(),
                 "context_lens": batch.context_lens.cpu().pin_memory(),
                 "out": torch.empty_like(q, device="cpu").pin_memory()}
-        # two staging sets: step i+1's inputs and step i-1's output cross the host
-        # link while step i computes (pa_pipeline); the split-K workspace is shared,
-        # since the computes themselves stay in order on one stream
         sets = []
         for _ in range(2):
-            d = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
-            d["workspace"] = batch.workspace
-            sets.append(d)
+            dset = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+            dset["workspace"] = batch.workspace
+            sets.append(dset)
         h2d = sum(host[k].numel() * host[k].element_size() for k in host if k != "out")
         d2h = host["out"].numel() * host["out"].element_size()
+        # (1) like `value`: pa_step per step (copy in, compute, copy out on one
+        # stream) between two events, L2 flushed between steps outside them
+        er = time_steps(pa, lambda: pa.pa_step(host, sets[0], batch.k_cache, batch.v_cache, cfg.scale,
+                                               batch.max_context_len, P),
+                        args.steps, args.warmup, flush, "decode", False, world)
+        ems = statistics.mean(er["step_ms"])
+        (ems,) = max_over_ranks([ems], dev)
+        # (2) a continuous serving loop without flushes (1.1 GB of K/V per step is
+        # larger than L2): pa_pipeline overlaps step i's copies with its neighbours'
+        # compute; the device-only step is timed over the same kind of loop
         pipe = pa.Pipeline(2)
+        n = args.steps
 
-        def e2e_run(n):
+        def pipe_run(k):
             pipe.begin(q)
-            for i in range(n):
+            for i in range(k):
                 pipe.step(i % 2, host, sets[i % 2], batch.k_cache, batch.v_cache, cfg.scale, batch.max_context_len, P)
             pipe.end(q)
 
-        e2e_run(3)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        # inputs (1.1 GB of K/V per step) are larger than L2: no flush inside this run
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        e2e_run(args.steps)
-        e1.record()
-        torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1) / args.steps
-        (ems,) = max_over_ranks([ems], dev)
-        e2e = {"value": whole_job_gbs(world, step_kv, ems), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": ems,
-               "tokens_per_s": world * len(lens) / (ems * 1e-3),
-               "how": "pa_pipeline: each step's H2D and D2H overlap the neighbouring steps' compute"}
+        def loop_ms(fn):
+            fn(3)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn(n)
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / n
 
-    peak, peak_kind = measured_peaks()
-    if Q > 1:
-        P = pa.pa_verify_partition_size(len(lens), Q, cfg.num_heads, cfg.num_kv_heads, P)   # what pa_verify used
-        dec_bytes = verify_kernel_bytes(cfg, lens, P, Q)
-    else:
-        dec_bytes = decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused")
+        def dev_run(k):
+            for _ in range(k):
+                step()
+        pms, dcont = max_over_ranks([loop_ms(pipe_run), loop_ms(dev_run)], dev)
+        e2e = {"value": whole_job_gbs(world, step_kv, ems), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": ems, "tokens_per_s": world * len(lens) / (ems * 1e-3),
+               "copy_ms_per_step": ems - ms,
+               "how": ("pa_step per step: H2D of q, k, v, slots, tables and lengths from pinned memory, the step, "
+                       "D2H of out, on one stream between two events; L2 flushed between steps outside them, "
+                       "as for value"),
+               "pipelined": {"value": whole_job_gbs(world, step_kv, pms), "ms_per_step": pms,
+                             "device_only_ms_per_step": dcont, "copy_ms_per_step": pms - dcont,
+                             "how": ("continuous loop, no flush: pa_pipeline (two staging sets, copies on their "
+                                     "own streams) against the device-only step over the same loop")}}
+
+    dec_bytes = (verify_kernel_bytes(cfg, lens, pa.pa_verify_partition_size(len(lens), Q, cfg.num_heads,
+                                                                           cfg.num_kv_heads, P), Q)
+                 if Q > 1 else decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused"))
     traffic = None if args.num_seqs else recorded_traffic(kname, args.workload, Q)
-    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     value = whole_job_gbs(world, step_kv, ms)
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAMES[args.workload], "num_seqs": len(lens),
-                   "context_tokens": int(lens.sum()), "kv_bytes_per_step": step_kv,
-                   "partition_size": P or 512, "decode_math": args.math, "split_merge": args.merge, "l2": "flushed between steps (256 MiB write, outside step events)",
-                   "parallelism": "replicas" if world > 1 else "single"},
+        "config": workload_config(args, cfg, lens, P, world),
         "pct_of_hbm_peak": value / world / peak,
         "ms_per_step_median": ms_median,
         "pct_of_spec_peak": value / world / SPEC_HBM_GBS,
         "tokens_per_s": world * len(lens) / (ms * 1e-3),
         "kernel_ms": {k: v[0] / max(1, v[1]) for k, v in prof.items() if v[1]},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": f"{kname}_kernel", "algorithmic_bytes": dec_bytes,
-                     "peak_source": peak_kind, "spec_peak": SPEC_HBM_GBS, "spec_frac": achieved / SPEC_HBM_GBS},
-        "gpu_launches": int(launches), "device_error_flags": err, "wall_s": wall,
+        "roofline": roofline(dec_bytes, dec_ms, peak, peak_kind, f"{kname}_kernel", traffic),
+        "gpu_launches": int(r["launches"]), "device_error_flags": err, "wall_s": r["wall"],
         "e2e": e2e, "clocks": clk,
     }
     if Q > 1:
@@ -563,6 +711,14 @@ def run_native(args):
         result["tensor"] = {"flops_per_launch": fl, "achieved_tflops": fl / (dec_ms * 1e-3) / 1e12,
                             "peak_tflops": tpeak, "frac": fl / (dec_ms * 1e-3) / 1e12 / tpeak,
                             "peak_source": tkind, "note": "plain flops; P.V runs as two mma (16-bit value + remainder)"}
+    del batch, q, out
+    torch.cuda.empty_cache()
+    # the other configurations of the path, on the default run (one GPU)
+    if world == 1 and Q == 1 and not args.no_extra and args.workload == "70b" and not args.num_seqs:
+        result["workloads"] = {w: sub_decode(pa, w, args.seed, dev, flush, peak, peak_kind) for w in ("7b", "long")}
+        result["trace"] = sub_trace(dev, peak)
+        result["verify_q6"] = sub_verify(pa, "70b", args.seed, dev, flush, peak, peak_kind)
+        result["device_error_flags"] |= pa.pa_get_device_error()
     if rank == 0 and world == 1 and not args.no_cpu_baseline and Q == 1:
         result["cpu_baseline"] = cpu_baseline(cfg, args.seed, lens, 1e9)
         try:        # a host without process spawning must not cost the run its line
