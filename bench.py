@@ -111,9 +111,7 @@ def traffic_profile_name(kernel, workload, queries):
     return f"{kernel}_{workload}_traffic.json" if queries == 1 else f"{kernel}_{workload}_q{queries}_traffic.json"
 
 
-def recorded_traffic(kernel, workload, queries=1):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary for this
-    workload, if it was taken on the current kernel source; else None."""
+def _current_record(kernel, workload, queries):
     path = os.path.join(ROOT, "profiles", traffic_profile_name(kernel, workload, queries))
     if not os.path.exists(path):
         return None
@@ -121,7 +119,21 @@ def recorded_traffic(kernel, workload, queries=1):
         j = json.load(f)
     if j.get("kernel_source_sha256_16") != kernel_hash(kernel):
         return None
-    return j.get("dram_bytes_per_launch")
+    return j
+
+
+def recorded_traffic(kernel, workload, queries=1):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary for this
+    workload, if it was taken on the current kernel source; else None."""
+    j = _current_record(kernel, workload, queries)
+    return None if j is None else j.get("dram_bytes_per_launch")
+
+
+def recorded_dram_pct(kernel, workload, queries=1):
+    """ncu's dram__throughput.avg.pct_of_peak_sustained_elapsed for `kernel` on
+    this workload (mean over the captured launches), under the same gate."""
+    j = _current_record(kernel, workload, queries)
+    return None if j is None else j.get("dram_throughput_pct_of_peak_ncu")
 
 
 def elt_bytes(dtype):
@@ -467,11 +479,12 @@ def time_steps(pa, step, steps, warmup, flush, kernel, profile_all=False, world=
     return {"step_ms": step_ms, "prof": prof, "launches": pa.launch_count() - launches0, "wall": wall}
 
 
-def roofline(bytes_per_launch, ms, peak, peak_kind, kernel, traffic):
+def roofline(bytes_per_launch, ms, peak, peak_kind, kernel, traffic, ncu_dram_pct=None):
     achieved = bytes_per_launch / (ms * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
             "traffic": traffic, "kernel": kernel, "algorithmic_bytes": int(bytes_per_launch), "peak_source": peak_kind,
-            "spec_peak": SPEC_HBM_GBS, "spec_frac": achieved / SPEC_HBM_GBS}
+            "spec_peak": SPEC_HBM_GBS, "spec_frac": achieved / SPEC_HBM_GBS,
+            "ncu_dram_throughput_pct": ncu_dram_pct}
 
 
 def sub_decode(pa, name, seed, dev, flush, peak, peak_kind, steps=100, warmup=5):
@@ -491,7 +504,7 @@ def sub_decode(pa, name, seed, dev, flush, peak, peak_kind, steps=100, warmup=5)
            "unit": "GB/s", "pct_of_hbm_peak": step_kv / (ms * 1e-3) / 1e9 / peak, "kv_bytes_per_step": step_kv,
            "tokens_per_s": len(lens) / (ms * 1e-3), "kernel_ms": {"decode": dec_ms},
            "roofline": roofline(decode_kernel_bytes(cfg, lens, P), dec_ms, peak, peak_kind, "decode_kernel",
-                                recorded_traffic("decode", name))}
+                                recorded_traffic("decode", name), recorded_dram_pct("decode", name))}
     del batch, q, out
     torch.cuda.empty_cache()
     return res
@@ -522,7 +535,7 @@ def sub_verify(pa, name, seed, dev, flush, peak, peak_kind, Q=6, steps=100, warm
            "value": step_kv / (ms * 1e-3) / 1e9, "unit": "GB/s", "tokens_per_s": len(lens) * Q / (ms * 1e-3),
            "kernel_ms": {"verify": k_ms},
            "roofline": roofline(verify_kernel_bytes(cfg, lens, P, Q), k_ms, peak, peak_kind, f"{kname}_kernel",
-                                recorded_traffic(kname, name, Q)),
+                                recorded_traffic(kname, name, Q), recorded_dram_pct(kname, name, Q)),
            "tensor": {"flops_per_launch": fl, "achieved_tflops": fl / (k_ms * 1e-3) / 1e12, "peak_tflops": tpeak,
                       "frac": fl / (k_ms * 1e-3) / 1e12 / tpeak, "peak_source": tkind,
                       "note": "plain flops; P.V runs as two products (16-bit value + remainder) for bf16"}}
@@ -686,6 +699,7 @@ def run_native(args):
                                                                            cfg.num_kv_heads, P), Q)
                  if Q > 1 else decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused"))
     traffic = None if args.num_seqs else recorded_traffic(kname, args.workload, Q)
+    dram_pct = None if args.num_seqs else recorded_dram_pct(kname, args.workload, Q)
     value = whole_job_gbs(world, step_kv, ms)
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -697,7 +711,7 @@ def run_native(args):
         "pct_of_spec_peak": value / world / SPEC_HBM_GBS,
         "tokens_per_s": world * len(lens) / (ms * 1e-3),
         "kernel_ms": {k: v[0] / max(1, v[1]) for k, v in prof.items() if v[1]},
-        "roofline": roofline(dec_bytes, dec_ms, peak, peak_kind, f"{kname}_kernel", traffic),
+        "roofline": roofline(dec_bytes, dec_ms, peak, peak_kind, f"{kname}_kernel", traffic, dram_pct),
         "gpu_launches": int(r["launches"]), "device_error_flags": err, "wall_s": r["wall"],
         "e2e": e2e, "clocks": clk,
     }

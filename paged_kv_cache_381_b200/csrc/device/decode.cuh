@@ -415,7 +415,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
         for (; i < total && ok; ++k) {
             // publish the item: descriptor, then its q rows by one bulk copy
             const int b = k & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&item_empty[b], ((k >> 1) & 1u) ^ 1u, abort_flag))) {
+            if (!mbar_wait_warp(&item_empty[b], ((k >> 1) & 1u) ^ 1u, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
                     for (int st = 0; st < nst; ++st, ++stage) {
                         const int slot = stage % C::NSTAGES;
                         const uint32_t parity = ((stage / C::NSTAGES) & 1u) ^ 1u;
-                        if (!__all_sync(0xffffffffu, mbar_wait(&empty[slot], parity, abort_flag))) {
+                        if (!mbar_wait_warp(&empty[slot], parity, abort_flag)) {
                             ok = false;
                             break;
                         }

@@ -109,12 +109,17 @@ __global__ void __launch_bounds__(256) write_plan_kernel(const WriteArgs w, int 
 // any of them is used, so a row of up to RB partitions costs one round trip to
 // L2, where the attention kernel has just left the partials.  Partials merge
 // in partition order (the bits do not depend on the grid).
+// Partials of a row a lane holds in flight (a build-time knob: more partials per
+// round trip against more registers, so fewer warps resident).
+#ifndef PA_REDUCE_RB
+#define PA_REDUCE_RB 16
+#endif
 constexpr int kReduceWarps = 8;                   // warps per reduce CTA
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const DecodeArgs a) {
     using Tr = ElemTraits<T>;
     constexpr int PER = D / 32;                   // floats of a partial row per lane
-    constexpr int RB = 16;                        // partials in flight per lane
+    constexpr int RB = PA_REDUCE_RB;              // partials in flight per lane
     using Vec = typename std::conditional<PER == 4, float4, float2>::type;
     grid_dependency_wait();                       // the plan and the partials must be complete
     const int warp = threadIdx.x >> 5;

@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(VerifyCfg<T, D>::THREADS, 2)
             for (int st = 0; st < nst; ++st, ++stage) {
                 const int slot = stage % C::NSTAGES;
                 const uint32_t parity = ((stage / C::NSTAGES) & 1u) ^ 1u;
-                if (!mbar_wait(&empty[slot], parity, abort_flag)) {
+                if (!mbar_wait_warp(&empty[slot], parity, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -195,7 +195,8 @@ __global__ void __launch_bounds__(VerifyCfg<T, D>::THREADS, 2)
     uint32_t stage = 0;
     auto acquire = [&](uint32_t c) -> bool {
         const int slot = c % C::NSTAGES;
-        if (*abort_flag || !mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag)) {
+        const bool got = !*abort_flag && mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
             *abort_flag = 1;
             return false;
         }

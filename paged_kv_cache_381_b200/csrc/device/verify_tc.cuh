@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                         const uint32_t prev = __shfl_sync(0xffffffffu, tag, (int)slot);
                         const uint32_t g = prev >> 1;
                         uint64_t* done = (prev & 1u) ? &o_full[g % C::NPH] : &s_full[g % C::NPH];
-                        if (!__all_sync(0xffffffffu, mbar_wait(done, (g / C::NPH) & 1u, abort_flag))) return false;
+                        if (!mbar_wait_warp(done, (g / C::NPH) & 1u, abort_flag)) return false;
                     }
                     const int rows = min(C::CHUNK, w.n - c * C::CHUNK);
                     const int nbk = (rows + bs - 1) >> a.log2_bs;          // whole blocks
@@ -325,12 +325,12 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         auto issue_s = [&](uint32_t pos, uint32_t g) -> bool {
             const uint32_t buf = g & 1u;
             const int slot = pos % C::NSLOTS;
-            if (!mbar_wait(&full[slot], (pos / C::NSLOTS) & 1u, abort_flag)) return false;
+            if (!mbar_wait_warp(&full[slot], (pos / C::NSLOTS) & 1u, abort_flag)) return false;
             if constexpr (C::PTMEM && PA_VERIFY_TC_PWAR) {
                 // the buffer holds p of chunk g - 2, read by P.V of that chunk: a later
                 // product may not overwrite an operand the tensor core may still read
                 // (nor, with two issuers, one not yet read), so that P.V completes first
-                if (g >= 2 && !mbar_wait(&o_full[(g - 2) % C::NPH], ((g - 2) / C::NPH) & 1u, abort_flag)) return false;
+                if (g >= 2 && !mbar_wait_warp(&o_full[(g - 2) % C::NPH], ((g - 2) / C::NPH) & 1u, abort_flag)) return false;
             }
             tc::fence_after_sync();
             if (lane == 0) {
@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         auto issue_pv = [&](uint32_t pos, int c, int n, uint32_t g, bool first) -> bool {
             const uint32_t pbuf = C::PBUF == 2 ? (g & 1u) : 0u;
             const int slot = pos % C::NSLOTS;
-            if (!mbar_wait(&full[slot], (pos / C::NSLOTS) & 1u, abort_flag)) return false;
+            if (!mbar_wait_warp(&full[slot], (pos / C::NSLOTS) & 1u, abort_flag)) return false;
             const int rows = min(C::CHUNK, n - c * C::CHUNK);
             if (rows < C::CHUNK) {
                 // rows past the partition (stale or unwritten rows, maybe NaN): zero them
@@ -389,10 +389,10 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         // P.V of chunk c, once its p is written (and, for the item's first chunk, the
         // previous item's O has been read out)
         auto pv_chunk = [&](uint32_t pos, int c, int n, uint32_t g) -> bool {
-            if (!mbar_wait(p_full, p_ph, abort_flag)) return false;
+            if (!mbar_wait_warp(p_full, p_ph, abort_flag)) return false;
             p_ph ^= 1u;
             if (c == 0) {
-                if (!mbar_wait(o_empty, oe_ph ^ 1u, abort_flag)) return false;
+                if (!mbar_wait_warp(o_empty, oe_ph ^ 1u, abort_flag)) return false;
                 oe_ph ^= 1u;
             }
             tc::fence_after_sync();
@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 return seq + (c + 1 < nc ? (uint32_t)(2 * c + 2) : (uint32_t)(2 * nc - 1));
             };
             if (do_s) {
-                if (!mbar_wait(q_full, q_ph, abort_flag)) {
+                if (!mbar_wait_warp(q_full, q_ph, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         uint32_t qe_ph = 0, gch = 0;
         // P.V of global chunk g done: barrier copy g % NPH, its (g / NPH)-th phase
         auto wait_pv = [&](uint32_t g) -> bool {
-            return mbar_wait(&o_full[g % C::NPH], (g / C::NPH) & 1u, abort_flag);
+            return mbar_wait_warp(&o_full[g % C::NPH], (g / C::NPH) & 1u, abort_flag);
         };
         // output row and query position of local row lr of item w (orow < 0: no row)
         auto row_in = [&](const WorkItem& w, int ctx, int lr, int64_t& orow, int& pos) {
@@ -485,7 +485,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         // item w's query rows as the A tile (rows past the chunk are zero), once the
         // previous item's last S product no longer reads the tile
         auto stage_q = [&](const WorkItem& w, int ctx) -> bool {
-            if (!mbar_wait(q_empty, qe_ph ^ 1u, abort_flag)) return false;
+            if (!mbar_wait_warp(q_empty, qe_ph ^ 1u, abort_flag)) return false;
             qe_ph ^= 1u;
             // all loads of this thread first, then the swizzled stores
             constexpr int VPR = D * 2 / 16;               // 16-byte chunks per row
@@ -535,7 +535,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
             for (int c = 0; c < nc && ok; ++c) {
                 const uint32_t buf = (gch + c) & 1u;
-                if (!(ok = mbar_wait(&s_full[(gch + c) % C::NPH], ((gch + c) / C::NPH) & 1u, abort_flag))) break;
+                if (!(ok = mbar_wait_warp(&s_full[(gch + c) % C::NPH], ((gch + c) / C::NPH) & 1u, abort_flag))) break;
                 tc::fence_after_sync();
                 uint32_t r[32];
                 tc::ld16x2(tmem + lane_addr + C::S_COL + buf * 64, r);
@@ -613,7 +613,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     // ahead of the others must not arrive before the previous chunk's phase
                     // completes, or its arrival would count toward that phase.  (With a
                     // single P buffer the wait for the previous P.V below implies this.)
-                    if (gc >= 1 && !(ok = mbar_wait(p_full, (gc - 1) & 1u, abort_flag))) break;
+                    if (gc >= 1 && !(ok = mbar_wait_warp(p_full, (gc - 1) & 1u, abort_flag))) break;
                 }
                 if constexpr (C::PTMEM) {
                     // p over this chunk's S columns (already read): tokens half*32 .. +31 of row m

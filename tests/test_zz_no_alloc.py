@@ -30,13 +30,14 @@ pytestmark = pytest.mark.gpu
 PA_ERR_UNSUPPORTED = 2
 
 
-def _call_noalloc(b, out, max_context_len, num_seqs=None, partition_size=0):
+def _call_noalloc(b, out, max_context_len, num_seqs=None, partition_size=0, tables=None):
     S, Hq, D = b.q.shape
+    tables = b.block_tables if tables is None else tables
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     return pa.lib().pa_decode_noalloc(
-        out.data_ptr(), b.q.data_ptr(), b.k_cache.data_ptr(), b.v_cache.data_ptr(), b.block_tables.data_ptr(),
+        out.data_ptr(), b.q.data_ptr(), b.k_cache.data_ptr(), b.v_cache.data_ptr(), tables.data_ptr(),
         b.context_lens.data_ptr(), b.cfg.scale, b.bs, b.cfg.num_kv_heads, S if num_seqs is None else num_seqs, Hq, D,
-        b.block_tables.shape[1], max_context_len, b.nb, {"f32": 0, "f16": 1, "bf16": 2}[b.dtype], partition_size,
+        tables.shape[1], max_context_len, b.nb, {"f32": 0, "f16": 1, "bf16": 2}[b.dtype], partition_size,
         stream)
 
 
@@ -86,11 +87,16 @@ def test_noalloc_single_pass_and_rejection():
     torch.cuda.synchronize()
     assert_close(to_storage(out, "f16"), widen(to_storage(ref, "f16"), "f16"), "f16", "single pass")
     # a batch whose scratch need exceeds the built-in array is refused before any
-    # launch (same tensors; a declared bound of 30000 tokens in 32-token
-    # partitions would need ~47 MB of scratch)
+    # launch: the same sequences with block tables wide enough for 30000 tokens
+    # (padded with -1) and that bound, in 32-token partitions, would need ~47 MB
+    # of scratch
     big = pa.pa_decode_workspace_size(3, 32, 128, 30000, 32)
     assert big > 32 * 1024 * 1024
-    assert _call_noalloc(b, out, 30000, partition_size=32) == PA_ERR_UNSUPPORTED
+    wide = torch.full((3, 30000 // b.bs + 1), -1, dtype=torch.int32, device="cuda")
+    wide[:, :b.block_tables.shape[1]] = b.block_tables
+    n0 = pa.launch_count()
+    assert _call_noalloc(b, out, 30000, partition_size=32, tables=wide) == PA_ERR_UNSUPPORTED
+    assert pa.launch_count() == n0
     assert pa.pa_get_device_error() == 0
 
 
