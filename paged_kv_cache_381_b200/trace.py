@@ -64,10 +64,10 @@ def _runs(kind, a, b, c):
     return runs
 
 
-def run(tc=wl.TRACE, seed=5, device="cuda", flush_bytes=256 << 20, partition_size=0):
-    """Run the trace; returns per-step host and device times and the work done."""
-    import torch
-    dev = torch.device(device)
+def schedule(tc=wl.TRACE, seed=5):
+    """The scheduler alone over every step of the trace (host only): per step
+    its device ops in issue order, packed tables and context lengths, and the
+    host time of the scheduling step and its table packing."""
     reqs = wl.make_trace_requests(tc, seed)
     nb = int(math.ceil(tc.pool_frac * dry_peak(tc, reqs)))
     order = np.random.default_rng(seed).permutation(nb).astype(np.int32)
@@ -76,17 +76,16 @@ def run(tc=wl.TRACE, seed=5, device="cuda", flush_bytes=256 << 20, partition_siz
     sch = Scheduler(bm, tc.max_running, wl.PREFIX_SEQ)
     for q in reqs:
         sch.add_request(q.seq_id, q.prompt_len, q.output_len, q.shares_prefix, q.fork_child, q.fork_output_len)
-    prefix_slots = bm.slots(wl.PREFIX_SEQ, 0, tc.prefix_len)
-
-    # ---- the scheduler alone: every step's decisions, timed on the host
+    prefix_slots = np.asarray(bm.slots(wl.PREFIX_SEQ, 0, tc.prefix_len), dtype=np.int64)
     steps, host_ms = [], []
-    max_rows, max_running, preempted, admitted = len(prefix_slots), 1, 0, 0
+    preempted = admitted = 0
     for _ in range(tc.steps):
         t0 = time.perf_counter()
         rec = sch.step(raw=True)
         running = rec["running"]
         if running:
-            width = max(len(bm.block_table(s)) for s in running)
+            # a table holds exactly ceil(context / block size) blocks
+            width = -(-max(rec["context_lens"]) // tc.block_size)
             tables, lens = bm.pack(running, width)
         host_ms.append((time.perf_counter() - t0) * 1e3)
         preempted += len(rec["preempted"])
@@ -95,11 +94,19 @@ def run(tc=wl.TRACE, seed=5, device="cuda", flush_bytes=256 << 20, partition_siz
             steps.append(None)
             continue
         runs = _runs(rec["op_kind"], rec["op_a"], rec["op_b"], rec["op_c"])
-        for kind, x in runs:
-            if kind == "w":
-                max_rows = max(max_rows, len(x))
-        max_running = max(max_running, len(running))
         steps.append((runs, np.ascontiguousarray(tables), np.ascontiguousarray(lens), int(lens.max())))
+    return {"steps": steps, "host_ms": host_ms, "num_blocks": nb, "prefix_slots": prefix_slots,
+            "preempted": preempted, "admitted": admitted}
+
+
+def run(tc=wl.TRACE, seed=5, device="cuda", flush_bytes=256 << 20, partition_size=0):
+    """Run the trace; returns per-step host and device times and the work done."""
+    import torch
+    dev = torch.device(device)
+    sc = schedule(tc, seed)
+    steps, host_ms, nb, prefix_slots = sc["steps"], sc["host_ms"], sc["num_blocks"], sc["prefix_slots"]
+    max_rows = max([len(prefix_slots)] + [len(x) for st in steps if st is not None for k, x in st[0] if k == "w"])
+    max_running = max([1] + [len(st[2]) for st in steps if st is not None])
 
     # ---- device buffers: pools, seeded rows, pinned metadata
     H, Hq, D, bs = tc.num_kv_heads, tc.num_heads, tc.head_dim, tc.block_size
@@ -124,8 +131,7 @@ def run(tc=wl.TRACE, seed=5, device="cuda", flush_bytes=256 << 20, partition_siz
             continue
         runs, tables, lens, mcl = s
         host_steps.append(([(k, pin(x)) for k, x in runs], pin(tables), pin(lens), mcl))
-    pa_cache_write(krows[:len(prefix_slots)], vrows[:len(prefix_slots)], kc, vc,
-                   torch.from_numpy(np.asarray(prefix_slots, dtype=np.int64)).to(dev))
+    pa_cache_write(krows[:len(prefix_slots)], vrows[:len(prefix_slots)], kc, vc, torch.from_numpy(prefix_slots).to(dev))
     torch.cuda.synchronize()
 
     # ---- the device work of every step, in issue order, between two events
@@ -167,4 +173,4 @@ def run(tc=wl.TRACE, seed=5, device="cuda", flush_bytes=256 << 20, partition_siz
     torch.cuda.synchronize()
     dev_ms = [x.elapsed_time(y) for x, y in ev]
     return {"device_ms": dev_ms, "host_ms": host_ms, "kv_bytes": kv_bytes, "num_blocks": nb,
-            "preempted": preempted, "admitted": admitted, "steps": len(dev_ms)}
+            "preempted": sc["preempted"], "admitted": sc["admitted"], "steps": len(dev_ms)}
