@@ -106,13 +106,17 @@ __global__ void __launch_bounds__(256) write_plan_kernel(const WriteArgs w, int 
 // partition, walked by a persistent grid; sequences with one partition were
 // finished by the attention kernel.  A row's statistics (lane i holds those of
 // partitions i and i + 32) and its first RB partials are all requested before
-// any of them is used, so a row of up to RB partitions costs one round trip to
-// L2, where the attention kernel has just left the partials.  Partials merge
-// in partition order (the bits do not depend on the grid).
+// any of them is used, then RB partials per round trip to L2, where the
+// attention kernel has just left them.  RB = 4 keeps the kernel near 50
+// registers, so about five CTAs of eight warps fit an SM and every split row
+// of the 70B-shaped batch (5,824) has its own warp: measured on B200, one step
+// of that batch took 0.2146 ms with RB = 4, 0.2160 ms with 8 and 0.2181 ms
+// with 16.  Partials merge in partition order (the bits do not depend on the
+// grid or on RB).
 // Partials of a row a lane holds in flight (a build-time knob: more partials per
 // round trip against more registers, so fewer warps resident).
 #ifndef PA_REDUCE_RB
-#define PA_REDUCE_RB 16
+#define PA_REDUCE_RB 4
 #endif
 constexpr int kReduceWarps = 8;                   // warps per reduce CTA
 template <typename T, int D>
