@@ -84,11 +84,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     }
 }
 
+// One answer for the whole warp (false if any lane says false): a wait that
+// expires in some lanes only must not split a warp in front of warp-wide
+// instructions.  All 32 lanes must call it.  PA_WAIT_VOTE=0 (a build-time
+// measurement knob) takes each lane's own answer instead.
+#ifndef PA_WAIT_VOTE
+#define PA_WAIT_VOTE 1
+#endif
+__device__ __forceinline__ bool warp_uniform(bool x) {
+#if PA_WAIT_VOTE
+    return __all_sync(0xffffffffu, x);
+#else
+    return x;
+#endif
+}
+
 // mbar_wait for a whole warp: every lane polls, and the answer is the same for
-// all of them (false if the wait gave up in any lane), so that a wait expiring
-// in some lanes only cannot split the warp.  All 32 lanes must call it.
+// all of them (false if the wait gave up in any lane).  All 32 lanes must call it.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const volatile int* abort) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+    return warp_uniform(mbar_wait(bar, parity, abort));
 }
 
 // Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from

@@ -14,9 +14,9 @@
 //    CTA handles all query heads of a kv-head group that share the K/V rows it
 //    streams, so each K/V byte leaves HBM once.  Contexts longer than the
 //    partition size are split.  A planning kernel sorts the items by length,
-//    longest first, and a persistent grid (a multiple of the SM count) deals
-//    them out in snake order (walk_first / walk_next), which evens out the
-//    CTAs' totals.
+//    longest first, and a persistent grid (a multiple of the SM count) walks
+//    them with a fixed stride (walk_first / walk_next): every round of the
+//    grid then takes items of nearly the same length.
 //  * One producer warp looks items up one ahead of their use, publishes each
 //    item's descriptor and q rows (one bulk copy) to the consumers through a
 //    double-buffered shared-memory slot, resolves block ids through the block
@@ -123,18 +123,28 @@ __device__ __forceinline__ WorkItem decode_item(const DecodeArgs& a, int i, bool
 }
 
 // The items a CTA of the persistent grid takes.  Round r covers items
-// [r * G, (r + 1) * G) with G = gridDim.x; CTA c takes item r * G + c in even
-// rounds and r * G + G - 1 - c in odd rounds (snake order).  With the plan
-// sorted longest first, the CTA that took a round's longest item takes the
-// next round's shortest, and the per-CTA sums of item lengths stay close to
-// their mean.  The sequence of items is increasing, so a walk ends at the
-// first index past the total.
+// [r * G, (r + 1) * G) with G = gridDim.x; CTA c takes item r * G + c (a fixed
+// stride), or, in snake order, r * G + c in even rounds and r * G + G - 1 - c
+// in odd rounds.  With the plan sorted longest first, every round holds items
+// of nearly the same length.  The sequence of items is increasing, so a walk
+// ends at the first index past the total.
+// Measured on B200 (70B-shaped batch, one box, two rounds each): the fixed
+// stride over the length-sorted plan gave 194.5 us per decode launch against
+// 196.6 us in snake order, although a model of per-CTA item lengths favours the
+// snake order; PA_DECODE_SNAKE=1 (a build-time knob) walks in snake order.
+#ifndef PA_DECODE_SNAKE
+#define PA_DECODE_SNAKE 0
+#endif
 __device__ __forceinline__ int walk_first() { return (int)blockIdx.x; }
 
 __device__ __forceinline__ int walk_next(int i) {
     const int64_t G = gridDim.x;
+#if PA_DECODE_SNAKE
     const int64_t r = i / G + 1;
     const int64_t n = r * G + ((r & 1) ? G - 1 - (int64_t)blockIdx.x : (int64_t)blockIdx.x);
+#else
+    const int64_t n = (int64_t)i + G;
+#endif
     return n > 0x7fffffff ? 0x7fffffff : (int)n;
 }
 
@@ -525,9 +535,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
     // same for every lane of the warp (the lanes poll on their own, and the
     // warp-wide matrix instructions that follow need all of them).
     auto acquire = [&](uint32_t c) -> bool {
-        const int slot = c % C::NSTAGES;
-        const bool got = !*abort_flag && mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) {
+        if (!mbar_wait_warp(&full[c % C::NSTAGES], (c / C::NSTAGES) & 1u, abort_flag)) {
             *abort_flag = 1;
             return false;
         }
@@ -546,7 +554,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
         WorkItem w;
         bool have_q = false;
         const bool got = !*abort_flag && mbar_wait(&item_full[b], (k >> 1) & 1u, abort_flag);
-        if (__all_sync(0xffffffffu, got)) {
+        if (warp_uniform(got)) {
             const int* src = info + b * 8;
             w.s = src[0];
             w.p = src[1];

@@ -12,8 +12,8 @@
 namespace pa_dev {
 
 // Orders the (sequence, partition) pairs that the attention kernels walk by
-// their token count, longest first, so that the snake walk (walk_next) deals
-// every CTA of the persistent grid about the same number of tokens.  Counts
+// their token count, longest first, so that each round of the persistent
+// grid's walk (walk_next) deals its CTAs items of nearly the same length.  Counts
 // are bucketed by 16-token step: a whole partition is bucket P / 16, a
 // sequence's last partition the bucket of what is left of it, an empty
 // context bucket 0.  One CTA: a histogram of the buckets, a descending scan

@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(VerifyCfg<T, D>::THREADS, 2)
     auto acquire = [&](uint32_t c) -> bool {
         const int slot = c % C::NSTAGES;
         const bool got = !*abort_flag && mbar_wait(&full[slot], (c / C::NSTAGES) & 1u, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) {
+        if (!warp_uniform(got)) {
             *abort_flag = 1;
             return false;
         }
