@@ -79,6 +79,8 @@ struct DecodeArgs {
     float* part_o;             // [num_seqs * num_heads, max_partitions, head_dim]
     int* merge_count;          // split mode, fused merge: finished partitions per (seq, kv head, chunk);
                                // nullptr: partitions are merged by reduce_kernel instead
+    int* work_counter;         // decode, split mode: items of the plan's tail handed out so far (zeroed by
+                               // the plan kernel); nullptr: every item is dealt by the fixed stride
     int num_queries;           // query rows per sequence and head (1: decode; > 1: verification pass)
 };
 
@@ -146,6 +148,29 @@ __device__ __forceinline__ int walk_next(int i) {
     const int64_t n = (int64_t)i + G;
 #endif
     return n > 0x7fffffff ? 0x7fffffff : (int)n;
+}
+
+// The decode kernel deals the last PA_DECODE_DYN_ROUNDS rounds of the sorted
+// plan (its shortest items) dynamically: a CTA that runs out of its own items
+// takes the next one from an atomic counter, so CTAs that ran faster absorb the
+// tail.  0: every item by the fixed stride.
+#ifndef PA_DECODE_DYN_ROUNDS
+#define PA_DECODE_DYN_ROUNDS 2
+#endif
+
+// Named barrier `id` over `threads` threads (a multiple of 32) that also returns
+// the AND of every participating thread's `pred`: one answer for all of them.
+__device__ __forceinline__ bool barrier_and(int id, int threads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(threads)
+        : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -412,10 +437,24 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
                 ids[k] = j < nblk ? trow[j] : 0;
             }
         };
+        // Items below dyn_start follow the fixed stride; the rest are handed out
+        // one at a time by the atomic counter (lane 0 takes, the warp shares).
+        const int dyn_start = a.work_counter ? max(0, total - PA_DECODE_DYN_ROUNDS * (int)gridDim.x) : total;
+        auto take_dynamic = [&]() -> int {
+            int d = 0;
+            if (lane == 0) d = atomicAdd(a.work_counter, 1);
+            d = __shfl_sync(0xffffffffu, d, 0);
+            return d >= total - dyn_start ? total : dyn_start + d;
+        };
+        auto next_item = [&](int cur) -> int {
+            const int nx = walk_next(cur);
+            return nx < dyn_start ? nx : (dyn_start < total ? take_dynamic() : total);
+        };
         uint32_t stage = 0;
         uint32_t k = 0;                                   // items published
         bool ok = true;
         int i = walk_first();
+        if (i >= dyn_start) i = dyn_start < total ? take_dynamic() : total;
         WorkItem w{};
         int32_t ids[C::TPL];
         if (i < total) {
@@ -431,6 +470,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
             }
             if (lane == 0) {
                 int* dst = info + b * 8;
+                dst[7] = 1;                   // an item (0: no more items)
                 dst[0] = w.s;
                 dst[1] = w.p;
                 dst[2] = w.h;
@@ -449,7 +489,7 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
                 }
             }
             // look the next item up while this item's stages wait for ring slots
-            const int inext = walk_next(i);
+            const int inext = next_item(i);
             WorkItem wn{};
             int32_t idn[C::TPL];
             if (inext < total) {
@@ -502,6 +542,19 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
 #pragma unroll
             for (int kk = 0; kk < C::TPL; ++kk) ids[kk] = idn[kk];
         }
+        if (ok) {
+            // no more items: the closing slot tells the consumers to stop
+            const int b = k & 1;
+            if (mbar_wait_warp(&item_empty[b], ((k >> 1) & 1u) ^ 1u, abort_flag)) {
+                if (lane == 0) {
+                    info[b * 8 + 7] = 0;
+                    mbar_arrive(&item_full[b]);
+                }
+                ++k;
+            } else {
+                ok = false;
+            }
+        }
         if (!ok) {
             if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
             *abort_flag = 1;
@@ -546,28 +599,28 @@ __global__ void __launch_bounds__(DecodeCfg<T, D, GC, TENSOR>::THREADS, TENSOR ?
         if (lane == 0) mbar_arrive(&empty[c % C::NSTAGES]);
     };
 
-    uint32_t k = 0;                                       // items taken
-    for (int i = walk_first(); i < total; i = walk_next(i), ++k) {
+    // Items in the order the producer publishes them, until its closing slot.
+    // Whether the slot arrived is agreed by all four warps in one barrier
+    // reduction, so that a wait giving up in one warp only cannot leave the
+    // others at a named barrier of an item it will not take.
+    for (uint32_t k = 0;; ++k) {
         const int b = k & 1;
-        // the item as the producer published it; after a give-up, looked up here
-        // (every warp then still takes the same items through the same barriers)
-        WorkItem w;
-        bool have_q = false;
-        const bool got = !*abort_flag && mbar_wait(&item_full[b], (k >> 1) & 1u, abort_flag);
-        if (warp_uniform(got)) {
-            const int* src = info + b * 8;
-            w.s = src[0];
-            w.p = src[1];
-            w.h = src[2];
-            w.gc = src[3];
-            w.t0 = src[4];
-            w.n = src[5];
-            w.np = src[6];
-            have_q = true;
-        } else {
+        const bool got = mbar_wait(&item_full[b], (k >> 1) & 1u, abort_flag);
+        if (!barrier_and(2, NCT, got)) {
             *abort_flag = 1;
-            w = decode_item(a, i, false);
+            break;
         }
+        const int* src = info + b * 8;
+        if (src[7] == 0) break;                       // no more items
+        WorkItem w;
+        w.s = src[0];
+        w.p = src[1];
+        w.h = src[2];
+        w.gc = src[3];
+        w.t0 = src[4];
+        w.n = src[5];
+        w.np = src[6];
+        const bool have_q = true;
         const int gq = min(GC, a.group - w.gc * GC);
         const int hq0 = w.h * a.group + w.gc * GC;
         const int64_t row0 = (int64_t)w.s * a.num_heads + hq0;

@@ -21,7 +21,8 @@ namespace pa_dev {
 // partitions together) and one per last partition.  The order inside a bucket
 // does not matter: results never depend on which CTA takes an item.  The plan
 // kernel also lists the sequences with more than one partition for the reduce
-// and clears the fused-merge counters for this call.
+// and clears the fused-merge counters and the decode kernel's item counter for
+// this call.
 constexpr int kPlanBuckets = 1024 / 16 + 1;        // partitions of up to 1024 tokens
 __device__ __forceinline__ void build_plan(const DecodeArgs& a, int2* plan, int* count, int* split_seqs,
                                            int* merge_count, int num_counters) {
@@ -33,7 +34,10 @@ __device__ __forceinline__ void build_plan(const DecodeArgs& a, int2* plan, int*
     const int full = P >> 4;                     // bucket of a whole partition
     for (int i = tid; i < kPlanBuckets; i += blockDim.x) hist[i] = 0;
     for (int i = tid; i < num_counters; i += blockDim.x) merge_count[i] = 0;
-    if (tid == 0) nsplit = 0;
+    if (tid == 0) {
+        nsplit = 0;
+        count[2] = 0;                            // the decode kernel's counter of dynamically dealt items
+    }
     __syncthreads();
     for (int s = tid; s < a.num_seqs; s += blockDim.x) {
         const int ctx = clamp_context(a, s, true);

@@ -183,8 +183,8 @@ WsLayout ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t maxP) {
     size_t off = 0;
     w.plan = off;
     off = align256(off + (size_t)(S * maxP) * sizeof(int2));
-    w.count = off;                                      // pairs in the plan, split sequences
-    off = align256(off + 2 * sizeof(int));
+    w.count = off;                                      // pairs in the plan, split sequences, items dealt
+    off = align256(off + 3 * sizeof(int));
     w.split = off;                                      // the split sequences
     off = align256(off + (size_t)S * sizeof(int));
     w.counters = off;                                   // fused-merge counters, <= S * Hq of them
@@ -497,6 +497,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
         int2* plan = reinterpret_cast<int2*>(ws + L.plan);
         int* count = reinterpret_cast<int*>(ws + L.count);
         int* split = reinterpret_cast<int*>(ws + L.split);
+        a.work_counter = count + 2;
         if (wr) {
             LaunchScope scope(PA_KERNEL_WRITE_PLAN, s);
             const unsigned wb = write_grid(*wr);
