@@ -113,7 +113,11 @@ struct VerifyTcCfg {
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
     static constexpr int OFF_TABLE = (OFF_ABORT + 4 + 15) / 16 * 16;
     static constexpr int MAX_TABLE = 1024 / 8;
-    static constexpr size_t SMEM = 1024 + (size_t)OFF_TABLE + MAX_TABLE * 4;
+    // 1024 bytes of slack let the kernel round its base up to 1024 bytes.  Six
+    // slots fit two CTAs on an SM only without the slack: the kernel then needs
+    // the base it is given to be 1024-byte aligned, and checks it.
+    static constexpr int ALIGN_SLACK = NSLOTS >= 6 ? 0 : 1024;
+    static constexpr size_t SMEM = ALIGN_SLACK + (size_t)OFF_TABLE + MAX_TABLE * 4;
     // A tcgen05.mma costs its issuing thread about 57 cycles whatever its N; two
     // issuing warps (S in warp 1, P.V in warp 6) double the rate the chunks need.
     // The S warp's wait for P.V of chunk g - 2 orders the two streams where they
@@ -143,6 +147,12 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    if constexpr (C::ALIGN_SLACK == 0) {
+        if (smem != smem_raw) {                  // no room to align: give up before any barrier
+            if (threadIdx.x == 0) flag_error(PA_DEVERR_TIMEOUT);
+            return;
+        }
+    }
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* full = bar;                        // [NSLOTS] a slot's TMA bytes landed
     uint64_t* s_full = bar + C::NSLOTS;          // [NPH] S of chunk g done (commit), copy g % NPH

@@ -249,6 +249,30 @@ bool encode_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, int hea
     return r == CUDA_SUCCESS;
 }
 
+// The pool as the 4-D tensor (128-byte head_dim slice, token row, slice index,
+// kv head), innermost first.  One box is one block of one kv head with every
+// slice: the slices land one after another, each as block_size rows of 128
+// bytes with the 128-byte swizzle (the decode kernel's stage layout).
+bool encode_pool_map_blocks(CUtensorMap* map, const void* pool, pa_dtype dtype, int head_dim, int num_kv_heads,
+                            int num_blocks, int block_size) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t elt = dtype == PA_F32 ? 4 : 2;
+    const CUtensorMapDataType t = dtype == PA_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                  : dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint32_t slices = (cuuint32_t)(head_dim * elt / 128);
+    cuuint64_t dims[4] = {128 / elt, (cuuint64_t)num_blocks * (cuuint64_t)block_size, slices,
+                          (cuuint64_t)num_kv_heads};
+    cuuint64_t strides[3] = {(cuuint64_t)num_kv_heads * head_dim * elt, 128, (cuuint64_t)head_dim * elt};
+    cuuint32_t box[4] = {(cuuint32_t)(128 / elt), (cuuint32_t)block_size, slices, 1u};
+    cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
+    CUresult r = enc(map, t, 4, const_cast<void*>(pool), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <typename T, int D, int GC, bool TENSOR>
 pa_status launch_decode(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                         int64_t pair_upper, cudaStream_t stream) {
@@ -474,11 +498,18 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
     a.max_partitions = (int)maxP;
     a.num_queries = 1;
 
-    const int box_rows = block_size;          // one TMA box = one block of one kv head, one 128-byte slice
     CUtensorMap tk, tv;
+#if PA_DECODE_BOX_BLOCK
+    // one TMA box = one block of one kv head, every 128-byte slice of head_dim
+    if (!encode_pool_map_blocks(&tk, k_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size) ||
+        !encode_pool_map_blocks(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size))
+        return PA_ERR_CUDA;
+#else
+    const int box_rows = block_size;          // one TMA box = one block of one kv head, one 128-byte slice
     if (!encode_pool_map(&tk, k_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, box_rows) ||
         !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, box_rows))
         return PA_ERR_CUDA;
+#endif
     if (maxP > 1) {
         const WsLayout L = ws_layout(num_seqs, num_heads, head_dim, maxP);
         if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
