@@ -85,6 +85,8 @@ typedef struct {
 #define PA_DEVERR_BLOCK_ID    0x2u  /* decode / copy: block id outside [0, num_blocks) (clamped / skipped) */
 #define PA_DEVERR_CONTEXT_LEN 0x4u  /* decode: context_len < 0, > max_context_len or > table width (clamped) */
 #define PA_DEVERR_TIMEOUT     0x8u  /* decode: a bounded wait on a staging barrier expired (CTA abandoned its work) */
+#define PA_DEVERR_SMEM_ALIGN  0x10u /* verify (tcgen05): the dynamic shared memory base was not 1024-byte aligned;
+                                       the kernel needs it aligned to fit two CTAs per SM and did no work */
 
 /* ------------------------------------------------------------------------ */
 /* Device hot path                                                           */

@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3:
                 4: "PA_ERR_CUDA", 5: "PA_ERR_DEVICE"}
 PA_ERR_NO_BLOCKS = 3
 DEVERR_SLOT, DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+DEVERR_SMEM_ALIGN = 0x10
 KERNELS = ("cache_write", "decode", "reduce", "plan", "copy_blocks", "verify", "swap", "write_plan")
 DEFAULT_PARTITION = 512
 

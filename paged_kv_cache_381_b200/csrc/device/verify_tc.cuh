@@ -11,7 +11,7 @@
 //    query rows).  The rows form one M = 64 tile; the partition is walked in
 //    chunks of 64 tokens.
 //  * Warp 0 streams K and V chunks through TMA tiled boxes into a ring of
-//    five slots (slot = 64 token rows of one kv head; each 128-byte head_dim
+//    six slots (slot = 64 token rows of one kv head; each 128-byte head_dim
 //    slice of the 64 rows is one 128-byte-swizzled array), K running one
 //    chunk ahead of V: K0 K1 V0 K2 V1 ... .  A slot is refilled once the
 //    products that read its previous contents are done: the producer waits
@@ -54,7 +54,10 @@ namespace pa_dev {
 #define PA_VERIFY_TC_PSPLIT 2
 #endif
 #ifndef PA_VERIFY_TC_SLOTS
-#define PA_VERIFY_TC_SLOTS 5
+// Measured on B200 (6 candidate tokens, two runs each): 6 slots 247.2 us vs 5
+// slots 252.8 us on the 70B-shaped batch, 213.4 vs 213.65 us (7B), 211.85 vs
+// 211.05 us (long contexts).
+#define PA_VERIFY_TC_SLOTS 6
 #endif
 #ifndef PA_VERIFY_TC_PTMEM
 #define PA_VERIFY_TC_PTMEM 1     // 1: p written to tensor memory over its S buffer, P.V reads A from there
@@ -149,7 +152,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     if constexpr (C::ALIGN_SLACK == 0) {
         if (smem != smem_raw) {                  // no room to align: give up before any barrier
-            if (threadIdx.x == 0) flag_error(PA_DEVERR_TIMEOUT);
+            if (threadIdx.x == 0) flag_error(PA_DEVERR_SMEM_ALIGN);
             return;
         }
     }
