@@ -82,8 +82,8 @@ struct DecodeArgs {
     float* part_o;             // [num_seqs * num_heads, max_partitions, head_dim]
     int* merge_count;          // split mode, fused merge: finished partitions per (seq, kv head, chunk);
                                // nullptr: partitions are merged by reduce_kernel instead
-    int* work_counter;         // decode, split mode: items of the plan's tail handed out so far (zeroed by
-                               // the plan kernel); nullptr: every item is dealt by the fixed stride
+    int* work_counter;         // split mode (decode, tcgen05 verification): items of the plan's tail handed
+                               // out so far (zeroed by the plan kernel); nullptr: every item by the stride
     int num_queries;           // query rows per sequence and head (1: decode; > 1: verification pass)
 };
 

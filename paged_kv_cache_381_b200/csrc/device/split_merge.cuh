@@ -36,7 +36,7 @@ __device__ __forceinline__ void build_plan(const DecodeArgs& a, int2* plan, int*
     for (int i = tid; i < num_counters; i += blockDim.x) merge_count[i] = 0;
     if (tid == 0) {
         nsplit = 0;
-        count[2] = 0;                            // the decode kernel's counter of dynamically dealt items
+        count[2] = 0;                            // the counter of dynamically dealt items (decode, verify)
     }
     __syncthreads();
     for (int s = tid; s < a.num_seqs; s += blockDim.x) {

@@ -9,7 +9,9 @@
 // Design (2 CTAs per SM, each holding 256 of the SM's 512 TMEM columns):
 //  * Item = (sequence, partition of 512 or 1024 tokens, kv head, chunk of <= 64
 //    query rows).  The rows form one M = 64 tile; the partition is walked in
-//    chunks of 64 tokens.
+//    chunks of 64 tokens.  A CTA walks the length-sorted plan with a fixed
+//    stride; the last rounds are dealt from an atomic counter by the producer,
+//    which publishes each item's index to the other warps in item slots.
 //  * Warp 0 streams K and V chunks through TMA tiled boxes into a ring of
 //    six slots (slot = 64 token rows of one kv head; each 128-byte head_dim
 //    slice of the 64 rows is one 128-byte-swizzled array), K running one
@@ -58,6 +60,15 @@ namespace pa_dev {
 // slots 252.8 us on the 70B-shaped batch, 213.4 vs 213.65 us (7B), 211.85 vs
 // 211.05 us (long contexts).
 #define PA_VERIFY_TC_SLOTS 6
+#endif
+#ifndef PA_VERIFY_TC_DYN_ROUNDS
+// The last rounds of the length-sorted plan (its shortest items) are handed out
+// one at a time from an atomic counter; 0: every item by the fixed stride.
+// Measured on B200 (6 candidate tokens, one box, three runs each): 0 / 2 / 3
+// rounds 249.9 / 247.7 / 248.2 us on the 70B-shaped batch, 215.6 / 212.2 /
+// 212.7 us (7B), 215.0 / 211.5 / 211.4 us (long contexts); the kernel without
+// the item slots 248.4 / 214.7 / 213.6 us.
+#define PA_VERIFY_TC_DYN_ROUNDS 2
 #endif
 #ifndef PA_VERIFY_TC_PTMEM
 #define PA_VERIFY_TC_PTMEM 1     // 1: p written to tensor memory over its S buffer, P.V reads A from there
@@ -110,11 +121,14 @@ struct VerifyTcCfg {
     static constexpr int OFF_Q = NSLOTS * SLOT_BYTES;
     static constexpr int OFF_P = OFF_Q + Q_BYTES;            // tile (buffer b, part h) at (2 b + h) * P_TILE
     static constexpr int OFF_BAR = OFF_P + 2 * PBUF * P_TILE;
-    // barriers: full[NSLOTS], s_full[NPH], q_full, q_empty, p_full, o_full[NPH], o_empty, drain
-    static constexpr int NBAR = NSLOTS + 2 * NPH + 5;
+    // barriers: full[NSLOTS], s_full[NPH], q_full, q_empty, p_full, o_full[NPH], o_empty, drain,
+    // dyn_full[NDYN], dyn_empty[NDYN]
+    static constexpr int NDYN = 4;                           // item slots of the dynamic tail
+    static constexpr int NBAR = NSLOTS + 2 * NPH + 5 + 2 * NDYN;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;      // allocated TMEM address
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
-    static constexpr int OFF_TABLE = (OFF_ABORT + 4 + 15) / 16 * 16;
+    static constexpr int OFF_DYN = OFF_ABORT + 4;            // item index per slot (-1: no more items)
+    static constexpr int OFF_TABLE = (OFF_DYN + NDYN * 4 + 15) / 16 * 16;
     static constexpr int MAX_TABLE = 1024 / 8;
     // 1024 bytes of slack let the kernel round its base up to 1024 bytes.  Six
     // slots fit two CTAs on an SM only without the slack: the kernel then needs
@@ -165,6 +179,9 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     uint64_t* o_full = q_full + 3;               // [NPH] P.V of chunk g done (commit), copy g % NPH
     uint64_t* o_empty = o_full + C::NPH;         // O read by the epilogue (128 arrivals)
     uint64_t* drain = o_empty + 1;               // every MMA done, before TMEM is freed (one commit per issuer)
+    uint64_t* dyn_full = drain + 1;              // [NDYN] item slot written by the producer
+    uint64_t* dyn_empty = dyn_full + C::NDYN;    // [NDYN] item slot read by the S, P.V and softmax warps
+    volatile int* dyn_item = reinterpret_cast<volatile int*>(smem + C::OFF_DYN);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + C::OFF_TABLE);
@@ -184,6 +201,10 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         mbar_init(p_full, 128);
         mbar_init(o_empty, 128);
         mbar_init(drain, C::TWO_ISSUERS ? 2 : 1);
+        for (int i = 0; i < C::NDYN; ++i) {
+            mbar_init(&dyn_full[i], 1);
+            mbar_init(&dyn_empty[i], C::TWO_ISSUERS ? 6 : 5);     // one per consumer warp
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -201,11 +222,39 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     // blockIdx.x, then + gridDim.x, ...): on the 70B-shaped batch with 6
     // candidate tokens this kernel measured 254.5 us with the stride and
     // 263.2 us in snake order (round r reversed when r is odd; same B200, same
-    // build otherwise).
+    // build otherwise, five ring slots, no dynamic tail).
     const int pairs = a.max_partitions == 1 ? a.num_seqs : *a.plan_count;
     const int total = pairs * a.num_kv_heads * a.n_gchunks;
     const int bs = 1 << a.log2_bs;
     const int box_bytes = bs * 128;
+    // A CTA takes items blockIdx.x, + gridDim.x, ... of the sorted plan while they
+    // lie below dyn_start; past it (the last rounds, the shortest items) the
+    // producer takes the next item from the counter and publishes its index in
+    // the next item slot for the other warps.  Each role walks the same sequence:
+    // next_static gives the successor of `cur` in the fixed-stride part (cur < 0:
+    // the first item), or -1 once the walk reaches the dynamic part.
+    const bool dyn_tail = a.work_counter != nullptr && PA_VERIFY_TC_DYN_ROUNDS > 0;
+    const int dyn_start = dyn_tail ? max(0, total - PA_VERIFY_TC_DYN_ROUNDS * (int)gridDim.x) : total;
+    auto next_static = [&](int cur) -> int {
+        if (cur >= dyn_start) return -1;
+        const int s = cur < 0 ? (int)blockIdx.x : cur + (int)gridDim.x;
+        return s < dyn_start ? s : -1;
+    };
+    // a consumer warp's next dynamic item (total when there is none); the whole
+    // warp reads the slot before its lane 0 releases it
+    auto read_dynamic = [&](uint32_t& dk, bool& ok) -> int {
+        if (!dyn_tail) return total;
+        const int slot = (int)(dk % C::NDYN);
+        if (!mbar_wait(&dyn_full[slot], (dk / C::NDYN) & 1u, abort_flag)) {
+            ok = false;
+            return total;
+        }
+        const int it = dyn_item[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dyn_empty[slot]);
+        ++dk;
+        return it < 0 ? total : it;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -221,7 +270,31 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
 #pragma unroll
         for (int k = 0; k < C::NSLOTS; ++k) hist[k] = 0;
         bool ok = true;
-        for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        uint32_t dk = 0;                                    // dynamic items taken so far
+        // the item after `cur`: by the stride, else the next one of the counter,
+        // published in the next item slot (-1 there: no more items)
+        auto take = [&](int cur) -> int {
+            if (!ok) return total;
+            const int st = next_static(cur);
+            if (st >= 0) return st;
+            if (!dyn_tail) return total;
+            const int slot = (int)(dk % C::NDYN);
+            if (!mbar_wait(&dyn_empty[slot], ((dk / C::NDYN) & 1u) ^ 1u, abort_flag)) {
+                ok = false;
+                return total;
+            }
+            int it = 0;
+            if (lane == 0) {
+                it = dyn_start + atomicAdd(a.work_counter, 1);
+                if (it >= total) it = -1;
+                dyn_item[slot] = it;
+                mbar_arrive(&dyn_full[slot]);
+            }
+            it = __shfl_sync(0xffffffffu, it, 0);
+            ++dk;
+            return it < 0 ? total : it;
+        };
+        for (int i = take(-1); i < total && ok; i = take(i)) {
             const WorkItem w = decode_item(a, i, lane == 0);
             if (w.n == 0) continue;
             const int nblk = (w.n + bs - 1) >> a.log2_bs;
@@ -375,7 +448,13 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             tc::fence_after_sync();
             return issue_pv(pos, c, n, g, c == 0);
         };
-        for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        uint32_t dk = 0;
+        auto next_item = [&](int cur) -> int {
+            if (!ok) return total;
+            const int st = next_static(cur);
+            return st >= 0 ? st : read_dynamic(dk, ok);
+        };
+        for (int i = next_item(-1); i < total && ok; i = next_item(i)) {
             const WorkItem w = decode_item(a, i, false);
             if (w.n == 0) continue;
             const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
@@ -490,7 +569,14 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         };
         bool ok = true;
         int staged = -1;                                 // item whose Q tile is already written
-        for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        uint32_t dk = 0;
+        auto next_item = [&](int cur) -> int {
+            if (!ok) return total;
+            const int st = next_static(cur);
+            return st >= 0 ? st : read_dynamic(dk, ok);
+        };
+        int i = next_item(-1);
+        while (i < total && ok) {
             const WorkItem w = decode_item(a, i, false);
             const int ctx = clamp_context(a, w.s, false);
             if (w.n == 0) {                              // empty context: zero rows
@@ -501,6 +587,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     row_in(w, ctx, e / D, orow, pos);
                     outg[orow * D + (e % D)] = Tr::from_float(0.f);
                 }
+                i = next_item(i);
                 continue;
             }
             if (staged != i && !(ok = stage_q(w, ctx))) break;
@@ -622,8 +709,9 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             if (!ok) break;
             // ---- the next item's Q tile now, so that its first S products run while
             // this item's epilogue does
+            const int inext = next_item(i);
+            if (!ok) break;
             {
-                const int inext = i + gridDim.x;
                 if (inext < total) {
                     const WorkItem wn = decode_item(a, inext, false);
                     if (wn.n > 0) {
@@ -672,6 +760,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             }
             tc::fence_before_sync();
             mbar_arrive(o_empty);
+            i = inext;
         }
         if (!ok) {
             if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);

@@ -849,6 +849,7 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
         a.part_l = reinterpret_cast<float*>(ws + L.l);
         a.part_o = reinterpret_cast<float*>(ws + L.o);
         a.merge_count = nullptr;
+        a.work_counter = reinterpret_cast<int*>(ws + L.count) + 2;   // zeroed by the plan kernel
         LaunchScope scope(PA_KERNEL_PLAN, s);
         const int threads = std::min(1024, std::max(32, (num_seqs + 31) / 32 * 32));
         if (launch_dependent(pa_dev::plan_kernel, dim3(1), dim3(threads), 0, s, a,
