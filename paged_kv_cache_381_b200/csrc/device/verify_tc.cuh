@@ -13,7 +13,8 @@
 //    stride; the last rounds are dealt from an atomic counter by the producer,
 //    which publishes each item's index to the other warps in item slots.
 //  * Warp 0 streams K and V chunks through TMA tiled boxes into a ring of
-//    six slots (slot = 64 token rows of one kv head; each 128-byte head_dim
+//    five slots, and each item's q rows into one of two q tiles an item ahead
+//    (slot = 64 token rows of one kv head; each 128-byte head_dim
 //    slice of the 64 rows is one 128-byte-swizzled array), K running one
 //    chunk ahead of V: K0 K1 V0 K2 V1 ... .  A slot is refilled once the
 //    products that read its previous contents are done: the producer waits
@@ -55,11 +56,19 @@ namespace pa_dev {
 // 2: split for bf16 only (an fp16 p already carries 11 significant bits)
 #define PA_VERIFY_TC_PSPLIT 2
 #endif
+#ifndef PA_VERIFY_TC_QTMA
+// 1: two q tiles; when an item's query rows are one tile (group x queries <= 64)
+// the producer brings its tile by TMA an item ahead.  0: one q tile, staged by
+// the softmax warps after the previous item's last chunk.  Measured on B200 (6
+// candidate tokens, one box, three runs each): 239.8 vs 248.2 us on the
+// 70B-shaped batch, 207.5 vs 210.3 us (7B), 206.2 vs 210.3 us (long contexts).
+#define PA_VERIFY_TC_QTMA 1
+#endif
 #ifndef PA_VERIFY_TC_SLOTS
 // Measured on B200 (6 candidate tokens, two runs each): 6 slots 247.2 us vs 5
 // slots 252.8 us on the 70B-shaped batch, 213.4 vs 213.65 us (7B), 211.85 vs
-// 211.05 us (long contexts).
-#define PA_VERIFY_TC_SLOTS 6
+// 211.05 us (long contexts).  With two q tiles, five slots fit.
+#define PA_VERIFY_TC_SLOTS (PA_VERIFY_TC_QTMA ? 5 : 6)
 #endif
 #ifndef PA_VERIFY_TC_DYN_ROUNDS
 // The last rounds of the length-sorted plan (its shortest items) are handed out
@@ -109,6 +118,7 @@ struct VerifyTcCfg {
     static constexpr int M = 64;                             // query rows per item
     static constexpr int Q_SLICE = M * 128;                  // one 128-byte slice of the Q tile
     static constexpr int Q_BYTES = NH * Q_SLICE;
+    static constexpr int QBUF = PA_VERIFY_TC_QTMA ? 2 : 1;   // q tiles (item k uses tile k % QBUF)
     static constexpr int P_TILE = M * 128;                   // 64 rows x 64 tokens, one 128-byte atom column
     static constexpr bool PTMEM = PA_VERIFY_TC_PTMEM != 0;
     static constexpr int PBUF = PTMEM ? 0 : PA_VERIFY_TC_PBUF;  // P tiles in shared memory
@@ -119,21 +129,22 @@ struct VerifyTcCfg {
     static constexpr int O_COL = 128;
     // shared memory: ring, Q, P (buffers x {value, remainder}), barriers, table
     static constexpr int OFF_Q = NSLOTS * SLOT_BYTES;
-    static constexpr int OFF_P = OFF_Q + Q_BYTES;            // tile (buffer b, part h) at (2 b + h) * P_TILE
+    static constexpr int OFF_P = OFF_Q + QBUF * Q_BYTES;     // tile (buffer b, part h) at (2 b + h) * P_TILE
     static constexpr int OFF_BAR = OFF_P + 2 * PBUF * P_TILE;
-    // barriers: full[NSLOTS], s_full[NPH], q_full, q_empty, p_full, o_full[NPH], o_empty, drain,
-    // dyn_full[NDYN], dyn_empty[NDYN]
+    // barriers: full[NSLOTS], s_full[NPH], p_full[2], o_full[NPH], o_empty, drain, q_full[QBUF],
+    // q_empty[QBUF], dyn_full[NDYN], dyn_empty[NDYN]
     static constexpr int NDYN = 4;                           // item slots of the dynamic tail
-    static constexpr int NBAR = NSLOTS + 2 * NPH + 5 + 2 * NDYN;
+    static constexpr int NBAR = NSLOTS + 2 * NPH + 4 + 2 * QBUF + 2 * NDYN;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;      // allocated TMEM address
     static constexpr int OFF_ABORT = OFF_TMEM + 4;
     static constexpr int OFF_DYN = OFF_ABORT + 4;            // item index per slot (-1: no more items)
     static constexpr int OFF_TABLE = (OFF_DYN + NDYN * 4 + 15) / 16 * 16;
     static constexpr int MAX_TABLE = 1024 / 8;
-    // 1024 bytes of slack let the kernel round its base up to 1024 bytes.  Six
-    // slots fit two CTAs on an SM only without the slack: the kernel then needs
-    // the base it is given to be 1024-byte aligned, and checks it.
-    static constexpr int ALIGN_SLACK = NSLOTS >= 6 ? 0 : 1024;
+    // 1024 bytes of slack let the kernel round its base up to 1024 bytes.  When
+    // two CTAs fit on an SM (228 KB, 1 KB reserved per CTA) only without the
+    // slack, the kernel needs the base it is given to be 1024-byte aligned, and
+    // checks it.
+    static constexpr int ALIGN_SLACK = 2 * (OFF_TABLE + MAX_TABLE * 4 + 2048) <= 228 * 1024 ? 1024 : 0;
     static constexpr size_t SMEM = ALIGN_SLACK + (size_t)OFF_TABLE + MAX_TABLE * 4;
     // A tcgen05.mma costs its issuing thread about 57 cycles whatever its N; two
     // issuing warps (S in warp 1, P.V in warp 6) double the rate the chunks need.
@@ -153,7 +164,7 @@ struct VerifyTcCfg {
 template <typename T, int D>
 __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     verify_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
-                     const __grid_constant__ CUtensorMap tmap_v) {
+                     const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_q) {
     using C = VerifyTcCfg<T, D>;
     using Tr = ElemTraits<T>;
     using MO = MmaOps<T>;
@@ -173,13 +184,22 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* full = bar;                        // [NSLOTS] a slot's TMA bytes landed
     uint64_t* s_full = bar + C::NSLOTS;          // [NPH] S of chunk g done (commit), copy g % NPH
-    uint64_t* q_full = s_full + C::NPH;          // Q tile written (128 arrivals)
-    uint64_t* q_empty = q_full + 1;              // last S of the item done (commit)
-    uint64_t* p_full = q_full + 2;               // chunk's S read, O rescaled, p written (128 arrivals)
-    uint64_t* o_full = q_full + 3;               // [NPH] P.V of chunk g done (commit), copy g % NPH
+    // [2] chunk g's S read, O rescaled, p written (128 arrivals), copy g % 2.  Two
+    // copies: the P.V warp waits for chunk g's phase in order, and one barrier
+    // could complete the phases of g and g + 1 before that warp looks (it may be
+    // reading the next item's descriptor while the softmax warps finish two
+    // chunks), after which the parity test would wait for a phase that never
+    // comes.  The arrivals for chunk g + 2 need S(g + 2), which waits for P.V of
+    // g, so copy g % 2 cannot move past the phase of g unseen; and a warp that
+    // arrives for chunk g has seen S(g) done, so the phase of g - 2 on the same
+    // copy is complete and the arrival counts toward the phase of g.
+    uint64_t* p_full = s_full + C::NPH;
+    uint64_t* o_full = p_full + 2;               // [NPH] P.V of chunk g done (commit), copy g % NPH
     uint64_t* o_empty = o_full + C::NPH;         // O read by the epilogue (128 arrivals)
     uint64_t* drain = o_empty + 1;               // every MMA done, before TMEM is freed (one commit per issuer)
-    uint64_t* dyn_full = drain + 1;              // [NDYN] item slot written by the producer
+    uint64_t* q_full = drain + 1;                // [QBUF] q tile written (TMA bytes, or 128 arrivals)
+    uint64_t* q_empty = q_full + C::QBUF;        // [QBUF] last S of the tile's item done (commit)
+    uint64_t* dyn_full = q_empty + C::QBUF;      // [NDYN] item slot written by the producer
     uint64_t* dyn_empty = dyn_full + C::NDYN;    // [NDYN] item slot read by the S, P.V and softmax warps
     volatile int* dyn_item = reinterpret_cast<volatile int*>(smem + C::OFF_DYN);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
@@ -190,15 +210,30 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // An item's query rows are one box of q viewed as (head_dim, head, sequence x
+    // query) when they are all of one kv head's group x queries (one row tile):
+    // then the producer loads the tile by TMA and rows past them stay zero.
+    const bool q_by_tma = C::QBUF == 2 && a.n_gchunks == 1;
+    if (q_by_tma) {
+        const int R = a.group * a.num_queries;
+        for (int e = threadIdx.x; e < C::QBUF * C::NH * C::M * 8; e += blockDim.x) {
+            const int row = (e >> 3) % C::M;
+            if (row >= R) reinterpret_cast<uint4*>(smem + C::OFF_Q)[e] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        tc::fence_proxy_async_smem();
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NSLOTS; ++i) mbar_init(&full[i], 1);
         for (int i = 0; i < C::NPH; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&o_full[i], 1);
         }
-        mbar_init(q_full, 128);
-        mbar_init(q_empty, 1);
-        mbar_init(p_full, 128);
+        for (int b = 0; b < C::QBUF; ++b) {
+            mbar_init(&q_full[b], q_by_tma ? 1 : 128);
+            mbar_init(&q_empty[b], 1);
+        }
+        mbar_init(&p_full[0], 128);
+        mbar_init(&p_full[1], 128);
         mbar_init(o_empty, 128);
         mbar_init(drain, C::TWO_ISSUERS ? 2 : 1);
         for (int i = 0; i < C::NDYN; ++i) {
@@ -270,6 +305,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
 #pragma unroll
         for (int k = 0; k < C::NSLOTS; ++k) hist[k] = 0;
         bool ok = true;
+        uint32_t kq = 0;                                    // q tiles loaded (items with tokens)
         uint32_t dk = 0;                                    // dynamic items taken so far
         // the item after `cur`: by the stride, else the next one of the counter,
         // published in the next item slot (-1 there: no more items)
@@ -310,6 +346,23 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             }
             __syncwarp();
             const int nc = (w.n + C::CHUNK - 1) / C::CHUNK;
+            if (q_by_tma) {
+                // the item's q rows into tile kq % 2 once the item two back has no S
+                // product left to read it: rows (query i, head h * group + g) for all i,
+                // g, i.e. row i * group + g of the tile
+                const uint32_t b = kq & 1u;
+                if (!mbar_wait(&q_empty[b], ((kq >> 1) & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0)
+                    mbar_arrive_expect_tx(&q_full[b], (uint32_t)(C::NH * a.group * a.num_queries * 128));
+                __syncwarp();
+                if (lane < C::NH)
+                    tma_load_3d(qs + b * C::Q_BYTES + lane * C::Q_SLICE, &tmap_q, lane * C::BOX_ELEMS,
+                                w.h * a.group, w.s * a.num_queries, &q_full[b], policy);
+                ++kq;
+            }
             // K or V of chunk c into the next slot, once the products that read the
             // slot's previous contents (the element NSLOTS back) are done
             auto issue = [&](int c, bool is_v) -> bool {
@@ -349,12 +402,16 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
             *abort_flag = 1;
             const uint32_t issued = seq;
+            const volatile int never = 0;
             for (int slot = lane; slot < C::NSLOTS; slot += 32) {
                 if ((uint32_t)slot < issued) {
                     const uint32_t last = issued - 1 - ((issued - 1 - slot) % C::NSLOTS);
-                    const volatile int never = 0;
                     mbar_wait(&full[slot], (last / C::NSLOTS) & 1u, &never);
                 }
+            }
+            if (lane < 2 && (uint32_t)lane < kq) {            // the q tiles' last loads
+                const uint32_t last = kq - 1 - ((kq - 1 - lane) & 1u);
+                mbar_wait(&q_full[lane], (last >> 1) & 1u, &never);
             }
         }
     }
@@ -362,7 +419,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         // ------------------------------------------------------------ MMA issue
         const bool do_s = warp == 1;                     // issues S products (and commits q_empty)
         const bool do_pv = warp == C::PV_WARP;           // issues P.V products
-        uint32_t seq = 0, q_ph = 0, p_ph = 0, oe_ph = 0, gch = 0;
+        uint32_t seq = 0, kq = 0, oe_ph = 0, gch = 0;
         bool ok = true;
         // operand descriptors built once; every MMA adds a byte offset to one of them
         const uint64_t qdesc = tc::sw128_desc(smem_addr(qs), 16, 1024);                 // Q, K-major
@@ -372,7 +429,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         // S of global chunk g = Q K^T over its 64 tokens (stream element pos), into S
         // buffer g & 1 (token columns past the partition read stale rows; the softmax
         // masks them)
-        auto issue_s = [&](uint32_t pos, uint32_t g) -> bool {
+        auto issue_s = [&](uint32_t pos, uint32_t g, uint32_t qb) -> bool {
             const uint32_t buf = g & 1u;
             const int slot = pos % C::NSLOTS;
             if (!mbar_wait(&full[slot], (pos / C::NSLOTS) & 1u, abort_flag)) return false;
@@ -390,7 +447,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 for (int kk = 0; kk < KS; ++kk) {
                     const uint32_t koff = (kk >> 2) * C::SLICE_BYTES + (kk & 3) * 32;
                     const uint32_t qoff = (kk >> 2) * C::Q_SLICE + (kk & 3) * 32;
-                    tc::mma_ss(d, tc::desc_add(qdesc, qoff), tc::desc_add(kd, koff), IDESC_S, kk > 0);
+                    tc::mma_ss(d, tc::desc_add(qdesc, qb * C::Q_BYTES + qoff), tc::desc_add(kd, koff), IDESC_S, kk > 0);
                 }
                 tc::commit(&s_full[g % C::NPH]);    // also frees the slot for the producer
             }
@@ -439,8 +496,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         // P.V of chunk c, once its p is written (and, for the item's first chunk, the
         // previous item's O has been read out)
         auto pv_chunk = [&](uint32_t pos, int c, int n, uint32_t g) -> bool {
-            if (!mbar_wait(p_full, p_ph, abort_flag)) return false;
-            p_ph ^= 1u;
+            if (!mbar_wait(&p_full[g & 1u], (g >> 1) & 1u, abort_flag)) return false;
             if (c == 0) {
                 if (!mbar_wait(o_empty, oe_ph ^ 1u, abort_flag)) return false;
                 oe_ph ^= 1u;
@@ -463,19 +519,19 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             auto vpos = [&](int c) -> uint32_t {
                 return seq + (c + 1 < nc ? (uint32_t)(2 * c + 2) : (uint32_t)(2 * nc - 1));
             };
+            const uint32_t qb = kq % C::QBUF;                   // the item's q tile
             if (do_s) {
-                if (!mbar_wait(q_full, q_ph, abort_flag)) {
+                if (!mbar_wait(&q_full[qb], (kq / C::QBUF) & 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
-                q_ph ^= 1u;
                 tc::fence_after_sync();
             }
             if constexpr (C::TWO_ISSUERS) {
                 if (do_s) {
                     for (int c = 0; c < nc && ok; ++c) {
-                        ok = issue_s(kpos(c), gch + c);
-                        if (ok && c + 1 == nc && lane == 0) tc::commit(q_empty);   // Q may be replaced
+                        ok = issue_s(kpos(c), gch + c, qb);
+                        if (ok && c + 1 == nc && lane == 0) tc::commit(&q_empty[qb]);   // the tile may be replaced
                         __syncwarp();
                     }
                 } else {
@@ -483,13 +539,13 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 }
             } else {
                 // one thread: S(c+1) is issued before P.V(c), so it runs during softmax(c)
-                if (!(ok = issue_s(kpos(0), gch))) break;
-                if (nc == 1 && lane == 0) tc::commit(q_empty);        // last S of the item: Q may be replaced
+                if (!(ok = issue_s(kpos(0), gch, qb))) break;
+                if (nc == 1 && lane == 0) tc::commit(&q_empty[qb]);   // last S of the item: the tile may be replaced
                 __syncwarp();
                 for (int c = 0; c < nc && ok; ++c) {
                     if (c + 1 < nc) {
-                        if (!(ok = issue_s(kpos(c + 1), gch + c + 1))) break;
-                        if (c + 2 == nc && lane == 0) tc::commit(q_empty);
+                        if (!(ok = issue_s(kpos(c + 1), gch + c + 1, qb))) break;
+                        if (c + 2 == nc && lane == 0) tc::commit(&q_empty[qb]);
                         __syncwarp();
                     }
                     ok = pv_chunk(vpos(c), c, w.n, gch + c);
@@ -497,6 +553,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             }
             seq += 2 * nc;
             gch += nc;
+            ++kq;
         }
         if (!ok) {
             if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
@@ -519,7 +576,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
         T* outg = static_cast<T*>(a.out);
         const int Q = a.num_queries;
         const int R = a.group * Q;
-        uint32_t qe_ph = 0, gch = 0;
+        uint32_t gch = 0;
         // P.V of global chunk g done: barrier copy g % NPH, its (g / NPH)-th phase
         auto wait_pv = [&](uint32_t g) -> bool {
             return mbar_wait(&o_full[g % C::NPH], (g / C::NPH) & 1u, abort_flag);
@@ -538,11 +595,13 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             orow = ((int64_t)w.s * Q + qi) * a.num_heads + (int64_t)w.h * a.group + g;
             pos = ctx - Q + qi;
         };
-        // item w's query rows as the A tile (rows past the chunk are zero), once the
-        // previous item's last S product no longer reads the tile
-        auto stage_q = [&](const WorkItem& w, int ctx) -> bool {
-            if (!mbar_wait(q_empty, qe_ph ^ 1u, abort_flag)) return false;
-            qe_ph ^= 1u;
+        // item w (the k-th item with tokens) as the A tile k % QBUF (rows past the
+        // chunk are zero), once the item that last used the tile has no S product
+        // left to read it
+        auto stage_q = [&](const WorkItem& w, int ctx, uint32_t k) -> bool {
+            const uint32_t b = k % C::QBUF;
+            if (!mbar_wait(&q_empty[b], ((k / C::QBUF) & 1u) ^ 1u, abort_flag)) return false;
+            unsigned char* qt = qs + b * C::Q_BYTES;
             // all loads of this thread first, then the swizzled stores
             constexpr int VPR = D * 2 / 16;               // 16-byte chunks per row
             constexpr int PER = C::M * VPR / 128;         // chunks per thread
@@ -561,10 +620,10 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 const int e = ctid + u * 128;
                 const int lr = e / VPR;
                 const int cc = e % VPR;
-                *reinterpret_cast<uint4*>(qs + (cc >> 3) * C::Q_SLICE + lr * 128 + (((cc & 7) ^ (lr & 7)) << 4)) = v[u];
+                *reinterpret_cast<uint4*>(qt + (cc >> 3) * C::Q_SLICE + lr * 128 + (((cc & 7) ^ (lr & 7)) << 4)) = v[u];
             }
             tc::fence_proxy_async_smem();
-            mbar_arrive(q_full);
+            mbar_arrive(&q_full[b]);
             return true;
         };
         bool ok = true;
@@ -575,10 +634,21 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             const int st = next_static(cur);
             return st >= 0 ? st : read_dynamic(dk, ok);
         };
+        uint32_t kq = 0;                                 // items with tokens so far
+        // the next item's descriptor, looked up while the current item ends
+        WorkItem wpre{};
+        int cpre = 0, ipre = -1;
         int i = next_item(-1);
         while (i < total && ok) {
-            const WorkItem w = decode_item(a, i, false);
-            const int ctx = clamp_context(a, w.s, false);
+            WorkItem w;
+            int ctx;
+            if (ipre == i) {
+                w = wpre;
+                ctx = cpre;
+            } else {
+                w = decode_item(a, i, false);
+                ctx = clamp_context(a, w.s, false);
+            }
             if (w.n == 0) {                              // empty context: zero rows
                 const int nr = min(C::M, R - w.gc * C::M);
                 for (int e = ctid; e < nr * D; e += 128) {
@@ -590,7 +660,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 i = next_item(i);
                 continue;
             }
-            if (staged != i && !(ok = stage_q(w, ctx))) break;
+            if (!q_by_tma && staged != i && !(ok = stage_q(w, ctx, kq))) break;
             int64_t orow;
             int pos;
             row_in(w, ctx, m, orow, pos);
@@ -671,12 +741,10 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                 }
                 m_run = m_new;
                 l_run = l_run * corr + lsum;
-                if constexpr (C::PTMEM || C::PBUF == 2) {
-                    // p_full counts one arrival per thread and phase: a warp that is a chunk
-                    // ahead of the others must not arrive before the previous chunk's phase
-                    // completes, or its arrival would count toward that phase.  (With a
-                    // single P buffer the wait for the previous P.V below implies this.)
-                    if (gc >= 1 && !(ok = mbar_wait(p_full, (gc - 1) & 1u, abort_flag))) break;
+                if constexpr (C::PTMEM && PA_VERIFY_TC_PWAR == 0) {
+                    // S(gc) did not wait for P.V(gc - 2) here, so the phase of gc - 2 on this
+                    // copy is not known complete: wait for chunk gc - 1's phase, which follows it
+                    if (gc >= 1 && !(ok = mbar_wait(&p_full[(gc - 1) & 1u], ((gc - 1) >> 1) & 1u, abort_flag))) break;
                 }
                 if constexpr (C::PTMEM) {
                     // p over this chunk's S columns (already read): tokens half*32 .. +31 of row m
@@ -703,21 +771,22 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
                     tc::fence_proxy_async_smem();
                 }
                 tc::fence_before_sync();
-                mbar_arrive(p_full);
+                mbar_arrive(&p_full[gc & 1u]);
             }
             gch += nc;
             if (!ok) break;
-            // ---- the next item's Q tile now, so that its first S products run while
-            // this item's epilogue does
+            // ---- the next item now: its descriptor, and its q tile when the softmax
+            // warps stage it, so that its first S products run while this item's
+            // epilogue does
             const int inext = next_item(i);
             if (!ok) break;
-            {
-                if (inext < total) {
-                    const WorkItem wn = decode_item(a, inext, false);
-                    if (wn.n > 0) {
-                        if (!(ok = stage_q(wn, clamp_context(a, wn.s, false)))) break;
-                        staged = inext;
-                    }
+            if (inext < total) {
+                wpre = decode_item(a, inext, false);
+                cpre = clamp_context(a, wpre.s, false);
+                ipre = inext;
+                if (!q_by_tma && wpre.n > 0) {
+                    if (!(ok = stage_q(wpre, cpre, kq + 1))) break;
+                    staged = inext;
                 }
             }
             // ---- epilogue: O after the last chunk, normalised row or partition partials
@@ -760,6 +829,7 @@ __global__ void __launch_bounds__(VerifyTcCfg<T, D>::THREADS, 2)
             }
             tc::fence_before_sync();
             mbar_arrive(o_empty);
+            ++kq;
             i = inext;
         }
         if (!ok) {

@@ -273,6 +273,26 @@ bool encode_pool_map_blocks(CUtensorMap* map, const void* pool, pa_dtype dtype, 
     return r == CUDA_SUCCESS;
 }
 
+// q [num_seqs, num_queries, num_heads, head_dim] as the 3-D tensor (head_dim,
+// num_heads, num_seqs * num_queries), innermost first.  One box is one 128-byte
+// slice of head_dim x `group` heads x `num_queries` rows: the query rows of one
+// (sequence, kv head), landing as row i * group + g with the 128-byte swizzle.
+bool encode_q_map(CUtensorMap* map, const void* q, pa_dtype dtype, int head_dim, int num_heads, int rows,
+                  int group, int num_queries) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc || dtype == PA_F32 || group > 256 || num_queries > 256) return false;
+    const cuuint64_t elt = 2;
+    const CUtensorMapDataType t = dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_heads, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)head_dim * elt, (cuuint64_t)num_heads * head_dim * elt};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / elt), (cuuint32_t)group, (cuuint32_t)num_queries};
+    cuuint32_t estride[3] = {1u, 1u, 1u};
+    CUresult r = enc(map, t, 3, const_cast<void*>(q), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <typename T, int D, int GC, bool TENSOR>
 pa_status launch_decode(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                         int64_t pair_upper, cudaStream_t stream) {
@@ -384,7 +404,7 @@ pa_status launch_verify(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, cons
 
 template <typename T, int D>
 pa_status launch_verify_tc(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                           int64_t pair_upper, cudaStream_t stream) {
+                           const CUtensorMap& tq, int64_t pair_upper, cudaStream_t stream) {
     using C = pa_dev::VerifyTcCfg<T, D>;
     auto kern = pa_dev::verify_tc_kernel<T, D>;
     int dev = 0;
@@ -422,7 +442,7 @@ pa_status launch_verify_tc(const pa_dev::DecodeArgs& a, const CUtensorMap& tk, c
     const int64_t items_upper = pair_upper * a.num_kv_heads * a.n_gchunks;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items_upper, (int64_t)device_sms(dev) * occ));
     LaunchScope scope(PA_KERNEL_VERIFY, stream);
-    return launch_dependent(kern, dim3((unsigned)grid), dim3(C::THREADS), smem, stream, a, tk, tv);
+    return launch_dependent(kern, dim3((unsigned)grid), dim3(C::THREADS), smem, stream, a, tk, tv, tq);
 }
 
 std::atomic<int> g_verify_kernel{PA_VERIFY_AUTO};
@@ -858,25 +878,32 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
                              0) != PA_OK)
             return PA_ERR_CUDA;
     }
-    CUtensorMap tk, tv;
+    CUtensorMap tk, tv, tq;
     if (!encode_pool_map(&tk, k_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, block_size) ||
         !encode_pool_map(&tv, v_cache, dtype, head_dim, num_kv_heads, num_blocks, block_size, block_size))
         return PA_ERR_CUDA;
     const int64_t pair_upper = (int64_t)num_seqs * maxP;
     const int vk = g_verify_kernel.load(std::memory_order_relaxed);
     const bool tc5 = vk != PA_VERIFY_MMA_SYNC;
+    // The tcgen05 kernel loads an item's q tile by TMA when its rows are one tile
+    // (group x queries <= 64): q as (head_dim, num_heads, num_seqs x num_queries),
+    // a box of one 128-byte slice x group heads x num_queries rows.
+    std::memset(&tq, 0, sizeof(tq));
+    if (tc5 && PA_VERIFY_TC_QTMA && n_chunks == 1 &&
+        !encode_q_map(&tq, q, dtype, head_dim, num_heads, num_seqs * num_queries, group, num_queries))
+        return PA_ERR_CUDA;
     pa_status st;
     if (dtype == PA_F16) {
         if (tc5)
-            st = head_dim == 64 ? launch_verify_tc<__half, 64>(a, tk, tv, pair_upper, s)
-                                : launch_verify_tc<__half, 128>(a, tk, tv, pair_upper, s);
+            st = head_dim == 64 ? launch_verify_tc<__half, 64>(a, tk, tv, tq, pair_upper, s)
+                                : launch_verify_tc<__half, 128>(a, tk, tv, tq, pair_upper, s);
         else
             st = head_dim == 64 ? launch_verify<__half, 64>(a, tk, tv, pair_upper, s)
                                 : launch_verify<__half, 128>(a, tk, tv, pair_upper, s);
     } else {
         if (tc5)
-            st = head_dim == 64 ? launch_verify_tc<__nv_bfloat16, 64>(a, tk, tv, pair_upper, s)
-                                : launch_verify_tc<__nv_bfloat16, 128>(a, tk, tv, pair_upper, s);
+            st = head_dim == 64 ? launch_verify_tc<__nv_bfloat16, 64>(a, tk, tv, tq, pair_upper, s)
+                                : launch_verify_tc<__nv_bfloat16, 128>(a, tk, tv, tq, pair_upper, s);
         else
             st = head_dim == 64 ? launch_verify<__nv_bfloat16, 64>(a, tk, tv, pair_upper, s)
                                 : launch_verify<__nv_bfloat16, 128>(a, tk, tv, pair_upper, s);

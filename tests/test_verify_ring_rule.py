@@ -22,8 +22,12 @@ SRC = os.path.join(ROOT, "paged_kv_cache_381_b200", "csrc", "device", "verify_tc
 
 
 def _constants():
+    """Ring depths the default build can take (one per q-tile mode), NPH and the
+    static_assert bound on NSLOTS."""
     src = open(SRC).read()
-    nslots = int(re.search(r"#define PA_VERIFY_TC_SLOTS (\d+)", src).group(1))
+    m = re.search(r"#define PA_VERIFY_TC_SLOTS \(PA_VERIFY_TC_QTMA \? (\d+) : (\d+)\)", src)
+    nslots = [int(m.group(1)), int(m.group(2))] if m else \
+        [int(re.search(r"#define PA_VERIFY_TC_SLOTS (\d+)", src).group(1))]
     nph = int(re.search(r"static constexpr int NPH = (\d+);", src).group(1))
     limit = int(re.search(r"static_assert\(NSLOTS >= 3 && NSLOTS <= (\d+)", src).group(1))
     return nslots, nph, limit
@@ -64,7 +68,7 @@ def test_stream_order_matches_the_kernel_description():
 def test_refill_rule_holds_for_the_kernel_constants():
     nslots, nph, limit = _constants()
     d = _min_distance(nph)
-    assert d >= nslots, (d, nslots, nph)
+    assert all(d >= n for n in nslots), (d, nslots, nph)
     # the static_assert bound on NSLOTS is exactly what the rule allows
     assert d == limit, (d, limit)
 
