@@ -517,7 +517,8 @@ def sub_verify(pa, name, seed, dev, flush, peak, peak_kind, Q=6, steps=100, warm
     cfg = wl.CONFIGS[name]
     batch, q, lens = decode_case(pa, cfg, seed, dev, 0, queries=Q)
     out = torch.empty_like(q)
-    P = pa.pa_verify_partition_size(len(lens), Q, cfg.num_heads, cfg.num_kv_heads, 0)
+    P = pa.pa_verify_partition_size(len(lens), Q, cfg.num_heads, cfg.num_kv_heads, batch.max_context_len,
+                                    cfg.block_size, 0)
     batch.ensure_workspace(cfg.num_heads, 0)
 
     def step():
@@ -696,7 +697,8 @@ def run_native(args):
                                      "own streams) against the device-only step over the same loop")}}
 
     dec_bytes = (verify_kernel_bytes(cfg, lens, pa.pa_verify_partition_size(len(lens), Q, cfg.num_heads,
-                                                                           cfg.num_kv_heads, P), Q)
+                                                                           cfg.num_kv_heads, batch.max_context_len,
+                                                                           cfg.block_size, P), Q)
                  if Q > 1 else decode_kernel_bytes(cfg, lens, P, fused=args.merge == "fused"))
     traffic = None if args.num_seqs else recorded_traffic(kname, args.workload, Q)
     dram_pct = None if args.num_seqs else recorded_dram_pct(kname, args.workload, Q)

@@ -179,12 +179,21 @@ size_t pa_verify_workspace_size(int num_seqs, int num_queries, int num_heads, in
 
 /*
  * The partition pa_verify uses for these shapes: partition_size itself when
- * non-zero, else 1024 tokens when a kv head carries R = num_heads /
- * num_kv_heads x num_queries >= 32 query rows and num_seqs x num_kv_heads x
- * ceil(R / 64) >= 592, else 512.  No device work; never fails (argument checks
- * are pa_verify's).
+ * non-zero.  Otherwise, with R = num_heads / num_kv_heads x num_queries query
+ * rows per kv head, C = ceil(R / 64) row chunks and the item bound
+ * items(P) = num_seqs x ceil(max_context_len / P) x num_kv_heads x C:
+ *   2048 tokens when R >= 32, block_size >= 16, num_seqs x num_kv_heads x C
+ *        >= 592 and items(2048) >= 1776;
+ *   1024 tokens when R >= 32 and items(1024) >= 1776;
+ *   512 otherwise.
+ * Larger partitions write fewer split-K partials (R x (head_dim + 2) floats per
+ * kv head and partition) and cross fewer item boundaries; the bound keeps about
+ * six items per CTA of the kernel's grid.  max_context_len is the longest
+ * context (pa_verify passes min(max_context_len, max_blocks_per_seq x
+ * block_size)).  No device work; never fails (argument checks are pa_verify's).
  */
-int pa_verify_partition_size(int num_seqs, int num_queries, int num_heads, int num_kv_heads, int partition_size);
+int pa_verify_partition_size(int num_seqs, int num_queries, int num_heads, int num_kv_heads, int max_context_len,
+                             int block_size, int partition_size);
 
 /*
  * pa_verify -- multi-query paged attention: the target model's verification
@@ -205,8 +214,10 @@ int pa_verify_partition_size(int num_seqs, int num_queries, int num_heads, int n
  * row.  fp16 and bf16 only (tensor cores; fp32 returns PA_ERR_UNSUPPORTED);
  * 1 <= Q <= 64.  Long contexts are split and merged as in pa_decode; the
  * workspace (>= pa_verify_workspace_size bytes, 256-byte aligned) holds the
- * partials.  partition_size 0 lets pa_verify_partition_size choose (512 or
- * 1024 tokens); pa_verify_workspace_size(..., 0) covers either.
+ * partials.  partition_size 0 lets pa_verify_partition_size choose (512, 1024
+ * or 2048 tokens); pa_verify_workspace_size(..., 0) covers each.  An explicit
+ * partition_size is a multiple of 32 from 32 to 2048 with at most 128 blocks
+ * (the kernels' block-id table).
  */
 pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, const int32_t* context_lens, float scale,

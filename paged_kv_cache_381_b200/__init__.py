@@ -203,9 +203,11 @@ def pa_write_decode(k, v, slot_mapping, out, q, k_cache, v_cache, block_tables, 
     return out
 
 
-def pa_verify_partition_size(num_seqs, num_queries, num_heads, num_kv_heads, partition_size=0):
+def pa_verify_partition_size(num_seqs, num_queries, num_heads, num_kv_heads, max_context_len, block_size,
+                             partition_size=0):
     """The partition (tokens) pa_verify uses for these shapes."""
-    return int(lib().pa_verify_partition_size(num_seqs, num_queries, num_heads, num_kv_heads, partition_size))
+    return int(lib().pa_verify_partition_size(num_seqs, num_queries, num_heads, num_kv_heads, int(max_context_len),
+                                              int(block_size), partition_size))
 
 
 def pa_verify_workspace_size(num_seqs, num_queries, num_heads, head_dim, max_context_len, partition_size=0):

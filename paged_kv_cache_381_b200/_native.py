@@ -54,7 +54,7 @@ SIGNATURES = {
                                 c_void_p, c_void_p, c_float, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                 c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "pa_verify_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
-    "pa_verify_partition_size": (c_int, [c_int, c_int, c_int, c_int, c_int]),
+    "pa_verify_partition_size": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_int]),
     "pa_verify": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int, c_int,
                           c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_size_t,
                           c_void_p]),

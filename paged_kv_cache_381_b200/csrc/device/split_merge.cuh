@@ -23,7 +23,7 @@ namespace pa_dev {
 // kernel also lists the sequences with more than one partition for the reduce
 // and clears the fused-merge counters and the decode kernel's item counter for
 // this call.
-constexpr int kPlanBuckets = 1024 / 16 + 1;        // partitions of up to 1024 tokens
+constexpr int kPlanBuckets = 2048 / 16 + 1;        // partitions of up to 2048 tokens
 __device__ __forceinline__ void build_plan(const DecodeArgs& a, int2* plan, int* count, int* split_seqs,
                                            int* merge_count, int num_counters) {
     __shared__ int hist[kPlanBuckets];

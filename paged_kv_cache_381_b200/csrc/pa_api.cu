@@ -202,6 +202,14 @@ WsLayout ws_layout(int64_t S, int64_t Hq, int64_t D, int64_t maxP) {
 int resolve_partition(int partition_size) { return partition_size == 0 ? kDefaultPartition : partition_size; }
 
 bool valid_partition(int p) { return p >= 32 && p <= 1024 && p % 32 == 0; }
+// The verification kernels walk one partition's block ids from a table of 128
+// entries in shared memory, and the plan sorts partitions of up to 2048 tokens.
+constexpr int kMaxVerifyPartition = 2048;
+constexpr int kVerifyTableEntries = 128;
+bool valid_verify_partition_size(int p) { return p >= 32 && p <= kMaxVerifyPartition && p % 32 == 0; }
+bool valid_verify_partition(int p, int block_size) {
+    return valid_verify_partition_size(p) && p / block_size <= kVerifyTableEntries;
+}
 
 int64_t partitions_for(int64_t ctx, int64_t P) { return ctx <= P ? 1 : (ctx + P - 1) / P; }
 
@@ -786,24 +794,39 @@ pa_status pa_write_decode(const void* k, const void* v, const int64_t* slot_mapp
                        workspace, workspace_bytes, stream, num_tokens > 0 ? &w : nullptr);
 }
 
-int pa_verify_partition_size(int num_seqs, int num_queries, int num_heads, int num_kv_heads, int partition_size) {
+int pa_verify_partition_size(int num_seqs, int num_queries, int num_heads, int num_kv_heads, int max_context_len,
+                             int block_size, int partition_size) {
     if (partition_size != 0) return partition_size;
-    if (num_seqs <= 0 || num_queries <= 0 || num_kv_heads <= 0 || num_heads <= 0) return kDefaultPartition;
+    if (num_seqs <= 0 || num_queries <= 0 || num_kv_heads <= 0 || num_heads <= 0 || block_size <= 0)
+        return kDefaultPartition;
     const int64_t rows = (int64_t)num_heads / num_kv_heads * num_queries;
-    const int64_t items = (int64_t)num_seqs * num_kv_heads * ((rows + 63) / 64);
+    const int64_t per_seq = (int64_t)num_kv_heads * ((rows + 63) / 64);
+    const int64_t ctx = std::max<int64_t>(1, max_context_len);
+    auto items = [&](int64_t P) { return (int64_t)num_seqs * ((ctx + P - 1) / P) * per_seq; };
     // A split partition writes rows x (head_dim + 2) fp32 partials per kv head, which
     // the reduce reads back: at 32 rows or more that is over a tenth of the K/V bytes
-    // of a 512-token partition.  There, and with enough (sequence, kv head) items to
-    // fill the GPU without splitting, 1024-token partitions halve the partials and the
-    // per-item start-up of the kernel (their workspace need is below the 512-token one
-    // that pa_verify_workspace_size reports for partition_size 0).
-    return rows >= 32 && items >= 4 * 148 ? 1024 : kDefaultPartition;
+    // of a 512-token partition.  There, larger partitions write fewer partials and
+    // cross fewer item boundaries, as long as the work still spreads over the grid:
+    // about six items per CTA of its 2 x 148 (the bound counts every sequence at the
+    // longest context), and, for 2048, enough (sequence, kv head) items without any
+    // split.  Their workspace need is below the 512-token one that
+    // pa_verify_workspace_size reports for partition_size 0.
+    constexpr int64_t kItems = 6 * 2 * 148;
+    if (rows < 32) return kDefaultPartition;
+    if (block_size >= 16 && num_seqs * per_seq >= 4 * 148 && items(2048) >= kItems) return 2048;
+    if (items(1024) >= kItems) return 1024;
+    return kDefaultPartition;
 }
 
 size_t pa_verify_workspace_size(int num_seqs, int num_queries, int num_heads, int head_dim, int max_context_len,
                                 int partition_size) {
-    if (num_queries <= 0) return 0;
-    return pa_decode_workspace_size(num_seqs, num_queries * num_heads, head_dim, max_context_len, partition_size);
+    const int P = resolve_partition(partition_size);
+    if (num_queries <= 0 || num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+        !valid_verify_partition_size(P))
+        return 0;
+    const int64_t maxP = partitions_for(max_context_len, P);
+    if (maxP <= 1) return 0;
+    return ws_layout(num_seqs, (int64_t)num_queries * num_heads, head_dim, maxP).total;
 }
 
 pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
@@ -820,8 +843,11 @@ pa_status pa_verify(void* out, const void* q, const void* k_cache, const void* v
     const int group = num_heads / num_kv_heads;
     const int rows = group * num_queries;
     const int n_chunks = (rows + 63) / 64;
-    const int P = pa_verify_partition_size(num_seqs, num_queries, num_heads, num_kv_heads, partition_size);
-    if (!valid_partition(P)) return PA_ERR_INVALID_ARG;
+    const int64_t table_cap0 = (int64_t)max_blocks_per_seq * block_size;
+    const int P = pa_verify_partition_size(num_seqs, num_queries, num_heads, num_kv_heads,
+                                           (int)std::min<int64_t>(max_context_len, table_cap0), block_size,
+                                           partition_size);
+    if (!valid_verify_partition(P, block_size)) return PA_ERR_INVALID_ARG;
     if (num_seqs == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;

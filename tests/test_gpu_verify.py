@@ -107,6 +107,25 @@ def test_split_partitions(P):
     assert_close(got, _oracle(inp, b, q), "f16", f"P{P}")
 
 
+@pytest.mark.parametrize("P,bs", [(1024, 16), (2048, 16), (2048, 32)])
+def test_large_partitions(P, bs):
+    """1024- and 2048-token partitions (the sizes pa_verify picks for many query
+    rows per kv head): contexts of one to three partitions and a last partition
+    shorter than Q, merged by the reduce kernel."""
+    lens = (4099, 2049, 2048, 1030, 6)
+    cfg = _cfg("bf16", 64, 8, 128, bs, lens=lens)
+    inp, b, q, got = _run(cfg, 6, seed=P + bs, partition_size=P)
+    assert_close(got, _oracle(inp, b, q), "bf16", f"P{P} bs{bs}")
+
+
+def test_partition_beyond_the_block_table_is_refused():
+    """A partition of more than 128 blocks (2048 tokens of 8-token blocks) does
+    not fit the kernels' block-id table: pa_verify refuses it."""
+    cfg = _cfg("bf16", 64, 8, 128, 8, lens=(3000, 40))
+    with pytest.raises(pa.PagedAttentionError):
+        _run(cfg, 6, partition_size=2048)
+
+
 def test_single_query_matches_decode_oracle():
     cfg = _cfg("bf16", 32, 8, 128, 16, lens=(1, 16, 17, 90, 777))
     inp, b, q, got = _run(cfg, 1)

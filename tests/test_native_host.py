@@ -279,19 +279,26 @@ def test_verify_workspace_and_argument_rules(pa):
 
 
 def test_verify_partition_choice(pa):
-    """partition_size 0: 1024 tokens once a kv head carries >= 32 query rows
-    and (sequence, kv head, 64-row chunk) items reach 592, else 512; an
-    explicit size is kept; the 0-partition workspace covers the 1024 choice."""
-    assert pa.pa_verify_partition_size(256, 6, 64, 8) == 1024       # 48 rows, 2048 items
-    assert pa.pa_verify_partition_size(64, 6, 32, 32) == 512        # 6 rows
-    assert pa.pa_verify_partition_size(8, 6, 64, 8) == 512          # 64 items
-    assert pa.pa_verify_partition_size(74, 4, 64, 8) == 1024        # 32 rows, 592 items
-    assert pa.pa_verify_partition_size(73, 4, 64, 8) == 512         # 584 items
-    assert pa.pa_verify_partition_size(256, 3, 64, 8) == 512        # 24 rows
-    assert pa.pa_verify_partition_size(8, 16, 64, 8) == 512         # 128 rows per kv head: 2 chunks, 128 items
-    assert pa.pa_verify_partition_size(256, 6, 64, 8, 256) == 256
+    """partition_size 0, R query rows per kv head, C = ceil(R / 64), items(P) =
+    seqs x ceil(ctx / P) x kv heads x C: 2048 tokens when R >= 32, blocks of 16
+    or more, seqs x kv heads x C >= 592 and items(2048) >= 1776; 1024 when
+    R >= 32 and items(1024) >= 1776; else 512.  An explicit size is kept; the
+    0-partition workspace covers every choice."""
+    P = pa.pa_verify_partition_size
+    assert P(256, 6, 64, 8, 7918, 16) == 2048       # 70b-shaped: 48 rows, items(2048) = 8192
+    assert P(256, 6, 64, 8, 7918, 8) == 1024        # 8-token blocks: 2048 tokens would be 256 blocks
+    assert P(8, 6, 64, 8, 32768, 16) == 1024        # long contexts: items(2048) = 1024, items(1024) = 2048
+    assert P(8, 6, 64, 8, 16384, 16) == 512         # items(1024) = 1024
+    assert P(64, 6, 32, 32, 2049, 16) == 512        # 7b-shaped: 6 rows
+    assert P(256, 3, 64, 8, 8192, 16) == 512        # 24 rows
+    assert P(73, 4, 64, 8, 8192, 16) == 1024        # 32 rows, 584 unsplit items: no 2048
+    assert P(74, 4, 64, 8, 8192, 16) == 2048        # 592 unsplit items, items(2048) = 2368
+    assert P(74, 4, 64, 8, 6144, 16) == 2048        # items(2048) = 74 x 3 x 8 = 1776, the bound itself
+    assert P(74, 4, 64, 8, 4096, 16) == 1024        # items(2048) = 1184, items(1024) = 2368
+    assert P(256, 6, 64, 8, 8192, 16, 256) == 256
     for S, Q, Hq, D, ctx in ((256, 6, 64, 128, 8192), (64, 6, 32, 128, 2048), (8, 4, 64, 64, 32768)):
-        assert pa.pa_verify_workspace_size(S, Q, Hq, D, ctx, 0) >= pa.pa_verify_workspace_size(S, Q, Hq, D, ctx, 1024)
+        for p in (1024, 2048):
+            assert pa.pa_verify_workspace_size(S, Q, Hq, D, ctx, 0) >= pa.pa_verify_workspace_size(S, Q, Hq, D, ctx, p)
 
 
 def test_verify_kernel_selection(pa):
