@@ -600,8 +600,12 @@ def run_native(args):
     cfg = wl.CONFIGS[args.workload]
     seed = args.seed + rank                       # independent replica per rank
     Q = args.queries
-    P = args.partition_size or cfg.partition_size
+    # decode: the workload's partition; verification: the one pa_verify picks
+    # (partition_size 0) unless --partition-size names one
+    P = args.partition_size or (0 if Q > 1 else cfg.partition_size)
     batch, q, lens = decode_case(pa, cfg, seed, dev, P, num_seqs=args.num_seqs, queries=Q)
+    P_used = (pa.pa_verify_partition_size(len(lens), Q, cfg.num_heads, cfg.num_kv_heads, batch.max_context_len,
+                                          cfg.block_size, P) if Q > 1 else P)
     out = torch.empty_like(q)
     batch.ensure_workspace(cfg.num_heads, P)
     step_kv = kv_bytes(cfg, lens)
@@ -707,7 +711,7 @@ def run_native(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-        "config": workload_config(args, cfg, lens, P, world),
+        "config": workload_config(args, cfg, lens, P_used, world),
         "pct_of_hbm_peak": value / world / peak,
         "ms_per_step_median": ms_median,
         "pct_of_spec_peak": value / world / SPEC_HBM_GBS,
