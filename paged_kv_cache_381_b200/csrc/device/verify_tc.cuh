@@ -7,8 +7,8 @@
 // items, partitions, partials and the reduce are shared with decode.
 //
 // Design (2 CTAs per SM, each holding 256 of the SM's 512 TMEM columns):
-//  * Item = (sequence, partition of 512 or 1024 tokens, kv head, chunk of <= 64
-//    query rows).  The rows form one M = 64 tile; the partition is walked in
+//  * Item = (sequence, partition of 512, 1024 or 2048 tokens, kv head, chunk of
+//    <= 64 query rows).  The rows form one M = 64 tile; the partition is walked in
 //    chunks of 64 tokens.  A CTA walks the length-sorted plan with a fixed
 //    stride; the last rounds are dealt from an atomic counter by the producer,
 //    which publishes each item's index to the other warps in item slots.
@@ -33,11 +33,12 @@
 //    issuers.
 //  * Warps 2-5 (one TMEM lane quarter each; a quarter's first 16 lanes hold 16
 //    rows of an M = 64 accumulator, read as two half-warps of 32 columns)
-//    stage q, take the exact max of the chunk (causal mask, only where a
+//    stage q when its rows are not one TMA box, take the exact max of the chunk (causal mask, only where a
 //    thread's tokens need it; max over raw scores, scaled once), rescale O in TMEM
 //    when the running max grows by more than 8 (base 2), write p over the
-//    chunk's S columns, and finally read O, normalise and store (or store the
-//    partition's partials).  For bf16, p is split into a 16-bit value and its
+//    chunk's S columns (arriving on one of two p_full copies), and finally read
+//    O, normalise and store (or store the partition's partials) and release O
+//    to the next item's first P.V.  For bf16, p is split into a 16-bit value and its
 //    remainder (two products, as in decode); an fp16 p keeps 11 significant
 //    bits and goes in one product.
 //  * All waits are bounded; TMEM is freed after a final commit has drained
