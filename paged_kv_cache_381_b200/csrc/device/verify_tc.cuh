@@ -74,11 +74,13 @@ namespace pa_dev {
 #ifndef PA_VERIFY_TC_DYN_ROUNDS
 // The last rounds of the length-sorted plan (its shortest items) are handed out
 // one at a time from an atomic counter; 0: every item by the fixed stride.
-// Measured on B200 (6 candidate tokens, one box, three runs each): 0 / 2 / 3
-// rounds 249.9 / 247.7 / 248.2 us on the 70B-shaped batch, 215.6 / 212.2 /
-// 212.7 us (7B), 215.0 / 211.5 / 211.4 us (long contexts); the kernel without
-// the item slots 248.4 / 214.7 / 213.6 us.
-#define PA_VERIFY_TC_DYN_ROUNDS 2
+// Measured on B200 (6 candidate tokens, one box, three runs each, each batch at
+// the partition pa_verify picks): 2 / 4 / 6 rounds 235.2 / 230.6 / 233.2 us on
+// the 70B-shaped batch (2048-token partitions), 207.3 / 207.9 / 208.8 us (7B,
+// 512), 195.5 / 196.5 / 196.9 us (long contexts, 1024); with the earlier
+// 512-token partitions on the 70B batch, 0 / 2 / 3 rounds 249.9 / 247.7 /
+// 248.2 us.
+#define PA_VERIFY_TC_DYN_ROUNDS 4
 #endif
 #ifndef PA_VERIFY_TC_PTMEM
 #define PA_VERIFY_TC_PTMEM 1     // 1: p written to tensor memory over its S buffer, P.V reads A from there
